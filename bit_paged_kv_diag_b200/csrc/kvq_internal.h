@@ -1,0 +1,72 @@
+// kvq_internal.h -- parameter blocks shared by the host code and the kernels of libkvq.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvq {
+
+// Device status bits (same values as KVQ_DEV_* in include/kvq.h).
+constexpr int KVQ_DEV_BAD_PAGE_BIT = 1;
+constexpr int KVQ_DEV_BAD_POS_BIT = 2;
+constexpr int KVQ_DEV_TIMEOUT_BIT = 4;
+
+struct AppendParams {
+  uint8_t* pool_layer;            // block(0, 0) of the layer
+  const __half* k;                // [T][Hkv][128]
+  const __half* v;                // [T][Hkv][128]
+  const int32_t* cu_new_tokens;   // [batch+1]
+  const int32_t* seq_lens;        // [batch], before the append
+  const int32_t* page_table;      // [batch][max_pages_per_seq]
+  int32_t* status;                // device status word
+  int batch;
+  int total_new_tokens;
+  int num_kv_heads;
+  int num_pages;
+  int page_size;
+  int max_pages_per_seq;
+  float cb;                       // fp32 nearest 1/sqrt(hadamard_block)
+};
+
+// Tokens per decode tile (one shared-memory ring slot per tile).
+constexpr int kTileTokens = 64;
+// fp32 words per (partial, query) record in the split scratch: o'[128], m, l, 2 pad.
+constexpr int kPartStride = 132;
+
+struct DecodeParams {
+  const uint8_t* pool_layer;      // block(0, 0) of the layer
+  const __half* q;                // [batch][Hq][128]
+  const int32_t* seq_lens;        // [batch], tokens to attend
+  const int32_t* page_table;      // [batch][max_pages_per_seq]
+  __half* out;                    // [batch][Hq][128]
+  float* part;                    // split partials [slots][G][kPartStride]
+  int32_t* tile_prefix;           // [batch+1] tiles-per-sequence prefix (per KV head)
+  int32_t* status;
+  int batch;
+  int num_kv_heads;
+  int group;                      // G = Hq / Hkv
+  int num_pages;
+  int page_size;
+  int max_pages_per_seq;
+  int hadamard_block;
+  float q_scale;                  // softmax_scale * log2(e)
+  float cb;                       // fp32 nearest 1/sqrt(hadamard_block)
+  int total_warps;                // W: warps in the split pass grid
+};
+
+// Host-side launchers (return 0 on success, <0 on an unsupported shape or a launch
+// error).
+int launch_append(const AppendParams& p, int block, cudaStream_t stream);
+
+struct DecodeLaunch {
+  int grid;          // CTAs of the split pass
+  int warps;         // total warps (grid * warps per CTA)
+  size_t smem;       // dynamic shared memory per CTA
+};
+// Shape of the split pass for a batch (grid sized to fill every SM).
+int plan_decode(int group, int page_size, int batch, int num_sms, DecodeLaunch* out);
+int max_decode_warps(int num_sms);
+int launch_decode(const DecodeParams& p, const DecodeLaunch& L, cudaStream_t stream);
+
+}  // namespace kvq

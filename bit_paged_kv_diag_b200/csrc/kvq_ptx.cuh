@@ -1,0 +1,183 @@
+// kvq_ptx.cuh -- thin inline-PTX wrappers used by the sm_100a kernels of libkvq.
+//
+// Bulk asynchronous copies (cp.async.bulk, the 1-D TMA form) with mbarrier
+// completion, bounded mbarrier waits, 256-bit global loads, the packed fp32x2
+// arithmetic of sm_100, and the legacy-path tensor-core MMA (mma.sync m16n8k16,
+// f16 x f16 -> f32).  No multicast form of any copy is used anywhere.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace kvq {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier --
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Order this thread's earlier generic-proxy shared-memory accesses before later
+// async-proxy accesses (a bulk copy overwriting a slot that was just read).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of a barrier, giving up after `limit_ns` nanoseconds.
+// Returns false on timeout (the caller records KVQ_DEV_TIMEOUT and stops using the
+// slot); never spins forever.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing bytes on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// --------------------------------------------------------------- global io --
+// 256-bit read-only global load (sm_100): 8 x 32-bit words.
+struct u32x8 {
+  uint32_t w[8];
+};
+
+__device__ __forceinline__ u32x8 ldg_256_stream(const void* p) {
+  u32x8 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]),
+                 "=r"(r.w[5]), "=r"(r.w[6]), "=r"(r.w[7])
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void stg_128(void* p, uint32_t a, uint32_t b, uint32_t c,
+                                        uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+// ------------------------------------------------------------ shared loads --
+__device__ __forceinline__ uint4 lds_128(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+
+__device__ __forceinline__ uint2 lds_64(uint32_t addr) {
+  uint2 r;
+  asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+  return r;
+}
+
+__device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
+  uint16_t r;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
+  return r;
+}
+
+// ------------------------------------------------------------- bit tricks --
+__device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t mask, uint32_t x) {
+  // (a & mask) ^ x in one LOP3.
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(a), "r"(mask), "r"(x));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Two signed 4-bit codes -> half2, exact.  The nibbles at bits [4s, 4s+4) and
+// [16+4s, 16+4s+4) of w (s = 0 or 1) become the low and high halves.
+//   s = 0: (w & 0x000F000F) ^ 0x64086408 = fp16(1024 + (n ^ 8)) per half, and
+//          n ^ 8 = n + 8 for a 4-bit two's-complement n, so subtracting 1032 gives n.
+//   s = 1: (w & 0x00F000F0) ^ 0x64806480 = fp16(1024 + 16 (n + 8)); times 1/16
+//          minus 72 gives n.  Every intermediate is an exactly representable fp16.
+__device__ __forceinline__ uint32_t nib_lo_to_half2(uint32_t w) {
+  uint32_t x = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);
+  const uint32_t k1032 = 0x64086408u;  // half2(1032, 1032)
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(k1032));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t nib_hi_to_half2(uint32_t w) {
+  uint32_t x = lop3_and_xor(w, 0x00F000F0u, 0x64806480u);
+  const uint32_t k16th = 0x2C002C00u;  // half2(1/16, 1/16)
+  const uint32_t km72 = 0xD480D480u;   // half2(-72, -72)
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(k16th), "r"(km72));
+  return r;
+}
+
+// --------------------------------------------------------------- tensor core --
+// D = A * B + D, m16n8k16, A row-major 16x16 f16, B col-major 16x8 f16, f32 accum.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
+  return static_cast<uint32_t>(__half_as_ushort(lo)) |
+         (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+}
+
+}  // namespace kvq

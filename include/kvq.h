@@ -1,0 +1,193 @@
+/*
+ * kvq.h -- C ABI of libkvq.so: rotated-INT4 paged KV cache on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources cited by page title and section):
+ *
+ *   [P1] "KVキャッシュを4ビットへ — SAW-INT4とシステムを踏まえたINT4量子化" (youngju.dev)
+ *   [P2] "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving"
+ *        (gist.science)
+ *
+ *   * Every new K/V row (fp16, head_dim = 128 channels) is rotated by an orthonormal
+ *     block-diagonal Hadamard transform (blocks of b = 32, 64 or 128 channels) [P1,
+ *     "回転のトリック — ブロック対角アダマール"], quantised token-wise to symmetric INT4
+ *     with one fp16 scale per token per KV head [P1, "素朴なINT4はなぜ崩れるのか"], and
+ *     appended into fixed-size pages addressed through a page table, without touching
+ *     past tokens [P1, "システムこそが設計である — 融合カーネル"].
+ *   * Paged GQA decode attention reads that cache: q is rotated with the same transform,
+ *     pages are dequantised in-kernel, softmax is computed online, and the output is
+ *     rotated back (the orthonormal Sylvester matrix is its own inverse) [P1,
+ *     "KVキャッシュこそが本当のボトルネックである理由": paged layout, fused attention].
+ *
+ * Readings of what the pages leave open (the CPU oracle takes the same readings):
+ *   rotation   fp32 butterfly, stages h = 1, 2, ..., b/2, then one multiply by the fp32
+ *              value nearest 1/sqrt(b); natural (Sylvester) order;
+ *   scale      s = fp16_rn(max_d |y_d| / 7) over all 128 channels, saturated at 65504;
+ *   codes      clamp(round_half_even(y_d / s), -8, 7), dividing by the stored fp16 s;
+ *              all codes 0 when s == 0;
+ *   packing    two codes per byte, low nibble = even channel, 4-bit two's complement;
+ *   GQA        query head hq reads KV head hq / (num_q_heads / num_kv_heads);
+ *   softmax    scale 1/sqrt(head_dim) unless given; an empty sequence outputs zeros.
+ *
+ * Pool layout (device memory, bytes; one pool holds every layer):
+ *   block(layer, page, kv_head) starts at
+ *       ((layer * num_pages + page) * num_kv_heads + kv_head) * page_size * 132
+ *   and holds, for the page_size token slots of that page:
+ *       [K codes  page_size x 64 B][V codes  page_size x 64 B]
+ *       [K scales page_size x fp16][V scales page_size x fp16]
+ *   Token at position pos of sequence b lives in page page_table[b][pos / page_size],
+ *   slot pos % page_size.  The page table is shared by all layers.
+ *
+ * Conventions for every call:
+ *   * Return value: KVQ_OK (0) or a negative status below.  Argument errors that the
+ *     host can see are returned before anything is launched.
+ *   * Calls that launch work are asynchronous and ordered on the given stream (a
+ *     cudaStream_t passed as void*; NULL = the legacy default stream).  They never
+ *     synchronise the host.  Asynchronous CUDA errors surface at the caller's next
+ *     synchronisation.
+ *   * A bad page id or an out-of-range position met on the device (a page-table entry
+ *     outside [0, num_pages), a position beyond max_pages_per_seq * page_size) is never
+ *     a trap: the kernel skips or redirects the access and ORs a code into the handle's
+ *     device status word, read with kvq_get_device_status().
+ *   * No C++ exception crosses this boundary.  No call changes seq_lens or the page
+ *     table; the caller advances seq_lens by the number of appended tokens.
+ *   * Ownership: the caller owns q, k, v, out, seq_lens, page_table and (optionally) the
+ *     pool; the library owns the handle, its split-KV scratch, its status word and the
+ *     pool when it allocated it.  One handle must not be used from two streams at once
+ *     (decode calls share the handle's scratch).
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define KVQ_OK 0
+#define KVQ_EINVAL (-1)        /* a null pointer, a negative size, a misaligned buffer  */
+#define KVQ_EUNSUPPORTED (-2)  /* a shape outside what the kernels implement            */
+#define KVQ_ENOPAGES (-3)      /* the pool or a sequence's page budget is too small      */
+#define KVQ_ECUDA (-4)         /* a CUDA runtime call failed (allocation, launch, copy)  */
+
+/* Bits of the device status word (kvq_get_device_status). */
+#define KVQ_DEV_BAD_PAGE 1     /* a page-table entry outside [0, num_pages)              */
+#define KVQ_DEV_BAD_POS 2      /* a position or length beyond the sequence's page budget */
+#define KVQ_DEV_TIMEOUT 4      /* a bounded wait in a kernel gave up (never expected)    */
+
+typedef struct kvq_cache kvq_cache; /* opaque, library-owned handle */
+
+/* Cache geometry; all values are host integers.
+ *   num_layers         layers sharing one pool and one page table            (>= 1)
+ *   num_kv_heads       Hkv                                                    (>= 1)
+ *   num_q_heads        Hq, a multiple of Hkv; G = Hq / Hkv must be 1, 2, 4 or 8
+ *   head_dim           D; only 128 is implemented
+ *   hadamard_block     b: 32, 64 or 128
+ *   page_size          S tokens per page: 16, 32, 64, 128 or 256
+ *   num_pages          pages per layer in the pool                            (>= 1)
+ *   max_batch          largest batch any call will pass                (1 .. 4096)
+ *   max_pages_per_seq  row length of the page table                          (>= 1) */
+typedef struct {
+  int32_t num_layers;
+  int32_t num_kv_heads;
+  int32_t num_q_heads;
+  int32_t head_dim;
+  int32_t hadamard_block;
+  int32_t page_size;
+  int32_t num_pages;
+  int32_t max_batch;
+  int32_t max_pages_per_seq;
+} kvq_desc;
+
+/* Bytes of the pool a descriptor needs:
+ * num_layers * num_pages * num_kv_heads * page_size * (head_dim + 4).
+ * Returns 0 for an invalid descriptor.  Host only. */
+KVQ_API size_t kvq_pool_bytes(const kvq_desc* d);
+
+/* Deterministic page assignment (host only; no CUDA call).  Walks page_order (host
+ * [num_pages], a permutation of 0..num_pages-1) or, when page_order is NULL, the pages
+ * 0..num_pages-1, and gives sequence b = 0, 1, ..., batch-1 in turn the next
+ * ceil(capacity_tokens[b] / page_size) pages.
+ *   capacity_tokens  host [batch], tokens each sequence must be able to hold (>= 0)
+ *   page_table       host out [batch][max_pages_per_seq]; unused entries are -1
+ * Returns KVQ_OK, KVQ_EINVAL, KVQ_EUNSUPPORTED (descriptor), or KVQ_ENOPAGES when a
+ * sequence needs more than max_pages_per_seq pages or the pool runs out.  The page
+ * table is then left partially written. */
+KVQ_API int kvq_assign_pages(const kvq_desc* d, int32_t batch, const int32_t* capacity_tokens,
+                     const int32_t* page_order, int32_t* page_table);
+
+/* Create a cache handle, the split-KV scratch and (optionally) the pool, and assign
+ * pages with kvq_assign_pages.
+ *   dev_pool    device buffer of >= kvq_pool_bytes(d) bytes, 16-byte aligned, owned by
+ *               the caller; NULL = the library allocates (cudaMalloc) and owns the pool
+ *   pool_bytes  size of dev_pool (ignored when dev_pool is NULL)
+ *   batch, capacity_tokens, page_order, page_table: as kvq_assign_pages; batch may be
+ *               0 (then no table is written) and must not exceed max_batch
+ *   out         receives the handle
+ * Uses the current CUDA device.  Blocks the host (allocation).  Returns KVQ_OK or a
+ * negative status; on failure nothing is left allocated and *out is NULL. */
+KVQ_API int kvq_alloc_pages(const kvq_desc* d, void* dev_pool, size_t pool_bytes, int32_t batch,
+                    const int32_t* capacity_tokens, const int32_t* page_order,
+                    int32_t* page_table, kvq_cache** out);
+
+/* Fused block-diagonal Hadamard rotation + token-wise INT4 quantisation + paged append
+ * for one layer [P1, "システムこそが設計である — 融合カーネル"].  One kernel launch.
+ *   layer             0 .. num_layers-1
+ *   k, v              device fp16 [total_new_tokens][num_kv_heads][128], token-major,
+ *                     32-byte aligned (rows are read with 256-bit loads)
+ *   cu_new_tokens     device int32 [batch+1], cu[0] = 0, non-decreasing,
+ *                     cu[batch] = total_new_tokens; sequence b appends tokens
+ *                     cu[b] .. cu[b+1]-1 of k/v
+ *   seq_lens          device int32 [batch], lengths BEFORE this append
+ *   page_table        device int32 [batch][max_pages_per_seq]
+ *   batch             0 .. max_batch;  total_new_tokens >= 0 (0 launches nothing)
+ * Token i of sequence b is written at position seq_lens[b] + i.  Nothing else in the
+ * pool is written.  Returns KVQ_OK or a negative status (before any launch). */
+KVQ_API int kvq_rotate_quant_append(kvq_cache* c, int32_t layer, const void* k, const void* v,
+                            const int32_t* cu_new_tokens, const int32_t* seq_lens,
+                            const int32_t* page_table, int32_t batch,
+                            int32_t total_new_tokens, void* stream);
+
+/* Paged GQA decode attention over the INT4 cache of one layer: one query token per
+ * sequence.  Two kernel launches (split-KV pass, then split combine + inverse rotation).
+ *   q              device fp16 [batch][num_q_heads][128], 16-byte aligned
+ *   seq_lens       device int32 [batch], lengths AFTER any append (tokens to attend)
+ *   page_table     device int32 [batch][max_pages_per_seq]
+ *   batch          0 .. max_batch
+ *   softmax_scale  multiplier of q.k; 0 means 1/sqrt(128)
+ *   out            device fp16 [batch][num_q_heads][128], 16-byte aligned; rows of
+ *                  empty sequences are zeros
+ * Uses the handle's scratch: calls on one handle must be ordered (one stream).
+ * Returns KVQ_OK or a negative status (before any launch). */
+KVQ_API int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, const int32_t* seq_lens,
+                         const int32_t* page_table, int32_t batch, float softmax_scale,
+                         void* out, void* stream);
+
+/* Device address of the pool (the caller's buffer, or the library's). NULL for NULL. */
+KVQ_API void* kvq_pool_ptr(const kvq_cache* c);
+
+/* Read and clear the handle's device status word (KVQ_DEV_* bits).  Synchronises the
+ * given stream.  Returns KVQ_OK or KVQ_ECUDA / KVQ_EINVAL. */
+KVQ_API int kvq_get_device_status(kvq_cache* c, int32_t* status, void* stream);
+
+/* Free library-owned memory (the handle, scratch, status word, and the pool if the
+ * library allocated it).  Synchronises the device first.  NULL is a no-op.  Returns
+ * KVQ_OK, or KVQ_ECUDA if an earlier asynchronous error is found. */
+KVQ_API int kvq_free(kvq_cache* c);
+
+/* Short static description of a status code. */
+KVQ_API const char* kvq_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,108 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol the header
+declares, its host-only page allocator is bit-exact with the oracle's, and argument errors
+are reported before any CUDA call."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_paged_kv_diag_b200 as kvq
+import oracle
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(kvq_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = kvq.lib()
+    declared = _declared_symbols()
+    assert declared, "no declarations found"
+    assert declared == set(kvq.EXPORTED)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def _desc(**kw):
+    base = dict(num_layers=2, num_kv_heads=8, num_q_heads=32, head_dim=128, hadamard_block=128,
+                page_size=16, num_pages=100, max_batch=16, max_pages_per_seq=20)
+    base.update(kw)
+    return kvq.Desc(**base)
+
+
+def test_pool_bytes_and_descriptor_validation():
+    d = _desc()
+    assert kvq.pool_bytes(d) == 2 * 100 * 8 * 16 * 132
+    for bad in [dict(head_dim=64), dict(hadamard_block=16), dict(page_size=24),
+                dict(num_q_heads=24), dict(num_q_heads=48), dict(max_batch=5000),
+                dict(num_layers=0), dict(num_pages=0)]:
+        assert kvq.pool_bytes(_desc(**bad)) == 0, bad
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3_4b_decode", "long_context", "ragged",
+                                  "prefill_append"])
+def test_page_assignment_bit_exact_with_oracle(name):
+    w = workloads.WORKLOADS[name]
+    lens = workloads.context_lengths(w) + w.new_tokens
+    P = workloads.pool_pages(w, lens)
+    mp = int(((lens.astype(np.int64) + w.page_size - 1) // w.page_size).max())
+    d = _desc(num_kv_heads=w.num_kv_heads, num_q_heads=w.num_q_heads, hadamard_block=w.block,
+              page_size=w.page_size, num_pages=P, max_batch=w.batch, max_pages_per_seq=mp)
+    order = workloads.page_order(w, P)
+    ours = kvq.assign_pages(d, lens, order)
+    ref = oracle.assign_pages(lens, w.page_size, P, mp, order)
+    assert np.array_equal(ours, ref)
+
+
+def test_page_assignment_random_and_errors():
+    rng = np.random.default_rng(0)
+    for trial in range(50):
+        B = int(rng.integers(1, 40))
+        S = int(rng.choice([16, 32, 64, 128, 256]))
+        cap = rng.integers(0, 2000, size=B).astype(np.int32)
+        need = (cap + S - 1) // S
+        P = int(need.sum()) + int(rng.integers(0, 10))
+        mp = int(need.max()) + int(rng.integers(0, 3))
+        order = rng.permutation(max(P, 1)).astype(np.int32) if trial % 2 else None
+        d = _desc(page_size=S, num_pages=max(P, 1), max_batch=B, max_pages_per_seq=max(mp, 1))
+        ours = kvq.assign_pages(d, cap, order)
+        ref = oracle.assign_pages(cap, S, max(P, 1), max(mp, 1), order)
+        assert np.array_equal(ours, ref)
+    d = _desc(num_pages=3, max_pages_per_seq=4, max_batch=2)
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.assign_pages(d, [40, 40])                       # 3 + 3 pages > 3
+    assert e.value.status == kvq.KVQ_ENOPAGES
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.assign_pages(d, [65])                           # 5 pages > 4 per sequence
+    assert e.value.status == kvq.KVQ_ENOPAGES
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.assign_pages(d, [-1])
+    assert e.value.status == kvq.KVQ_EINVAL
+
+
+def test_calls_reject_bad_arguments_before_any_cuda_call():
+    L = kvq.lib()
+    d = _desc()
+    h = ctypes.c_void_p()
+    # unsupported descriptor, null out pointer, misaligned caller pool: host-side errors
+    assert L.kvq_alloc_pages(ctypes.byref(_desc(head_dim=96)), None, 0, 0, None, None, None,
+                             ctypes.byref(h)) == kvq.KVQ_EUNSUPPORTED
+    assert L.kvq_alloc_pages(ctypes.byref(d), None, 0, 0, None, None, None, None) == kvq.KVQ_EINVAL
+    assert L.kvq_alloc_pages(ctypes.byref(d), 0x1003, 1 << 40, 0, None, None, None,
+                             ctypes.byref(h)) == kvq.KVQ_EINVAL
+    assert L.kvq_rotate_quant_append(None, 0, None, None, None, None, None, 0, 0, None) == kvq.KVQ_EINVAL
+    assert L.kvq_decode_attention(None, 0, None, None, None, 0, 0.0, None, None) == kvq.KVQ_EINVAL
+    assert L.kvq_free(None) == kvq.KVQ_OK
+    assert L.kvq_pool_ptr(None) is None
+    assert kvq.status_string(kvq.KVQ_ENOPAGES) == "not enough pages"

@@ -183,3 +183,38 @@ def scale_down(w: Workload, max_tokens: int, batch: Optional[int] = None) -> Wor
             v.context.append(v.context[-1] if v.context else max_tokens)
     v.num_layers = min(v.num_layers, 1)
     return v
+
+
+# ---------------------------------------------------------------- on-device ---
+# The same recipes drawn with torch's generator on a CUDA device, for workloads too
+# large to generate on the host (full-size benchmarks and sampled parity checks, which
+# copy back only the rows they check).  Values differ from the numpy draws above (a
+# different generator) but follow the same distributions.
+def kv_rows_torch(w: Workload, layer: int, kv: int, n_tokens: int, stream: int = 0,
+                  device="cuda"):
+    import torch
+    D, H = w.head_dim, w.num_kv_heads
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(np.random.SeedSequence([w.seed, _S_KV, layer, kv, stream]).generate_state(1)[0]))
+    if w.dist == "student_t3":
+        # t(3) = N(0,1) / sqrt(chi2(3)/3), chi2(3) = sum of 3 squared normals
+        z = torch.randn((n_tokens, H, D), generator=gen, device=device, dtype=torch.float32)
+        c = torch.randn((3, n_tokens, H, D), generator=gen, device=device, dtype=torch.float32)
+        x = z / torch.sqrt((c * c).sum(0) / 3.0)
+        return x.clamp_(-65504.0, 65504.0).to(torch.float16)
+    x = torch.randn((n_tokens, H, D), generator=gen, device=device, dtype=torch.float32)
+    ch, fac = _outlier_channels(w, layer, kv)
+    for h in range(H):
+        x[:, h, torch.as_tensor(ch[h], device=device)] *= torch.as_tensor(
+            fac[h], device=device, dtype=torch.float32)
+    if w.dist == "lognormal_outliers":
+        x *= torch.exp(0.5 * torch.randn((n_tokens, H, 1), generator=gen, device=device))
+    return x.clamp_(-65504.0, 65504.0).to(torch.float16)
+
+
+def q_rows_torch(w: Workload, layer: int, stream: int = 0, device="cuda"):
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(np.random.SeedSequence([w.seed, _S_Q, layer, stream]).generate_state(1)[0]))
+    x = torch.randn((w.batch, w.num_q_heads, w.head_dim), generator=gen, device=device)
+    return x.to(torch.float16)
