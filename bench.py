@@ -1,0 +1,534 @@
+#!/usr/bin/env python
+"""Benchmark of the rotated-INT4 paged KV-cache hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+
+One step = one decode step of the Qwen3-4B-shaped workload (36 layers, 8 KV heads, 32
+query heads, head_dim 128, Hadamard block 128, page 16, 16 sequences of 4096 cached
+tokens): for every layer, the fused rotate-quant-append of the step's token of each
+sequence, then paged GQA decode attention over 4097 tokens.  The step is captured once
+as a CUDA graph and replayed.  ``value`` is effective HBM GB/s: the step's algorithmic
+bytes (132 B per cached (token, KV head) + page-table, q and out bytes for decode; 2 x 256
+B read + 132 B written per appended (token, KV head)) over the device time per step, all
+ranks summed.  The cache (2.5 GB) is far larger than the 126 MB L2, so nothing is reused
+across steps.
+
+Also reported: the roofline of the decode-attention call, the prefill-append throughput
+(8 x 8192 new tokens in one call, b = 32/64/128), end-to-end throughput through the C ABI
+with host buffers, and the CPU oracle timed on a bounded sample of the same workload.
+
+Multi-GPU: replicas only (each rank runs the whole workload on its own GPU; the path has
+no exchange step), timing = max over ranks.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = ("INT4 paged decode-attn effective HBM GB/s (% of peak); fused quant-append tok/s")
+WORKLOAD = "qwen3_4b_decode"
+BYTES_PER_TOKEN_HEAD = 132
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def decode_bytes(lengths_after, num_kv_heads, num_q_heads, page_size):
+    lengths_after = np.asarray(lengths_after, np.int64)
+    cache = int(lengths_after.sum()) * num_kv_heads * BYTES_PER_TOKEN_HEAD
+    table = int(((lengths_after + page_size - 1) // page_size).sum()) * 4
+    qo = 2 * len(lengths_after) * num_q_heads * 128 * 2
+    return cache + table + qo
+
+
+def append_bytes(tokens, num_kv_heads):
+    return int(tokens) * num_kv_heads * (2 * 256 + 132)
+
+
+# --------------------------------------------------------------------- clocks --
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.2)
+        return self
+
+    def __exit__(self, *a):
+        self.result = None
+        if self.proc is None:
+            return False
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if sm:
+            self.result = {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                           "reasons": sorted(reasons), "samples": len(sm)}
+        return False
+
+
+# ------------------------------------------------------------------- GPU arm --
+def run_kvq(args, rank, world, local_rank):
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.WORKLOADS[WORKLOAD]
+    L = np.asarray(w.context, np.int32)                 # cached before the step
+    B, H, HQ, S, NL = w.batch, w.num_kv_heads, w.num_q_heads, w.page_size, w.num_layers
+    cap = L + 1
+    P = workloads.pool_pages(w, cap)
+    mp = int((cap.max() + S - 1) // S)
+    desc = kvq.Desc(NL, H, HQ, 128, w.block, S, P, B, mp)
+    cache, pt = kvq.alloc_pages(desc, cap, None)
+    ptd = torch.from_numpy(pt).to(dev)
+
+    # Prefill the cache through the append kernel (not timed).
+    zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+    cu_pre = torch.from_numpy(workloads.cu_seqlens(L)).to(dev)
+    for layer in range(NL):
+        kp = workloads.kv_rows_torch(w, layer, 0, int(L.sum()), stream=1, device=dev)
+        vp = workloads.kv_rows_torch(w, layer, 1, int(L.sum()), stream=1, device=dev)
+        kvq.rotate_quant_append(cache, layer, kp, vp, cu_pre, zeros, ptd)
+        del kp, vp
+    torch.cuda.synchronize()
+
+    # Step inputs, resident in HBM.
+    q = torch.stack([workloads.q_rows_torch(w, l, device=dev) for l in range(NL)])
+    kn = torch.stack([workloads.kv_rows_torch(w, l, 0, B, stream=2, device=dev) for l in range(NL)])
+    vn = torch.stack([workloads.kv_rows_torch(w, l, 1, B, stream=2, device=dev) for l in range(NL)])
+    out = torch.empty_like(q)
+    lens_before = torch.from_numpy(L).to(dev)
+    lens_after = torch.from_numpy(cap).to(dev)
+    cu_new = torch.arange(B + 1, dtype=torch.int32, device=dev)
+
+    # Timing events captured into the graph as event-record nodes ("external" events),
+    # so every replay stamps the start and end of each layer's decode-attention call.
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(NL)]
+
+    def step(instrument):
+        for l in range(NL):
+            kvq.rotate_quant_append(cache, l, kn[l], vn[l], cu_new, lens_before, ptd)
+            if instrument:
+                ev[l][0].record()
+            kvq.decode_attention(cache, l, q[l], lens_after, ptd, out=out[l])
+            if instrument:
+                ev[l][1].record()
+
+    # Eager warm-up (also initialises the library's launch state), then graph capture.
+    step(False)
+    torch.cuda.synchronize()
+    assert kvq.get_device_status(cache) == 0
+    side = torch.cuda.Stream(device=dev)
+    graph = torch.cuda.CUDAGraph()
+    instrumented = True
+    try:
+        with torch.cuda.graph(graph, stream=side):
+            step(True)
+    except Exception:
+        instrumented = False
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            step(False)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize()
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        t0.record()
+        for _ in range(args.steps):
+            graph.replay()
+        t1.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    dec_ms, dec_how = None, None
+    if instrumented:
+        try:  # the last timed replay's stamps
+            dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+            dec_how = "events inside the step graph (last timed step, mean of 36 layers)"
+        except Exception:
+            dec_ms = None
+    if dec_ms is None:
+        # Fallback: a graph of the 36 decode calls alone, timed around its replays.
+        dgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(dgraph, stream=side):
+            for l in range(NL):
+                kvq.decode_attention(cache, l, q[l], lens_after, ptd, out=out[l])
+        for _ in range(3):
+            dgraph.replay()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(3, args.steps // 4)
+        d0.record()
+        for _ in range(reps):
+            dgraph.replay()
+        d1.record()
+        torch.cuda.synchronize()
+        dec_ms = d0.elapsed_time(d1) / (reps * NL)
+        dec_how = "graph of the 36 decode calls alone, replayed back to back"
+        del dgraph
+    if world > 1:
+        import torch.distributed as dist
+        tms = torch.tensor([ms], device=dev)
+        dist.all_reduce(tms, op=dist.ReduceOp.MAX)
+        ms = float(tms.item())
+    status = kvq.get_device_status(cache)
+
+    ms_step = ms / args.steps
+    dec_b = decode_bytes(cap, H, HQ, S)
+    app_b = append_bytes(B, H)
+    step_bytes = NL * (dec_b + app_b)
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+
+    # End to end through the C ABI with host buffers: per step, H2D of q and the step's
+    # K/V rows from pinned memory, the step, D2H of the outputs.
+    hq = q.cpu().pin_memory()
+    hk, hv = kn.cpu().pin_memory(), vn.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        kn.copy_(hk, non_blocking=True)
+        vn.copy_(hv, non_blocking=True)
+        graph.replay()
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        import torch.distributed as dist
+        tms = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tms, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tms.item())
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
+    d2h = hout.numel() * 2
+
+    del graph
+    cache.close()
+    append = run_append_bench(dev) if rank == 0 else None
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4+fp16",
+        "data": "synthetic (seeded K/V with lognormal outlier channels and RMS multipliers)",
+        "config": {"workload": WORKLOAD, "layers": NL, "batch": B, "context": int(L[0]),
+                   "kv_heads": H, "q_heads": HQ, "head_dim": 128, "hadamard_block": w.block,
+                   "page_size": S, "global_batch": B * world, "seq_len": int(cap[0]),
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: 2.5 GB cache per step vs 126 MB L2",
+                   "graph": "one CUDA graph per step"},
+        "gpu_launches": args.steps * NL * 3,
+        "device_status": status,
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": round(e2e_ms, 5)},
+    }
+    if dec_ms is not None:
+        ach = dec_b / (dec_ms * 1e-3) / 1e9
+        line["roofline"] = {
+            "kernel": "decode attention (split pass + combine), one layer",
+            "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(ach / peak, 4), "peak_kind": peak_kind,
+            "traffic": _traffic("decode", dec_b), "us_per_launch": round(dec_ms * 1e3, 3),
+            "bytes_per_launch": dec_b, "timing": dec_how}
+    line["append"] = append
+    line["clocks"] = clk.result
+    return line
+
+
+def _traffic(kernel, alg_bytes):
+    """DRAM bytes per launch from the committed ncu summary, if it is for the current
+    kernel source; else None."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, "bit_paged_kv_diag_b200", "csrc", rec["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h != rec["source_sha256_16"]:
+            return None
+        return int(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def run_append_bench(dev, reps=20):
+    """Prefill-append stress: 8 x 8192 new tokens through one call, b = 32, 64, 128."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    w = workloads.WORKLOADS["prefill_append"]
+    B, H, S, T = w.batch, w.num_kv_heads, w.page_size, w.batch * w.new_tokens
+    cap = np.full(B, w.new_tokens, np.int32)
+    P = workloads.pool_pages(w, cap)
+    mp = int((cap.max() + S - 1) // S)
+    k = workloads.kv_rows_torch(w, 0, 0, T, stream=1, device=dev)
+    v = workloads.kv_rows_torch(w, 0, 1, T, stream=1, device=dev)
+    cu = torch.from_numpy(workloads.cu_seqlens(cap)).to(dev)
+    z = torch.zeros(B, dtype=torch.int32, device=dev)
+    res = {}
+    peak, _ = _peaks()
+    for block in w.blocks_sweep:
+        desc = kvq.Desc(1, H, w.num_q_heads, 128, block, S, P, B, mp)
+        cache, pt = kvq.alloc_pages(desc, cap, None)
+        ptd = torch.from_numpy(pt).to(dev)
+        for _ in range(3):
+            kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
+        b.record()
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) * 1e3 / reps
+        gbs = append_bytes(T, H) / (us * 1e-6) / 1e9
+        res[f"b{block}"] = {"us_per_call": round(us, 2), "tok_s": round(T / (us * 1e-6), 1),
+                            "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        assert kvq.get_device_status(cache) == 0
+        cache.close()
+    res["workload"] = "prefill_append: 8 x 8192 tokens, 8 KV heads, page 16, Student-t(3)"
+    res["traffic"] = _traffic("append", append_bytes(T, H))
+    return res
+
+
+# ------------------------------------------------------------- CPU oracle arm --
+def oracle_sample(budget_s, n_units_max=None):
+    """Time the CPU oracle on whole (sequence, KV head) units of one layer of the decode
+    workload: its step append (one token per sequence, all heads) and decode attention of
+    the unit's G query heads, fp64, one thread.  Returns (GB/s, description)."""
+    import oracle
+    w = workloads.WORKLOADS[WORKLOAD]
+    G, H, S = w.group, w.num_kv_heads, w.page_size
+    L = int(w.context[0])
+    nseq = 1
+    g = oracle.Geometry(1, H, w.num_q_heads, 128, w.block, S, nseq * ((L + 1 + S - 1) // S),
+                        (L + 1 + S - 1) // S)
+    cap = np.full(nseq, L + 1, np.int32)
+    pt = oracle.assign_pages(cap, S, g.num_pages, g.max_pages_per_seq)
+    pool = g.new_pool()
+    kp, vp = workloads.kv_rows(w, 0, 0, L * nseq, 1), workloads.kv_rows(w, 0, 1, L * nseq, 1)
+    oracle.rotate_quant_append(g, pool, 0, kp, vp, workloads.cu_seqlens([L] * nseq),
+                               np.zeros(nseq, np.int32), pt)
+    kn, vn = workloads.kv_rows(w, 0, 0, nseq, 2), workloads.kv_rows(w, 0, 1, nseq, 2)
+    q = workloads.q_rows(w, 0)[:nseq]
+    units, byt = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.rotate_quant_append(g, pool, 0, kn, vn, workloads.cu_seqlens([1] * nseq),
+                                   np.full(nseq, L, np.int32), pt)
+        byt += append_bytes(nseq, H)
+        for h in range(H):
+            for qi in range(G):
+                oracle.decode_one(g, pool, 0, q, cap, pt, 0, h * G + qi)
+            units += 1
+            byt += (L + 1) * BYTES_PER_TOKEN_HEAD + 2 * G * 256
+            if (time.perf_counter() - t0 >= budget_s) or (n_units_max and units >= n_units_max):
+                el = time.perf_counter() - t0
+                desc = (f"oracle (C, fp64 attention, 1 thread): step append of 1 token x {H} "
+                        f"KV heads + decode of {units} (sequence, KV head) units x {G} query "
+                        f"heads at {L + 1} tokens, one layer of {WORKLOAD}; {el:.2f} s")
+                return byt / el / 1e9, desc
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle as it stands, on host cores, same metric and
+    workload; each step a bounded sample sized so the whole run ends in a few minutes."""
+    if rank != 0:
+        return None
+    total = max(1, args.steps + args.warmup)
+    per_step = max(0.02, min(2.0, 150.0 / total))
+    for _ in range(args.warmup):
+        oracle_sample(per_step, n_units_max=1)
+    vals, descs = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, d = oracle_sample(per_step)
+        vals.append(v)
+        descs.append(d)
+    el = time.perf_counter() - t0
+    val = float(np.mean(vals))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": "bounded per step"},
+        "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": descs[-1] if descs else ""},
+        "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------ profiling cases --
+def run_kernel_case(which, calls):
+    """A small case of one kernel for ncu captures: ``decode`` = decode attention on one
+    layer of the Qwen3-4B-shaped workload (69 MB of cache); ``append`` = the prefill-append
+    call (8 x 8192 tokens, b = 128; 268 MB read, 69 MB written).  The kernel is launched
+    ``calls`` times after the setup."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    dev = torch.device("cuda", 0)
+    if which == "append":
+        w = workloads.WORKLOADS["prefill_append"]
+        B, H, S, T = w.batch, w.num_kv_heads, w.page_size, w.batch * w.new_tokens
+        cap = np.full(B, w.new_tokens, np.int32)
+        P = workloads.pool_pages(w, cap)
+        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S))
+        cache, pt = kvq.alloc_pages(desc, cap, None)
+        ptd = torch.from_numpy(pt).to(dev)
+        k = workloads.kv_rows_torch(w, 0, 0, T, stream=1, device=dev)
+        v = workloads.kv_rows_torch(w, 0, 1, T, stream=1, device=dev)
+        cu = torch.from_numpy(workloads.cu_seqlens(cap)).to(dev)
+        z = torch.zeros(B, dtype=torch.int32, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(calls):
+            kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
+    else:
+        w = workloads.WORKLOADS[WORKLOAD]
+        L = np.asarray(w.context, np.int32)
+        B, H, S = w.batch, w.num_kv_heads, w.page_size
+        cap = L + 1
+        P = workloads.pool_pages(w, cap)
+        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S))
+        cache, pt = kvq.alloc_pages(desc, cap, None)
+        ptd = torch.from_numpy(pt).to(dev)
+        kp = workloads.kv_rows_torch(w, 0, 0, int(cap.sum()), stream=1, device=dev)
+        vp = workloads.kv_rows_torch(w, 0, 1, int(cap.sum()), stream=1, device=dev)
+        kvq.rotate_quant_append(cache, 0, kp, vp, torch.from_numpy(workloads.cu_seqlens(cap)).to(dev),
+                                torch.zeros(B, dtype=torch.int32, device=dev), ptd)
+        del kp, vp
+        q = workloads.q_rows_torch(w, 0, device=dev)
+        lens = torch.from_numpy(cap).to(dev)
+        torch.cuda.synchronize()
+        for _ in range(calls):
+            kvq.decode_attention(cache, 0, q, lens, ptd)
+    torch.cuda.synchronize()
+    assert kvq.get_device_status(cache) == 0
+    cache.close()
+    print(json.dumps({"kernel_case": which, "calls": calls, "ok": True}))
+
+
+# ----------------------------------------------------------------------- main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", choices=["decode", "append"], default=None,
+                    help="run one small case of one kernel (for ncu captures) and exit")
+    ap.add_argument("--calls", type=int, default=3)
+    args = ap.parse_args()
+    if args.kernel_case:
+        run_kernel_case(args.kernel_case, args.calls)
+        return
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_kvq(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                v, d = oracle_sample(12.0)
+                line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": 1,
+                                        "kind": "oracle", "sample": d}
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

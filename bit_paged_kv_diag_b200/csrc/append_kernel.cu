@@ -8,24 +8,28 @@
 // kernel that rotates, quantises and appends into paged KV blocks without revisiting
 // past tokens).
 //
-// Work decomposition.  One group of 4 lanes handles one (token, KV head) pair: both
-// its K row and its V row (128 fp16 channels each).  Lane l of the group holds
-// channels [16l, 16l+16) and [64+16l, 64+16l+16), loaded as two 256-bit reads, so the
-// 4 lanes read the row's 256 bytes as two fully used 128-byte lines.  In channel-index
-// bits, bits 0-3 and bit 6 are inside a lane and bits 4-5 are across lanes, so the
-// butterfly stages h = 1, 2, 4, 8 and 64 are register-only and stages h = 16, 32 are
-// warp shuffles (xor 1, xor 2).  The stage order and every add/subtract are those of
-// the fixed-order fp32 butterfly (stages h = 1, 2, ..., b/2, pairs (i, i+h) with bit h
-// of i clear -> (a+c, a-c)), then one multiply by the fp32 constant nearest 1/sqrt(b),
-// each as a single IEEE operation, so rotated values, scales and codes are bit-exact
-// with any implementation of the same fixed-order butterfly.
+// Work decomposition.  Two lanes handle one row (the K row or the V row of one
+// (token, KV head) pair, 128 fp16 channels); a warp handles the K and V rows of 8 pairs.
+// Lane l of a row holds the 16-channel chunks 2j + l (j = 0..3), read with 256-bit loads:
+// channel index bits 0-3 and 5-6 are inside the lane and bit 4 is across the lane pair.
+// So the butterfly stages h = 1, 2, 4, 8, 32, 64 are register-only and stage h = 16 is one
+// warp shuffle.  Stages run in the fixed order h = 1, 2, ..., b/2, each pair (i, i+h) with
+// bit h of i clear becoming (a + c, a - c) as one IEEE fp32 add and one subtract, then one
+// multiply by the fp32 constant nearest 1/sqrt(b): rotated values are bit-exact with any
+// implementation of that fixed-order butterfly.  Pairs of channels go through the packed
+// fp32x2 add/sub/mul of sm_100 (each lane of the pair is still one IEEE operation), and
+// fp16 -> fp32 conversion rides in the first stage's mixed-precision adds.
 //
-// The row's absmax is a 2-step shuffle reduction over the group; the scale is
-// fp16_rn(max/7) (IEEE division); codes are round-half-even of y / s (IEEE division by
-// the stored fp16 scale), clamped to [-8, 7], packed two per byte (low nibble = even
-// channel).  After one 8-byte exchange with the neighbouring lane, every lane holds 16
-// contiguous code bytes and writes them with one 128-bit store; lanes 0 and 1 store the
-// K and V scales.
+// Quantisation: m = max |y| (lane-pair shuffle), s = fp16_rn(m / 7) (IEEE division, once
+// per row).  Codes are round-half-even of y / s, clamped to [-8, 7].  The fast path
+// multiplies by r = 1/s (IEEE reciprocal, once per row) and rounds with the 1.5 * 2^23
+// magic addend, whose sum carries the integer code in its low mantissa bits.  The
+// product y*r is within 2^-19 of the IEEE quotient y/s for |y/s| < 8, so whenever every
+// fractional part stays more than 2^-19 away from one half, both round to the same
+// integer; otherwise (a near-tie), and whenever s is subnormal or saturated, the lane
+// recomputes its codes with IEEE division -- codes stay bit-exact with division by the
+// stored fp16 scale.  Codes are packed two per byte (low nibble = even channel) and
+// written with 64-bit stores; lane 0 of the row stores the fp16 scale.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -37,97 +41,160 @@ namespace kvq {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kPairsPerBlock = 64;            // (token, head) pairs per CTA
-constexpr int kThreads = kPairsPerBlock * 4;  // 4 lanes per pair
+constexpr int kRowsPerBlock = 128;           // rows (K or V) per CTA
+constexpr int kThreads = kRowsPerBlock * 2;  // 2 lanes per row
+constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23
 
-// x[0..15] = channels [16l, 16l+16), x[16..31] = channels [64+16l, 64+16l+16).
-template <int BLOCK>
-__device__ __forceinline__ void rotate_row(float (&x)[32], int lane4, unsigned gmask, float cb) {
-  // In-lane stages: h = 1, 2, 4, 8 act on bits 0-3 of the in-group index.
-#pragma unroll
-  for (int h = 1; h <= 8; h *= 2) {
-    if (h < BLOCK) {
-#pragma unroll
-      for (int grp = 0; grp < 2; grp++) {
-#pragma unroll
-        for (int i = 0; i < 16; i++) {
-          if (i & h) continue;
-          const float a = x[grp * 16 + i];
-          const float c = x[grp * 16 + i + h];
-          x[grp * 16 + i] = __fadd_rn(a, c);
-          x[grp * 16 + i + h] = __fsub_rn(a, c);
-        }
-      }
-    }
-  }
-  // Cross-lane stages h = 16 (partner lane ^ 1) and h = 32 (partner lane ^ 2).  The
-  // lane holding the lower index computes own + other; the upper one other - own.  A
-  // single fused multiply-add with a +-1 multiplier rounds once, so
-  // fma(own, -1, other) is bit-identical to the IEEE difference other - own.
-#pragma unroll
-  for (int s = 0; s < 2; s++) {
-    const int h = 16 << s;
-    if (h < BLOCK) {
-      const int bit = 1 << s;
-      const float sgn = (lane4 & bit) ? -1.0f : 1.0f;
-#pragma unroll
-      for (int i = 0; i < 32; i++) {
-        const float other = __shfl_xor_sync(gmask, x[i], bit);
-        x[i] = __fmaf_rn(x[i], sgn, other);
-      }
-    }
-  }
-  // In-lane stage h = 64: channel 16l+i pairs with channel 64+16l+i.
-  if (64 < BLOCK) {
-#pragma unroll
-    for (int i = 0; i < 16; i++) {
-      const float a = x[i];
-      const float c = x[16 + i];
-      x[i] = __fadd_rn(a, c);
-      x[16 + i] = __fsub_rn(a, c);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 32; i++) x[i] = __fmul_rn(x[i], cb);
+__device__ __forceinline__ float cvt_f16(uint16_t h) {
+  // Exact fp16 -> fp32 through the mixed-precision add (h + -0.0 keeps signed zeros).
+  float d;
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(h), "f"(-0.0f));
+  return d;
 }
 
-__device__ __forceinline__ void load_row(const __half* row, int lane4, float (&x)[32]) {
+// Butterfly on two pairs at once: (a0,a1),(c0,c1) -> (a+c, a-c) per lane, IEEE fp32.
+__device__ __forceinline__ void bfly2(float& a0, float& a1, float& c0, float& c1) {
+  asm("{\n\t.reg .b64 pa, pc, ps, pd;\n\t"
+      "mov.b64 pa, {%0, %1};\n\tmov.b64 pc, {%2, %3};\n\t"
+      "add.rn.f32x2 ps, pa, pc;\n\tsub.rn.f32x2 pd, pa, pc;\n\t"
+      "mov.b64 {%0, %1}, ps;\n\tmov.b64 {%2, %3}, pd;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(c0), "+f"(c1));
+}
+
+// (x0, x1) <- (x0 * s + o0, x1 * s + o1), one rounding each: with s = +-1 this is the
+// IEEE sum or difference of the two operands.
+__device__ __forceinline__ void fma2(float& x0, float& x1, float s, float o0, float o1) {
+  asm("{\n\t.reg .b64 px, ps, po, pd;\n\t"
+      "mov.b64 px, {%0, %1};\n\tmov.b64 ps, {%2, %2};\n\tmov.b64 po, {%3, %4};\n\t"
+      "fma.rn.f32x2 pd, px, ps, po;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(s), "f"(o0), "f"(o1));
+}
+
+__device__ __forceinline__ void mul2(float& x0, float& x1, float s) {
+  asm("{\n\t.reg .b64 px, ps, pd;\n\t"
+      "mov.b64 px, {%0, %1};\n\tmov.b64 ps, {%2, %2};\n\t"
+      "mul.rn.f32x2 pd, px, ps;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(s));
+}
+
+// x[16j + e] = channel 16(2j + l) + e.
+template <int BLOCK>
+__device__ __forceinline__ void load_rotate(const __half* row, int l, unsigned pmask, float cb,
+                                            float (&x)[64]) {
+  u32x8 raw[4];
 #pragma unroll
-  for (int j = 0; j < 2; j++) {
-    // 32 bytes = 16 channels starting at channel 64j + 16*lane4.
-    const u32x8 r = ldg_256_stream(row + 64 * j + 16 * lane4);
+  for (int j = 0; j < 4; j++) raw[j] = ldg_256_stream(row + 16 * (2 * j + l));
+  // Stage h = 1 fused with the conversion: (a, c) -> (a + c, a - c).
+#pragma unroll
+  for (int j = 0; j < 4; j++)
 #pragma unroll
     for (int w = 0; w < 8; w++) {
-      const __half2 h2 = *reinterpret_cast<const __half2*>(&r.w[w]);
-      const float2 f = __half22float2(h2);
-      x[16 * j + 2 * w] = f.x;
-      x[16 * j + 2 * w + 1] = f.y;
+      const uint16_t lo = static_cast<uint16_t>(raw[j].w[w] & 0xffffu);
+      const uint16_t hi = static_cast<uint16_t>(raw[j].w[w] >> 16);
+      const float c = cvt_f16(hi);
+      float s, d;
+      asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(s) : "h"(lo), "f"(c));
+      asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(lo), "f"(c));
+      x[16 * j + 2 * w] = s;
+      x[16 * j + 2 * w + 1] = d;
+    }
+  // In-lane stages h = 2, 4, 8 (bits 1-3 of the chunk-local index).
+#pragma unroll
+  for (int h = 2; h <= 8; h *= 2)
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+#pragma unroll
+      for (int e = 0; e < 16; e += 2)
+        if (!(e & h)) bfly2(x[16 * j + e], x[16 * j + e + 1], x[16 * j + e + h], x[16 * j + e + h + 1]);
+  // Cross-lane stage h = 16: the lane holding the lower index computes own + other, the
+  // upper one other - own (fma with a +-1 multiplier rounds once: bit-identical).
+  if (16 < BLOCK) {
+    const float sgn = l ? -1.0f : 1.0f;
+#pragma unroll
+    for (int i = 0; i < 64; i += 2) {
+      const float o0 = __shfl_xor_sync(pmask, x[i], 1);
+      const float o1 = __shfl_xor_sync(pmask, x[i + 1], 1);
+      fma2(x[i], x[i + 1], sgn, o0, o1);
     }
   }
+  // In-lane stages h = 32 (chunk j with j ^ 1) and h = 64 (chunk j with j ^ 2).
+  if (32 < BLOCK) {
+#pragma unroll
+    for (int j = 0; j < 4; j += 2)
+#pragma unroll
+      for (int e = 0; e < 16; e += 2)
+        bfly2(x[16 * j + e], x[16 * j + e + 1], x[16 * (j + 1) + e], x[16 * (j + 1) + e + 1]);
+  }
+  if (64 < BLOCK) {
+#pragma unroll
+    for (int j = 0; j < 2; j++)
+#pragma unroll
+      for (int e = 0; e < 16; e += 2)
+        bfly2(x[16 * j + e], x[16 * j + e + 1], x[16 * (j + 2) + e], x[16 * (j + 2) + e + 1]);
+  }
+#pragma unroll
+  for (int i = 0; i < 64; i += 2) mul2(x[i], x[i + 1], cb);
 }
 
-// Quantise the rotated row; returns the fp16 scale bits and the packed codes, 8
-// channels per word: q[0], q[1] = group A (channels 16l..16l+15), q[2], q[3] = group
-// B (channels 64+16l..64+16l+15).
-__device__ __forceinline__ uint16_t quantise_row(const float (&y)[32], unsigned gmask,
-                                                 uint32_t (&q)[4]) {
+// Codes of 8 channels from their magic-rounded sums (low nibble = code & 0xF).
+__device__ __forceinline__ uint32_t pack8_magic(const float (&m)[8]) {
+  uint32_t b[4];
+#pragma unroll
+  for (int k = 0; k < 4; k++)
+    b[k] = (__float_as_uint(m[2 * k]) & 0xFu) | ((__float_as_uint(m[2 * k + 1]) & 0xFu) << 4);
+  return prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
+}
+
+// Quantise this lane's 64 rotated values of a row; q[2j], q[2j+1] = packed codes of
+// chunk j.  Returns the fp16 scale bits (identical on both lanes of the row).
+__device__ __forceinline__ uint16_t quantise(const float (&x)[64], unsigned pmask,
+                                             uint32_t (&q)[8]) {
   float m = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 32; i++) m = fmaxf(m, fabsf(y[i]));
-  m = fmaxf(m, __shfl_xor_sync(gmask, m, 1));
-  m = fmaxf(m, __shfl_xor_sync(gmask, m, 2));
+  for (int i = 0; i < 64; i += 2) m = fmaxf(m, fmaxf(fabsf(x[i]), fabsf(x[i + 1])));
+  m = fmaxf(m, __shfl_xor_sync(pmask, m, 1));
   const float s32 = __fdiv_rn(m, 7.0f);
-  const __half sh = (s32 > 65504.0f) ? __ushort_as_half(0x7BFF) : __float2half_rn(s32);
+  const bool sat = s32 > 65504.0f;
+  const __half sh = sat ? __ushort_as_half(0x7BFF) : __float2half_rn(s32);
   const float s = __half2float(sh);
+  // Fast path: s a normal fp16 number and not saturated (then |y/s| <= 7.004).
+  bool exact = !sat && s >= 6.103515625e-05f;
+  if (exact) {
+    const float r = __frcp_rn(s);
+    float dmax = 0.0f;
 #pragma unroll
-  for (int w = 0; w < 4; w++) q[w] = 0u;
-  if (s != 0.0f) {
+    for (int c8 = 0; c8 < 8; c8++) {
+      float mg[8];
 #pragma unroll
-    for (int i = 0; i < 32; i++) {
-      float t = rintf(__fdiv_rn(y[i], s));
-      t = fminf(fmaxf(t, -8.0f), 7.0f);
-      const uint32_t nib = static_cast<uint32_t>(static_cast<int>(t)) & 0xFu;
-      q[i / 8] |= nib << (4 * (i % 8));
+      for (int e = 0; e < 8; e += 2) {
+        float t0 = x[8 * c8 + e], t1 = x[8 * c8 + e + 1];
+        mul2(t0, t1, r);
+        float m0 = t0, m1 = t1;
+        fma2(m0, m1, 1.0f, kMagic, kMagic);           // t + 1.5*2^23, rounded: rint
+        float r0 = m0, r1 = m1;
+        fma2(r0, r1, 1.0f, -kMagic, -kMagic);         // the integer, exactly
+        float d0 = r0, d1 = r1;
+        fma2(d0, d1, -1.0f, t0, t1);                  // t - rint(t), exactly
+        dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
+        mg[e] = m0;
+        mg[e + 1] = m1;
+      }
+      q[c8] = pack8_magic(mg);
+    }
+    exact = dmax < 0.5f - 0x1p-19f;
+  }
+  if (!exact) {  // near-tie, subnormal or saturated scale, or s == 0
+#pragma unroll
+    for (int w = 0; w < 8; w++) q[w] = 0u;
+    if (s != 0.0f) {
+#pragma unroll
+      for (int i = 0; i < 64; i++) {
+        float t = rintf(__fdiv_rn(x[i], s));
+        t = fminf(fmaxf(t, -8.0f), 7.0f);
+        q[i / 8] |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xFu) << (4 * (i % 8));
+      }
     }
   }
   return __half_as_ushort(sh);
@@ -135,25 +202,22 @@ __device__ __forceinline__ uint16_t quantise_row(const float (&y)[32], unsigned 
 
 template <int BLOCK>
 __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
-  const int lane4 = threadIdx.x & 3;
-  // Shuffles never leave the 4-lane group, so they name only the group's lanes.
-  const unsigned gmask = 0xFu << (threadIdx.x & 28);
-  const long long pair = static_cast<long long>(blockIdx.x) * kPairsPerBlock + (threadIdx.x >> 2);
-  const long long npairs = static_cast<long long>(p.total_new_tokens) * p.num_kv_heads;
-  // Whole groups of 4 share validity and shuffle only among themselves, so a group
-  // past the end may leave early.
-  if (pair >= npairs) return;
+  const int l = threadIdx.x & 1;
+  // Shuffles never leave the lane pair of a row, so they name only those two lanes.
+  const unsigned pmask = 0x3u << (threadIdx.x & 30);
+  const long long row = static_cast<long long>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 1);
+  const long long nrows = 2LL * p.total_new_tokens * p.num_kv_heads;
+  if (row >= nrows) return;  // both lanes of a row leave together
+  const long long pair = row >> 1;
+  const int kv = static_cast<int>(row & 1);
   const int t = static_cast<int>(pair / p.num_kv_heads);
   const int h = static_cast<int>(pair % p.num_kv_heads);
 
-  // Issue the K/V loads first; the page lookup below overlaps their latency.
-  float xk[32], xv[32];
-  const size_t row_off = (static_cast<size_t>(t) * p.num_kv_heads + h) * kD;
-  load_row(p.k + row_off, lane4, xk);
-  load_row(p.v + row_off, lane4, xv);
+  float x[64];
+  load_rotate<BLOCK>((kv ? p.v : p.k) + static_cast<size_t>(pair) * kD, l, pmask, p.cb, x);
 
   // Sequence of token t: the b with cu[b] <= t < cu[b+1] (binary search).
-  int lo = 0, hi = p.batch;  // invariant: cu[lo] <= t < cu[hi]
+  int lo = 0, hi = p.batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (__ldg(p.cu_new_tokens + mid) <= t) lo = mid; else hi = mid;
@@ -166,14 +230,10 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
     page = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + lp);
   const bool ok = pos >= 0 && lp < p.max_pages_per_seq && page >= 0 && page < p.num_pages;
 
-  rotate_row<BLOCK>(xk, lane4, gmask, p.cb);
-  rotate_row<BLOCK>(xv, lane4, gmask, p.cb);
-  uint32_t qk[4], qv[4];
-  const uint16_t sk = quantise_row(xk, gmask, qk);
-  const uint16_t sv = quantise_row(xv, gmask, qv);
-
+  uint32_t q[8];
+  const uint16_t sbits = quantise(x, pmask, q);
   if (!ok) {
-    if (lane4 == 0)
+    if (l == 0 && kv == 0)
       atomicOr(p.status, (pos < 0 || lp >= p.max_pages_per_seq) ? KVQ_DEV_BAD_POS_BIT
                                                                   : KVQ_DEV_BAD_PAGE_BIT);
     return;
@@ -182,33 +242,21 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
   const int slot = pos - lp * S;
   uint8_t* blk = p.pool_layer + (static_cast<size_t>(page) * p.num_kv_heads + h) *
                                     (static_cast<size_t>(S) * (kD + 4));
-  // Exchange 8 bytes with the neighbour so each lane owns 16 contiguous code bytes:
-  // even lane l stores bytes [8l, 8l+16) = (own A, neighbour A); odd lane l stores
-  // bytes [24+8l, 40+8l) = (neighbour B, own B).
-  const bool odd = lane4 & 1;
+  uint8_t* crow = blk + static_cast<size_t>(kv) * S * (kD / 2) + static_cast<size_t>(slot) * (kD / 2);
 #pragma unroll
-  for (int kv = 0; kv < 2; kv++) {
-    const uint32_t* q = kv == 0 ? qk : qv;
-    const uint32_t s0 = odd ? q[0] : q[2], s1 = odd ? q[1] : q[3];
-    const uint32_t r0 = __shfl_xor_sync(gmask, s0, 1);
-    const uint32_t r1 = __shfl_xor_sync(gmask, s1, 1);
-    uint8_t* row = blk + static_cast<size_t>(kv) * S * (kD / 2) + static_cast<size_t>(slot) * (kD / 2);
-    if (!odd) stg_128(row + 8 * lane4, q[0], q[1], r0, r1);
-    else stg_128(row + 24 + 8 * lane4, r0, r1, q[2], q[3]);
-  }
-  if (lane4 < 2) {
-    uint8_t* sp = blk + static_cast<size_t>(S) * kD + static_cast<size_t>(lane4) * S * 2 +
-                  static_cast<size_t>(slot) * 2;
-    *reinterpret_cast<uint16_t*>(sp) = lane4 == 0 ? sk : sv;
-  }
+  for (int j = 0; j < 4; j++)
+    *reinterpret_cast<uint2*>(crow + 8 * (2 * j + l)) = make_uint2(q[2 * j], q[2 * j + 1]);
+  if (l == 0)
+    *reinterpret_cast<uint16_t*>(blk + static_cast<size_t>(S) * kD + static_cast<size_t>(kv) * S * 2 +
+                                 static_cast<size_t>(slot) * 2) = sbits;
 }
 
 }  // namespace
 
 int launch_append(const AppendParams& p, int block, cudaStream_t stream) {
-  const long long npairs = static_cast<long long>(p.total_new_tokens) * p.num_kv_heads;
-  if (npairs == 0) return 0;
-  const long long grid = (npairs + kPairsPerBlock - 1) / kPairsPerBlock;
+  const long long nrows = 2LL * p.total_new_tokens * p.num_kv_heads;
+  if (nrows == 0) return 0;
+  const long long grid = (nrows + kRowsPerBlock - 1) / kRowsPerBlock;
   if (grid > 0x7fffffffLL) return -1;
   switch (block) {
     case 32: append_kernel<32><<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(p); break;

@@ -20,9 +20,9 @@ struct kvq_cache {
   uint8_t* pool;
   size_t pool_bytes;
   bool own_pool;
-  void* scratch;             // one allocation: status word, tile prefix, partials
+  void* scratch;             // one allocation: status word, unit counters, partials
   int32_t* status;
-  int32_t* tile_prefix;
+  int32_t* counters;
   float* part;
   int device;
   int num_sms;
@@ -147,19 +147,22 @@ int kvq_alloc_pages(const kvq_desc* d, void* dev_pool, size_t pool_bytes, int32_
     delete c;
     return KVQ_ECUDA;
   }
-  // Scratch: status word (padded to 256 B), tile prefix [max_batch+1] (padded), and the
-  // split partials [(max_batch * Hkv + W) * G * kPartStride] fp32.
-  const size_t prefix_bytes = ((static_cast<size_t>(d->max_batch) + 1) * 4 + 255) & ~size_t(255);
-  const size_t slots = static_cast<size_t>(d->max_batch) * d->num_kv_heads + c->launch.warps;
+  // Scratch: status word (padded to 256 B), one arrival counter per unit (zero between
+  // calls; the decode kernel resets what it uses), and the per-(unit, CTA) partials
+  // [(max_batch * Hkv + grid) * G * kPartStride] fp32.
+  const size_t units = static_cast<size_t>(d->max_batch) * d->num_kv_heads;
+  const size_t counter_bytes = (units * 4 + 255) & ~size_t(255);
+  const size_t slots = units + static_cast<size_t>(c->launch.grid);
   const size_t part_bytes = slots * g * kvq::kPartStride * sizeof(float);
-  if (cudaMalloc(&c->scratch, 256 + prefix_bytes + part_bytes) != cudaSuccess) {
+  if (cudaMalloc(&c->scratch, 256 + counter_bytes + part_bytes) != cudaSuccess) {
     delete c;
     return KVQ_ECUDA;
   }
   c->status = static_cast<int32_t*>(c->scratch);
-  c->tile_prefix = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(c->scratch) + 256);
-  c->part = reinterpret_cast<float*>(static_cast<uint8_t*>(c->scratch) + 256 + prefix_bytes);
-  if (cudaMemset(c->status, 0, 256) != cudaSuccess) {
+  c->counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(c->scratch) + 256);
+  c->part = reinterpret_cast<float*>(static_cast<uint8_t*>(c->scratch) + 256 + counter_bytes);
+  if (cudaMemset(c->scratch, 0, 256 + counter_bytes) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(c->scratch);
     delete c;
     return KVQ_ECUDA;
@@ -233,7 +236,7 @@ int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, const int32
   p.page_table = page_table;
   p.out = static_cast<__half*>(out);
   p.part = c->part;
-  p.tile_prefix = c->tile_prefix;
+  p.counters = c->counters;
   p.status = c->status;
   p.batch = batch;
   p.num_kv_heads = c->d.num_kv_heads;
@@ -246,7 +249,7 @@ int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, const int32
                                           : static_cast<double>(softmax_scale);
   p.q_scale = static_cast<float>(sm * 1.4426950408889634);  // log2(e)
   p.cb = c->cb;
-  p.total_warps = c->launch.warps;
+  p.total_ctas = c->launch.grid;
   const int rc = kvq::launch_decode(p, c->launch, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;

@@ -30,7 +30,7 @@ struct AppendParams {
 };
 
 // Tokens per decode tile (one shared-memory ring slot per tile).
-constexpr int kTileTokens = 64;
+constexpr int kTileTokens = 32;
 // fp32 words per (partial, query) record in the split scratch: o'[128], m, l, 2 pad.
 constexpr int kPartStride = 132;
 
@@ -40,8 +40,8 @@ struct DecodeParams {
   const int32_t* seq_lens;        // [batch], tokens to attend
   const int32_t* page_table;      // [batch][max_pages_per_seq]
   __half* out;                    // [batch][Hq][128]
-  float* part;                    // split partials [slots][G][kPartStride]
-  int32_t* tile_prefix;           // [batch+1] tiles-per-sequence prefix (per KV head)
+  float* part;                    // per-(unit, CTA) partials [slots][G][kPartStride]
+  int32_t* counters;              // [max_batch * Hkv] arrival counters, zero between calls
   int32_t* status;
   int batch;
   int num_kv_heads;
@@ -52,7 +52,7 @@ struct DecodeParams {
   int hadamard_block;
   float q_scale;                  // softmax_scale * log2(e)
   float cb;                       // fp32 nearest 1/sqrt(hadamard_block)
-  int total_warps;                // W: warps in the split pass grid
+  int total_ctas;                 // C: CTAs in the grid
 };
 
 // Host-side launchers (return 0 on success, <0 on an unsupported shape or a launch
@@ -60,13 +60,11 @@ struct DecodeParams {
 int launch_append(const AppendParams& p, int block, cudaStream_t stream);
 
 struct DecodeLaunch {
-  int grid;          // CTAs of the split pass
-  int warps;         // total warps (grid * warps per CTA)
+  int grid;          // CTAs (a multiple of the SM count)
   size_t smem;       // dynamic shared memory per CTA
 };
-// Shape of the split pass for a batch (grid sized to fill every SM).
-int plan_decode(int group, int page_size, int batch, int num_sms, DecodeLaunch* out);
-int max_decode_warps(int num_sms);
+// Shape of the decode pass for a batch capacity (grid sized to fill every SM).
+int plan_decode(int group, int page_size, int max_batch, int num_sms, DecodeLaunch* out);
 int launch_decode(const DecodeParams& p, const DecodeLaunch& L, cudaStream_t stream);
 
 }  // namespace kvq

@@ -157,7 +157,8 @@ KVQ_API int kvq_rotate_quant_append(kvq_cache* c, int32_t layer, const void* k, 
                             int32_t total_new_tokens, void* stream);
 
 /* Paged GQA decode attention over the INT4 cache of one layer: one query token per
- * sequence.  Two kernel launches (split-KV pass, then split combine + inverse rotation).
+ * sequence.  One kernel launch: a split-KV pass whose last-arriving CTA per (sequence,
+ * KV head) merges the splits and applies the inverse rotation.
  *   q              device fp16 [batch][num_q_heads][128], 16-byte aligned
  *   seq_lens       device int32 [batch], lengths AFTER any append (tokens to attend)
  *   page_table     device int32 [batch][max_pages_per_seq]

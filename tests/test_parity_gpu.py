@@ -115,3 +115,35 @@ def test_empty_batch_calls_are_no_ops():
     assert not out.any()
     assert kvq.get_device_status(cache) == 0
     cache.close()
+
+
+def test_repeated_decode_is_bit_identical():
+    """The cross-CTA merge counters reset themselves: the same call twice gives the same
+    bytes (long units split over many CTAs, plus short ones finished inside one CTA)."""
+    import torch
+    import bit_paged_kv_diag_b200 as kvq
+    w = W["long_context"]
+    case = make_case(w, [5000, 31, 1, 2600], [1, 1, 1, 1])
+    from harness import GpuRun, host_inputs
+    kp, vp, kn, vn, q = host_inputs(case)
+    run = GpuRun(case, kp, vp, kn, vn, q)
+    try:
+        pt = torch.from_numpy(run.page_table).cuda()
+        lens = torch.as_tensor(run.lens_after).cuda()
+        qd = torch.as_tensor(q).cuda()
+        a = kvq.decode_attention(run.cache, 0, qd, lens, pt)
+        b = kvq.decode_attention(run.cache, 0, qd, lens, pt)
+        torch.cuda.synchronize()
+        assert torch.equal(a, b)
+        assert torch.equal(a.float().cpu(), torch.from_numpy(run.host_out))
+        assert kvq.get_device_status(run.cache) == 0
+    finally:
+        run.close()
+
+
+def test_many_short_units_per_cta():
+    """Hundreds of sequences of 1..40 tokens: many units inside one CTA's range."""
+    w = dataclasses.replace(W["ragged"], num_kv_heads=2, num_q_heads=8)
+    rng = np.random.default_rng(5)
+    lengths = rng.integers(0, 40, size=300).tolist()
+    full_parity(make_case(w, lengths, [1] * 300, pool_factor=1.1))
