@@ -9,21 +9,23 @@
 // moving with few instructions per byte.
 //
 // Work split (one launch).  The cache is cut into tiles of 32 tokens of one (sequence,
-// KV head) "unit", numbered unit-major.  CTA k of C takes the contiguous tile range
-// [k*T/C, (k+1)*T/C) of the T tiles, so every CTA streams the same number of bytes
-// whatever the length mix.  Its 4 warps take the range's tiles of each unit in turn
-// (tile xs + w, xs + w + 4, ...), each keeping an online-softmax state; at the end of
-// each unit the warps merge through shared memory.  A unit inside one CTA is finished
+// KV head) "unit", numbered unit-major.  CTA k takes the contiguous tile range
+// [k*chunk, (k+1)*chunk) of the T tiles, chunk = ceil(T/C), so every CTA streams the
+// same number of bytes whatever the length mix.  Its 4 warps take the range's tiles in
+// turn (tile X0 + w, X0 + w + 4, ...), each keeping an online-softmax state per unit; at
+// the end of each unit the warps merge through shared memory.  A unit inside one CTA is finished
 // there (normalise, inverse rotation, fp16 store).  A unit spanning several CTAs leaves
 // one (o', m, l) partial per CTA in scratch slot unit + k (unique along the staircase of
 // ranges); the last CTA to arrive (an atomic counter per unit, reset after use) merges
-// them and finishes the unit.
+// them and finishes the unit.  The rotated, sliced q of a unit is prepared once per CTA
+// (warp w takes query w) into a shared table the warps load their fragments from.
 //
 // Loads.  Each warp owns a ring of 3 shared-memory slots of one tile each.  Per tile one
 // lane per page issues a 1-D bulk copy (cp.async.bulk, TMA engine, no multicast) of the
 // contiguous (page, head) block -- codes and scales together -- into a slot, completing
-// on the slot's mbarrier; page ids three tiles ahead are read while the current tile
-// computes.
+// on the slot's mbarrier.  Page ids are read in batches, one per lane, a batch ahead of
+// use, and sequence lengths are kept in shared memory, so no global-memory latency sits
+// between consuming a tile and issuing the copy that refills its slot.
 //
 // QK^T on tensor cores in exact integer arithmetic: mma.sync m16n8k32 s8 x s8 -> s32 with
 // A = K codes (16 tokens x 32 channels) and B = the rotated, scaled q cut into three int8
@@ -35,7 +37,9 @@
 // PV on tensor cores: mma.sync m16n8k16 f16 x f16 -> f32 with A = V codes transposed
 // (16 channels x 16 tokens, gathered with byte permutes, exact fp16 integers) and B = P'
 // = p * s_v (the V scale folded into the probabilities) as fp16 hi + lo parts: for G <= 4
-// the two parts sit in neighbouring columns, for G = 8 two MMAs accumulate them.  The GQA group is the N = 8
+// the two parts sit in neighbouring columns, for G = 8 two MMAs accumulate them.  (The
+// integer values go in exactly, without a constant offset: the tensor core's internal
+// sum is not precise enough to cancel a large offset afterwards.)  The GQA group is the N = 8
 // side of both products; the dequantised cache is the M side.  The K scale multiplies the
 // fp32 score of its token; softmax runs in the log2 domain with exp2.
 #include <cuda_fp16.h>
@@ -66,94 +70,86 @@ __device__ __forceinline__ int clamp_len(int L, int cap, int32_t* status) {
   return L;
 }
 
-// One (sequence, KV head) unit and its place in the tile sequence.
+// One (sequence, KV head) unit and its place in the tile sequence.  pre[] (tiles per
+// sequence, exclusive prefix) and lens[] (clamped lengths) live in shared memory.
 struct Unit {
-  int b, h;       // sequence, KV head
-  int n;          // tiles in the unit
-  int L;          // tokens (clamped to the page budget)
-  long long U;    // global index of the unit's first tile
+  int b, h;  // sequence, KV head
+  int n;     // tiles in the unit
+  int L;     // tokens
+  int U;     // global index of the unit's first tile
 };
 
-__device__ __forceinline__ void unit_of_tile(Unit& u, long long x, const int32_t* pre,
+__device__ __forceinline__ void unit_of_tile(Unit& u, int x, const int32_t* pre, const int32_t* lens,
                                              const DecodeParams& p) {
   int lo = 0, hi = p.batch;  // pre[lo]*Hkv <= x < pre[hi]*Hkv
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (static_cast<long long>(pre[mid]) * p.num_kv_heads <= x) lo = mid; else hi = mid;
+    if (pre[mid] * p.num_kv_heads <= x) lo = mid; else hi = mid;
   }
   u.b = lo;
   u.n = pre[lo + 1] - pre[lo];
-  const long long base = static_cast<long long>(pre[lo]) * p.num_kv_heads;
-  u.h = static_cast<int>((x - base) / u.n);
-  u.U = base + static_cast<long long>(u.h) * u.n;
-  u.L = clamp_len(__ldg(p.seq_lens + u.b), p.max_pages_per_seq * p.page_size, p.status);
+  const int base = pre[lo] * p.num_kv_heads;
+  u.h = (x - base) / u.n;
+  u.U = base + u.h * u.n;
+  u.L = lens[lo];
 }
 
 // The next non-empty unit.  Callers only ask while one exists.
-__device__ __forceinline__ void unit_next(Unit& u, const int32_t* pre, const DecodeParams& p) {
+__device__ __forceinline__ void unit_next(Unit& u, const int32_t* pre, const int32_t* lens,
+                                          const DecodeParams& p) {
   if (++u.h == p.num_kv_heads) {
     u.h = 0;
     do { ++u.b; } while (u.b < p.batch && pre[u.b + 1] == pre[u.b]);
     if (u.b >= p.batch) return;
     u.n = pre[u.b + 1] - pre[u.b];
-    u.L = clamp_len(__ldg(p.seq_lens + u.b), p.max_pages_per_seq * p.page_size, p.status);
+    u.L = lens[u.b];
   }
-  u.U = static_cast<long long>(pre[u.b]) * p.num_kv_heads + static_cast<long long>(u.h) * u.n;
-}
-
-// CTA whose tile range holds tile x (ranges [k*T/C, (k+1)*T/C)).
-__device__ __forceinline__ long long cta_of(long long x, long long T, long long C) {
-  return ((x + 1) * C - 1) / T;
-}
-
-// A warp's walk over its tiles: units overlapping [X0, X1), tiles xs + w + 4i of each.
-struct Walk {
-  Unit u;
-  long long x, xe;
-  bool valid;
-};
-
-__device__ __forceinline__ void walk_settle(Walk& wk, long long X1, int w, const int32_t* pre,
-                                            const DecodeParams& p) {
-  while (wk.x >= wk.xe) {
-    if (wk.xe >= X1) {
-      wk.valid = false;
-      return;
-    }
-    unit_next(wk.u, pre, p);
-    wk.x = wk.u.U + w;
-    wk.xe = min(X1, wk.u.U + wk.u.n);
-  }
+  u.U = pre[u.b] * p.num_kv_heads + u.h * u.n;
 }
 
 // ------------------------------------------------------------------- copies --
-// Page id lane `lane` needs for tile k of unit u (or -1): for pages of <= 32 tokens the
-// tile's pages (<= 2), else the page holding the tile.
+// Page ids of a warp's upcoming tiles, one per lane: a batch covers kBatch tiles of
+// kPPT pages (tile t of the warp = CTA tile X0 + w + kWarps*t).  Entry lane: tile
+// tb + lane / kPPT, page lane % kPPT of the tile; -1 where no page is needed.
 template <int SEFF>
-__device__ __forceinline__ int tile_page_id(const Unit& u, long long k, int lane,
-                                            const DecodeParams& p) {
-  const int S = p.page_size;
-  const int t0 = static_cast<int>(k) * kTileTokens;
-  int npg = 1;
-  if (S <= kTileTokens) npg = (min(t0 + kTileTokens, u.L) - 1) / S - t0 / S + 1;
-  if (lane >= npg) return -1;
-  return __ldg(p.page_table + static_cast<size_t>(u.b) * p.max_pages_per_seq + t0 / S + lane);
+struct PageBatch {
+  static constexpr int kPPT = (SEFF < kTileTokens) ? kTileTokens / SEFF : 1;
+  static constexpr int kBatch = 32 / kPPT;
+};
+
+template <int SEFF>
+__device__ __forceinline__ int load_page_batch(int tb, int X0, int X1, int w, int lane,
+                                               const int32_t* pre, const int32_t* lens,
+                                               const DecodeParams& p) {
+  constexpr int kPPT = PageBatch<SEFF>::kPPT;
+  const int x = X0 + w + kWarps * (tb + lane / kPPT);
+  int pid = -1;
+  if (x < X1) {
+    Unit u;
+    unit_of_tile(u, x, pre, lens, p);
+    const int t0 = (x - u.U) * kTileTokens;
+    const int lp = (t0 >> p.page_shift) + lane % kPPT;
+    if ((lp << p.page_shift) < u.L)
+      pid = __ldg(p.page_table + static_cast<size_t>(u.b) * p.max_pages_per_seq + lp);
+  }
+  return pid;
 }
 
-// Issue the bulk copies of tile k of unit u into a ring slot (the whole warp calls).
-// The slot holds a virtual page of SEFF = min(S, 32) token slots per copied page,
-// [K codes][V codes][K scales][V scales], the pool's own block layout.
+// Issue the bulk copies of tile k of unit u into a ring slot (the whole warp calls; lane
+// j < pages-needed holds that page's id).  The slot holds a virtual page of SEFF =
+// min(S, 32) token slots per copied page, [K codes][V codes][K scales][V scales], the
+// pool's own block layout.
 template <int SEFF>
-__device__ __forceinline__ void tile_issue(const Unit& u, long long k, int pid, uint32_t slot,
+__device__ __forceinline__ void tile_issue(const Unit& u, int k, int pid, uint32_t slot,
                                            uint32_t bar, int lane, uint64_t pol,
                                            const DecodeParams& p) {
-  const int S = p.page_size;
+  const int S = p.page_size, sh = p.page_shift;
   const uint32_t blk_bytes = static_cast<uint32_t>(S) * (kD + 4);
-  const int t0 = static_cast<int>(k) * kTileTokens;
+  const int t0 = k * kTileTokens;
   int npg = 1;
   uint32_t total = kSlotBytes;
-  if (S <= kTileTokens) {
-    npg = (min(t0 + kTileTokens, u.L) - 1) / S - t0 / S + 1;
+  if (SEFF < kTileTokens) {
+    npg = ((min(t0 + kTileTokens, u.L) - 1) >> sh) - (t0 >> sh) + 1;
     total = npg * blk_bytes;
   }
   const bool bad = lane < npg && (pid < 0 || pid >= p.num_pages);
@@ -161,14 +157,14 @@ __device__ __forceinline__ void tile_issue(const Unit& u, long long k, int pid, 
   if (bad) pid = 0;  // keep the barrier's byte count; the status word flags the result
   if (lane == 0) mbar_arrive_expect_tx(bar, total);
   __syncwarp();
-  if (S <= kTileTokens) {
+  if (SEFF < kTileTokens || S == kTileTokens) {
     if (lane < npg)
       bulk_copy_g2s(slot + lane * blk_bytes,
                     p.pool_layer + (static_cast<size_t>(pid) * p.num_kv_heads + u.h) * blk_bytes,
                     blk_bytes, bar, pol);
   } else {
     const int pid0 = __shfl_sync(kFull, pid, 0);
-    const size_t o = static_cast<size_t>(t0 % S);  // first token of the tile in the page
+    const size_t o = static_cast<size_t>(t0 & (S - 1));  // first token of the tile in the page
     const uint8_t* blk = p.pool_layer + (static_cast<size_t>(pid0) * p.num_kv_heads + u.h) * blk_bytes;
     if (lane == 0) bulk_copy_g2s(slot, blk + o * 64, 2048, bar, pol);
     if (lane == 1) bulk_copy_g2s(slot + 2048, blk + static_cast<size_t>(S) * 64 + o * 64, 2048, bar, pol);
@@ -177,140 +173,186 @@ __device__ __forceinline__ void tile_issue(const Unit& u, long long k, int pid, 
   }
 }
 
+// A warp's producer: issues its tiles t = 0, 1, ... (CTA tile X0 + w + kWarps*t) in
+// order into its ring, slot t % kStages; page ids come from prefetched batches.
+template <int SEFF>
+struct Producer {
+  int t;        // next tile to issue
+  int nT;       // tiles of this warp
+  Unit u;       // unit of tile t
+  int tb;       // first tile of the current page-id batch
+  int pid_cur;  // this lane's entry of the current batch
+  int pid_nxt;  // ... of the next batch (loaded one batch ahead)
+};
+
+template <int SEFF>
+__device__ __forceinline__ void producer_issue(Producer<SEFF>& pr, int X0, int X1, int w, int lane,
+                                               uint32_t ring_s, uint32_t bar_s, uint64_t pol,
+                                               const int32_t* pre, const int32_t* lens,
+                                               const DecodeParams& p) {
+  constexpr int kPPT = PageBatch<SEFF>::kPPT, kBatch = PageBatch<SEFF>::kBatch;
+  if (pr.t >= pr.tb + kBatch) {
+    pr.tb += kBatch;
+    pr.pid_cur = pr.pid_nxt;
+    pr.pid_nxt = load_page_batch<SEFF>(pr.tb + kBatch, X0, X1, w, lane, pre, lens, p);
+  }
+  const int x = X0 + w + kWarps * pr.t;
+  while (x >= pr.u.U + pr.u.n && pr.u.b < p.batch) unit_next(pr.u, pre, lens, p);
+  const int src = (pr.t - pr.tb) * kPPT + lane;
+  const int pid = __shfl_sync(kFull, pr.pid_cur, src < 32 ? src : 31);
+  const int s = pr.t % kStages;
+  tile_issue<SEFF>(pr.u, x - pr.u.U, pid, ring_s + s * kSlotBytes, bar_s + 8 * s, lane, pol, p);
+  pr.t++;
+}
+
 // ------------------------------------------------------------------------ q --
+// int8 B fragments of the rotated, scaled q, per k32 chunk jj: [jj][0] = k 4c..4c+3,
+// [jj][1] = k 16+4c..16+4c+3, where k = 4c + e <-> channel 32c + 8jj + 2e and
+// k = 16 + 4c + e <-> channel 32c + 8jj + 2e + 1.
+// G <= 4: A = column g holds slice 1 (g even) or 2 (g odd) of query g/2, B = slice 3
+// (g even) or zero.  G == 8: A, B, C = slices 1, 2, 3 of query g.
 template <int G>
 struct QFrag {
   static constexpr int NQ = (G == 8) ? 2 : 1;  // queries owned by one thread
-  // int8 B fragments per k32 chunk jj: [jj][0] = k 4c..4c+3, [jj][1] = k 16+4c..16+4c+3.
-  // G <= 4: A = column g holds slice 1 (g even) or 2 (g odd) of query g/2, B = slice 3
-  // (g even) or zero.  G == 8: A, B, C = slices 1, 2, 3 of query g.
   uint32_t A[4][2], B[4][2], C[4][2];
   float sf[NQ];  // M / 1024 of the owned queries
 };
 
-// Raw fp16 q row of this thread's column: channels [32c, 32c+32).
+// Raw fp16 q for the cooperative preparation: warp w handles query w (and w + 4 when
+// G == 8); lane holds channels 4*lane..4*lane+3.
 template <int G>
-__device__ __forceinline__ void load_q_raw(uint4 (&raw)[4], const Unit& u, int lane,
-                                           const DecodeParams& p) {
-  const int g = lane >> 2, c = lane & 3;
-  const int qi = (G == 8) ? g : (g >> 1);
-  if (qi < G) {
-    const uint4* src = reinterpret_cast<const uint4*>(
-        p.q + (static_cast<size_t>(u.b) * p.num_kv_heads * G + u.h * G + qi) * kD + 32 * c);
+__device__ __forceinline__ void load_q_coop(uint2 (&raw)[2], const Unit& u, int w, int lane,
+                                            const DecodeParams& p) {
 #pragma unroll
-    for (int v = 0; v < 4; v++) raw[v] = __ldg(src + v);
-  } else {
-#pragma unroll
-    for (int v = 0; v < 4; v++) raw[v] = make_uint4(0u, 0u, 0u, 0u);
+  for (int r = 0; r < 2; r++) {
+    const int qi = w + kWarps * r;
+    raw[r] = make_uint2(0u, 0u);
+    if (qi < G)
+      raw[r] = __ldg(reinterpret_cast<const uint2*>(
+                         p.q + (static_cast<size_t>(u.b) * p.num_kv_heads * G + u.h * G + qi) * kD) +
+                     lane);
   }
 }
 
-__device__ __forceinline__ uint32_t int8x4(const float (&m)[32], int i0, int step) {
-  // Low bytes of four magic-rounded sums (each holds an integer in [-64, 64]).
-  const uint32_t b0 = __float_as_uint(m[i0]), b1 = __float_as_uint(m[i0 + step]);
-  const uint32_t b2 = __float_as_uint(m[i0 + 2 * step]), b3 = __float_as_uint(m[i0 + 3 * step]);
-  return prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
-}
-
-// Rotate q (same fixed-order butterfly: bits 0-4 in registers, bits 5-6 across the 4
-// lanes of the row group), scale by c_b * softmax_scale * log2(e), cut into int8 slices.
+// Rotate (the fixed-order butterfly: stages h = 1, 2 in registers, h = 4..64 across
+// lanes), scale by c_b * softmax_scale * log2(e), and cut query qi into three int8
+// slices q' = M/64 * (q1 + q2/128 + q3/16384), M the power of two >= max|q'| (1 for a
+// zero row); write them to the shared table in fragment order:
+//   qfb word ((qi*3 + s)*4 + c)*8 + 2*jj + half, byte e  <->  channel 32c + 8jj + 2e + half.
 template <int G>
-__device__ __forceinline__ void make_qfrag(QFrag<G>& f, const uint4 (&raw)[4], int lane,
-                                           const DecodeParams& p) {
-  const int g = lane >> 2, c = lane & 3;
-  float x[32];
+__device__ __forceinline__ void prep_q(uint32_t* qfb, float* sfb, const uint2 (&raw)[2], int w,
+                                       int lane, const DecodeParams& p) {
 #pragma unroll
-  for (int v = 0; v < 4; v++) {
-    const uint32_t w[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
+  for (int r = 0; r < 2; r++) {
+    const int qi = w + kWarps * r;
+    if (qi >= G) continue;  // warp-uniform
+    float x[4];
+    {
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw[r].x));
+      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw[r].y));
+      x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    }
+    float t0 = x[0], t1 = x[1];
+    x[0] = __fadd_rn(t0, t1); x[1] = __fsub_rn(t0, t1);
+    t0 = x[2]; t1 = x[3];
+    x[2] = __fadd_rn(t0, t1); x[3] = __fsub_rn(t0, t1);
+    t0 = x[0]; t1 = x[2];
+    x[0] = __fadd_rn(t0, t1); x[2] = __fsub_rn(t0, t1);
+    t0 = x[1]; t1 = x[3];
+    x[1] = __fadd_rn(t0, t1); x[3] = __fsub_rn(t0, t1);
+#pragma unroll
+    for (int s = 0; s < 5; s++) {
+      if ((4 << s) < p.hadamard_block) {
+        const float sgn = ((lane >> s) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int e = 0; e < 4; e++) x[e] = __fmaf_rn(x[e], sgn, __shfl_xor_sync(kFull, x[e], 1 << s));
+      }
+    }
+    float amax = 0.0f;
 #pragma unroll
     for (int e = 0; e < 4; e++) {
-      const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
-      x[8 * v + 2 * e] = t.x;
-      x[8 * v + 2 * e + 1] = t.y;
+      x[e] = __fmul_rn(__fmul_rn(x[e], p.cb), p.q_scale);
+      amax = fmaxf(amax, fabsf(x[e]));
+    }
+#pragma unroll
+    for (int d = 1; d < 32; d *= 2) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, d));
+    float M = 1.0f;
+    if (amax > 1e-30f) {
+      const uint32_t bits = __float_as_uint(amax);
+      M = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax;
+    }
+    const float inv = __fdiv_rn(64.0f, M);  // exact: powers of two
+    uint32_t ms[3][4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const float t = x[e] * inv;                         // |t| <= 64, exact scaling
+      const float m1 = t + kMagic;                        // rint(t) in the low mantissa bits
+      const float r1 = (t - (m1 - kMagic)) * 128.0f;      // exact
+      const float m2 = r1 + kMagic;
+      const float r2 = (r1 - (m2 - kMagic)) * 128.0f;
+      const float m3 = r2 + kMagic;
+      ms[0][e] = __float_as_uint(m1);
+      ms[1][e] = __float_as_uint(m2);
+      ms[2][e] = __float_as_uint(m3);
+    }
+    // Channels 4*lane + i: c = lane/8, jj = (lane/2)%4, half = i%2, byte e0 + i/2 with
+    // e0 = (2*lane)%4: a 2-byte store per (slice, half).
+    const int c = lane >> 3, jj = (lane >> 1) & 3, e0 = (2 * lane) & 3;
+    uint8_t* base = reinterpret_cast<uint8_t*>(qfb);
+#pragma unroll
+    for (int s = 0; s < 3; s++) {
+      const int word = ((qi * 3 + s) * 4 + c) * 8 + 2 * jj;
+      const uint16_t h0 = static_cast<uint16_t>((ms[s][0] & 0xFFu) | ((ms[s][2] & 0xFFu) << 8));
+      const uint16_t h1 = static_cast<uint16_t>((ms[s][1] & 0xFFu) | ((ms[s][3] & 0xFFu) << 8));
+      *reinterpret_cast<uint16_t*>(base + word * 4 + e0) = h0;
+      *reinterpret_cast<uint16_t*>(base + (word + 1) * 4 + e0) = h1;
+    }
+    if (lane == 0) sfb[qi] = M * (1.0f / 1024.0f);
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void qfrag_load(QFrag<G>& f, const uint32_t* qfb, const float* sfb,
+                                           int lane) {
+  const int g = lane >> 2, c = lane & 3;
+  const int qi = (G == 8) ? g : (g >> 1);
+  const bool ok = qi < G;
+  uint4 s[3][2];
+#pragma unroll
+  for (int sl = 0; sl < 3; sl++) {
+    s[sl][0] = s[sl][1] = make_uint4(0u, 0u, 0u, 0u);
+    if (ok) {
+      const uint4* src = reinterpret_cast<const uint4*>(qfb + ((qi * 3 + sl) * 4 + c) * 8);
+      s[sl][0] = src[0];
+      s[sl][1] = src[1];
     }
   }
-  const int block = p.hadamard_block;
-#pragma unroll
-  for (int h = 1; h <= 16; h *= 2) {
-    if (h < block) {
-#pragma unroll
-      for (int i = 0; i < 32; i++) {
-        if (i & h) continue;
-        const float a = x[i], d = x[i + h];
-        x[i] = __fadd_rn(a, d);
-        x[i + h] = __fsub_rn(a, d);
-      }
-    }
-  }
-#pragma unroll
-  for (int s = 0; s < 2; s++) {
-    if ((32 << s) < block) {
-      const int bit = 1 << s;
-      const float sgn = (c & bit) ? -1.0f : 1.0f;
-#pragma unroll
-      for (int i = 0; i < 32; i++) {
-        const float other = __shfl_xor_sync(kFull, x[i], bit);
-        x[i] = __fmaf_rn(x[i], sgn, other);
-      }
-    }
-  }
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; i++) {
-    x[i] = __fmul_rn(__fmul_rn(x[i], p.cb), p.q_scale);
-    amax = fmaxf(amax, fabsf(x[i]));
-  }
-  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
-  // M = the smallest power of two >= amax (1 for a zero row).
-  float M = 1.0f;
-  if (amax > 1e-30f) {
-    const uint32_t bits = __float_as_uint(amax);
-    M = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax;
-  }
-  const float inv = __fdiv_rn(64.0f, M);  // exact: powers of two
-  float m1[32], m2[32], m3[32];
-#pragma unroll
-  for (int i = 0; i < 32; i++) {
-    const float t = x[i] * inv;                 // |t| <= 64, exact scaling
-    m1[i] = t + kMagic;                         // rint(t) in the low mantissa bits
-    const float r1 = (t - (m1[i] - kMagic)) * 128.0f;  // |r1| <= 64, exact
-    m2[i] = r1 + kMagic;
-    const float r2 = (r1 - (m2[i] - kMagic)) * 128.0f;
-    m3[i] = r2 + kMagic;
-  }
-  uint32_t s1[4][2], s2[4][2], s3[4][2];
-#pragma unroll
-  for (int jj = 0; jj < 4; jj++) {
-    // k = 4c + e <-> channel 32c + 8jj + 2e; k = 16 + 4c + e <-> channel 32c + 8jj + 2e + 1.
-    s1[jj][0] = int8x4(m1, 8 * jj, 2);
-    s1[jj][1] = int8x4(m1, 8 * jj + 1, 2);
-    s2[jj][0] = int8x4(m2, 8 * jj, 2);
-    s2[jj][1] = int8x4(m2, 8 * jj + 1, 2);
-    s3[jj][0] = int8x4(m3, 8 * jj, 2);
-    s3[jj][1] = int8x4(m3, 8 * jj + 1, 2);
-  }
-  const float sf_col = M * (1.0f / 1024.0f);
 #pragma unroll
   for (int jj = 0; jj < 4; jj++)
 #pragma unroll
     for (int e = 0; e < 2; e++) {
+      uint32_t v[3];
+#pragma unroll
+      for (int sl = 0; sl < 3; sl++) {
+        const uint4 q4 = s[sl][jj >> 1];
+        const uint32_t wds[4] = {q4.x, q4.y, q4.z, q4.w};
+        v[sl] = wds[2 * (jj & 1) + e];
+      }
       if (G == 8) {
-        f.A[jj][e] = s1[jj][e];
-        f.B[jj][e] = s2[jj][e];
-        f.C[jj][e] = s3[jj][e];
+        f.A[jj][e] = v[0];
+        f.B[jj][e] = v[1];
+        f.C[jj][e] = v[2];
       } else {
-        const bool col_ok = (g >> 1) < G;
-        f.A[jj][e] = col_ok ? ((g & 1) ? s2[jj][e] : s1[jj][e]) : 0u;
-        f.B[jj][e] = (col_ok && !(g & 1)) ? s3[jj][e] : 0u;
+        f.A[jj][e] = (g & 1) ? v[1] : v[0];
+        f.B[jj][e] = (g & 1) ? 0u : v[2];
         f.C[jj][e] = 0u;
       }
     }
   if (G == 8) {
-    f.sf[0] = __shfl_sync(kFull, sf_col, 4 * (2 * c));
-    f.sf[QFrag<G>::NQ - 1] = __shfl_sync(kFull, sf_col, 4 * (2 * c + 1));
+    f.sf[0] = sfb[2 * c];
+    f.sf[QFrag<G>::NQ - 1] = sfb[2 * c + 1];
   } else {
-    f.sf[0] = __shfl_sync(kFull, sf_col, 8 * c);
+    f.sf[0] = c < G ? sfb[c] : 1.0f;
   }
 }
 
@@ -336,27 +378,24 @@ __device__ __forceinline__ void state_reset(State<G>& st) {
   }
 }
 
-__device__ __forceinline__ float half_at(uint32_t addr) {
-  return __half2float(__ushort_as_half(lds_u16(addr)));
-}
 
-// One tile (2 k-steps of 16 tokens) from a ring slot; ntok valid tokens.
+// One tile = 2 k-steps of 16 tokens in a ring slot (a shared-memory pointer); ntok
+// valid tokens.  The work is split in three so that the QK^T of the next tile and the
+// PV of the current one sit in one straight-line block the compiler can interleave.
+
+// Scores (log2 domain) of the tile: sc[k-step][owned query][row], -inf past ntok.
 template <int G, int SEFF>
-__device__ __forceinline__ void tile_compute(State<G>& st, const QFrag<G>& qf, uint32_t slot,
-                                             int ntok, int lane) {
-  constexpr int NQ = State<G>::NQ;
+__device__ __forceinline__ void tile_qk(const QFrag<G>& qf, const uint8_t* slot, int ntok, int lane,
+                                        float (&sc)[2][QFrag<G>::NQ][2]) {
   const int g = lane >> 2, c = lane & 3;
-  const int tau0 = (g < 4) ? g : g + 4;  // token of A row g (QK^T)
+  const int tau0 = (g < 4) ? g : g + 4;  // token of A row g
   const int tau1 = tau0 + 4;             // token of A row g + 8
-  float sc[2][NQ][2];                    // scores (log2 domain): [k-step][query][row]
-
 #pragma unroll
   for (int j = 0; j < 2; j++) {
-    const uint32_t pbase = slot + (16 * j / SEFF) * (SEFF * 132);
+    const uint8_t* pbase = slot + (16 * j / SEFF) * (SEFF * 132);
     const int sl = (16 * j) % SEFF;
-    const uint32_t kb = pbase + sl * 64;
-    const uint4 ka = lds_128(kb + tau0 * 64 + 16 * c);
-    const uint4 kc = lds_128(kb + tau1 * 64 + 16 * c);
+    const uint4 ka = *reinterpret_cast<const uint4*>(pbase + (sl + tau0) * 64 + 16 * c);
+    const uint4 kc = *reinterpret_cast<const uint4*>(pbase + (sl + tau1) * 64 + 16 * c);
     const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
     const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
     int accA[4] = {0, 0, 0, 0}, accB[4] = {0, 0, 0, 0}, accC[4] = {0, 0, 0, 0};
@@ -368,8 +407,8 @@ __device__ __forceinline__ void tile_compute(State<G>& st, const QFrag<G>& qf, u
       mma_16832_s8(accB, a0, a1, a2, a3, qf.B[jj][0], qf.B[jj][1]);
       if (G == 8) mma_16832_s8(accC, a0, a1, a2, a3, qf.C[jj][0], qf.C[jj][1]);
     }
-    const uint32_t skb = pbase + SEFF * 128 + sl * 2;
-    const float sk0 = half_at(skb + tau0 * 2), sk1 = half_at(skb + tau1 * 2);
+    const __half* skp = reinterpret_cast<const __half*>(pbase + SEFF * 128) + sl;
+    const float sk0 = __half2float(skp[tau0]), sk1 = __half2float(skp[tau1]);
     const bool v0 = 16 * j + tau0 < ntok, v1 = 16 * j + tau1 < ntok;
     const float k14 = 1.0f / 16384.0f;
     if (G == 8) {
@@ -380,18 +419,22 @@ __device__ __forceinline__ void tile_compute(State<G>& st, const QFrag<G>& qf, u
         for (int r = 0; r < 2; r++) {
           const int e = 2 * r + qq;
           const float v = static_cast<float>(accA[e]) + static_cast<float>(accB[e] * 128 + accC[e]) * k14;
-          sc[j][qq][r] = (r ? v1 : v0) ? v * (r ? sk1 : sk0) * qf.sf[qq] : -CUDART_INF_F;
+          sc[j][qq][r] = (r ? v1 : v0) ? v * ((r ? sk1 : sk0) * qf.sf[qq]) : -CUDART_INF_F;
         }
     } else {
       // Column 2c = slices 1 (A) and 3 (B) of query c, 2c+1 = slice 2 (A) of query c.
       const float va = static_cast<float>(accA[0]) + static_cast<float>(accA[1] * 128 + accB[0]) * k14;
       const float vc = static_cast<float>(accA[2]) + static_cast<float>(accA[3] * 128 + accB[2]) * k14;
-      sc[j][0][0] = v0 ? va * sk0 * qf.sf[0] : -CUDART_INF_F;
-      sc[j][0][1] = v1 ? vc * sk1 * qf.sf[0] : -CUDART_INF_F;
+      sc[j][0][0] = v0 ? va * (sk0 * qf.sf[0]) : -CUDART_INF_F;
+      sc[j][0][1] = v1 ? vc * (sk1 * qf.sf[0]) : -CUDART_INF_F;
     }
   }
+}
 
-  // Online softmax over the tile (log2 domain).
+// Online softmax update with the tile's scores; sc becomes p = exp2(score - m).
+template <int G>
+__device__ __forceinline__ void tile_softmax(State<G>& st, float (&sc)[2][QFrag<G>::NQ][2]) {
+  constexpr int NQ = State<G>::NQ;
   float alpha[NQ];
   bool rescale = false;
 #pragma unroll
@@ -424,19 +467,26 @@ __device__ __forceinline__ void tile_compute(State<G>& st, const QFrag<G>& qf, u
       st.o[i][3] *= alpha[NQ - 1];
     }
   }
+}
 
-  // PV.  B fragment of thread (g, c): tokens c, c+4 (b0) and c+8, c+12 (b1) of the
-  // k-step for column g, taken from the lanes that scored them (rows c and c + 4 of
-  // the QK^T fragment).
+// PV of the tile with probabilities pr.  B fragment of thread (g, c): tokens c, c+4 (b0)
+// and c+8, c+12 (b1) of the k-step for column g, taken from the lanes that scored them
+// (rows c and c + 4 of the QK^T fragment).
+template <int G, int SEFF>
+__device__ __forceinline__ void tile_pv(State<G>& st, const uint8_t* slot, int ntok, int lane,
+                                        const float (&pr)[2][QFrag<G>::NQ][2]) {
+  const int g = lane >> 2, c = lane & 3;
+  const int tau0 = (g < 4) ? g : g + 4;
+  const int tau1 = tau0 + 4;
   const int srcA = 4 * c + (g >> 1);
   const int srcB = srcA + 16;
 #pragma unroll
   for (int j = 0; j < 2; j++) {
-    const uint32_t pbase = slot + (16 * j / SEFF) * (SEFF * 132);
+    const uint8_t* pbase = slot + (16 * j / SEFF) * (SEFF * 132);
     const int sl = (16 * j) % SEFF;
-    const uint32_t vb = pbase + SEFF * 64 + sl * 64;
-    const uint32_t svb = pbase + SEFF * 130 + sl * 2;
-    const float sv0 = half_at(svb + tau0 * 2), sv1 = half_at(svb + tau1 * 2);
+    const uint8_t* vb = pbase + SEFF * 64 + sl * 64;
+    const __half* svp = reinterpret_cast<const __half*>(pbase + SEFF * 130) + sl;
+    const float sv0 = __half2float(svp[tau0]), sv1 = __half2float(svp[tau1]);
     const bool v0 = 16 * j + tau0 < ntok, v1 = 16 * j + tau1 < ntok;
     // P' = p * s_v carried as fp16 hi + lo (relative precision ~2^-22).
     uint32_t bh0, bh1, bl0 = 0u, bl1 = 0u;
@@ -444,7 +494,7 @@ __device__ __forceinline__ void tile_compute(State<G>& st, const QFrag<G>& qf, u
       uint32_t xh[2], xl[2];
 #pragma unroll
       for (int qq = 0; qq < 2; qq++) {
-        const float p0 = v0 ? sc[j][qq][0] * sv0 : 0.0f, p1 = v1 ? sc[j][qq][1] * sv1 : 0.0f;
+        const float p0 = v0 ? pr[j][qq][0] * sv0 : 0.0f, p1 = v1 ? pr[j][qq][1] * sv1 : 0.0f;
         const __half h0 = __float2half_rn(p0), h1 = __float2half_rn(p1);
         xh[qq] = pack_half2(h0, h1);
         xl[qq] = pack_half2(__float2half_rn(p0 - __half2float(h0)),
@@ -460,7 +510,7 @@ __device__ __forceinline__ void tile_compute(State<G>& st, const QFrag<G>& qf, u
       bl0 = (g & 1) ? dO : dE;
       bl1 = (g & 1) ? eO : eE;
     } else {
-      const float p0 = v0 ? sc[j][0][0] * sv0 : 0.0f, p1 = v1 ? sc[j][0][1] * sv1 : 0.0f;
+      const float p0 = v0 ? pr[j][0][0] * sv0 : 0.0f, p1 = v1 ? pr[j][0][1] * sv1 : 0.0f;
       const __half h0 = __float2half_rn(p0), h1 = __float2half_rn(p1);
       const uint32_t xh = pack_half2(h0, h1);
       const uint32_t xl = pack_half2(__float2half_rn(p0 - __half2float(h0)),
@@ -473,10 +523,10 @@ __device__ __forceinline__ void tile_compute(State<G>& st, const QFrag<G>& qf, u
       if ((g >> 1) >= G) bh0 = bh1 = 0u;
     }
     // V rows of tokens c, c+4, c+8, c+12; this thread's channels [16g, 16g+16).
-    const uint2 t0 = lds_64(vb + (c + 0) * 64 + 8 * g);
-    const uint2 t1 = lds_64(vb + (c + 4) * 64 + 8 * g);
-    const uint2 t2 = lds_64(vb + (c + 8) * 64 + 8 * g);
-    const uint2 t3 = lds_64(vb + (c + 12) * 64 + 8 * g);
+    const uint2 t0 = *reinterpret_cast<const uint2*>(vb + (c + 0) * 64 + 8 * g);
+    const uint2 t1 = *reinterpret_cast<const uint2*>(vb + (c + 4) * 64 + 8 * g);
+    const uint2 t2 = *reinterpret_cast<const uint2*>(vb + (c + 8) * 64 + 8 * g);
+    const uint2 t3 = *reinterpret_cast<const uint2*>(vb + (c + 12) * 64 + 8 * g);
     const uint32_t w0[2] = {t0.x, t0.y}, w1[2] = {t1.x, t1.y};
     const uint32_t w2[2] = {t2.x, t2.y}, w3[2] = {t3.x, t3.y};
 #pragma unroll
@@ -566,8 +616,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
   uint8_t* ring = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kSlotBytes);
-  float* mbuf = reinterpret_cast<float*>(bars + kWarps * kStages);  // [kWarps][G][132]
-  int32_t* pre = reinterpret_cast<int32_t*>(mbuf + kWarps * G * kPartStride);
+  float* mbuf = reinterpret_cast<float*>(bars + kWarps * kStages);               // [kWarps][G][132]
+  uint32_t* qfb = reinterpret_cast<uint32_t*>(mbuf + kWarps * G * kPartStride);  // [G][3][4][8]
+  float* sfb = reinterpret_cast<float*>(qfb + G * 96);                           // [G]
+  int32_t* pre = reinterpret_cast<int32_t*>(sfb + 8);                            // [batch + 1]
+  int32_t* lens = pre + p.batch + 1;                                             // [batch]
   __shared__ int warp_sum[kWarps];
   __shared__ int running;
   __shared__ int last_flag;
@@ -575,13 +628,17 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int cap = p.max_pages_per_seq * p.page_size;
 
-  // Tiles per sequence -> exclusive prefix pre[0..batch] (block-wide scan).
+  // Clamped lengths, and tiles per sequence -> exclusive prefix pre[0..batch].
   if (tid == 0) running = 0;
   __syncthreads();
   for (int base = 0; base < p.batch; base += kThreads) {
     const int i = base + tid;
     int n = 0;
-    if (i < p.batch) n = (clamp_len(__ldg(p.seq_lens + i), cap, p.status) + kTileTokens - 1) / kTileTokens;
+    if (i < p.batch) {
+      const int L = clamp_len(__ldg(p.seq_lens + i), cap, p.status);
+      lens[i] = L;
+      n = (L + kTileTokens - 1) / kTileTokens;
+    }
     int incl = n;
 #pragma unroll
     for (int d = 1; d < 32; d *= 2) {
@@ -608,13 +665,18 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
         reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.num_kv_heads * G * kD)[i] =
             make_uint4(0u, 0u, 0u, 0u);
 
-  const long long T = static_cast<long long>(pre[p.batch]) * p.num_kv_heads;
-  const long long C = p.total_ctas;
-  const long long kc = blockIdx.x;
-  const long long X0 = T * kc / C, X1 = T * (kc + 1) / C;
-  if (X0 >= X1) return;  // the whole CTA: nothing to do
+  // CTA k takes tiles [k*chunk, (k+1)*chunk) of the T tiles (the host bounds T < 2^30);
+  // warp w of it takes tiles X0 + w, X0 + w + kWarps, ...
+  const int T = pre[p.batch] * p.num_kv_heads;
+  if (T == 0) return;
+  const int chunk = (T + p.total_ctas - 1) / p.total_ctas;
+  const int kc = blockIdx.x;
+  const int X0 = kc * chunk;
+  if (X0 >= T) return;  // the whole CTA: nothing to do
+  const int X1 = min(T, X0 + chunk);
 
-  const uint32_t ring_s = smem_addr(ring + w * kStages * kSlotBytes);
+  const uint8_t* ring_p = ring + w * kStages * kSlotBytes;
+  const uint32_t ring_s = smem_addr(ring_p);
   const uint32_t bar_s = smem_addr(bars + w * kStages);
   if (lane == 0) {
 #pragma unroll
@@ -624,73 +686,107 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   __syncwarp();
   const uint64_t pol = l2_policy_evict_first();
 
-  // Producer walk: issue the first kStages tiles.
-  Walk pw;
-  unit_of_tile(pw.u, X0, pre, p);
-  pw.x = X0 + w;
-  pw.xe = min(X1, pw.u.U + pw.u.n);
-  pw.valid = true;
-  walk_settle(pw, X1, w, pre, p);
-  int issued = 0;
-  for (int s = 0; s < kStages && pw.valid; s++) {
-    const int pid = tile_page_id<SEFF>(pw.u, pw.x - pw.u.U, lane, p);
-    tile_issue<SEFF>(pw.u, pw.x - pw.u.U, pid, ring_s + s * kSlotBytes, bar_s + 8 * s, lane, pol, p);
-    issued++;
-    pw.x += kWarps;
-    walk_settle(pw, X1, w, pre, p);
-  }
+  // Producer: page-id batches 0 and 1, then the first kStages tiles.
+  constexpr int kBatch = PageBatch<SEFF>::kBatch;
+  Producer<SEFF> pr;
+  pr.t = 0;
+  pr.nT = (X1 - X0 - w + kWarps - 1) / kWarps;
+  pr.tb = 0;
+  pr.pid_cur = load_page_batch<SEFF>(0, X0, X1, w, lane, pre, lens, p);
+  pr.pid_nxt = load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p);
+  if (pr.nT > 0) unit_of_tile(pr.u, X0 + w, pre, lens, p);
+  while (pr.t < pr.nT && pr.t < kStages)
+    producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
 
-  // Consumer: the CTA's units in order; this warp's tiles of each.
-  Unit cu = pw.u;  // overwritten just below
-  unit_of_tile(cu, X0, pre, p);
-  long long xs = X0;
-  uint4 qraw[4];
-  load_q_raw<G>(qraw, cu, lane, p);
-  int consumed = 0;
+  // q of the first unit, prepared cooperatively while the first copies fly.
+  Unit cu;
+  unit_of_tile(cu, X0, pre, lens, p);
+  uint2 qraw[2];
+  load_q_coop<G>(qraw, cu, w, lane, p);
+  prep_q<G>(qfb, sfb, qraw, w, lane, p);
+  __syncthreads();
+
+  int consumed = 0;   // tiles of this warp consumed (tile t uses slot t % kStages)
   bool dead = false;  // a bounded wait gave up: stop touching the ring
   State<G> st;
   QFrag<G> qf;
+  constexpr int NQ = QFrag<G>::NQ;
   while (true) {
-    const long long xe = min(X1, cu.U + cu.n);
-    make_qfrag<G>(qf, qraw, lane, p);
+    const int ux0 = max(X0, cu.U), ux1 = min(X1, cu.U + cu.n);
+    qfrag_load<G>(qf, qfb, sfb, lane);
     Unit nu = cu;
-    const bool has_next = xe < X1;
+    const bool has_next = ux1 < X1;
     if (has_next) {
-      unit_next(nu, pre, p);
-      load_q_raw<G>(qraw, nu, lane, p);  // prefetch the next unit's q
+      unit_next(nu, pre, lens, p);
+      load_q_coop<G>(qraw, nu, w, lane, p);  // prefetch the next unit's q
     }
     state_reset<G>(st);
-    for (long long x = xs + w; x < xe && !dead; x += kWarps) {
-      const int s = consumed % kStages;
-      const uint32_t parity = static_cast<uint32_t>((consumed / kStages) & 1);
-      const bool more = pw.valid;
-      const int pid_next = more ? tile_page_id<SEFF>(pw.u, pw.x - pw.u.U, lane, p) : -1;
-      if (!mbar_wait_bounded(bar_s + 8 * s, parity, kWaitLimitNs)) {
-        dead = true;
-        if (lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
-        break;
-      }
-      const int k = static_cast<int>(x - cu.U);
-      const int ntok = min(kTileTokens, cu.L - k * kTileTokens);
-      tile_compute<G, SEFF>(st, qf, ring_s + s * kSlotBytes, ntok, lane);
-      consumed++;
+    // This warp's tiles of the unit: x = first + kWarps*i < ux1.  Pipelined: the QK^T
+    // of the next tile is computed next to the PV of the current one.
+    const int first = ux0 + ((X0 + w - ux0) & (kWarps - 1));
+    const int nt = first < ux1 ? (ux1 - first + kWarps - 1) / kWarps : 0;
+    float sc[2][NQ][2];
+    int slot_i = consumed % kStages;
+    uint32_t parity = static_cast<uint32_t>((consumed / kStages) & 1);
+    auto ntok_of = [&](int x) { return min(kTileTokens, cu.L - (x - cu.U) * kTileTokens); };
+    // Release a consumed slot and refill it with the warp's tile kStages ahead.
+    auto refill = [&]() {
       __syncwarp();
-      if (more) {
+      if (pr.t < pr.nT) {
         fence_proxy_async_smem();
-        tile_issue<SEFF>(pw.u, pw.x - pw.u.U, pid_next, ring_s + s * kSlotBytes, bar_s + 8 * s,
-                         lane, pol, p);
-        issued++;
-        pw.x += kWarps;
-        walk_settle(pw, X1, w, pre, p);
+        producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
+      }
+    };
+    if (nt > 0 && !dead) {
+      if (!mbar_wait_bounded(bar_s + 8 * slot_i, parity, kWaitLimitNs)) {
+        dead = true;
+      } else {
+        tile_qk<G, SEFF>(qf, ring_p + slot_i * kSlotBytes, ntok_of(first), lane, sc);
+        tile_softmax<G>(st, sc);
       }
     }
+    // Steady state: a next tile always exists.
+    for (int i = 0; i + 1 < nt && !dead; i++) {
+      const int x = first + kWarps * i;
+      const int cur = slot_i;
+      const int nslot = cur + 1 == kStages ? 0 : cur + 1;
+      const uint32_t npar = cur + 1 == kStages ? parity ^ 1u : parity;
+      if (!mbar_wait_bounded(bar_s + 8 * nslot, npar, kWaitLimitNs)) {
+        dead = true;
+        break;
+      }
+      float sn[2][NQ][2];
+      tile_qk<G, SEFF>(qf, ring_p + nslot * kSlotBytes, ntok_of(x + kWarps), lane, sn);
+      tile_pv<G, SEFF>(st, ring_p + cur * kSlotBytes, ntok_of(x), lane, sc);
+      consumed++;
+      slot_i = nslot;
+      parity = npar;
+      refill();
+      tile_softmax<G>(st, sn);
+#pragma unroll
+      for (int j = 0; j < 2; j++)
+#pragma unroll
+        for (int qq = 0; qq < NQ; qq++)
+#pragma unroll
+          for (int r = 0; r < 2; r++) sc[j][qq][r] = sn[j][qq][r];
+    }
+    // Last tile of the unit for this warp.
+    if (nt > 0 && !dead) {
+      const int cur = slot_i;
+      tile_pv<G, SEFF>(st, ring_p + cur * kSlotBytes, ntok_of(first + kWarps * (nt - 1)), lane, sc);
+      consumed++;
+      slot_i = cur + 1 == kStages ? 0 : cur + 1;
+      refill();
+    }
+    if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
 
     // Merge the 4 warps' partials of this unit.
     state_to_smem<G>(st, mbuf, w, lane);
     __syncthreads();
-    const long long unit = static_cast<long long>(cu.b) * p.num_kv_heads + cu.h;
-    const long long k_first = cta_of(cu.U, T, C), k_last = cta_of(cu.U + cu.n - 1, T, C);
+    const int unit = cu.b * p.num_kv_heads + cu.h;
+    const int k_first = cu.U / chunk, k_last = (cu.U + cu.n - 1) / chunk;
     const bool alone = k_first == k_last;
+    __half* orow = p.out + (static_cast<size_t>(cu.b) * p.num_kv_heads * G + cu.h * G) * kD;
     for (int qi = w; qi < G; qi += kWarps) {
       float M = -CUDART_INF_F;
 #pragma unroll
@@ -709,10 +805,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
         l += e * rec[kD + 1];
       }
       if (alone) {
-        finish_query(o, l, p.out + (static_cast<size_t>(cu.b) * p.num_kv_heads * G + cu.h * G + qi) * kD,
-                     lane, p);
+        finish_query(o, l, orow + qi * kD, lane, p);
       } else {
-        float* rec = p.part + ((unit + kc) * G + qi) * kPartStride;
+        float* rec = p.part + (static_cast<size_t>(unit + kc) * G + qi) * kPartStride;
         *reinterpret_cast<float4*>(rec + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
         if (lane == 0) {
           rec[kD] = M;
@@ -721,14 +816,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       }
     }
     if (!alone) {
-      // Last CTA to arrive merges every CTA's partial of the unit.
+      // The last CTA to arrive merges every CTA's partial of the unit (CTAs k_first ..
+      // k_last all hold tiles of it).
       __threadfence();
       __syncthreads();
       if (tid == 0) {
-        int expect = 0;
-        for (long long k2 = k_first; k2 <= k_last; k2++) expect += (T * k2 / C < T * (k2 + 1) / C);
         const int old = atomicAdd(p.counters + unit, 1);
-        last_flag = (old == expect - 1);
+        last_flag = (old == k_last - k_first);
         if (last_flag) p.counters[unit] = 0;  // ready for the next call
       }
       __syncthreads();
@@ -736,14 +830,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
         __threadfence();
         for (int qi = w; qi < G; qi += kWarps) {
           float M = -CUDART_INF_F;
-          for (long long k2 = k_first; k2 <= k_last; k2++) {
-            if (T * k2 / C == T * (k2 + 1) / C) continue;
-            M = fmaxf(M, __ldcg(p.part + ((unit + k2) * G + qi) * kPartStride + kD));
-          }
+          for (int k2 = k_first; k2 <= k_last; k2++)
+            M = fmaxf(M, __ldcg(p.part + (static_cast<size_t>(unit + k2) * G + qi) * kPartStride + kD));
           float o[4] = {0.0f, 0.0f, 0.0f, 0.0f}, l = 0.0f;
-          for (long long k2 = k_first; k2 <= k_last; k2++) {
-            if (T * k2 / C == T * (k2 + 1) / C) continue;
-            const float* rec = p.part + ((unit + k2) * G + qi) * kPartStride;
+          for (int k2 = k_first; k2 <= k_last; k2++) {
+            const float* rec = p.part + (static_cast<size_t>(unit + k2) * G + qi) * kPartStride;
             const float e = exp2f(__ldcg(rec + kD) - M);
             const float4 v = __ldcg(reinterpret_cast<const float4*>(rec + 4 * lane));
             o[0] += e * v.x;
@@ -752,21 +843,20 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
             o[3] += e * v.w;
             l += e * __ldcg(rec + kD + 1);
           }
-          finish_query(o, l,
-                       p.out + (static_cast<size_t>(cu.b) * p.num_kv_heads * G + cu.h * G + qi) * kD,
-                       lane, p);
+          finish_query(o, l, orow + qi * kD, lane, p);
         }
       }
     }
-    __syncthreads();  // the merge buffer is reused by the next unit
+    // Everyone has read this unit's q fragments and merge buffer: prepare the next q.
+    if (has_next) prep_q<G>(qfb, sfb, qraw, w, lane, p);
+    __syncthreads();
     if (!has_next) break;
     cu = nu;
-    xs = cu.U;
   }
 
   if (dead) {
     // Let copies still in flight land before the CTA's shared memory is released.
-    for (int j = consumed + 1; j < issued; j++)
+    for (int j = consumed + 1; j < pr.t; j++)
       mbar_wait_bounded(bar_s + 8 * (j % kStages), static_cast<uint32_t>((j / kStages) & 1),
                         kWaitLimitNs);
   }
@@ -795,7 +885,8 @@ size_t smem_bytes(int group, int max_batch) {
   size_t s = static_cast<size_t>(kWarps) * kStages * kSlotBytes;
   s += sizeof(uint64_t) * kWarps * kStages;
   s += sizeof(float) * kWarps * group * kPartStride;
-  s += static_cast<size_t>(max_batch + 1) * sizeof(int32_t);
+  s += sizeof(uint32_t) * group * 96 + sizeof(float) * 8;  // q fragment table, M factors
+  s += static_cast<size_t>(2 * max_batch + 1) * sizeof(int32_t);  // prefix, lengths
   s += 128;  // alignment slack for the ring base
   return (s + 15) & ~static_cast<size_t>(15);
 }

@@ -50,6 +50,10 @@ bool desc_ok(const kvq_desc* d, int* why) {
   if (d->max_batch > 4096) return false;
   if (static_cast<long long>(d->max_pages_per_seq) * S > (1LL << 30)) return false;
   if (static_cast<long long>(d->max_batch) * d->max_pages_per_seq > (1LL << 31) - 1) return false;
+  // The decode kernel numbers 32-token tiles of all (sequence, KV head) pairs in 32 bits.
+  const long long tiles_per_seq = (static_cast<long long>(d->max_pages_per_seq) * S + 31) / 32;
+  if (static_cast<long long>(d->max_batch) * d->num_kv_heads * tiles_per_seq >= (1LL << 30))
+    return false;
   *why = KVQ_OK;
   return true;
 }
@@ -243,6 +247,7 @@ int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, const int32
   p.group = c->d.num_q_heads / c->d.num_kv_heads;
   p.num_pages = c->d.num_pages;
   p.page_size = c->d.page_size;
+  p.page_shift = __builtin_ctz(static_cast<unsigned>(c->d.page_size));
   p.max_pages_per_seq = c->d.max_pages_per_seq;
   p.hadamard_block = c->d.hadamard_block;
   const double sm = softmax_scale == 0.0f ? 1.0 / sqrt(static_cast<double>(c->d.head_dim))

@@ -48,6 +48,7 @@ struct DecodeParams {
   int group;                      // G = Hq / Hkv
   int num_pages;
   int page_size;
+  int page_shift;                 // log2(page_size)
   int max_pages_per_seq;
   int hadamard_block;
   float q_scale;                  // softmax_scale * log2(e)
