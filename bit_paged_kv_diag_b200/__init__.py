@@ -22,7 +22,8 @@ from . import build as _build
 
 __all__ = [
     "KVQError", "Desc", "Cache", "lib", "pool_bytes", "assign_pages", "alloc_pages",
-    "rotate_quant_append", "decode_attention", "free", "get_device_status", "status_string",
+    "rotate_quant_append", "decode_attention", "decode_attention_noalloc", "free",
+    "get_device_status", "status_string",
     "EXPORTED",
 ]
 
@@ -32,7 +33,7 @@ KVQ_DEV_BAD_PAGE, KVQ_DEV_BAD_POS, KVQ_DEV_TIMEOUT = 1, 2, 4
 EXPORTED = (
     "kvq_pool_bytes", "kvq_assign_pages", "kvq_alloc_pages", "kvq_rotate_quant_append",
     "kvq_decode_attention", "kvq_pool_ptr", "kvq_get_device_status", "kvq_free",
-    "kvq_status_string",
+    "kvq_status_string", "kvq_decode_attention_noalloc",
 )
 
 
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "kvq_get_device_status": (ctypes.c_int, [vp, i32p, vp]),
             "kvq_free": (ctypes.c_int, [vp]),
             "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "kvq_decode_attention_noalloc": (ctypes.c_int, [dp, vp, i32, vp, vp, vp, i32,
+                                                            ctypes.c_float, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -208,6 +211,23 @@ def decode_attention(cache: Cache, layer: int, q, seq_lens, page_table, softmax_
         _dev_ptr(seq_lens, "seq_lens", torch.int32), _dev_ptr(page_table, "page_table", torch.int32),
         batch, float(softmax_scale), _dev_ptr(out, "out", torch.float16), _stream_ptr(stream))
     _check(rc, "kvq_decode_attention")
+    return out
+
+
+def decode_attention_noalloc(desc: Desc, pool, layer: int, q, seq_lens, page_table,
+                             softmax_scale=0.0, out=None, stream=None):
+    """Decode attention without a handle and without any device allocation by the library
+    (scratch lives in a fixed device array; see include/kvq.h for its limits)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    batch = int(seq_lens.shape[0])
+    rc = lib().kvq_decode_attention_noalloc(
+        ctypes.byref(desc), _dev_ptr(pool, "pool", torch.uint8), int(layer),
+        _dev_ptr(q, "q", torch.float16), _dev_ptr(seq_lens, "seq_lens", torch.int32),
+        _dev_ptr(page_table, "page_table", torch.int32), batch, float(softmax_scale),
+        _dev_ptr(out, "out", torch.float16), _stream_ptr(stream))
+    _check(rc, "kvq_decode_attention_noalloc")
     return out
 
 

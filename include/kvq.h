@@ -172,6 +172,33 @@ KVQ_API int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, con
                          const int32_t* page_table, int32_t batch, float softmax_scale,
                          void* out, void* stream);
 
+/* Decode attention that allocates nothing.  The pages have no counterpart of this call;
+ * it exists for callers that cannot call cudaMalloc: an inference runtime that has
+ * reserved all of device memory for its own pool and forbids stray allocations, a plugin
+ * whose host framework owns every device allocation, or a latency-critical path where
+ * cudaMalloc's implicit device synchronisation is not acceptable.  Those callers cannot
+ * create a kvq_cache (kvq_alloc_pages allocates the split scratch), so this call takes the
+ * geometry and the pool directly and keeps its scratch in one fixed-size device array
+ * inside the library (about 2.2 MB, held by every GPU that loads the library until exit).
+ *   d              cache geometry (as for kvq_alloc_pages); only read
+ *   pool           device pool of kvq_pool_bytes(d) bytes, 16-byte aligned, laid out as
+ *                  kvq_rotate_quant_append writes it (caller-owned)
+ *   layer, q, seq_lens, page_table, batch, softmax_scale, out, stream: as for
+ *                  kvq_decode_attention
+ * Limits of the fixed scratch: batch * num_kv_heads <= 4096 and
+ * (batch * num_kv_heads + C) * G <= 4096, C = the kernel's grid (up to 3 CTAs per SM);
+ * larger calls return KVQ_EUNSUPPORTED before anything is launched.
+ * The first call on a device sets the array up (looks up its device address and zeroes
+ * its counters, synchronising the device); make that first call before any stream
+ * capture.  Every call shares the array: calls that overlap on the GPU (two streams, or
+ * two devices' contexts racing on one device) race on it and must be ordered by the
+ * caller.  Device-side range errors are not reported by this call (they still never
+ * fault).  Returns KVQ_OK or a negative status. */
+KVQ_API int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, int32_t layer,
+                                         const void* q, const int32_t* seq_lens,
+                                         const int32_t* page_table, int32_t batch,
+                                         float softmax_scale, void* out, void* stream);
+
 /* Device address of the pool (the caller's buffer, or the library's). NULL for NULL. */
 KVQ_API void* kvq_pool_ptr(const kvq_cache* c);
 
