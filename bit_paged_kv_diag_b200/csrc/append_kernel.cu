@@ -202,6 +202,9 @@ __device__ __forceinline__ uint16_t quantise(const float (&x)[64], unsigned pmas
 
 template <int BLOCK>
 __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
+  // The next kernel may start its own prologue; the pool stores below wait for every
+  // earlier kernel (griddep_wait), so they never race with a decode still reading.
+  griddep_launch_dependents();
   const int l = threadIdx.x & 1;
   // Shuffles never leave the lane pair of a row, so they name only those two lanes.
   const unsigned pmask = 0x3u << (threadIdx.x & 30);
@@ -232,6 +235,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
 
   uint32_t q[8];
   const uint16_t sbits = quantise(x, pmask, q);
+  griddep_wait();
   if (!ok) {
     if (l == 0 && kv == 0)
       atomicOr(p.status, (pos < 0 || lp >= p.max_pages_per_seq) ? KVQ_DEV_BAD_POS_BIT
@@ -258,13 +262,23 @@ int launch_append(const AppendParams& p, int block, cudaStream_t stream) {
   if (nrows == 0) return 0;
   const long long grid = (nrows + kRowsPerBlock - 1) / kRowsPerBlock;
   if (grid > 0x7fffffffLL) return -1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   switch (block) {
-    case 32: append_kernel<32><<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(p); break;
-    case 64: append_kernel<64><<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(p); break;
-    case 128: append_kernel<128><<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(p); break;
+    case 32: e = cudaLaunchKernelEx(&cfg, append_kernel<32>, p); break;
+    case 64: e = cudaLaunchKernelEx(&cfg, append_kernel<64>, p); break;
+    case 128: e = cudaLaunchKernelEx(&cfg, append_kernel<128>, p); break;
     default: return -1;
   }
-  return cudaGetLastError() == cudaSuccess ? 0 : -2;
+  return e == cudaSuccess ? 0 : -2;
 }
 
 }  // namespace kvq

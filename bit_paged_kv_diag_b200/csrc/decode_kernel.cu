@@ -627,6 +627,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int cap = p.max_pages_per_seq * p.page_size;
+  // The prologue below reads only seq_lens and the page table, which no kernel of this
+  // library writes; everything an earlier kernel may write or read (pool, q, out, the
+  // scratch) is touched only after griddep_wait().
+  griddep_launch_dependents();
 
   // Clamped lengths, and tiles per sequence -> exclusive prefix pre[0..batch].
   if (tid == 0) running = 0;
@@ -657,23 +661,14 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   if (tid == 0) pre[p.batch] = running;
   __syncthreads();
 
-  // An empty sequence has no tiles: its output rows are zeros (CTAs share the writes).
-  const int row_words = p.num_kv_heads * G * kD / 8;  // 16-byte words per sequence
-  for (int b = blockIdx.x; b < p.batch; b += p.total_ctas)
-    if (pre[b + 1] == pre[b])
-      for (int i = tid; i < row_words; i += kThreads)
-        reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.num_kv_heads * G * kD)[i] =
-            make_uint4(0u, 0u, 0u, 0u);
-
   // CTA k takes tiles [k*chunk, (k+1)*chunk) of the T tiles (the host bounds T < 2^30);
   // warp w of it takes tiles X0 + w, X0 + w + kWarps, ...
   const int T = pre[p.batch] * p.num_kv_heads;
-  if (T == 0) return;
   const int chunk = (T + p.total_ctas - 1) / p.total_ctas;
   const int kc = blockIdx.x;
   const int X0 = kc * chunk;
-  if (X0 >= T) return;  // the whole CTA: nothing to do
   const int X1 = min(T, X0 + chunk);
+  const bool has_tiles = T > 0 && X0 < T;
 
   const uint8_t* ring_p = ring + w * kStages * kSlotBytes;
   const uint32_t ring_s = smem_addr(ring_p);
@@ -686,15 +681,28 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   __syncwarp();
   const uint64_t pol = l2_policy_evict_first();
 
-  // Producer: page-id batches 0 and 1, then the first kStages tiles.
+  // Producer: page-id batches 0 and 1 (page table only: before the wait).
   constexpr int kBatch = PageBatch<SEFF>::kBatch;
   Producer<SEFF> pr;
   pr.t = 0;
-  pr.nT = (X1 - X0 - w + kWarps - 1) / kWarps;
+  pr.nT = has_tiles ? (X1 - X0 - w + kWarps - 1) / kWarps : 0;
   pr.tb = 0;
-  pr.pid_cur = load_page_batch<SEFF>(0, X0, X1, w, lane, pre, lens, p);
-  pr.pid_nxt = load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p);
+  pr.pid_cur = has_tiles ? load_page_batch<SEFF>(0, X0, X1, w, lane, pre, lens, p) : -1;
+  pr.pid_nxt = has_tiles ? load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p) : -1;
   if (pr.nT > 0) unit_of_tile(pr.u, X0 + w, pre, lens, p);
+
+  griddep_wait();
+
+  // An empty sequence has no tiles: its output rows are zeros (CTAs share the writes).
+  const int row_words = p.num_kv_heads * G * kD / 8;  // 16-byte words per sequence
+  for (int b = blockIdx.x; b < p.batch; b += p.total_ctas)
+    if (pre[b + 1] == pre[b])
+      for (int i = tid; i < row_words; i += kThreads)
+        reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.num_kv_heads * G * kD)[i] =
+            make_uint4(0u, 0u, 0u, 0u);
+  if (!has_tiles) return;  // the whole CTA: nothing else to do
+
+  // The first kStages tiles.
   while (pr.t < pr.nT && pr.t < kStages)
     producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
 
@@ -918,8 +926,17 @@ int launch_decode(const DecodeParams& p, const DecodeLaunch& L, cudaStream_t str
   DecodeParams q = p;
   q.total_ctas = L.grid;
   void* args[] = {&q};
-  if (cudaLaunchKernel(fn, dim3(L.grid), dim3(kThreads), args, L.smem, stream) != cudaSuccess)
-    return -2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(L.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return -2;
   return 0;
 }
 
