@@ -55,7 +55,7 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kSlotBytes = kTileTokens * (kD + 4);  // 4224: one tile of codes + scales
-constexpr int kWarps = 4;                           // warps per CTA
+constexpr int kWarps = kDecodeWarps;                // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 3;                          // ring slots per warp
 constexpr uint64_t kWaitLimitNs = 2000000000ull;    // bounded waits: 2 s
@@ -218,97 +218,96 @@ struct QFrag {
   float sf[NQ];  // M / 1024 of the owned queries
 };
 
-// Raw fp16 q for the cooperative preparation: warp w handles query w (and w + 4 when
-// G == 8); lane holds channels 4*lane..4*lane+3.
-template <int G>
-__device__ __forceinline__ void load_q_coop(uint2 (&raw)[2], const Unit& u, int w, int lane,
-                                            const DecodeParams& p) {
-#pragma unroll
-  for (int r = 0; r < 2; r++) {
-    const int qi = w + kWarps * r;
-    raw[r] = make_uint2(0u, 0u);
-    if (qi < G)
-      raw[r] = __ldg(reinterpret_cast<const uint2*>(
-                         p.q + (static_cast<size_t>(u.b) * p.num_kv_heads * G + u.h * G + qi) * kD) +
-                     lane);
-  }
-}
-
 // Rotate (the fixed-order butterfly: stages h = 1, 2 in registers, h = 4..64 across
-// lanes), scale by c_b * softmax_scale * log2(e), and cut query qi into three int8
-// slices q' = M/64 * (q1 + q2/128 + q3/16384), M the power of two >= max|q'| (1 for a
-// zero row); write them to the shared table in fragment order:
-//   qfb word ((qi*3 + s)*4 + c)*8 + 2*jj + half, byte e  <->  channel 32c + 8jj + 2e + half.
+// lanes), scale by c_b * softmax_scale * log2(e), and cut every query of the unit into
+// three int8 slices q' = M/64 * (q1 + q2/128 + q3/16384), M the power of two >= max|q'|
+// (1 for a zero row).  qraw: the unit's G fp16 rows in shared memory; the slices go to the
+// warp's fragment table in fragment order:
+//   frag word ((qi*3 + s)*4 + c)*8 + 2*jj + half, byte e  <->  channel 32c + 8jj + 2e + half.
 template <int G>
-__device__ __forceinline__ void prep_q(uint32_t* qfb, float* sfb, const uint2 (&raw)[2], int w,
-                                       int lane, const DecodeParams& p) {
+__device__ __forceinline__ void prep_q_warp(const uint8_t* qraw, uint32_t* frag, float* sf, int lane,
+                                            const DecodeParams& p) {
+  // Up to four queries at a time: their shuffle chains are independent and interleave.
+  constexpr int QB = G < 4 ? G : 4;
+  const int c = lane >> 3, jj = (lane >> 1) & 3, e0 = (2 * lane) & 3;
+  uint8_t* base = reinterpret_cast<uint8_t*>(frag);
+#pragma unroll 1
+  for (int q0 = 0; q0 < G; q0 += QB) {
+    float x[QB][4];
 #pragma unroll
-  for (int r = 0; r < 2; r++) {
-    const int qi = w + kWarps * r;
-    if (qi >= G) continue;  // warp-uniform
-    float x[4];
-    {
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw[r].x));
-      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw[r].y));
-      x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    for (int b = 0; b < QB; b++) {
+      const uint2 raw = *reinterpret_cast<const uint2*>(qraw + (q0 + b) * kD * 2 + 8 * lane);
+      const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+      const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+      float t0 = lo.x, t1 = lo.y, t2 = hi.x, t3 = hi.y;
+      const float a0 = __fadd_rn(t0, t1), a1 = __fsub_rn(t0, t1);
+      const float a2 = __fadd_rn(t2, t3), a3 = __fsub_rn(t2, t3);
+      x[b][0] = __fadd_rn(a0, a2);
+      x[b][2] = __fsub_rn(a0, a2);
+      x[b][1] = __fadd_rn(a1, a3);
+      x[b][3] = __fsub_rn(a1, a3);
     }
-    float t0 = x[0], t1 = x[1];
-    x[0] = __fadd_rn(t0, t1); x[1] = __fsub_rn(t0, t1);
-    t0 = x[2]; t1 = x[3];
-    x[2] = __fadd_rn(t0, t1); x[3] = __fsub_rn(t0, t1);
-    t0 = x[0]; t1 = x[2];
-    x[0] = __fadd_rn(t0, t1); x[2] = __fsub_rn(t0, t1);
-    t0 = x[1]; t1 = x[3];
-    x[1] = __fadd_rn(t0, t1); x[3] = __fsub_rn(t0, t1);
 #pragma unroll
     for (int s = 0; s < 5; s++) {
       if ((4 << s) < p.hadamard_block) {
         const float sgn = ((lane >> s) & 1) ? -1.0f : 1.0f;
 #pragma unroll
-        for (int e = 0; e < 4; e++) x[e] = __fmaf_rn(x[e], sgn, __shfl_xor_sync(kFull, x[e], 1 << s));
+        for (int b = 0; b < QB; b++)
+#pragma unroll
+          for (int e = 0; e < 4; e++)
+            x[b][e] = __fmaf_rn(x[b][e], sgn, __shfl_xor_sync(kFull, x[b][e], 1 << s));
       }
     }
-    float amax = 0.0f;
+    float amax[QB];
 #pragma unroll
-    for (int e = 0; e < 4; e++) {
-      x[e] = __fmul_rn(__fmul_rn(x[e], p.cb), p.q_scale);
-      amax = fmaxf(amax, fabsf(x[e]));
+    for (int b = 0; b < QB; b++) {
+      amax[b] = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        x[b][e] = __fmul_rn(__fmul_rn(x[b][e], p.cb), p.q_scale);
+        amax[b] = fmaxf(amax[b], fabsf(x[b][e]));
+      }
     }
 #pragma unroll
-    for (int d = 1; d < 32; d *= 2) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, d));
-    float M = 1.0f;
-    if (amax > 1e-30f) {
-      const uint32_t bits = __float_as_uint(amax);
-      M = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax;
-    }
-    const float inv = __fdiv_rn(64.0f, M);  // exact: powers of two
-    uint32_t ms[3][4];
+    for (int d = 1; d < 32; d *= 2)
 #pragma unroll
-    for (int e = 0; e < 4; e++) {
-      const float t = x[e] * inv;                         // |t| <= 64, exact scaling
-      const float m1 = t + kMagic;                        // rint(t) in the low mantissa bits
-      const float r1 = (t - (m1 - kMagic)) * 128.0f;      // exact
-      const float m2 = r1 + kMagic;
-      const float r2 = (r1 - (m2 - kMagic)) * 128.0f;
-      const float m3 = r2 + kMagic;
-      ms[0][e] = __float_as_uint(m1);
-      ms[1][e] = __float_as_uint(m2);
-      ms[2][e] = __float_as_uint(m3);
-    }
-    // Channels 4*lane + i: c = lane/8, jj = (lane/2)%4, half = i%2, byte e0 + i/2 with
-    // e0 = (2*lane)%4: a 2-byte store per (slice, half).
-    const int c = lane >> 3, jj = (lane >> 1) & 3, e0 = (2 * lane) & 3;
-    uint8_t* base = reinterpret_cast<uint8_t*>(qfb);
+      for (int b = 0; b < QB; b++) amax[b] = fmaxf(amax[b], __shfl_xor_sync(kFull, amax[b], d));
 #pragma unroll
-    for (int s = 0; s < 3; s++) {
-      const int word = ((qi * 3 + s) * 4 + c) * 8 + 2 * jj;
-      const uint16_t h0 = static_cast<uint16_t>((ms[s][0] & 0xFFu) | ((ms[s][2] & 0xFFu) << 8));
-      const uint16_t h1 = static_cast<uint16_t>((ms[s][1] & 0xFFu) | ((ms[s][3] & 0xFFu) << 8));
-      *reinterpret_cast<uint16_t*>(base + word * 4 + e0) = h0;
-      *reinterpret_cast<uint16_t*>(base + (word + 1) * 4 + e0) = h1;
+    for (int b = 0; b < QB; b++) {
+      float M = 1.0f;
+      if (amax[b] > 1e-30f) {
+        const uint32_t bits = __float_as_uint(amax[b]);
+        M = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax[b];
+      }
+      const float inv = __fdiv_rn(64.0f, M);  // exact: powers of two
+      uint32_t ms[3][4];
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        const float t = x[b][e] * inv;                      // |t| <= 64, exact scaling
+        const float m1 = t + kMagic;                        // rint(t) in the low mantissa bits
+        const float r1 = (t - (m1 - kMagic)) * 128.0f;      // exact
+        const float m2 = r1 + kMagic;
+        const float r2 = (r1 - (m2 - kMagic)) * 128.0f;
+        const float m3 = r2 + kMagic;
+        ms[0][e] = __float_as_uint(m1);
+        ms[1][e] = __float_as_uint(m2);
+        ms[2][e] = __float_as_uint(m3);
+      }
+      // Channels 4*lane + i: c = lane/8, jj = (lane/2)%4, half = i%2, byte e0 + i/2 with
+      // e0 = (2*lane)%4: a 2-byte store per (slice, half).
+      const int qi = q0 + b;
+#pragma unroll
+      for (int sl = 0; sl < 3; sl++) {
+        const int word = ((qi * 3 + sl) * 4 + c) * 8 + 2 * jj;
+        const uint16_t h0 = static_cast<uint16_t>((ms[sl][0] & 0xFFu) | ((ms[sl][2] & 0xFFu) << 8));
+        const uint16_t h1 = static_cast<uint16_t>((ms[sl][1] & 0xFFu) | ((ms[sl][3] & 0xFFu) << 8));
+        *reinterpret_cast<uint16_t*>(base + word * 4 + e0) = h0;
+        *reinterpret_cast<uint16_t*>(base + (word + 1) * 4 + e0) = h1;
+      }
+      if (lane == 0) sf[qi] = M * (1.0f / 1024.0f);
     }
-    if (lane == 0) sfb[qi] = M * (1.0f / 1024.0f);
   }
+  __syncwarp();
 }
 
 template <int G>
@@ -543,9 +542,11 @@ __device__ __forceinline__ void tile_pv(State<G>& st, const uint8_t* slot, int n
   }
 }
 
-// Warp partial (owned queries) -> shared merge buffer buf[w][qi][kPartStride].
+// Warp partial of one unit (its owned queries) -> a record block [G][kPartStride] at rec
+// (shared or global memory): o'[128], m, l per query.  With qsel >= 0 only query qsel is
+// written, at rec itself.
 template <int G>
-__device__ __forceinline__ void state_to_smem(const State<G>& st, float* buf, int w, int lane) {
+__device__ __forceinline__ void state_write(const State<G>& st, float* rec, int lane, int qsel = -1) {
   constexpr int NQ = State<G>::NQ;
   const int g = lane >> 2, c = lane & 3;
 #pragma unroll
@@ -555,7 +556,7 @@ __device__ __forceinline__ void state_to_smem(const State<G>& st, float* buf, in
     l += __shfl_xor_sync(kFull, l, 8);
     l += __shfl_xor_sync(kFull, l, 16);
     const int qi = (G == 8) ? 2 * c + qq : c;
-    if (qi >= G) continue;
+    if (qi >= G || (qsel >= 0 && qi != qsel)) continue;
     float v[16];
 #pragma unroll
     for (int i = 0; i < 8; i++) {
@@ -567,13 +568,13 @@ __device__ __forceinline__ void state_to_smem(const State<G>& st, float* buf, in
         v[2 * i + 1] = st.o[i][2] + st.o[i][3];
       }
     }
-    float* rec = buf + (w * G + qi) * kPartStride;
-    float4* dst = reinterpret_cast<float4*>(rec + 16 * g);
+    float* r = rec + (qsel >= 0 ? 0 : qi * kPartStride);
+    float4* dst = reinterpret_cast<float4*>(r + 16 * g);
 #pragma unroll
     for (int e = 0; e < 4; e++) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
     if (g == 0) {
-      rec[kD] = st.m[qq];
-      rec[kD + 1] = l;
+      r[kD] = st.m[qq];
+      r[kD + 1] = l;
     }
   }
 }
@@ -608,22 +609,148 @@ __device__ __forceinline__ void finish_query(const float (&o)[4], float l, __hal
   *reinterpret_cast<uint2*>(dst + 4 * lane) = make_uint2(lo, hi);
 }
 
+// A unit with a single contributing warp (one tile): finish it from the warp's registers,
+// one query at a time through a staging area of kPartStride floats.
+template <int G>
+__device__ __forceinline__ void finish_from_state(const State<G>& st, float* stage, __half* orow,
+                                                  int lane, const DecodeParams& p) {
+#pragma unroll 1
+  for (int qi = 0; qi < G; qi++) {
+    __syncwarp();
+    state_write<G>(st, stage, lane, qi);
+    __syncwarp();
+    const float4 v = *reinterpret_cast<const float4*>(stage + 4 * lane);
+    const float o[4] = {v.x, v.y, v.z, v.w};
+    finish_query(o, stage[kD + 1], orow + qi * kD, lane, p);
+  }
+  __syncwarp();
+}
+
+template <bool GLOBAL>
+__device__ __forceinline__ float2 ld_rec2(const float* a) {
+  if (GLOBAL) return __ldcg(reinterpret_cast<const float2*>(a));
+  return *reinterpret_cast<const float2*>(a);
+}
+template <bool GLOBAL>
+__device__ __forceinline__ float4 ld_rec4(const float* a) {
+  if (GLOBAL) return __ldcg(reinterpret_cast<const float4*>(a));
+  return *reinterpret_cast<const float4*>(a);
+}
+
+// Merge nrec partial records of one unit (record j: [G][kPartStride] floats at rec(j)) for
+// the queries q0, q0 + QSTEP, ... < G (one warp; lane: channels 4*lane..4*lane+3), then
+// either finish them into orow or, with crec != nullptr, store the merged record there.
+// Records are taken 32 at a time with an online rescale: lane j fetches (m, l) of record j
+// of the chunk for every owned query, in the same round as the o' rows of the chunk's
+// first records (8 float4 per lane a round), so a merge of a few records costs one round
+// trip to L2.
+// GLOBAL: the records were written by other warps or CTAs and are read from L2.
+template <int G, int QSTEP, bool GLOBAL, typename F>
+__device__ __forceinline__ void merge_records(int nrec, F&& rec, int q0, __half* orow, float* crec,
+                                              int lane, const DecodeParams& p) {
+  constexpr int NQW = (G + QSTEP - 1) / QSTEP;       // queries this warp handles (at most)
+  constexpr int R = (8 / NQW) < 1 ? 1 : 8 / NQW;     // records per round of o' loads
+  if (q0 >= G) return;
+  float M[NQW], l[NQW], o[NQW][4];
+#pragma unroll
+  for (int i = 0; i < NQW; i++) {
+    M[i] = -CUDART_INF_F;
+    l[i] = 0.0f;
+    o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+  }
+  for (int base = 0; base < nrec; base += 32) {
+    const bool mine = base + lane < nrec;
+    const float* rj = mine ? rec(base + lane) : nullptr;
+    const int cnt = min(32, nrec - base);
+    // o' rows of records base .. base + R - 1, fetched together with the (m, l) pairs.
+    float4 v[R][NQW];
+    auto fetch = [&](int j0) {
+#pragma unroll
+      for (int r = 0; r < R; r++) {
+        const int j = j0 + r;
+        const float* rr = (j < cnt) ? rec(base + j) : nullptr;
+#pragma unroll
+        for (int i = 0; i < NQW; i++) {
+          const int qi = min(q0 + i * QSTEP, G - 1);
+          v[r][i] = rr ? ld_rec4<GLOBAL>(rr + qi * kPartStride + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    };
+    fetch(0);
+    float e[NQW];
+    float2 ml[NQW];
+#pragma unroll
+    for (int i = 0; i < NQW; i++) {
+      const int qi = min(q0 + i * QSTEP, G - 1);
+      ml[i] = mine ? ld_rec2<GLOBAL>(rj + qi * kPartStride + kD) : make_float2(-CUDART_INF_F, 0.0f);
+    }
+#pragma unroll
+    for (int i = 0; i < NQW; i++) {
+      float mc = ml[i].x;
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) mc = fmaxf(mc, __shfl_xor_sync(kFull, mc, d));
+      const float Mn = fmaxf(M[i], mc);  // finite: every record holds at least one token
+      const float r = (M[i] == -CUDART_INF_F) ? 0.0f : exp2f(M[i] - Mn);
+      M[i] = Mn;
+      l[i] *= r;
+#pragma unroll
+      for (int c = 0; c < 4; c++) o[i][c] *= r;
+      e[i] = (ml[i].x == -CUDART_INF_F) ? 0.0f : exp2f(ml[i].x - Mn);
+      float le = e[i] * ml[i].y;
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) le += __shfl_xor_sync(kFull, le, d);
+      l[i] += le;
+    }
+    for (int j0 = 0; j0 < cnt; j0 += R) {
+      if (j0 > 0) fetch(j0);
+#pragma unroll
+      for (int r = 0; r < R; r++) {
+#pragma unroll
+        for (int i = 0; i < NQW; i++) {
+          const float ej = __shfl_sync(kFull, e[i], (j0 + r) & 31);  // 0 past cnt: v is 0 too
+          o[i][0] += ej * v[r][i].x;
+          o[i][1] += ej * v[r][i].y;
+          o[i][2] += ej * v[r][i].z;
+          o[i][3] += ej * v[r][i].w;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NQW; i++) {
+    const int qi = q0 + i * QSTEP;
+    if (qi >= G) continue;
+    if (crec) {
+      float* r = crec + qi * kPartStride;
+      *reinterpret_cast<float4*>(r + 4 * lane) = make_float4(o[i][0], o[i][1], o[i][2], o[i][3]);
+      if (lane == 0) *reinterpret_cast<float2*>(r + kD) = make_float2(M[i], l[i]);
+    } else {
+      finish_query(o[i], l[i], orow + qi * kD, lane, p);
+    }
+  }
+}
+
+// Per-warp fragment table: G queries x 96 words, at least one staging record.
+constexpr int frag_words(int g) { return g * 96 > kPartStride ? g * 96 : kPartStride; }
+
 template <int G, int SEFF>
 __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
+  constexpr int kFragWords = frag_words(G);
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  // Bulk copies need 16-byte aligned destinations; align the ring to 128 bytes (the
-  // allocation carries 128 spare bytes for this).
+  // Bulk copies need 16-byte aligned destinations; align to 128 bytes (the allocation
+  // carries 128 spare bytes for this).
   uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
-  uint8_t* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kSlotBytes);
-  float* mbuf = reinterpret_cast<float*>(bars + kWarps * kStages);               // [kWarps][G][132]
-  uint32_t* qfb = reinterpret_cast<uint32_t*>(mbuf + kWarps * G * kPartStride);  // [G][3][4][8]
-  float* sfb = reinterpret_cast<float*>(qfb + G * 96);                           // [G]
-  int32_t* pre = reinterpret_cast<int32_t*>(sfb + 8);                            // [batch + 1]
-  int32_t* lens = pre + p.batch + 1;                                             // [batch]
+  uint8_t* ring = smem;                                                      // [w][stage][4224]
+  uint8_t* qraw_all = ring + kWarps * kStages * kSlotBytes;                  // [w][G][128] fp16
+  uint32_t* frag_all = reinterpret_cast<uint32_t*>(qraw_all + kWarps * G * kD * 2);  // [w][kFragWords]
+  float* sf_all = reinterpret_cast<float*>(frag_all + kWarps * kFragWords);    // [w][8]
+  float* mbuf = sf_all + kWarps * 8;                                         // [w][G][132]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(mbuf + kWarps * G * kPartStride);  // [w][kStages+1]
+  int32_t* pre = reinterpret_cast<int32_t*>(bars + kWarps * (kStages + 1));  // [batch + 1]
+  int32_t* lens = pre + p.batch + 1;                                         // [batch]
   __shared__ int warp_sum[kWarps];
   __shared__ int running;
-  __shared__ int last_flag;
+  __shared__ int last_flag_e[2];
 
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int cap = p.max_pages_per_seq * p.page_size;
@@ -670,12 +797,16 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   const int X1 = min(T, X0 + chunk);
   const bool has_tiles = T > 0 && X0 < T;
 
+  uint8_t* qraw = qraw_all + w * G * kD * 2;
+  uint32_t* frag = frag_all + w * kFragWords;
+  float* sf = sf_all + w * 8;
   const uint8_t* ring_p = ring + w * kStages * kSlotBytes;
   const uint32_t ring_s = smem_addr(ring_p);
-  const uint32_t bar_s = smem_addr(bars + w * kStages);
+  const uint32_t bar_s = smem_addr(bars + w * (kStages + 1));
+  const uint32_t qbar = bar_s + 8 * kStages;
   if (lane == 0) {
 #pragma unroll
-    for (int s = 0; s < kStages; s++) mbar_init(bar_s + 8 * s, 1);
+    for (int s = 0; s <= kStages; s++) mbar_init(bar_s + 8 * s, 1);
     fence_mbar_init();
   }
   __syncwarp();
@@ -685,13 +816,36 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   constexpr int kBatch = PageBatch<SEFF>::kBatch;
   Producer<SEFF> pr;
   pr.t = 0;
-  pr.nT = has_tiles ? (X1 - X0 - w + kWarps - 1) / kWarps : 0;
+  pr.nT = has_tiles ? max(0, (X1 - X0 - w + kWarps - 1) / kWarps) : 0;
   pr.tb = 0;
   pr.pid_cur = has_tiles ? load_page_batch<SEFF>(0, X0, X1, w, lane, pre, lens, p) : -1;
   pr.pid_nxt = has_tiles ? load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p) : -1;
   if (pr.nT > 0) unit_of_tile(pr.u, X0 + w, pre, lens, p);
 
+  // This warp's q rows of a unit: one bulk copy into its raw-q buffer, completing on qbar.
+  int q_issued = 0, q_done = 0;  // q copies issued / waited for (one in flight at most)
+  auto q_fetch = [&](const Unit& u) {
+    q_issued++;
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(qbar, G * kD * 2);
+      bulk_copy_g2s(smem_addr(qraw),
+                    p.q + (static_cast<size_t>(u.b) * p.num_kv_heads * G + u.h * G) * kD,
+                    G * kD * 2, qbar, 0ull);
+    }
+    __syncwarp();
+  };
+  int x = X0 + w;
+  Unit cu;
+  if (x < X1) unit_of_tile(cu, x, pre, lens, p);
+
   griddep_wait();
+
+  // q of the first unit goes ahead of the tile copies, so that it is not queued behind
+  // them; then the first kStages tiles.
+  if (x < X1) q_fetch(cu);
+  while (pr.t < pr.nT && pr.t < kStages)
+    producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
 
   // An empty sequence has no tiles: its output rows are zeros (CTAs share the writes).
   const int row_words = p.num_kv_heads * G * kD / 8;  // 16-byte words per sequence
@@ -700,43 +854,52 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       for (int i = tid; i < row_words; i += kThreads)
         reinterpret_cast<uint4*>(p.out + static_cast<size_t>(b) * p.num_kv_heads * G * kD)[i] =
             make_uint4(0u, 0u, 0u, 0u);
-  if (!has_tiles) return;  // the whole CTA: nothing else to do
+  if (!has_tiles) return;  // the whole CTA (no copies were issued): nothing else to do
 
-  // The first kStages tiles.
-  while (pr.t < pr.nT && pr.t < kStages)
-    producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
-
-  // q of the first unit, prepared cooperatively while the first copies fly.
-  Unit cu;
-  unit_of_tile(cu, X0, pre, lens, p);
-  uint2 qraw[2];
-  load_q_coop<G>(qraw, cu, w, lane, p);
-  prep_q<G>(qfb, sfb, qraw, w, lane, p);
-  __syncthreads();
+  // The units of the CTA's range: the first (uf) and the last (ul) may be shared with
+  // other CTAs; the units between them lie wholly inside the range.  A warp's partial of uf
+  // goes to its part of the merge buffer and its partial of ul (always its last segment,
+  // when its ring has drained) to its ring's first slot; partials of the units between go
+  // to the warp's global slot.  All of them are merged at the CTA's end.
+  Unit uf, ul;
+  unit_of_tile(uf, X0, pre, lens, p);
+  unit_of_tile(ul, X1 - 1, pre, lens, p);
+  const int unit_f = uf.b * p.num_kv_heads + uf.h;
+  const int unit_l = ul.b * p.num_kv_heads + ul.h;
+  auto out_row = [&](int b, int h) {
+    return p.out + (static_cast<size_t>(b) * p.num_kv_heads * G + h * G) * kD;
+  };
+  auto warp_slot = [&](int unit, int ww) {
+    return p.part + (static_cast<size_t>(unit + kc) * kWarps + ww) * G * kPartStride;
+  };
+  float* const rec_f = mbuf;                             // [kWarps][G][kPartStride]
+  float* const rec_l = reinterpret_cast<float*>(ring);   // warp ww's: + ww*kStages*kSlotBytes
 
   int consumed = 0;   // tiles of this warp consumed (tile t uses slot t % kStages)
   bool dead = false;  // a bounded wait gave up: stop touching the ring
   State<G> st;
+  state_reset<G>(st);
   QFrag<G> qf;
   constexpr int NQ = QFrag<G>::NQ;
-  while (true) {
-    const int ux0 = max(X0, cu.U), ux1 = min(X1, cu.U + cu.n);
-    qfrag_load<G>(qf, qfb, sfb, lane);
+  while (x < X1) {
+    const int seg_end = min(X1, cu.U + cu.n);
+    const int nt = (seg_end - x + kWarps - 1) / kWarps;
+    const int x_next = x + kWarps * nt;
+    const bool has_next = x_next < X1;
     Unit nu = cu;
-    const bool has_next = ux1 < X1;
-    if (has_next) {
-      unit_next(nu, pre, lens, p);
-      load_q_coop<G>(qraw, nu, w, lane, p);  // prefetch the next unit's q
+    if (has_next) unit_of_tile(nu, x_next, pre, lens, p);
+    // q of this unit: rotate and slice into the warp's fragment table; then fetch the
+    // next unit's rows into the freed buffer.
+    if (!dead) {
+      if (mbar_wait_bounded(qbar, static_cast<uint32_t>(q_done & 1), kWaitLimitNs)) q_done++;
+      else dead = true;
     }
+    if (!dead) prep_q_warp<G>(qraw, frag, sf, lane, p);
+    qfrag_load<G>(qf, frag, sf, lane);
+    if (has_next && !dead) q_fetch(nu);
     state_reset<G>(st);
-    // This warp's tiles of the unit: x = first + kWarps*i < ux1.  Pipelined: the QK^T
-    // of the next tile is computed next to the PV of the current one.
-    const int first = ux0 + ((X0 + w - ux0) & (kWarps - 1));
-    const int nt = first < ux1 ? (ux1 - first + kWarps - 1) / kWarps : 0;
-    float sc[2][NQ][2];
-    int slot_i = consumed % kStages;
-    uint32_t parity = static_cast<uint32_t>((consumed / kStages) & 1);
-    auto ntok_of = [&](int x) { return min(kTileTokens, cu.L - (x - cu.U) * kTileTokens); };
+
+    auto ntok_of = [&](int xx) { return min(kTileTokens, cu.L - (xx - cu.U) * kTileTokens); };
     // Release a consumed slot and refill it with the warp's tile kStages ahead.
     auto refill = [&]() {
       __syncwarp();
@@ -745,17 +908,21 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
         producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
       }
     };
-    if (nt > 0 && !dead) {
+    float sc[2][NQ][2];
+    int slot_i = consumed % kStages;
+    uint32_t parity = static_cast<uint32_t>((consumed / kStages) & 1);
+    if (!dead) {
       if (!mbar_wait_bounded(bar_s + 8 * slot_i, parity, kWaitLimitNs)) {
         dead = true;
       } else {
-        tile_qk<G, SEFF>(qf, ring_p + slot_i * kSlotBytes, ntok_of(first), lane, sc);
+        tile_qk<G, SEFF>(qf, ring_p + slot_i * kSlotBytes, ntok_of(x), lane, sc);
         tile_softmax<G>(st, sc);
       }
     }
-    // Steady state: a next tile always exists.
+    // Steady state: a next tile of the unit always exists.  The QK^T of the next tile is
+    // computed next to the PV of the current one.
     for (int i = 0; i + 1 < nt && !dead; i++) {
-      const int x = first + kWarps * i;
+      const int xi = x + kWarps * i;
       const int cur = slot_i;
       const int nslot = cur + 1 == kStages ? 0 : cur + 1;
       const uint32_t npar = cur + 1 == kStages ? parity ^ 1u : parity;
@@ -764,8 +931,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
         break;
       }
       float sn[2][NQ][2];
-      tile_qk<G, SEFF>(qf, ring_p + nslot * kSlotBytes, ntok_of(x + kWarps), lane, sn);
-      tile_pv<G, SEFF>(st, ring_p + cur * kSlotBytes, ntok_of(x), lane, sc);
+      tile_qk<G, SEFF>(qf, ring_p + nslot * kSlotBytes, ntok_of(xi + kWarps), lane, sn);
+      tile_pv<G, SEFF>(st, ring_p + cur * kSlotBytes, ntok_of(xi), lane, sc);
       consumed++;
       slot_i = nslot;
       parity = npar;
@@ -778,95 +945,96 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 #pragma unroll
           for (int r = 0; r < 2; r++) sc[j][qq][r] = sn[j][qq][r];
     }
-    // Last tile of the unit for this warp.
-    if (nt > 0 && !dead) {
-      const int cur = slot_i;
-      tile_pv<G, SEFF>(st, ring_p + cur * kSlotBytes, ntok_of(first + kWarps * (nt - 1)), lane, sc);
+    if (!dead) {  // last tile of the unit for this warp
+      tile_pv<G, SEFF>(st, ring_p + slot_i * kSlotBytes, ntok_of(x + kWarps * (nt - 1)), lane, sc);
       consumed++;
-      slot_i = cur + 1 == kStages ? 0 : cur + 1;
       refill();
     }
     if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
 
-    // Merge the 4 warps' partials of this unit.
-    state_to_smem<G>(st, mbuf, w, lane);
-    __syncthreads();
     const int unit = cu.b * p.num_kv_heads + cu.h;
-    const int k_first = cu.U / chunk, k_last = (cu.U + cu.n - 1) / chunk;
-    const bool alone = k_first == k_last;
-    __half* orow = p.out + (static_cast<size_t>(cu.b) * p.num_kv_heads * G + cu.h * G) * kD;
-    for (int qi = w; qi < G; qi += kWarps) {
-      float M = -CUDART_INF_F;
-#pragma unroll
-      for (int w2 = 0; w2 < kWarps; w2++) M = fmaxf(M, mbuf[(w2 * G + qi) * kPartStride + kD]);
-      float o[4] = {0.0f, 0.0f, 0.0f, 0.0f}, l = 0.0f;
-#pragma unroll
-      for (int w2 = 0; w2 < kWarps; w2++) {
-        const float* rec = mbuf + (w2 * G + qi) * kPartStride;
-        const float mw = rec[kD];
-        const float e = (mw == -CUDART_INF_F) ? 0.0f : exp2f(mw - M);
-        const float4 v = *reinterpret_cast<const float4*>(rec + 4 * lane);
-        o[0] += e * v.x;
-        o[1] += e * v.y;
-        o[2] += e * v.z;
-        o[3] += e * v.w;
-        l += e * rec[kD + 1];
-      }
-      if (alone) {
-        finish_query(o, l, orow + qi * kD, lane, p);
-      } else {
-        float* rec = p.part + (static_cast<size_t>(unit + kc) * G + qi) * kPartStride;
-        *reinterpret_cast<float4*>(rec + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-        if (lane == 0) {
-          rec[kD] = M;
-          rec[kD + 1] = l;
-        }
-      }
+    if (cu.n == 1) {
+      // This warp is the unit's only contributor: finish it now (the fragment table is
+      // free until the next unit's q is prepared).
+      finish_from_state<G>(st, reinterpret_cast<float*>(frag), out_row(cu.b, cu.h), lane, p);
+    } else if (unit == unit_f) {
+      state_write<G>(st, rec_f + w * G * kPartStride, lane);
+    } else if (unit == unit_l) {
+      state_write<G>(st, rec_l + w * (kStages * kSlotBytes / 4), lane);
+    } else {
+      state_write<G>(st, warp_slot(unit, w), lane);
     }
-    if (!alone) {
-      // The last CTA to arrive merges every CTA's partial of the unit (CTAs k_first ..
-      // k_last all hold tiles of it).
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) {
-        const int old = atomicAdd(p.counters + unit, 1);
-        last_flag = (old == k_last - k_first);
-        if (last_flag) p.counters[unit] = 0;  // ready for the next call
-      }
-      __syncthreads();
-      if (last_flag) {
-        __threadfence();
-        for (int qi = w; qi < G; qi += kWarps) {
-          float M = -CUDART_INF_F;
-          for (int k2 = k_first; k2 <= k_last; k2++)
-            M = fmaxf(M, __ldcg(p.part + (static_cast<size_t>(unit + k2) * G + qi) * kPartStride + kD));
-          float o[4] = {0.0f, 0.0f, 0.0f, 0.0f}, l = 0.0f;
-          for (int k2 = k_first; k2 <= k_last; k2++) {
-            const float* rec = p.part + (static_cast<size_t>(unit + k2) * G + qi) * kPartStride;
-            const float e = exp2f(__ldcg(rec + kD) - M);
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(rec + 4 * lane));
-            o[0] += e * v.x;
-            o[1] += e * v.y;
-            o[2] += e * v.z;
-            o[3] += e * v.w;
-            l += e * __ldcg(rec + kD + 1);
-          }
-          finish_query(o, l, orow + qi * kD, lane, p);
-        }
-      }
-    }
-    // Everyone has read this unit's q fragments and merge buffer: prepare the next q.
-    if (has_next) prep_q<G>(qfb, sfb, qraw, w, lane, p);
-    __syncthreads();
-    if (!has_next) break;
+    x = x_next;
     cu = nu;
+  }
+
+  // ---- CTA end: every partial of the range is written (shared or global memory).
+  __syncthreads();
+  // The (one or two) edge units: merge the warps' partials from shared memory, queries
+  // split over the warps.  A unit inside the range is finished here; a shared one leaves
+  // one record per CTA at the CTA's slot (warp slot 0).
+  const int nedge = unit_l == unit_f ? 1 : 2;
+  bool shared_edge[2] = {false, false};
+#pragma unroll
+  for (int e = 0; e < 2; e++) {
+    if (e >= nedge) break;
+    const Unit& u = e == 0 ? uf : ul;
+    const int unit = e == 0 ? unit_f : unit_l;
+    const int a = max(X0, u.U), c = min(X1, u.U + u.n) - a;  // this CTA's tiles of u
+    shared_edge[e] = !(u.U >= X0 && u.U + u.n <= X1);
+    if (u.n == 1) continue;  // already finished by its warp
+    float* base = e == 0 ? rec_f : rec_l;
+    const int wstride = e == 0 ? G * kPartStride : kStages * kSlotBytes / 4;
+    auto rec = [&](int j) -> const float* { return base + ((a - X0 + j) & (kWarps - 1)) * wstride; };
+    merge_records<G, kWarps, false>(min(kWarps, c), rec, w, out_row(u.b, u.h),
+                                    shared_edge[e] ? warp_slot(unit, 0) : nullptr, lane, p);
+  }
+  // Units between the edges (wholly inside the range, at least two tiles): their warps'
+  // records are in global memory; warp w merges every kWarps-th of them.
+  if (nedge == 2) {
+    Unit u = uf;
+    unit_next(u, pre, lens, p);
+    for (int i = 0; !(u.b == ul.b && u.h == ul.h); i++, unit_next(u, pre, lens, p)) {
+      if ((i & (kWarps - 1)) != w || u.n == 1) continue;
+      const int unit = u.b * p.num_kv_heads + u.h;
+      auto rec = [&](int j) -> const float* { return warp_slot(unit, (u.U - X0 + j) & (kWarps - 1)); };
+      merge_records<G, 1, true>(min(kWarps, u.n), rec, 0, out_row(u.b, u.h), nullptr, lane, p);
+    }
+  }
+  // Shared edge units: publish this CTA's record (a CTA barrier, then one acquire-release
+  // arrival per unit); the last of the unit's CTAs merges.
+  if (shared_edge[0] || shared_edge[1]) {
+    __syncthreads();
+    if (lane == 0 && w < nedge && shared_edge[w]) {
+      const Unit& u = w == 0 ? uf : ul;
+      const int unit = w == 0 ? unit_f : unit_l;
+      const int ncta = (u.U + u.n - 1) / chunk - u.U / chunk + 1;
+      const int old = atom_add_acq_rel_gpu(p.counters + unit, 1);
+      const int last = old == ncta - 1;
+      if (last) p.counters[unit] = 0;  // ready for the next call
+      last_flag_e[w] = last;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+      if (e >= nedge || !shared_edge[e] || !last_flag_e[e]) continue;
+      const Unit& u = e == 0 ? uf : ul;
+      const int unit = e == 0 ? unit_f : unit_l;
+      const int k0 = u.U / chunk, ncta = (u.U + u.n - 1) / chunk - k0 + 1;
+      auto rec = [&](int j) -> const float* {
+        return p.part + (static_cast<size_t>(unit + k0 + j) * kWarps) * G * kPartStride;
+      };
+      merge_records<G, kWarps, true>(ncta, rec, w, out_row(u.b, u.h), nullptr, lane, p);
+    }
   }
 
   if (dead) {
     // Let copies still in flight land before the CTA's shared memory is released.
-    for (int j = consumed + 1; j < pr.t; j++)
+    for (int j = consumed; j < pr.t; j++)
       mbar_wait_bounded(bar_s + 8 * (j % kStages), static_cast<uint32_t>((j / kStages) & 1),
                         kWaitLimitNs);
+    for (; q_done < q_issued; q_done++)
+      mbar_wait_bounded(qbar, static_cast<uint32_t>(q_done & 1), kWaitLimitNs);
   }
 }
 
@@ -890,12 +1058,14 @@ void* pick_kernel(int group, int seff) {
 }
 
 size_t smem_bytes(int group, int max_batch) {
-  size_t s = static_cast<size_t>(kWarps) * kStages * kSlotBytes;
-  s += sizeof(uint64_t) * kWarps * kStages;
-  s += sizeof(float) * kWarps * group * kPartStride;
-  s += sizeof(uint32_t) * group * 96 + sizeof(float) * 8;  // q fragment table, M factors
-  s += static_cast<size_t>(2 * max_batch + 1) * sizeof(int32_t);  // prefix, lengths
-  s += 128;  // alignment slack for the ring base
+  size_t s = static_cast<size_t>(kWarps) * kStages * kSlotBytes;      // rings
+  s += static_cast<size_t>(kWarps) * group * kD * 2;                 // raw q rows
+  s += sizeof(uint32_t) * kWarps * frag_words(group);                // q fragment tables
+  s += sizeof(float) * kWarps * 8;                                   // M factors
+  s += sizeof(float) * kWarps * group * kPartStride;                 // CTA merge buffer
+  s += sizeof(uint64_t) * kWarps * (kStages + 1);                    // mbarriers
+  s += static_cast<size_t>(2 * max_batch + 1) * sizeof(int32_t);     // prefix, lengths
+  s += 128;                                                          // alignment slack
   return (s + 15) & ~static_cast<size_t>(15);
 }
 

@@ -152,11 +152,11 @@ int kvq_alloc_pages(const kvq_desc* d, void* dev_pool, size_t pool_bytes, int32_
     return KVQ_ECUDA;
   }
   // Scratch: status word (padded to 256 B), one arrival counter per unit (zero between
-  // calls; the decode kernel resets what it uses), and the per-(unit, CTA) partials
-  // [(max_batch * Hkv + grid) * G * kPartStride] fp32.
+  // calls; the decode kernel resets what it uses), and the per-(unit, CTA, warp) partials
+  // [(max_batch * Hkv + grid) * kDecodeWarps * G * kPartStride] fp32.
   const size_t units = static_cast<size_t>(d->max_batch) * d->num_kv_heads;
   const size_t counter_bytes = (units * 4 + 255) & ~size_t(255);
-  const size_t slots = units + static_cast<size_t>(c->launch.grid);
+  const size_t slots = (units + static_cast<size_t>(c->launch.grid)) * kvq::kDecodeWarps;
   const size_t part_bytes = slots * g * kvq::kPartStride * sizeof(float);
   if (cudaMalloc(&c->scratch, 256 + counter_bytes + part_bytes) != cudaSuccess) {
     delete c;

@@ -33,6 +33,8 @@ struct AppendParams {
 constexpr int kTileTokens = 32;
 // fp32 words per (partial, query) record in the split scratch: o'[128], m, l, 2 pad.
 constexpr int kPartStride = 132;
+// Warps per decode CTA; each (unit, CTA) partial slot holds one record per warp.
+constexpr int kDecodeWarps = 4;
 
 struct DecodeParams {
   const uint8_t* pool_layer;      // block(0, 0) of the layer

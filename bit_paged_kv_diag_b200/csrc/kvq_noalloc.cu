@@ -23,9 +23,10 @@ constexpr int kNoAllocMaxUnits = 4096;    // batch * num_kv_heads
 constexpr int kNoAllocMaxRecords = 4096;  // (batch * num_kv_heads + grid CTAs) * G
 constexpr size_t kNoAllocCounterBytes = kNoAllocMaxUnits * sizeof(int32_t);
 constexpr size_t kNoAllocBytes =
-    256 + kNoAllocCounterBytes + static_cast<size_t>(kNoAllocMaxRecords) * kvq::kPartStride * sizeof(float);
+    256 + kNoAllocCounterBytes + static_cast<size_t>(kNoAllocMaxRecords) * kvq::kDecodeWarps *
+                                     kvq::kPartStride * sizeof(float);
 
-// Every GPU that loads the library holds this array (about 2.2 MB) until exit.
+// Every GPU that loads the library holds this array (about 8.7 MB) until exit.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 constexpr int kMaxDevices = 64;

@@ -78,6 +78,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Device-scope fetch-and-add with acquire-release semantics: the caller's earlier writes
+// (and, after a CTA barrier, those of its CTA) are visible to whoever observes the new
+// value, and writes released by earlier arrivals are visible to the caller.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing bytes on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.  No multicast.
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes,

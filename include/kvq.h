@@ -179,7 +179,7 @@ KVQ_API int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, con
  * cudaMalloc's implicit device synchronisation is not acceptable.  Those callers cannot
  * create a kvq_cache (kvq_alloc_pages allocates the split scratch), so this call takes the
  * geometry and the pool directly and keeps its scratch in one fixed-size device array
- * inside the library (about 2.2 MB, held by every GPU that loads the library until exit).
+ * inside the library (about 8.7 MB, held by every GPU that loads the library until exit).
  *   d              cache geometry (as for kvq_alloc_pages); only read
  *   pool           device pool of kvq_pool_bytes(d) bytes, 16-byte aligned, laid out as
  *                  kvq_rotate_quant_append writes it (caller-owned)
