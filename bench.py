@@ -284,7 +284,7 @@ def run_kvq(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: 2.5 GB cache per step vs 126 MB L2",
                    "graph": "one CUDA graph per step"},
-        "gpu_launches": args.steps * NL * 3,
+        "gpu_launches": args.steps * NL * 2,  # per layer: one append, one decode launch
         "device_status": status,
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
