@@ -108,81 +108,94 @@ __device__ __forceinline__ void unit_next(Unit& u, const int32_t* pre, const int
 }
 
 // ------------------------------------------------------------------- copies --
-// Page ids of a warp's upcoming tiles, one per lane: a batch covers kBatch tiles of
+// Page entries of a warp's upcoming tiles, one per lane: a batch covers kBatch tiles of
 // kPPT pages (tile t of the warp = CTA tile X0 + w + kWarps*t).  Entry lane: tile
-// tb + lane / kPPT, page lane % kPPT of the tile; -1 where no page is needed.
+// tb + lane / kPPT, page lane % kPPT of the tile, as the address of that (page, head)
+// block with flags in its low 4 bits (blocks are 16-byte aligned): bits 0-2 = the
+// tile's first token in the page / 32 (pages of 64+ tokens), bit 3 = the page id was out
+// of range (page 0 is read instead and the status word is flagged at issue); 0 where no
+// page is needed.
 template <int SEFF>
 struct PageBatch {
   static constexpr int kPPT = (SEFF < kTileTokens) ? kTileTokens / SEFF : 1;
   static constexpr int kBatch = 32 / kPPT;
 };
 
+constexpr uint64_t kEntryBad = 8u;
+
 template <int SEFF>
-__device__ __forceinline__ int load_page_batch(int tb, int X0, int X1, int w, int lane,
-                                               const int32_t* pre, const int32_t* lens,
-                                               const DecodeParams& p) {
+__device__ __forceinline__ uint64_t load_page_batch(int tb, int X0, int X1, int w, int lane,
+                                                    const int32_t* pre, const int32_t* lens,
+                                                    const DecodeParams& p) {
   constexpr int kPPT = PageBatch<SEFF>::kPPT;
   const int x = X0 + w + kWarps * (tb + lane / kPPT);
-  int pid = -1;
+  uint64_t e = 0;
   if (x < X1) {
     Unit u;
     unit_of_tile(u, x, pre, lens, p);
     const int t0 = (x - u.U) * kTileTokens;
     const int lp = (t0 >> p.page_shift) + lane % kPPT;
-    if ((lp << p.page_shift) < u.L)
-      pid = __ldg(p.page_table + static_cast<size_t>(u.b) * p.max_pages_per_seq + lp);
+    if ((lp << p.page_shift) < u.L) {
+      int pid = __ldg(p.page_table + static_cast<size_t>(u.b) * p.max_pages_per_seq + lp);
+      uint64_t flags = 0;
+      if (pid < 0 || pid >= p.num_pages) {
+        pid = 0;
+        flags = kEntryBad;
+      }
+      const size_t blk_bytes = static_cast<size_t>(p.page_size) * (kD + 4);
+      e = reinterpret_cast<uint64_t>(p.pool_layer +
+                                     (static_cast<size_t>(pid) * p.num_kv_heads + u.h) * blk_bytes);
+      if (SEFF == kTileTokens) e |= static_cast<uint64_t>((t0 & (p.page_size - 1)) / kTileTokens);
+      e |= flags;
+    }
   }
-  return pid;
+  return e;
 }
 
-// Issue the bulk copies of tile k of unit u into a ring slot (the whole warp calls; lane
-// j < pages-needed holds that page's id).  The slot holds a virtual page of SEFF =
-// min(S, 32) token slots per copied page, [K codes][V codes][K scales][V scales], the
-// pool's own block layout.
+// Issue the bulk copies of one tile into a ring slot (the whole warp calls; lane j <
+// kPPT holds the tile's page entry j).  The slot holds a virtual page of SEFF = min(S, 32)
+// token slots per copied page, [K codes][V codes][K scales][V scales], the pool's own
+// block layout.
 template <int SEFF>
-__device__ __forceinline__ void tile_issue(const Unit& u, int k, int pid, uint32_t slot,
-                                           uint32_t bar, int lane, uint64_t pol,
-                                           const DecodeParams& p) {
-  const int S = p.page_size, sh = p.page_shift;
-  const uint32_t blk_bytes = static_cast<uint32_t>(S) * (kD + 4);
-  const int t0 = k * kTileTokens;
-  int npg = 1;
-  uint32_t total = kSlotBytes;
-  if (SEFF < kTileTokens) {
-    npg = ((min(t0 + kTileTokens, u.L) - 1) >> sh) - (t0 >> sh) + 1;
-    total = npg * blk_bytes;
-  }
-  const bool bad = lane < npg && (pid < 0 || pid >= p.num_pages);
-  if (__any_sync(kFull, bad) && lane == 0) atomicOr(p.status, KVQ_DEV_BAD_PAGE_BIT);
-  if (bad) pid = 0;  // keep the barrier's byte count; the status word flags the result
-  if (lane == 0) mbar_arrive_expect_tx(bar, total);
-  __syncwarp();
+__device__ __forceinline__ void tile_issue(uint64_t e, uint32_t slot, uint32_t bar, int lane,
+                                           uint64_t pol, const DecodeParams& p) {
+  constexpr int kPPT = PageBatch<SEFF>::kPPT;
+  const bool have = lane < kPPT && e != 0;
+  if (__any_sync(kFull, have && (e & kEntryBad)) && lane == 0) atomicOr(p.status, KVQ_DEV_BAD_PAGE_BIT);
+  const int S = p.page_size;
   if (SEFF < kTileTokens || S == kTileTokens) {
-    if (lane < npg)
-      bulk_copy_g2s(slot + lane * blk_bytes,
-                    p.pool_layer + (static_cast<size_t>(pid) * p.num_kv_heads + u.h) * blk_bytes,
-                    blk_bytes, bar, pol);
+    const uint8_t* blk = reinterpret_cast<const uint8_t*>(e & ~static_cast<uint64_t>(15));
+    const uint32_t blk_bytes = static_cast<uint32_t>(S) * (kD + 4);
+    const int npg = __popc(__ballot_sync(kFull, have));
+    if (lane == 0) mbar_arrive_expect_tx(bar, npg * blk_bytes);
+    __syncwarp();
+    if (have) bulk_copy_g2s(slot + lane * blk_bytes, blk, blk_bytes, bar, pol);
   } else {
-    const int pid0 = __shfl_sync(kFull, pid, 0);
-    const size_t o = static_cast<size_t>(t0 & (S - 1));  // first token of the tile in the page
-    const uint8_t* blk = p.pool_layer + (static_cast<size_t>(pid0) * p.num_kv_heads + u.h) * blk_bytes;
-    if (lane == 0) bulk_copy_g2s(slot, blk + o * 64, 2048, bar, pol);
-    if (lane == 1) bulk_copy_g2s(slot + 2048, blk + static_cast<size_t>(S) * 64 + o * 64, 2048, bar, pol);
-    if (lane == 2) bulk_copy_g2s(slot + 4096, blk + static_cast<size_t>(S) * 128 + o * 2, 64, bar, pol);
-    if (lane == 3) bulk_copy_g2s(slot + 4160, blk + static_cast<size_t>(S) * 130 + o * 2, 64, bar, pol);
+    // One page per tile; lanes 0-3 copy its K codes, V codes, K scales and V scales.
+    const uint64_t e0 = __shfl_sync(kFull, e, 0);
+    const uint8_t* blk = reinterpret_cast<const uint8_t*>(e0 & ~static_cast<uint64_t>(15));
+    const size_t o = static_cast<size_t>(e0 & 7u) * kTileTokens;  // tile's first token in the page
+    const uint8_t* src = blk + o * 64;
+    uint32_t dst = slot, bytes = 2048;
+    if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + 2048; }
+    if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 2; dst = slot + 4096; bytes = 64; }
+    if (lane == 3) { src = blk + static_cast<size_t>(S) * 130 + o * 2; dst = slot + 4160; bytes = 64; }
+    if (lane == 0) mbar_arrive_expect_tx(bar, kSlotBytes);
+    __syncwarp();
+    if (lane < 4) bulk_copy_g2s(dst, src, bytes, bar, pol);
   }
 }
 
 // A warp's producer: issues its tiles t = 0, 1, ... (CTA tile X0 + w + kWarps*t) in
-// order into its ring, slot t % kStages; page ids come from prefetched batches.
+// order into its ring, slot t % kStages; page entries come from batches loaded one
+// batch ahead.
 template <int SEFF>
 struct Producer {
-  int t;        // next tile to issue
-  int nT;       // tiles of this warp
-  Unit u;       // unit of tile t
-  int tb;       // first tile of the current page-id batch
-  int pid_cur;  // this lane's entry of the current batch
-  int pid_nxt;  // ... of the next batch (loaded one batch ahead)
+  int t;         // next tile to issue
+  int nT;        // tiles of this warp
+  int tb;        // first tile of the current batch
+  uint64_t cur;  // this lane's entry of the current batch
+  uint64_t nxt;  // ... of the next batch
 };
 
 template <int SEFF>
@@ -193,15 +206,13 @@ __device__ __forceinline__ void producer_issue(Producer<SEFF>& pr, int X0, int X
   constexpr int kPPT = PageBatch<SEFF>::kPPT, kBatch = PageBatch<SEFF>::kBatch;
   if (pr.t >= pr.tb + kBatch) {
     pr.tb += kBatch;
-    pr.pid_cur = pr.pid_nxt;
-    pr.pid_nxt = load_page_batch<SEFF>(pr.tb + kBatch, X0, X1, w, lane, pre, lens, p);
+    pr.cur = pr.nxt;
+    pr.nxt = load_page_batch<SEFF>(pr.tb + kBatch, X0, X1, w, lane, pre, lens, p);
   }
-  const int x = X0 + w + kWarps * pr.t;
-  while (x >= pr.u.U + pr.u.n && pr.u.b < p.batch) unit_next(pr.u, pre, lens, p);
   const int src = (pr.t - pr.tb) * kPPT + lane;
-  const int pid = __shfl_sync(kFull, pr.pid_cur, src < 32 ? src : 31);
+  const uint64_t e = __shfl_sync(kFull, pr.cur, src & 31);
   const int s = pr.t % kStages;
-  tile_issue<SEFF>(pr.u, x - pr.u.U, pid, ring_s + s * kSlotBytes, bar_s + 8 * s, lane, pol, p);
+  tile_issue<SEFF>(e, ring_s + s * kSlotBytes, bar_s + 8 * s, lane, pol, p);
   pr.t++;
 }
 
@@ -224,19 +235,23 @@ struct QFrag {
 // (1 for a zero row).  qraw: the unit's G fp16 rows in shared memory; the slices go to the
 // warp's fragment table in fragment order:
 //   frag word ((qi*3 + s)*4 + c)*8 + 2*jj + half, byte e  <->  channel 32c + 8jj + 2e + half.
-template <int G>
+// The warp prepares queries q0, q0 + QSTEP, ... < G (all of them for QSTEP = 1; a
+// quarter each when the CTA's warps share one unit's rows).
+template <int G, int QSTEP>
 __device__ __forceinline__ void prep_q_warp(const uint8_t* qraw, uint32_t* frag, float* sf, int lane,
-                                            const DecodeParams& p) {
+                                            const DecodeParams& p, int q0 = 0) {
   // Up to four queries at a time: their shuffle chains are independent and interleave.
-  constexpr int QB = G < 4 ? G : 4;
+  constexpr int NQW = (G + QSTEP - 1) / QSTEP;
+  constexpr int QB = NQW < 4 ? NQW : 4;
   const int c = lane >> 3, jj = (lane >> 1) & 3, e0 = (2 * lane) & 3;
   uint8_t* base = reinterpret_cast<uint8_t*>(frag);
 #pragma unroll 1
-  for (int q0 = 0; q0 < G; q0 += QB) {
+  for (int qb = q0; qb < G; qb += QB * QSTEP) {
     float x[QB][4];
 #pragma unroll
     for (int b = 0; b < QB; b++) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(qraw + (q0 + b) * kD * 2 + 8 * lane);
+      const int qi = min(qb + b * QSTEP, G - 1);  // a clamped duplicate is computed, not stored
+      const uint2 raw = *reinterpret_cast<const uint2*>(qraw + qi * kD * 2 + 8 * lane);
       const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
       const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
       float t0 = lo.x, t1 = lo.y, t2 = hi.x, t3 = hi.y;
@@ -295,7 +310,8 @@ __device__ __forceinline__ void prep_q_warp(const uint8_t* qraw, uint32_t* frag,
       }
       // Channels 4*lane + i: c = lane/8, jj = (lane/2)%4, half = i%2, byte e0 + i/2 with
       // e0 = (2*lane)%4: a 2-byte store per (slice, half).
-      const int qi = q0 + b;
+      const int qi = qb + b * QSTEP;
+      if (qi >= G) continue;
 #pragma unroll
       for (int sl = 0; sl < 3; sl++) {
         const int word = ((qi * 3 + sl) * 4 + c) * 8 + 2 * jj;
@@ -443,7 +459,7 @@ __device__ __forceinline__ void tile_softmax(State<G>& st, float (&sc)[2][QFrag<
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
     const float mnew = fmaxf(st.m[qq], mx);
-    alpha[qq] = exp2f(st.m[qq] - mnew);
+    alpha[qq] = ex2_approx(st.m[qq] - mnew);
     rescale |= alpha[qq] != 1.0f;
     st.m[qq] = mnew;
     float ps = 0.0f;
@@ -451,7 +467,7 @@ __device__ __forceinline__ void tile_softmax(State<G>& st, float (&sc)[2][QFrag<
     for (int j = 0; j < 2; j++)
 #pragma unroll
       for (int r = 0; r < 2; r++) {
-        sc[j][qq][r] = exp2f(sc[j][qq][r] - mnew);
+        sc[j][qq][r] = ex2_approx(sc[j][qq][r] - mnew);
         ps += sc[j][qq][r];
       }
     st.l[qq] = st.l[qq] * alpha[qq] + ps;
@@ -466,6 +482,15 @@ __device__ __forceinline__ void tile_softmax(State<G>& st, float (&sc)[2][QFrag<
       st.o[i][3] *= alpha[NQ - 1];
     }
   }
+}
+
+// (p0, p1) -> fp16 pairs hi = rn(p), lo = rn(p - hi): p carried to about 2^-22.
+__device__ __forceinline__ void split_hi_lo(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(p0, p1);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(p0 - f.x, p1 - f.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // PV of the tile with probabilities pr.  B fragment of thread (g, c): tokens c, c+4 (b0)
@@ -494,10 +519,7 @@ __device__ __forceinline__ void tile_pv(State<G>& st, const uint8_t* slot, int n
 #pragma unroll
       for (int qq = 0; qq < 2; qq++) {
         const float p0 = v0 ? pr[j][qq][0] * sv0 : 0.0f, p1 = v1 ? pr[j][qq][1] * sv1 : 0.0f;
-        const __half h0 = __float2half_rn(p0), h1 = __float2half_rn(p1);
-        xh[qq] = pack_half2(h0, h1);
-        xl[qq] = pack_half2(__float2half_rn(p0 - __half2float(h0)),
-                            __float2half_rn(p1 - __half2float(h1)));
+        split_hi_lo(p0, p1, xh[qq], xl[qq]);
       }
       // Column g = query g, owned by lane group c' = g/2 as its query (g & 1).
       const uint32_t aE = __shfl_sync(kFull, xh[0], srcA), aO = __shfl_sync(kFull, xh[1], srcA);
@@ -510,10 +532,8 @@ __device__ __forceinline__ void tile_pv(State<G>& st, const uint8_t* slot, int n
       bl1 = (g & 1) ? eO : eE;
     } else {
       const float p0 = v0 ? pr[j][0][0] * sv0 : 0.0f, p1 = v1 ? pr[j][0][1] * sv1 : 0.0f;
-      const __half h0 = __float2half_rn(p0), h1 = __float2half_rn(p1);
-      const uint32_t xh = pack_half2(h0, h1);
-      const uint32_t xl = pack_half2(__float2half_rn(p0 - __half2float(h0)),
-                                     __float2half_rn(p1 - __half2float(h1)));
+      uint32_t xh, xl;
+      split_hi_lo(p0, p1, xh, xl);
       // Column g = 2q + part holds query q's hi (part 0) or lo (part 1) part.
       const uint32_t aH = __shfl_sync(kFull, xh, srcA), aL = __shfl_sync(kFull, xl, srcA);
       const uint32_t cH = __shfl_sync(kFull, xh, srcB), cL = __shfl_sync(kFull, xl, srcB);
@@ -741,12 +761,14 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   // carries 128 spare bytes for this).
   uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
   uint8_t* ring = smem;                                                      // [w][stage][4224]
-  uint8_t* qraw_all = ring + kWarps * kStages * kSlotBytes;                  // [w][G][128] fp16
-  uint32_t* frag_all = reinterpret_cast<uint32_t*>(qraw_all + kWarps * G * kD * 2);  // [w][kFragWords]
-  float* sf_all = reinterpret_cast<float*>(frag_all + kWarps * kFragWords);    // [w][8]
-  float* mbuf = sf_all + kWarps * 8;                                         // [w][G][132]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(mbuf + kWarps * G * kPartStride);  // [w][kStages+1]
-  int32_t* pre = reinterpret_cast<int32_t*>(bars + kWarps * (kStages + 1));  // [batch + 1]
+  // Per warp (index w) and one more for the CTA (index kWarps): raw q rows, fragment
+  // table, M factors.
+  uint8_t* qraw_all = ring + kWarps * kStages * kSlotBytes;                  // [w+1][G][128] fp16
+  uint32_t* frag_all = reinterpret_cast<uint32_t*>(qraw_all + (kWarps + 1) * G * kD * 2);  // [w+1][kFragWords]
+  float* sf_all = reinterpret_cast<float*>(frag_all + (kWarps + 1) * kFragWords);  // [w+1][8]
+  float* mbuf = sf_all + (kWarps + 1) * 8;                                   // [w][G][132]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(mbuf + kWarps * G * kPartStride);  // [w][kStages+1], CTA q
+  int32_t* pre = reinterpret_cast<int32_t*>(bars + kWarps * (kStages + 1) + 1);  // [batch + 1]
   int32_t* lens = pre + p.batch + 1;                                         // [batch]
   __shared__ int warp_sum[kWarps];
   __shared__ int running;
@@ -758,6 +780,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   // library writes; everything an earlier kernel may write or read (pool, q, out, the
   // scratch) is touched only after griddep_wait().
   griddep_launch_dependents();
+
+  const uint32_t qbar_cta = smem_addr(bars + kWarps * (kStages + 1));
+  if (tid == 0) {
+    mbar_init(qbar_cta, 1);
+    fence_mbar_init();
+  }
 
   // Clamped lengths, and tiles per sequence -> exclusive prefix pre[0..batch].
   if (tid == 0) running = 0;
@@ -818,9 +846,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   pr.t = 0;
   pr.nT = has_tiles ? max(0, (X1 - X0 - w + kWarps - 1) / kWarps) : 0;
   pr.tb = 0;
-  pr.pid_cur = has_tiles ? load_page_batch<SEFF>(0, X0, X1, w, lane, pre, lens, p) : -1;
-  pr.pid_nxt = has_tiles ? load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p) : -1;
-  if (pr.nT > 0) unit_of_tile(pr.u, X0 + w, pre, lens, p);
+  pr.cur = has_tiles ? load_page_batch<SEFF>(0, X0, X1, w, lane, pre, lens, p) : 0;
+  pr.nxt = has_tiles ? load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p) : 0;
 
   // This warp's q rows of a unit: one bulk copy into its raw-q buffer, completing on qbar.
   int q_issued = 0, q_done = 0;  // q copies issued / waited for (one in flight at most)
@@ -835,15 +862,30 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     }
     __syncwarp();
   };
+  // The units of the CTA's range: the first (uf) and the last (ul) may be shared with
+  // other CTAs; the units between them lie wholly inside the range.
+  Unit uf, ul;
+  if (has_tiles) {
+    unit_of_tile(uf, X0, pre, lens, p);
+    unit_of_tile(ul, X1 - 1, pre, lens, p);
+  }
   int x = X0 + w;
   Unit cu;
   if (x < X1) unit_of_tile(cu, x, pre, lens, p);
+  // Warps whose first unit is uf share one copy of its q rows, prepared by all warps.
+  const bool first_uf = x < X1 && cu.b == uf.b && cu.h == uf.h;
 
   griddep_wait();
 
-  // q of the first unit goes ahead of the tile copies, so that it is not queued behind
-  // them; then the first kStages tiles.
-  if (x < X1) q_fetch(cu);
+  // q goes ahead of the tile copies, so that it is not queued behind them; then the first
+  // kStages tiles.
+  if (has_tiles && tid == 0) {
+    mbar_arrive_expect_tx(qbar_cta, G * kD * 2);
+    bulk_copy_g2s(smem_addr(qraw_all + kWarps * G * kD * 2),
+                  p.q + (static_cast<size_t>(uf.b) * p.num_kv_heads * G + uf.h * G) * kD,
+                  G * kD * 2, qbar_cta, 0ull);
+  }
+  if (x < X1 && !first_uf) q_fetch(cu);
   while (pr.t < pr.nT && pr.t < kStages)
     producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
 
@@ -856,14 +898,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
             make_uint4(0u, 0u, 0u, 0u);
   if (!has_tiles) return;  // the whole CTA (no copies were issued): nothing else to do
 
-  // The units of the CTA's range: the first (uf) and the last (ul) may be shared with
-  // other CTAs; the units between them lie wholly inside the range.  A warp's partial of uf
-  // goes to its part of the merge buffer and its partial of ul (always its last segment,
-  // when its ring has drained) to its ring's first slot; partials of the units between go
-  // to the warp's global slot.  All of them are merged at the CTA's end.
-  Unit uf, ul;
-  unit_of_tile(uf, X0, pre, lens, p);
-  unit_of_tile(ul, X1 - 1, pre, lens, p);
+  // A warp's partial of uf goes to its part of the merge buffer and its partial of ul
+  // (always its last segment, when its ring has drained) to its ring's first slot;
+  // partials of the units between go to the warp's global slot.  All of them are merged
+  // at the CTA's end.
   const int unit_f = uf.b * p.num_kv_heads + uf.h;
   const int unit_l = ul.b * p.num_kv_heads + ul.h;
   auto out_row = [&](int b, int h) {
@@ -877,6 +915,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 
   int consumed = 0;   // tiles of this warp consumed (tile t uses slot t % kStages)
   bool dead = false;  // a bounded wait gave up: stop touching the ring
+  // uf's q rows: every warp rotates and slices its share of the queries.
+  if (!mbar_wait_bounded(qbar_cta, 0u, kWaitLimitNs)) dead = true;
+  if (!dead)
+    prep_q_warp<G, kWarps>(qraw_all + kWarps * G * kD * 2, frag_all + kWarps * kFragWords,
+                           sf_all + kWarps * 8, lane, p, w);
+  if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
+  __syncthreads();
   State<G> st;
   state_reset<G>(st);
   QFrag<G> qf;
@@ -890,12 +935,16 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     if (has_next) unit_of_tile(nu, x_next, pre, lens, p);
     // q of this unit: rotate and slice into the warp's fragment table; then fetch the
     // next unit's rows into the freed buffer.
-    if (!dead) {
-      if (mbar_wait_bounded(qbar, static_cast<uint32_t>(q_done & 1), kWaitLimitNs)) q_done++;
-      else dead = true;
+    if (first_uf && x == X0 + w) {
+      qfrag_load<G>(qf, frag_all + kWarps * kFragWords, sf_all + kWarps * 8, lane);
+    } else {
+      if (!dead) {
+        if (mbar_wait_bounded(qbar, static_cast<uint32_t>(q_done & 1), kWaitLimitNs)) q_done++;
+        else dead = true;
+      }
+      if (!dead) prep_q_warp<G, 1>(qraw, frag, sf, lane, p);
+      qfrag_load<G>(qf, frag, sf, lane);
     }
-    if (!dead) prep_q_warp<G>(qraw, frag, sf, lane, p);
-    qfrag_load<G>(qf, frag, sf, lane);
     if (has_next && !dead) q_fetch(nu);
     state_reset<G>(st);
 
@@ -1035,6 +1084,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
                         kWaitLimitNs);
     for (; q_done < q_issued; q_done++)
       mbar_wait_bounded(qbar, static_cast<uint32_t>(q_done & 1), kWaitLimitNs);
+    mbar_wait_bounded(qbar_cta, 0u, kWaitLimitNs);
   }
 }
 
@@ -1059,11 +1109,11 @@ void* pick_kernel(int group, int seff) {
 
 size_t smem_bytes(int group, int max_batch) {
   size_t s = static_cast<size_t>(kWarps) * kStages * kSlotBytes;      // rings
-  s += static_cast<size_t>(kWarps) * group * kD * 2;                 // raw q rows
-  s += sizeof(uint32_t) * kWarps * frag_words(group);                // q fragment tables
-  s += sizeof(float) * kWarps * 8;                                   // M factors
+  s += static_cast<size_t>(kWarps + 1) * group * kD * 2;             // raw q rows
+  s += sizeof(uint32_t) * (kWarps + 1) * frag_words(group);          // q fragment tables
+  s += sizeof(float) * (kWarps + 1) * 8;                             // M factors
   s += sizeof(float) * kWarps * group * kPartStride;                 // CTA merge buffer
-  s += sizeof(uint64_t) * kWarps * (kStages + 1);                    // mbarriers
+  s += sizeof(uint64_t) * (kWarps * (kStages + 1) + 1);              // mbarriers
   s += static_cast<size_t>(2 * max_batch + 1) * sizeof(int32_t);     // prefix, lengths
   s += 128;                                                          // alignment slack
   return (s + 15) & ~static_cast<size_t>(15);

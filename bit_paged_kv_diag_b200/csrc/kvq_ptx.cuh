@@ -87,6 +87,14 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* addr, int v) {
   return old;
 }
 
+// 2^x with the hardware approximation (relative error about 2^-22; subnormal results
+// flush to zero, -inf gives +0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing bytes on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.  No multicast.
 __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes,
