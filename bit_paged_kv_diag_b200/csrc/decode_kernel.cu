@@ -207,7 +207,7 @@ __device__ __forceinline__ void producer_issue(Producer<SEFF>& pr, int X0, int X
   if (pr.t >= pr.tb + kBatch) {
     pr.tb += kBatch;
     pr.cur = pr.nxt;
-    pr.nxt = load_page_batch<SEFF>(pr.tb + kBatch, X0, X1, w, lane, pre, lens, p);
+    pr.nxt = pr.tb + kBatch < pr.nT ? load_page_batch<SEFF>(pr.tb + kBatch, X0, X1, w, lane, pre, lens, p) : 0;
   }
   const int src = (pr.t - pr.tb) * kPPT + lane;
   const uint64_t e = __shfl_sync(kFull, pr.cur, src & 31);
@@ -446,11 +446,14 @@ __device__ __forceinline__ void tile_qk(const QFrag<G>& qf, const uint8_t* slot,
   }
 }
 
-// Online softmax update with the tile's scores; sc becomes p = exp2(score - m).
+// Online softmax update with the tile's scores, in two parts.  The statistics part moves
+// m and l to the tile's frame and turns sc into p = exp2(score - m); it leaves the o'
+// accumulators alone, so it can run next to the previous tile's PV.  The rescale part
+// then brings o' to the new frame (alpha = exp2(m_old - m_new)).
 template <int G>
-__device__ __forceinline__ void tile_softmax(State<G>& st, float (&sc)[2][QFrag<G>::NQ][2]) {
+__device__ __forceinline__ bool tile_softmax_stats(State<G>& st, float (&sc)[2][QFrag<G>::NQ][2],
+                                                   float (&alpha)[QFrag<G>::NQ]) {
   constexpr int NQ = State<G>::NQ;
-  float alpha[NQ];
   bool rescale = false;
 #pragma unroll
   for (int qq = 0; qq < NQ; qq++) {
@@ -472,15 +475,19 @@ __device__ __forceinline__ void tile_softmax(State<G>& st, float (&sc)[2][QFrag<
       }
     st.l[qq] = st.l[qq] * alpha[qq] + ps;
   }
-  if (__any_sync(kFull, rescale)) {
+  return __any_sync(kFull, rescale);
+}
+
+template <int G>
+__device__ __forceinline__ void tile_rescale(State<G>& st, const float (&alpha)[QFrag<G>::NQ]) {
+  constexpr int NQ = State<G>::NQ;
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-      // G <= 4: columns 2c, 2c+1 are query c's hi and lo parts; G == 8: queries 2c, 2c+1.
-      st.o[i][0] *= alpha[0];
-      st.o[i][2] *= alpha[0];
-      st.o[i][1] *= alpha[NQ - 1];
-      st.o[i][3] *= alpha[NQ - 1];
-    }
+  for (int i = 0; i < 8; i++) {
+    // G <= 4: columns 2c, 2c+1 are query c's hi and lo parts; G == 8: queries 2c, 2c+1.
+    st.o[i][0] *= alpha[0];
+    st.o[i][2] *= alpha[0];
+    st.o[i][1] *= alpha[NQ - 1];
+    st.o[i][3] *= alpha[NQ - 1];
   }
 }
 
@@ -761,12 +768,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   // carries 128 spare bytes for this).
   uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
   uint8_t* ring = smem;                                                      // [w][stage][4224]
-  // Per warp (index w) and one more for the CTA (index kWarps): raw q rows, fragment
-  // table, M factors.
-  uint8_t* qraw_all = ring + kWarps * kStages * kSlotBytes;                  // [w+1][G][128] fp16
-  uint32_t* frag_all = reinterpret_cast<uint32_t*>(qraw_all + (kWarps + 1) * G * kD * 2);  // [w+1][kFragWords]
-  float* sf_all = reinterpret_cast<float*>(frag_all + (kWarps + 1) * kFragWords);  // [w+1][8]
-  float* mbuf = sf_all + (kWarps + 1) * 8;                                   // [w][G][132]
+  // Per warp (index w) and two more for the CTA's first and last unit (indices kWarps,
+  // kWarps + 1): raw q rows, fragment table, M factors.
+  constexpr int kQT = kWarps + 2;
+  uint8_t* qraw_all = ring + kWarps * kStages * kSlotBytes;                  // [kQT][G][128] fp16
+  uint32_t* frag_all = reinterpret_cast<uint32_t*>(qraw_all + kQT * G * kD * 2);  // [kQT][kFragWords]
+  float* sf_all = reinterpret_cast<float*>(frag_all + kQT * kFragWords);     // [kQT][8]
+  float* mbuf = sf_all + kQT * 8;                                            // [w][G][132]
   uint64_t* bars = reinterpret_cast<uint64_t*>(mbuf + kWarps * G * kPartStride);  // [w][kStages+1], CTA q
   int32_t* pre = reinterpret_cast<int32_t*>(bars + kWarps * (kStages + 1) + 1);  // [batch + 1]
   int32_t* lens = pre + p.batch + 1;                                         // [batch]
@@ -847,7 +855,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   pr.nT = has_tiles ? max(0, (X1 - X0 - w + kWarps - 1) / kWarps) : 0;
   pr.tb = 0;
   pr.cur = has_tiles ? load_page_batch<SEFF>(0, X0, X1, w, lane, pre, lens, p) : 0;
-  pr.nxt = has_tiles ? load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p) : 0;
+  pr.nxt = pr.nT > kBatch ? load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p) : 0;
 
   // This warp's q rows of a unit: one bulk copy into its raw-q buffer, completing on qbar.
   int q_issued = 0, q_done = 0;  // q copies issued / waited for (one in flight at most)
@@ -872,20 +880,27 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   int x = X0 + w;
   Unit cu;
   if (x < X1) unit_of_tile(cu, x, pre, lens, p);
-  // Warps whose first unit is uf share one copy of its q rows, prepared by all warps.
-  const bool first_uf = x < X1 && cu.b == uf.b && cu.h == uf.h;
+  // uf and ul have one copy of their q rows each, prepared by all warps together; only
+  // units between them are prepared by the warp that walks them.
+  auto is_uf = [&](const Unit& u) { return u.b == uf.b && u.h == uf.h; };
+  auto is_ul = [&](const Unit& u) { return u.b == ul.b && u.h == ul.h; };
+  const bool two_edges = has_tiles && !is_uf(ul);
 
   griddep_wait();
 
   // q goes ahead of the tile copies, so that it is not queued behind them; then the first
   // kStages tiles.
   if (has_tiles && tid == 0) {
-    mbar_arrive_expect_tx(qbar_cta, G * kD * 2);
+    mbar_arrive_expect_tx(qbar_cta, (two_edges ? 2 : 1) * G * kD * 2);
     bulk_copy_g2s(smem_addr(qraw_all + kWarps * G * kD * 2),
                   p.q + (static_cast<size_t>(uf.b) * p.num_kv_heads * G + uf.h * G) * kD,
                   G * kD * 2, qbar_cta, 0ull);
+    if (two_edges)
+      bulk_copy_g2s(smem_addr(qraw_all + (kWarps + 1) * G * kD * 2),
+                    p.q + (static_cast<size_t>(ul.b) * p.num_kv_heads * G + ul.h * G) * kD,
+                    G * kD * 2, qbar_cta, 0ull);
   }
-  if (x < X1 && !first_uf) q_fetch(cu);
+  if (x < X1 && !is_uf(cu) && !is_ul(cu)) q_fetch(cu);
   while (pr.t < pr.nT && pr.t < kStages)
     producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
 
@@ -915,11 +930,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 
   int consumed = 0;   // tiles of this warp consumed (tile t uses slot t % kStages)
   bool dead = false;  // a bounded wait gave up: stop touching the ring
-  // uf's q rows: every warp rotates and slices its share of the queries.
+  // uf's and ul's q rows: every warp rotates and slices its share of the queries.
   if (!mbar_wait_bounded(qbar_cta, 0u, kWaitLimitNs)) dead = true;
   if (!dead)
-    prep_q_warp<G, kWarps>(qraw_all + kWarps * G * kD * 2, frag_all + kWarps * kFragWords,
-                           sf_all + kWarps * 8, lane, p, w);
+    for (int t = 0; t < (two_edges ? 2 : 1); t++)
+      prep_q_warp<G, kWarps>(qraw_all + (kWarps + t) * G * kD * 2, frag_all + (kWarps + t) * kFragWords,
+                             sf_all + (kWarps + t) * 8, lane, p, w);
   if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
   __syncthreads();
   State<G> st;
@@ -935,8 +951,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     if (has_next) unit_of_tile(nu, x_next, pre, lens, p);
     // q of this unit: rotate and slice into the warp's fragment table; then fetch the
     // next unit's rows into the freed buffer.
-    if (first_uf && x == X0 + w) {
-      qfrag_load<G>(qf, frag_all + kWarps * kFragWords, sf_all + kWarps * 8, lane);
+    const int table = is_uf(cu) ? kWarps : (is_ul(cu) ? kWarps + 1 : -1);
+    if (table >= 0) {
+      qfrag_load<G>(qf, frag_all + table * kFragWords, sf_all + table * 8, lane);
     } else {
       if (!dead) {
         if (mbar_wait_bounded(qbar, static_cast<uint32_t>(q_done & 1), kWaitLimitNs)) q_done++;
@@ -945,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       if (!dead) prep_q_warp<G, 1>(qraw, frag, sf, lane, p);
       qfrag_load<G>(qf, frag, sf, lane);
     }
-    if (has_next && !dead) q_fetch(nu);
+    if (has_next && !dead && !is_ul(nu)) q_fetch(nu);
     state_reset<G>(st);
 
     auto ntok_of = [&](int xx) { return min(kTileTokens, cu.L - (xx - cu.U) * kTileTokens); };
@@ -965,11 +982,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
         dead = true;
       } else {
         tile_qk<G, SEFF>(qf, ring_p + slot_i * kSlotBytes, ntok_of(x), lane, sc);
-        tile_softmax<G>(st, sc);
+        float alpha[NQ];
+        if (tile_softmax_stats<G>(st, sc, alpha)) tile_rescale<G>(st, alpha);
       }
     }
-    // Steady state: a next tile of the unit always exists.  The QK^T of the next tile is
-    // computed next to the PV of the current one.
+    // Steady state: a next tile of the unit always exists.  The QK^T and softmax statistics
+    // of the next tile are computed next to the PV of the current one; only the rescale
+    // of o' has to follow that PV.
     for (int i = 0; i + 1 < nt && !dead; i++) {
       const int xi = x + kWarps * i;
       const int cur = slot_i;
@@ -979,14 +998,15 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
         dead = true;
         break;
       }
-      float sn[2][NQ][2];
+      float sn[2][NQ][2], alpha[NQ];
       tile_qk<G, SEFF>(qf, ring_p + nslot * kSlotBytes, ntok_of(xi + kWarps), lane, sn);
+      const bool rescale = tile_softmax_stats<G>(st, sn, alpha);
       tile_pv<G, SEFF>(st, ring_p + cur * kSlotBytes, ntok_of(xi), lane, sc);
       consumed++;
       slot_i = nslot;
       parity = npar;
       refill();
-      tile_softmax<G>(st, sn);
+      if (rescale) tile_rescale<G>(st, alpha);
 #pragma unroll
       for (int j = 0; j < 2; j++)
 #pragma unroll
@@ -1109,9 +1129,9 @@ void* pick_kernel(int group, int seff) {
 
 size_t smem_bytes(int group, int max_batch) {
   size_t s = static_cast<size_t>(kWarps) * kStages * kSlotBytes;      // rings
-  s += static_cast<size_t>(kWarps + 1) * group * kD * 2;             // raw q rows
-  s += sizeof(uint32_t) * (kWarps + 1) * frag_words(group);          // q fragment tables
-  s += sizeof(float) * (kWarps + 1) * 8;                             // M factors
+  s += static_cast<size_t>(kWarps + 2) * group * kD * 2;             // raw q rows
+  s += sizeof(uint32_t) * (kWarps + 2) * frag_words(group);          // q fragment tables
+  s += sizeof(float) * (kWarps + 2) * 8;                             // M factors
   s += sizeof(float) * kWarps * group * kPartStride;                 // CTA merge buffer
   s += sizeof(uint64_t) * (kWarps * (kStages + 1) + 1);              // mbarriers
   s += static_cast<size_t>(2 * max_batch + 1) * sizeof(int32_t);     // prefix, lengths
