@@ -611,8 +611,9 @@ __device__ __forceinline__ void state_write(const State<G>& st, float* rec, int 
 __device__ __forceinline__ void finish_query(const float (&o)[4], float l, __half* dst, int lane,
                                              const DecodeParams& p) {
   float x[4];
+  const float rl = __frcp_rn(l);
 #pragma unroll
-  for (int e = 0; e < 4; e++) x[e] = __fdiv_rn(o[e], l);
+  for (int e = 0; e < 4; e++) x[e] = o[e] * rl;
   const int block = p.hadamard_block;
   float a, c;
   a = x[0]; c = x[1]; x[0] = a + c; x[1] = a - c;
@@ -662,6 +663,50 @@ template <bool GLOBAL>
 __device__ __forceinline__ float4 ld_rec4(const float* a) {
   if (GLOBAL) return __ldcg(reinterpret_cast<const float4*>(a));
   return *reinterpret_cast<const float4*>(a);
+}
+
+// Merge of at most RMAX records (the common case: a unit's CTAs or a CTA's warps): every
+// lane loads the (m, l) pairs and its o' slice of all records at once (the (m, l) loads
+// are broadcasts), so a query costs one round trip and no cross-lane reduction.  Same
+// contract as merge_records below.
+template <int G, int QSTEP, bool GLOBAL, int RMAX, typename F>
+__device__ __forceinline__ void merge_few(int nrec, F&& rec, int q0, __half* orow, float* crec,
+                                          int lane, const DecodeParams& p) {
+#pragma unroll 1
+  for (int qi = q0; qi < G; qi += QSTEP) {
+    float2 ml[RMAX];
+    float4 v[RMAX];
+#pragma unroll
+    for (int r = 0; r < RMAX; r++) {
+      ml[r] = make_float2(-CUDART_INF_F, 0.0f);
+      v[r] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (r < nrec) {
+        const float* rr = rec(r) + qi * kPartStride;
+        ml[r] = ld_rec2<GLOBAL>(rr + kD);
+        v[r] = ld_rec4<GLOBAL>(rr + 4 * lane);
+      }
+    }
+    float M = ml[0].x;
+#pragma unroll
+    for (int r = 1; r < RMAX; r++) M = fmaxf(M, ml[r].x);
+    float o[4] = {0.0f, 0.0f, 0.0f, 0.0f}, l = 0.0f;
+#pragma unroll
+    for (int r = 0; r < RMAX; r++) {
+      const float e = (ml[r].x == -CUDART_INF_F) ? 0.0f : ex2_approx(ml[r].x - M);
+      l += e * ml[r].y;
+      o[0] += e * v[r].x;
+      o[1] += e * v[r].y;
+      o[2] += e * v[r].z;
+      o[3] += e * v[r].w;
+    }
+    if (crec) {
+      float* r = crec + qi * kPartStride;
+      *reinterpret_cast<float4*>(r + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+      if (lane == 0) *reinterpret_cast<float2*>(r + kD) = make_float2(M, l);
+    } else {
+      finish_query(o, l, orow + qi * kD, lane, p);
+    }
+  }
 }
 
 // Merge nrec partial records of one unit (record j: [G][kPartStride] floats at rec(j)) for
@@ -1055,8 +1100,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     float* base = e == 0 ? rec_f : rec_l;
     const int wstride = e == 0 ? G * kPartStride : kStages * kSlotBytes / 4;
     auto rec = [&](int j) -> const float* { return base + ((a - X0 + j) & (kWarps - 1)) * wstride; };
-    merge_records<G, kWarps, false>(min(kWarps, c), rec, w, out_row(u.b, u.h),
-                                    shared_edge[e] ? warp_slot(unit, 0) : nullptr, lane, p);
+    merge_few<G, kWarps, false, kWarps>(min(kWarps, c), rec, w, out_row(u.b, u.h),
+                                        shared_edge[e] ? warp_slot(unit, 0) : nullptr, lane, p);
   }
   // Units between the edges (wholly inside the range, at least two tiles): their warps'
   // records are in global memory; warp w merges every kWarps-th of them.
@@ -1067,7 +1112,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       if ((i & (kWarps - 1)) != w || u.n == 1) continue;
       const int unit = u.b * p.num_kv_heads + u.h;
       auto rec = [&](int j) -> const float* { return warp_slot(unit, (u.U - X0 + j) & (kWarps - 1)); };
-      merge_records<G, 1, true>(min(kWarps, u.n), rec, 0, out_row(u.b, u.h), nullptr, lane, p);
+      merge_few<G, 1, true, kWarps>(min(kWarps, u.n), rec, 0, out_row(u.b, u.h), nullptr, lane, p);
     }
   }
   // Shared edge units: publish this CTA's record (a CTA barrier, then one acquire-release
@@ -1093,7 +1138,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       auto rec = [&](int j) -> const float* {
         return p.part + (static_cast<size_t>(unit + k0 + j) * kWarps) * G * kPartStride;
       };
-      merge_records<G, kWarps, true>(ncta, rec, w, out_row(u.b, u.h), nullptr, lane, p);
+      if (ncta <= 8)
+        merge_few<G, kWarps, true, 8>(ncta, rec, w, out_row(u.b, u.h), nullptr, lane, p);
+      else
+        merge_records<G, kWarps, true>(ncta, rec, w, out_row(u.b, u.h), nullptr, lane, p);
     }
   }
 
