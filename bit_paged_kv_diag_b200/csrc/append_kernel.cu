@@ -79,10 +79,29 @@ __device__ __forceinline__ void mul2(float& x0, float& x1, float s) {
       : "f"(s));
 }
 
-// x[16j + e] = channel 16(2j + l) + e.
+// x[16j + e] = channel 16(2j + l) + e.  b = 1 (plain INT4): the transform of size 1 is
+// the identity and c_b = 1, so the row is only converted.
+template <int BLOCK>
+__device__ __forceinline__ void load_plain(const __half* row, int l, float (&x)[64]) {
+  u32x8 raw[4];
+#pragma unroll
+  for (int j = 0; j < 4; j++) raw[j] = ldg_256_stream(row + 16 * (2 * j + l));
+#pragma unroll
+  for (int j = 0; j < 4; j++)
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+      x[16 * j + 2 * w] = cvt_f16(static_cast<uint16_t>(raw[j].w[w] & 0xffffu));
+      x[16 * j + 2 * w + 1] = cvt_f16(static_cast<uint16_t>(raw[j].w[w] >> 16));
+    }
+}
+
 template <int BLOCK>
 __device__ __forceinline__ void load_rotate(const __half* row, int l, unsigned pmask, float cb,
                                             float (&x)[64]) {
+  if constexpr (BLOCK == 1) {
+    load_plain<BLOCK>(row, l, x);
+    return;
+  } else {
   u32x8 raw[4];
 #pragma unroll
   for (int j = 0; j < 4; j++) raw[j] = ldg_256_stream(row + 16 * (2 * j + l));
@@ -136,6 +155,7 @@ __device__ __forceinline__ void load_rotate(const __half* row, int l, unsigned p
   }
 #pragma unroll
   for (int i = 0; i < 64; i += 2) mul2(x[i], x[i + 1], cb);
+  }
 }
 
 // Codes of 8 channels from their magic-rounded sums (low nibble = code & 0xF).
@@ -273,6 +293,7 @@ int launch_append(const AppendParams& p, int block, cudaStream_t stream) {
   cfg.numAttrs = 1;
   cudaError_t e;
   switch (block) {
+    case 1: e = cudaLaunchKernelEx(&cfg, append_kernel<1>, p); break;
     case 32: e = cudaLaunchKernelEx(&cfg, append_kernel<32>, p); break;
     case 64: e = cudaLaunchKernelEx(&cfg, append_kernel<64>, p); break;
     case 128: e = cudaLaunchKernelEx(&cfg, append_kernel<128>, p); break;

@@ -254,13 +254,14 @@ __device__ __forceinline__ void prep_q_warp(const uint8_t* qraw, uint32_t* frag,
       const uint2 raw = *reinterpret_cast<const uint2*>(qraw + qi * kD * 2 + 8 * lane);
       const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
       const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      float t0 = lo.x, t1 = lo.y, t2 = hi.x, t3 = hi.y;
+      const float t0 = lo.x, t1 = lo.y, t2 = hi.x, t3 = hi.y;
       const float a0 = __fadd_rn(t0, t1), a1 = __fsub_rn(t0, t1);
       const float a2 = __fadd_rn(t2, t3), a3 = __fsub_rn(t2, t3);
-      x[b][0] = __fadd_rn(a0, a2);
-      x[b][2] = __fsub_rn(a0, a2);
-      x[b][1] = __fadd_rn(a1, a3);
-      x[b][3] = __fsub_rn(a1, a3);
+      const bool rot = p.hadamard_block > 1;  // b = 1 (plain INT4): no rotation
+      x[b][0] = rot ? __fadd_rn(a0, a2) : t0;
+      x[b][2] = rot ? __fsub_rn(a0, a2) : t2;
+      x[b][1] = rot ? __fadd_rn(a1, a3) : t1;
+      x[b][3] = rot ? __fsub_rn(a1, a3) : t3;
     }
 #pragma unroll
     for (int s = 0; s < 5; s++) {
@@ -615,11 +616,14 @@ __device__ __forceinline__ void finish_query(const float (&o)[4], float l, __hal
 #pragma unroll
   for (int e = 0; e < 4; e++) x[e] = o[e] * rl;
   const int block = p.hadamard_block;
-  float a, c;
-  a = x[0]; c = x[1]; x[0] = a + c; x[1] = a - c;
-  a = x[2]; c = x[3]; x[2] = a + c; x[3] = a - c;
-  a = x[0]; c = x[2]; x[0] = a + c; x[2] = a - c;
-  a = x[1]; c = x[3]; x[1] = a + c; x[3] = a - c;
+  {
+    const bool rot = block > 1;  // b = 1 (plain INT4): no rotation
+    const float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
+    x[0] = rot ? a0 + a2 : x[0];
+    x[1] = rot ? a1 + a3 : x[1];
+    x[2] = rot ? a0 - a2 : x[2];
+    x[3] = rot ? a1 - a3 : x[3];
+  }
 #pragma unroll
   for (int s = 0; s < 5; s++) {
     if ((4 << s) < block) {

@@ -63,7 +63,8 @@ bool noalloc_desc_ok(const kvq_desc* d) {
   const int g = d->num_q_heads / d->num_kv_heads;
   if (g != 1 && g != 2 && g != 4 && g != 8) return false;
   if (d->head_dim != 128) return false;
-  if (d->hadamard_block != 32 && d->hadamard_block != 64 && d->hadamard_block != 128) return false;
+  const int hb = d->hadamard_block;
+  if (hb != 1 && hb != 32 && hb != 64 && hb != 128) return false;  // 1: plain INT4, no rotation
   const int S = d->page_size;
   if (S != 16 && S != 32 && S != 64 && S != 128 && S != 256) return false;
   if (d->max_batch > 4096) return false;

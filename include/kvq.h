@@ -90,7 +90,8 @@ typedef struct kvq_cache kvq_cache; /* opaque, library-owned handle */
  *   num_kv_heads       Hkv                                                    (>= 1)
  *   num_q_heads        Hq, a multiple of Hkv; G = Hq / Hkv must be 1, 2, 4 or 8
  *   head_dim           D; only 128 is implemented
- *   hadamard_block     b: 32, 64 or 128
+ *   hadamard_block     b: 32, 64 or 128; or 1 for plain token-wise INT4 without the
+ *                      rotation (the transform with b = 1 is the identity and c_b = 1)
  *   page_size          S tokens per page: 16, 32, 64, 128 or 256
  *   num_pages          pages per layer in the pool                            (>= 1)
  *   max_batch          largest batch any call will pass                (1 .. 4096)

@@ -44,7 +44,9 @@ def _desc(**kw):
 def test_pool_bytes_and_descriptor_validation():
     d = _desc()
     assert kvq.pool_bytes(d) == 2 * 100 * 8 * 16 * 132
-    for bad in [dict(head_dim=64), dict(hadamard_block=16), dict(page_size=24),
+    assert kvq.pool_bytes(_desc(hadamard_block=1)) == 2 * 100 * 8 * 16 * 132  # plain INT4
+    for bad in [dict(head_dim=64), dict(hadamard_block=16), dict(hadamard_block=2),
+                dict(page_size=24),
                 dict(num_q_heads=24), dict(num_q_heads=48), dict(max_batch=5000),
                 dict(num_layers=0), dict(num_pages=0)]:
         assert kvq.pool_bytes(_desc(**bad)) == 0, bad

@@ -152,6 +152,22 @@ def test_fwht_special_cases(b):
     assert abs(float(y[0]) - np.sqrt(b)) < 1e-6 * np.sqrt(b)
 
 
+def test_block_of_one_is_plain_int4():
+    """b = 1 (the plain token-wise INT4 variant): the transform is the identity (no stage,
+    c_1 = 1), so the appended codes are those of the unrotated row: every code is within
+    s/2 of the raw value and the largest |value| maps to |code| = 7."""
+    assert oracle.hadamard_scale_f32(1) == 1.0
+    x = np.random.default_rng(11).standard_normal(128).astype(np.float32)
+    assert np.array_equal(oracle.fwht_f32(x, 1), x)
+    assert np.array_equal(oracle.fwht_f64(x.astype(np.float64), 1), x.astype(np.float64))
+    x16 = x.astype(np.float16).astype(np.float32)
+    bits, codes = oracle.quant_row(x16)
+    s = float(np.array([bits], np.uint16).view(np.float16)[0])
+    deq = codes.astype(np.float64) * s
+    assert np.all(np.abs(x16 - deq) <= s / 2 + 1e-12)
+    assert abs(int(codes[np.argmax(np.abs(x16))])) == 7
+
+
 # ------------------------------------------------------------ fp16 -----------
 def test_fp16_rounding_matches_numpy():
     """The oracle's float->fp16 is IEEE nearest-even (numpy's independent conversion),

@@ -48,6 +48,22 @@ def test_prefill_append_student_t(block):
     full_parity(make_case(w, [0, 0, 0, 0], [300, 257, 64, 1], block=block))
 
 
+@pytest.mark.parametrize("name,lengths", [
+    ("qwen3_4b_decode", [517, 300, 64, 1, 0, 129, 63, 65]),
+    ("long_context", [1000, 2049, 64, 777]),
+])
+def test_plain_int4_variant(name, lengths):
+    """b = 1: the same kernels without the rotation (plain token-wise INT4)."""
+    w = W[name]
+    r = full_parity(make_case(w, lengths, [1] * len(lengths), block=1))
+    assert r["flips"] == 0
+
+
+def test_plain_int4_prefill_student_t():
+    w = W["prefill_append"]
+    full_parity(make_case(w, [0, 0, 0, 0], [300, 257, 64, 1], block=1))
+
+
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])
 def test_group_and_page_size_grid(group, page_size):
