@@ -272,6 +272,7 @@ def run_kvq(args, rank, world, local_rank):
     del graph
     cache.close()
     append = run_append_bench(dev) if rank == 0 else None
+    plain = run_plain_decode_bench(dev) if rank == 0 else None
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -299,6 +300,7 @@ def run_kvq(args, rank, world, local_rank):
         "us_per_launch_alone": round(iso_ms * 1e3, 3),
         "bytes_per_launch": dec_b, "timing": dec_how}
     line["append"] = append
+    line["plain_int4"] = plain
     line["clocks"] = clk.result
     return line
 
@@ -320,7 +322,8 @@ def _traffic(kernel, alg_bytes):
 
 
 def run_append_bench(dev, reps=20):
-    """Prefill-append stress: 8 x 8192 new tokens through one call, b = 32, 64, 128."""
+    """Prefill-append stress: 8 x 8192 new tokens through one call, b = 32, 64, 128, and
+    b = 1 (the plain INT4 variant, no rotation)."""
     import torch
 
     import bit_paged_kv_diag_b200 as kvq
@@ -335,7 +338,7 @@ def run_append_bench(dev, reps=20):
     z = torch.zeros(B, dtype=torch.int32, device=dev)
     res = {}
     peak, _ = _peaks()
-    for block in w.blocks_sweep:
+    for block in [1] + list(w.blocks_sweep):
         desc = kvq.Desc(1, H, w.num_q_heads, 128, block, S, P, B, mp)
         cache, pt = kvq.alloc_pages(desc, cap, None)
         ptd = torch.from_numpy(pt).to(dev)
@@ -354,8 +357,62 @@ def run_append_bench(dev, reps=20):
                             "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
         assert kvq.get_device_status(cache) == 0
         cache.close()
-    res["workload"] = "prefill_append: 8 x 8192 tokens, 8 KV heads, page 16, Student-t(3)"
+    res["workload"] = ("prefill_append: 8 x 8192 tokens, 8 KV heads, page 16, Student-t(3); "
+                       "b1 = plain INT4 (no rotation)")
     res["traffic"] = _traffic("append", append_bytes(T, H))
+    return res
+
+
+def run_plain_decode_bench(dev, reps=10):
+    """Rotated (b = 128) against plain INT4 (b = 1) decode on the Qwen3-4B-shaped layer
+    shape: a graph of 36 decode calls cycling over 4 layer pools (276 MB > L2), per-launch
+    device time from events around the replays."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    w = workloads.WORKLOADS[WORKLOAD]
+    L = np.asarray(w.context, np.int32)
+    B, H, HQ, S, NL = w.batch, w.num_kv_heads, w.num_q_heads, w.page_size, 4
+    cap = L + 1
+    P = workloads.pool_pages(w, cap)
+    mp = int((cap.max() + S - 1) // S)
+    res = {}
+    for block in (w.block, 1):
+        desc = kvq.Desc(NL, H, HQ, 128, block, S, P, B, mp)
+        cache, pt = kvq.alloc_pages(desc, cap, None)
+        ptd = torch.from_numpy(pt).to(dev)
+        zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+        cu = torch.from_numpy(workloads.cu_seqlens(cap)).to(dev)
+        for layer in range(NL):
+            kp = workloads.kv_rows_torch(w, layer, 0, int(cap.sum()), stream=1, device=dev)
+            vp = workloads.kv_rows_torch(w, layer, 1, int(cap.sum()), stream=1, device=dev)
+            kvq.rotate_quant_append(cache, layer, kp, vp, cu, zeros, ptd)
+            del kp, vp
+        q = torch.stack([workloads.q_rows_torch(w, l, device=dev) for l in range(NL)])
+        out = torch.empty_like(q)
+        lens = torch.from_numpy(cap).to(dev)
+        side = torch.cuda.Stream(device=dev)
+        kvq.decode_attention(cache, 0, q[0], lens, ptd, out=out[0])
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(36):
+                kvq.decode_attention(cache, i % NL, q[i % NL], lens, ptd, out=out[i % NL])
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        res[f"decode_us_b{block}"] = round(a.elapsed_time(b) * 1e3 / (reps * 36), 3)
+        assert kvq.get_device_status(cache) == 0
+        del g
+        cache.close()
+    res["how"] = ("graph of 36 decode calls over 4 layer pools of the qwen3_4b_decode shape, "
+                  "b = 128 (rotated) and b = 1 (plain INT4)")
     return res
 
 

@@ -79,13 +79,15 @@ __device__ __forceinline__ void mul2(float& x0, float& x1, float s) {
       : "f"(s));
 }
 
-// x[16j + e] = channel 16(2j + l) + e.  b = 1 (plain INT4): the transform of size 1 is
-// the identity and c_b = 1, so the row is only converted.
-template <int BLOCK>
-__device__ __forceinline__ void load_plain(const __half* row, int l, float (&x)[64]) {
-  u32x8 raw[4];
+// This lane's half of a row: the 16-channel chunks 2j + l (j = 0..3), 256-bit loads.
+__device__ __forceinline__ void load_row(const __half* row, int l, u32x8 (&raw)[4]) {
 #pragma unroll
   for (int j = 0; j < 4; j++) raw[j] = ldg_256_stream(row + 16 * (2 * j + l));
+}
+
+// x[16j + e] = channel 16(2j + l) + e.  b = 1 (plain INT4): the transform of size 1 is
+// the identity and c_b = 1, so the row is only converted.
+__device__ __forceinline__ void convert_plain(const u32x8 (&raw)[4], float (&x)[64]) {
 #pragma unroll
   for (int j = 0; j < 4; j++)
 #pragma unroll
@@ -96,15 +98,12 @@ __device__ __forceinline__ void load_plain(const __half* row, int l, float (&x)[
 }
 
 template <int BLOCK>
-__device__ __forceinline__ void load_rotate(const __half* row, int l, unsigned pmask, float cb,
-                                            float (&x)[64]) {
+__device__ __forceinline__ void rotate_row(const u32x8 (&raw)[4], int l, unsigned pmask, float cb,
+                                           float (&x)[64]) {
   if constexpr (BLOCK == 1) {
-    load_plain<BLOCK>(row, l, x);
+    convert_plain(raw, x);
     return;
   } else {
-  u32x8 raw[4];
-#pragma unroll
-  for (int j = 0; j < 4; j++) raw[j] = ldg_256_stream(row + 16 * (2 * j + l));
   // Stage h = 1 fused with the conversion: (a, c) -> (a + c, a - c).
 #pragma unroll
   for (int j = 0; j < 4; j++)
@@ -220,68 +219,100 @@ __device__ __forceinline__ uint16_t quantise(const float (&x)[64], unsigned pmas
   return __half_as_ushort(sh);
 }
 
+// The K or V row r of the call: (token, head) pair r / 2, tensor r % 2.
+__device__ __forceinline__ const __half* row_src(const AppendParams& p, long long r) {
+  return ((r & 1) ? p.v : p.k) + static_cast<size_t>(r >> 1) * kD;
+}
+
+// Persistent: CTA i takes row blocks i, i + grid, ...; the loads of a lane's next row are
+// issued before the current row is rotated, quantised and stored, so they are in flight
+// while it computes.
 template <int BLOCK>
-__global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
+__global__ void __launch_bounds__(kThreads, 2) append_kernel(AppendParams p) {
   // The next kernel may start its own prologue; the pool stores below wait for every
   // earlier kernel (griddep_wait), so they never race with a decode still reading.
   griddep_launch_dependents();
   const int l = threadIdx.x & 1;
   // Shuffles never leave the lane pair of a row, so they name only those two lanes.
   const unsigned pmask = 0x3u << (threadIdx.x & 30);
-  const long long row = static_cast<long long>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 1);
   const long long nrows = 2LL * p.total_new_tokens * p.num_kv_heads;
-  if (row >= nrows) return;  // both lanes of a row leave together
-  const long long pair = row >> 1;
-  const int kv = static_cast<int>(row & 1);
-  const int t = static_cast<int>(pair / p.num_kv_heads);
-  const int h = static_cast<int>(pair % p.num_kv_heads);
-
-  float x[64];
-  load_rotate<BLOCK>((kv ? p.v : p.k) + static_cast<size_t>(pair) * kD, l, pmask, p.cb, x);
-
-  // Sequence of token t: the b with cu[b] <= t < cu[b+1] (binary search).
-  int lo = 0, hi = p.batch;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(p.cu_new_tokens + mid) <= t) lo = mid; else hi = mid;
+  const long long nblk = (nrows + kRowsPerBlock - 1) / kRowsPerBlock;
+  const int r_in = threadIdx.x >> 1;
+  long long rb = blockIdx.x;
+  u32x8 raw[4];
+  {
+    const long long row = rb * kRowsPerBlock + r_in;
+    if (row < nrows) load_row(row_src(p, row), l, raw);
   }
-  const int b = lo;
-  const int pos = __ldg(p.seq_lens + b) + (t - __ldg(p.cu_new_tokens + b));
-  const int lp = pos / p.page_size;
-  int page = -1;
-  if (pos >= 0 && lp < p.max_pages_per_seq)
-    page = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + lp);
-  const bool ok = pos >= 0 && lp < p.max_pages_per_seq && page >= 0 && page < p.num_pages;
+  bool waited = false;
+  for (; rb < nblk; rb += gridDim.x) {
+    const long long row = rb * kRowsPerBlock + r_in;
+    const long long row_next = (rb + gridDim.x) * kRowsPerBlock + r_in;
+    u32x8 nxt[4];
+    if (rb + gridDim.x < nblk && row_next < nrows) load_row(row_src(p, row_next), l, nxt);
+    if (row < nrows) {  // both lanes of a row take the same branch
+      const long long pair = row >> 1;
+      const int kv = static_cast<int>(row & 1);
+      const int t = static_cast<int>(pair / p.num_kv_heads);
+      const int h = static_cast<int>(pair % p.num_kv_heads);
 
-  uint32_t q[8];
-  const uint16_t sbits = quantise(x, pmask, q);
-  griddep_wait();
-  if (!ok) {
-    if (l == 0 && kv == 0)
-      atomicOr(p.status, (pos < 0 || lp >= p.max_pages_per_seq) ? KVQ_DEV_BAD_POS_BIT
-                                                                  : KVQ_DEV_BAD_PAGE_BIT);
-    return;
-  }
-  const int S = p.page_size;
-  const int slot = pos - lp * S;
-  uint8_t* blk = p.pool_layer + (static_cast<size_t>(page) * p.num_kv_heads + h) *
-                                    (static_cast<size_t>(S) * (kD + 4));
-  uint8_t* crow = blk + static_cast<size_t>(kv) * S * (kD / 2) + static_cast<size_t>(slot) * (kD / 2);
+      float x[64];
+      rotate_row<BLOCK>(raw, l, pmask, p.cb, x);
+
+      // Sequence of token t: the b with cu[b] <= t < cu[b+1] (binary search).
+      int lo = 0, hi = p.batch;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(p.cu_new_tokens + mid) <= t) lo = mid; else hi = mid;
+      }
+      const int b = lo;
+      const int pos = __ldg(p.seq_lens + b) + (t - __ldg(p.cu_new_tokens + b));
+      const int lp = pos / p.page_size;
+      int page = -1;
+      if (pos >= 0 && lp < p.max_pages_per_seq)
+        page = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + lp);
+      const bool ok = pos >= 0 && lp < p.max_pages_per_seq && page >= 0 && page < p.num_pages;
+
+      uint32_t q[8];
+      const uint16_t sbits = quantise(x, pmask, q);
+      if (!waited) {
+        griddep_wait();
+        waited = true;
+      }
+      if (!ok) {
+        if (l == 0 && kv == 0)
+          atomicOr(p.status, (pos < 0 || lp >= p.max_pages_per_seq) ? KVQ_DEV_BAD_POS_BIT
+                                                                      : KVQ_DEV_BAD_PAGE_BIT);
+      } else {
+        const int S = p.page_size;
+        const int slot = pos - lp * S;
+        uint8_t* blk = p.pool_layer + (static_cast<size_t>(page) * p.num_kv_heads + h) *
+                                          (static_cast<size_t>(S) * (kD + 4));
+        uint8_t* crow =
+            blk + static_cast<size_t>(kv) * S * (kD / 2) + static_cast<size_t>(slot) * (kD / 2);
 #pragma unroll
-  for (int j = 0; j < 4; j++)
-    *reinterpret_cast<uint2*>(crow + 8 * (2 * j + l)) = make_uint2(q[2 * j], q[2 * j + 1]);
-  if (l == 0)
-    *reinterpret_cast<uint16_t*>(blk + static_cast<size_t>(S) * kD + static_cast<size_t>(kv) * S * 2 +
-                                 static_cast<size_t>(slot) * 2) = sbits;
+        for (int j = 0; j < 4; j++)
+          *reinterpret_cast<uint2*>(crow + 8 * (2 * j + l)) = make_uint2(q[2 * j], q[2 * j + 1]);
+        if (l == 0)
+          *reinterpret_cast<uint16_t*>(blk + static_cast<size_t>(S) * kD +
+                                       static_cast<size_t>(kv) * S * 2 + static_cast<size_t>(slot) * 2) =
+              sbits;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; j++) raw[j] = nxt[j];
+  }
 }
 
 }  // namespace
 
-int launch_append(const AppendParams& p, int block, cudaStream_t stream) {
+int launch_append(const AppendParams& p, int block, int num_sms, cudaStream_t stream) {
   const long long nrows = 2LL * p.total_new_tokens * p.num_kv_heads;
   if (nrows == 0) return 0;
-  const long long grid = (nrows + kRowsPerBlock - 1) / kRowsPerBlock;
-  if (grid > 0x7fffffffLL) return -1;
+  const long long nblk = (nrows + kRowsPerBlock - 1) / kRowsPerBlock;
+  if (nblk > 0x7fffffffLL) return -1;
+  // One wave of persistent CTAs (2 per SM), or fewer for a small call.
+  const long long grid = nblk < 2LL * num_sms ? nblk : 2LL * num_sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);

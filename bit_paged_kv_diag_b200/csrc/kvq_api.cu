@@ -218,7 +218,7 @@ int kvq_rotate_quant_append(kvq_cache* c, int32_t layer, const void* k, const vo
   p.page_size = c->d.page_size;
   p.max_pages_per_seq = c->d.max_pages_per_seq;
   p.cb = c->cb;
-  const int rc = kvq::launch_append(p, c->d.hadamard_block, static_cast<cudaStream_t>(stream));
+  const int rc = kvq::launch_append(p, c->d.hadamard_block, c->num_sms, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;
 }

@@ -60,7 +60,7 @@ struct DecodeParams {
 
 // Host-side launchers (return 0 on success, <0 on an unsupported shape or a launch
 // error).
-int launch_append(const AppendParams& p, int block, cudaStream_t stream);
+int launch_append(const AppendParams& p, int block, int num_sms, cudaStream_t stream);
 
 struct DecodeLaunch {
   int grid;          // CTAs (a multiple of the SM count)
