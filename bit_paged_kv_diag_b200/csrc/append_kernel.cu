@@ -21,15 +21,14 @@
 // fp16 -> fp32 conversion rides in the first stage's mixed-precision adds.
 //
 // Quantisation: m = max |y| (lane-pair shuffle), s = fp16_rn(m / 7) (IEEE division, once
-// per row).  Codes are round-half-even of y / s, clamped to [-8, 7].  The fast path
-// multiplies by r = 1/s (IEEE reciprocal, once per row) and rounds with the 1.5 * 2^23
-// magic addend, whose sum carries the integer code in its low mantissa bits.  The
-// product y*r is within 2^-19 of the IEEE quotient y/s for |y/s| < 8, so whenever every
-// fractional part stays more than 2^-19 away from one half, both round to the same
-// integer; otherwise (a near-tie), and whenever s is subnormal or saturated, the lane
-// recomputes its codes with IEEE division -- codes stay bit-exact with division by the
+// per row).  Codes are round-half-even of y / s, clamped to [-8, 7], computed without
+// dividing: a fast multiply-by-reciprocal path, and an exact half-point comparison for
+// groups with a near-tie (see quantise()); codes stay bit-exact with division by the
 // stored fp16 scale.  Codes are packed two per byte (low nibble = even channel) and
 // written with 64-bit stores; lane 0 of the row stores the fp16 scale.
+//
+// The CTAs are persistent (one wave, two per SM): each takes row blocks i, i + grid, ...
+// and issues the loads of its next rows before computing the current ones.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -168,6 +167,17 @@ __device__ __forceinline__ uint32_t pack8_magic(const float (&m)[8]) {
 
 // Quantise this lane's 64 rotated values of a row; q[2j], q[2j+1] = packed codes of
 // chunk j.  Returns the fp16 scale bits (identical on both lanes of the row).
+//
+// Codes are round-half-even of y / s with s the stored fp16 scale.  Fast path (a normal,
+// unsaturated s, so |y/s| <= 7.004): multiply by r = 1/s and round with the magic addend;
+// y*r is within 2^-19 of y/s, so the result is exact unless the fraction is within 2^-19
+// of one half.  A group of 8 values with such a near-tie -- frequent for rows that are
+// not rotated, whose fp16 values meet exact ties -- and every group when s is subnormal
+// or saturated is recomputed exactly without dividing: k = floor(y*r) is within one of
+// the true floor, and (k + 1/2)*s is exact in fp32 (an fp16 scale times a number of 5
+// bits), so comparing y with it chooses between k and k + 1, an exact tie going to the
+// even one.  (If y*r fell on the wrong side of an integer n, y/s is within 2^-16 of n
+// and both candidates' half points place it at n.)  Codes are clamped to [-8, 7].
 __device__ __forceinline__ uint16_t quantise(const float (&x)[64], unsigned pmask,
                                              uint32_t (&q)[8]) {
   float m = 0.0f;
@@ -178,43 +188,45 @@ __device__ __forceinline__ uint16_t quantise(const float (&x)[64], unsigned pmas
   const bool sat = s32 > 65504.0f;
   const __half sh = sat ? __ushort_as_half(0x7BFF) : __float2half_rn(s32);
   const float s = __half2float(sh);
-  // Fast path: s a normal fp16 number and not saturated (then |y/s| <= 7.004).
-  bool exact = !sat && s >= 6.103515625e-05f;
-  if (exact) {
-    const float r = __frcp_rn(s);
-    float dmax = 0.0f;
-#pragma unroll
-    for (int c8 = 0; c8 < 8; c8++) {
-      float mg[8];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        float t0 = x[8 * c8 + e], t1 = x[8 * c8 + e + 1];
-        mul2(t0, t1, r);
-        float m0 = t0, m1 = t1;
-        fma2(m0, m1, 1.0f, kMagic, kMagic);           // t + 1.5*2^23, rounded: rint
-        float r0 = m0, r1 = m1;
-        fma2(r0, r1, 1.0f, -kMagic, -kMagic);         // the integer, exactly
-        float d0 = r0, d1 = r1;
-        fma2(d0, d1, -1.0f, t0, t1);                  // t - rint(t), exactly
-        dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
-        mg[e] = m0;
-        mg[e + 1] = m1;
-      }
-      q[c8] = pack8_magic(mg);
-    }
-    exact = dmax < 0.5f - 0x1p-19f;
-  }
-  if (!exact) {  // near-tie, subnormal or saturated scale, or s == 0
+  if (s == 0.0f) {  // an all-zero row (or a scale that underflows): every code is 0
 #pragma unroll
     for (int w = 0; w < 8; w++) q[w] = 0u;
-    if (s != 0.0f) {
+    return __half_as_ushort(sh);
+  }
+  const bool normal = !sat && s >= 6.103515625e-05f;
+  const float r = __frcp_rn(s);
+  const float hs = 0.5f * s;
 #pragma unroll
-      for (int i = 0; i < 64; i++) {
-        float t = rintf(__fdiv_rn(x[i], s));
-        t = fminf(fmaxf(t, -8.0f), 7.0f);
-        q[i / 8] |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xFu) << (4 * (i % 8));
+  for (int c8 = 0; c8 < 8; c8++) {
+    float mg[8];
+    float dmax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      float t0 = x[8 * c8 + e], t1 = x[8 * c8 + e + 1];
+      mul2(t0, t1, r);
+      float m0 = t0, m1 = t1;
+      fma2(m0, m1, 1.0f, kMagic, kMagic);           // t + 1.5*2^23, rounded: rint
+      float r0 = m0, r1 = m1;
+      fma2(r0, r1, 1.0f, -kMagic, -kMagic);         // the integer, exactly
+      float d0 = r0, d1 = r1;
+      fma2(d0, d1, -1.0f, t0, t1);                  // t - rint(t), exactly
+      dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
+      mg[e] = m0;
+      mg[e + 1] = m1;
+    }
+    if (!normal || !(dmax < 0.5f - 0x1p-19f)) {
+#pragma unroll
+      for (int e = 0; e < 8; e++) {
+        const float y = x[8 * c8 + e];
+        const float k = floorf(__fmul_rn(y, r));
+        const float h = __fmaf_rn(k, s, hs);  // (k + 1/2) * s, exact
+        const bool odd = (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) != 0u;
+        const bool up = y > h || (y == h && odd);
+        const float t = fminf(fmaxf(up ? k + 1.0f : k, -8.0f), 7.0f);
+        mg[e] = __fadd_rn(t, kMagic);
       }
     }
+    q[c8] = pack8_magic(mg);
   }
   return __half_as_ushort(sh);
 }
