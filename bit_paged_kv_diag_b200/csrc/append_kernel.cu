@@ -96,8 +96,10 @@ __device__ __forceinline__ void convert_plain(const u32x8 (&raw)[4], float (&x)[
     }
 }
 
+// The butterfly without its final scale: x = z, the rotated row being y = fl(c_b * z),
+// which quantise() applies where it needs y itself.
 template <int BLOCK>
-__device__ __forceinline__ void rotate_row(const u32x8 (&raw)[4], int l, unsigned pmask, float cb,
+__device__ __forceinline__ void rotate_row(const u32x8 (&raw)[4], int l, unsigned pmask,
                                            float (&x)[64]) {
   if constexpr (BLOCK == 1) {
     convert_plain(raw, x);
@@ -151,8 +153,6 @@ __device__ __forceinline__ void rotate_row(const u32x8 (&raw)[4], int l, unsigne
       for (int e = 0; e < 16; e += 2)
         bfly2(x[16 * j + e], x[16 * j + e + 1], x[16 * (j + 2) + e], x[16 * (j + 2) + e + 1]);
   }
-#pragma unroll
-  for (int i = 0; i < 64; i += 2) mul2(x[i], x[i + 1], cb);
   }
 }
 
@@ -169,21 +169,30 @@ __device__ __forceinline__ uint32_t pack8_magic(const float (&m)[8]) {
 // chunk j.  Returns the fp16 scale bits (identical on both lanes of the row).
 //
 // Codes are round-half-even of y / s with s the stored fp16 scale.  Fast path (a normal,
-// unsaturated s, so |y/s| <= 7.004): multiply by r = 1/s and round with the magic addend;
-// y*r is within 2^-19 of y/s, so the result is exact unless the fraction is within 2^-19
-// of one half.  A group of 8 values with such a near-tie -- frequent for rows that are
+// unsaturated s, so |y/s| <= 7.004): multiply the unscaled butterfly output z by
+// fl(c_b * fl(1/s)) and round with the magic addend; the product is within 2^-19 of y/s,
+// so the result is exact unless the fraction is within 2^-19 of one half.  A group of 8 values with such a near-tie -- frequent for rows that are
 // not rotated, whose fp16 values meet exact ties -- and every group when s is subnormal
 // or saturated is recomputed exactly without dividing: k = floor(y*r) is within one of
 // the true floor, and (k + 1/2)*s is exact in fp32 (an fp16 scale times a number of 5
 // bits), so comparing y with it chooses between k and k + 1, an exact tie going to the
 // even one.  (If y*r fell on the wrong side of an integer n, y/s is within 2^-16 of n
 // and both candidates' half points place it at n.)  Codes are clamped to [-8, 7].
-__device__ __forceinline__ uint16_t quantise(const float (&x)[64], unsigned pmask,
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint16_t quantise(const float (&z)[64], float cb, unsigned pmask,
                                              uint32_t (&q)[8]) {
-  float m = 0.0f;
+  // m = max |y| = fl(c_b * max |z|): rounding is monotonic, so scaling after the max gives
+  // the max of the scaled values.
+  float zmax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 64; i += 2) m = fmaxf(m, fmaxf(fabsf(x[i]), fabsf(x[i + 1])));
-  m = fmaxf(m, __shfl_xor_sync(pmask, m, 1));
+  for (int i = 0; i < 64; i += 2) zmax = max3(zmax, fabsf(z[i]), fabsf(z[i + 1]));
+  zmax = fmaxf(zmax, __shfl_xor_sync(pmask, zmax, 1));
+  const float m = __fmul_rn(cb, zmax);
   const float s32 = __fdiv_rn(m, 7.0f);
   const bool sat = s32 > 65504.0f;
   const __half sh = sat ? __ushort_as_half(0x7BFF) : __float2half_rn(s32);
@@ -195,6 +204,9 @@ __device__ __forceinline__ uint16_t quantise(const float (&x)[64], unsigned pmas
   }
   const bool normal = !sat && s >= 6.103515625e-05f;
   const float r = __frcp_rn(s);
+  // Fast path on z directly: t = z * fl(c_b * r) is within 4 roundings (< 2^-19 for
+  // |y/s| <= 7.004) of y / s.
+  const float rz = __fmul_rn(cb, r);
   const float hs = 0.5f * s;
 #pragma unroll
   for (int c8 = 0; c8 < 8; c8++) {
@@ -202,22 +214,22 @@ __device__ __forceinline__ uint16_t quantise(const float (&x)[64], unsigned pmas
     float dmax = 0.0f;
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
-      float t0 = x[8 * c8 + e], t1 = x[8 * c8 + e + 1];
-      mul2(t0, t1, r);
+      float t0 = z[8 * c8 + e], t1 = z[8 * c8 + e + 1];
+      mul2(t0, t1, rz);
       float m0 = t0, m1 = t1;
       fma2(m0, m1, 1.0f, kMagic, kMagic);           // t + 1.5*2^23, rounded: rint
       float r0 = m0, r1 = m1;
       fma2(r0, r1, 1.0f, -kMagic, -kMagic);         // the integer, exactly
       float d0 = r0, d1 = r1;
       fma2(d0, d1, -1.0f, t0, t1);                  // t - rint(t), exactly
-      dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
+      dmax = max3(dmax, fabsf(d0), fabsf(d1));
       mg[e] = m0;
       mg[e + 1] = m1;
     }
     if (!normal || !(dmax < 0.5f - 0x1p-19f)) {
 #pragma unroll
       for (int e = 0; e < 8; e++) {
-        const float y = x[8 * c8 + e];
+        const float y = __fmul_rn(z[8 * c8 + e], cb);  // the rotated value
         const float k = floorf(__fmul_rn(y, r));
         const float h = __fmaf_rn(k, s, hs);  // (k + 1/2) * s, exact
         const bool odd = (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) != 0u;
@@ -269,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 2) append_kernel(AppendParams p) {
       const int h = static_cast<int>(pair % p.num_kv_heads);
 
       float x[64];
-      rotate_row<BLOCK>(raw, l, pmask, p.cb, x);
+      rotate_row<BLOCK>(raw, l, pmask, x);
 
       // Sequence of token t: the b with cu[b] <= t < cu[b+1] (binary search).
       int lo = 0, hi = p.batch;
@@ -286,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 2) append_kernel(AppendParams p) {
       const bool ok = pos >= 0 && lp < p.max_pages_per_seq && page >= 0 && page < p.num_pages;
 
       uint32_t q[8];
-      const uint16_t sbits = quantise(x, pmask, q);
+      const uint16_t sbits = quantise(x, p.cb, pmask, q);
       if (!waited) {
         griddep_wait();
         waited = true;
