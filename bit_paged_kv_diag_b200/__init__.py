@@ -6,6 +6,7 @@ The names mirror the C ABI in ``include/kvq.h``:
 * ``kvq_alloc_pages``          -> :func:`alloc_pages`
 * ``kvq_rotate_quant_append``  -> :func:`rotate_quant_append`
 * ``kvq_decode_attention``     -> :func:`decode_attention`
+* ``kvq_append_decode_attention`` -> :func:`append_decode_attention`
 * ``kvq_free``                 -> :func:`free`
 * ``kvq_assign_pages``, ``kvq_pool_bytes``, ``kvq_get_device_status`` likewise.
 
@@ -22,7 +23,8 @@ from . import build as _build
 
 __all__ = [
     "KVQError", "Desc", "Cache", "lib", "pool_bytes", "assign_pages", "alloc_pages",
-    "rotate_quant_append", "decode_attention", "decode_attention_noalloc", "free",
+    "rotate_quant_append", "decode_attention", "append_decode_attention",
+    "decode_attention_noalloc", "free",
     "get_device_status", "status_string",
     "EXPORTED",
 ]
@@ -33,7 +35,7 @@ KVQ_DEV_BAD_PAGE, KVQ_DEV_BAD_POS, KVQ_DEV_TIMEOUT = 1, 2, 4
 EXPORTED = (
     "kvq_pool_bytes", "kvq_assign_pages", "kvq_alloc_pages", "kvq_rotate_quant_append",
     "kvq_decode_attention", "kvq_pool_ptr", "kvq_get_device_status", "kvq_free",
-    "kvq_status_string", "kvq_decode_attention_noalloc",
+    "kvq_status_string", "kvq_decode_attention_noalloc", "kvq_append_decode_attention",
 )
 
 
@@ -78,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "kvq_decode_attention_noalloc": (ctypes.c_int, [dp, vp, i32, vp, vp, vp, i32,
                                                             ctypes.c_float, vp, vp]),
+            "kvq_append_decode_attention": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, i32,
+                                                           ctypes.c_float, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -211,6 +215,23 @@ def decode_attention(cache: Cache, layer: int, q, seq_lens, page_table, softmax_
         _dev_ptr(seq_lens, "seq_lens", torch.int32), _dev_ptr(page_table, "page_table", torch.int32),
         batch, float(softmax_scale), _dev_ptr(out, "out", torch.float16), _stream_ptr(stream))
     _check(rc, "kvq_decode_attention")
+    return out
+
+
+def append_decode_attention(cache: Cache, layer: int, k_new, v_new, q, seq_lens, page_table,
+                            softmax_scale=0.0, out=None, stream=None):
+    """One new token per sequence appended at seq_lens[b] (lengths before the append) and
+    decode attention over seq_lens[b] + 1 tokens, in one launch."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    batch = int(seq_lens.shape[0])
+    rc = lib().kvq_append_decode_attention(
+        cache.handle, int(layer), _dev_ptr(k_new, "k_new", torch.float16),
+        _dev_ptr(v_new, "v_new", torch.float16), _dev_ptr(q, "q", torch.float16),
+        _dev_ptr(seq_lens, "seq_lens", torch.int32), _dev_ptr(page_table, "page_table", torch.int32),
+        batch, float(softmax_scale), _dev_ptr(out, "out", torch.float16), _stream_ptr(stream))
+    _check(rc, "kvq_append_decode_attention")
     return out
 
 

@@ -806,10 +806,123 @@ __device__ __forceinline__ void merge_records(int nrec, F&& rec, int q0, __half*
   }
 }
 
+// --------------------------------------------------------- fused append --
+// One new token of one (sequence, KV head): its K or V row rotated and quantised by a
+// warp, bit-identical to the append kernel (the fixed-order butterfly: stages h = 1, 2
+// inside a lane's 4 channels, h = 4..64 across lanes as fma(own, +-1, other), one rounding
+// each; then y = fl(y * c_b); s = fp16(fl(max|y| / 7)); codes = round-half-even of y / s
+// decided exactly by comparing y with (k + 1/2) * s, clamped to [-8, 7]).  Lane L gets the
+// 16 code bits of channels 4L..4L+3 (low nibble = even channel) and the fp16 scale bits.
+struct NewRow {
+  uint32_t codes16;  // this lane's 2 bytes of the packed row
+  uint32_t scale;    // fp16 bits, same in every lane
+};
+
+__device__ __forceinline__ NewRow quantise_new_row(const __half* row, int lane, const DecodeParams& p) {
+  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+  const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+  const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+  float x[4] = {lo.x, lo.y, hi.x, hi.y};
+  if (p.hadamard_block > 1) {
+    const float a0 = __fadd_rn(x[0], x[1]), a1 = __fsub_rn(x[0], x[1]);
+    const float a2 = __fadd_rn(x[2], x[3]), a3 = __fsub_rn(x[2], x[3]);
+    x[0] = __fadd_rn(a0, a2);
+    x[2] = __fsub_rn(a0, a2);
+    x[1] = __fadd_rn(a1, a3);
+    x[3] = __fsub_rn(a1, a3);
+#pragma unroll
+    for (int st = 0; st < 5; st++) {
+      if ((4 << st) < p.hadamard_block) {
+        const float sgn = ((lane >> st) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int e = 0; e < 4; e++) x[e] = __fmaf_rn(x[e], sgn, __shfl_xor_sync(kFull, x[e], 1 << st));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.cb);
+  }
+  float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+  for (int d = 1; d < 32; d *= 2) m = fmaxf(m, __shfl_xor_sync(kFull, m, d));
+  const float s32 = __fdiv_rn(m, 7.0f);
+  const __half sh = s32 > 65504.0f ? __ushort_as_half(0x7BFF) : __float2half_rn(s32);
+  const float s = __half2float(sh);
+  NewRow r;
+  r.scale = __half_as_ushort(sh);
+  r.codes16 = 0u;
+  if (s != 0.0f) {
+    const float rc = __frcp_rn(s), hs = 0.5f * s;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const float k = floorf(__fmul_rn(x[e], rc));
+      const float h = __fmaf_rn(k, s, hs);  // (k + 1/2) * s, exact
+      const bool odd = (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) != 0u;
+      const bool up = x[e] > h || (x[e] == h && odd);
+      const int c = static_cast<int>(fminf(fmaxf(up ? k + 1.0f : k, -8.0f), 7.0f));
+      r.codes16 |= (static_cast<uint32_t>(c) & 0xFu) << (4 * e);
+    }
+  }
+  return r;
+}
+
+// The new token of unit (b, h): rotate and quantise its K and V rows, store them at
+// position seq_lens[b] of the pool (skipped, with the status flagged, when the position or
+// its page is out of range) and, in the block layout of one token, into the warp's patch
+// buffer (shared memory): [K codes 64 B][V codes 64 B][K scale][V scale].  Returns
+// whether the rows are stored and belong in the decode.
+__device__ __forceinline__ bool fused_append(int b, int h, int lane, uint8_t* patch,
+                                             const DecodeParams& p) {
+  const size_t row = (static_cast<size_t>(b) * p.num_kv_heads + h) * kD;
+  const NewRow kr = quantise_new_row(p.k_new + row, lane, p);
+  const NewRow vr = quantise_new_row(p.v_new + row, lane, p);
+  *reinterpret_cast<uint16_t*>(patch + 2 * lane) = static_cast<uint16_t>(kr.codes16);
+  *reinterpret_cast<uint16_t*>(patch + 64 + 2 * lane) = static_cast<uint16_t>(vr.codes16);
+  if (lane == 0) {
+    *reinterpret_cast<uint16_t*>(patch + 128) = static_cast<uint16_t>(kr.scale);
+    *reinterpret_cast<uint16_t*>(patch + 130) = static_cast<uint16_t>(vr.scale);
+  }
+  __syncwarp();
+  const int pos = __ldg(p.seq_lens + b);
+  const int S = p.page_size;
+  const int lp = pos >> p.page_shift;
+  if (pos < 0 || lp >= p.max_pages_per_seq) return false;  // flagged by the length clamp
+  const int page = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + lp);
+  if (page < 0 || page >= p.num_pages) return false;     // flagged when the tile is issued
+  const int slot = pos & (S - 1);
+  uint8_t* blk = const_cast<uint8_t*>(p.pool_layer) + (static_cast<size_t>(page) * p.num_kv_heads + h) *
+                                      (static_cast<size_t>(S) * (kD + 4));
+  *reinterpret_cast<uint16_t*>(blk + slot * 64 + 2 * lane) = static_cast<uint16_t>(kr.codes16);
+  *reinterpret_cast<uint16_t*>(blk + S * 64 + slot * 64 + 2 * lane) = static_cast<uint16_t>(vr.codes16);
+  if (lane == 0) {
+    *reinterpret_cast<uint16_t*>(blk + S * 128 + slot * 2) = static_cast<uint16_t>(kr.scale);
+    *reinterpret_cast<uint16_t*>(blk + S * 130 + slot * 2) = static_cast<uint16_t>(vr.scale);
+  }
+  return true;
+}
+
+// Overwrite token j (0..31, kept at byte 132 of the patch buffer) of a landed ring slot
+// with the patch buffer's token (the slot's copy of the pool may predate the store above).  The warp syncs before the slot
+// is read.
+template <int SEFF>
+__device__ __forceinline__ void patch_slot(uint8_t* slot, int lane, const uint8_t* patch) {
+  const int j = *reinterpret_cast<const int*>(patch + 132);  // the token's place in the tile
+  uint8_t* base = slot + (j / SEFF) * (SEFF * 132);
+  const int jj = j % SEFF;
+  const uint32_t wv = reinterpret_cast<const uint32_t*>(patch)[lane];  // bytes 4*lane..
+  uint8_t* dst = lane < 16 ? base + jj * 64 + 4 * lane : base + SEFF * 64 + jj * 64 + 4 * (lane - 16);
+  *reinterpret_cast<uint32_t*>(dst) = wv;
+  if (lane == 0) {
+    *reinterpret_cast<uint16_t*>(base + SEFF * 128 + jj * 2) = *reinterpret_cast<const uint16_t*>(patch + 128);
+    *reinterpret_cast<uint16_t*>(base + SEFF * 130 + jj * 2) = *reinterpret_cast<const uint16_t*>(patch + 130);
+  }
+  __syncwarp();
+}
+
 // Per-warp fragment table: G queries x 96 words, at least one staging record.
 constexpr int frag_words(int g) { return g * 96 > kPartStride ? g * 96 : kPartStride; }
 
-template <int G, int SEFF>
+// FUSED: the one-token append runs inside (p.k_new, p.v_new set).
+template <int G, int SEFF, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   constexpr int kFragWords = frag_words(G);
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -834,8 +947,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int cap = p.max_pages_per_seq * p.page_size;
   // The prologue below reads only seq_lens and the page table, which no kernel of this
-  // library writes; everything an earlier kernel may write or read (pool, q, out, the
-  // scratch) is touched only after griddep_wait().
+  // library writes (and may OR bits into the status word); everything else an earlier
+  // kernel may write or read (pool, q, new K/V rows, out, the scratch) is touched only
+  // after griddep_wait().
   griddep_launch_dependents();
 
   const uint32_t qbar_cta = smem_addr(bars + kWarps * (kStages + 1));
@@ -851,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     const int i = base + tid;
     int n = 0;
     if (i < p.batch) {
-      const int L = clamp_len(__ldg(p.seq_lens + i), cap, p.status);
+      const int L = clamp_len(__ldg(p.seq_lens + i) + (FUSED ? 1 : 0), cap, p.status);
       lens[i] = L;
       n = (L + kTileTokens - 1) / kTileTokens;
     }
@@ -885,7 +999,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   uint8_t* qraw = qraw_all + w * G * kD * 2;
   uint32_t* frag = frag_all + w * kFragWords;
   float* sf = sf_all + w * 8;
-  const uint8_t* ring_p = ring + w * kStages * kSlotBytes;
+  uint8_t* ring_w = ring + w * kStages * kSlotBytes;
+  const uint8_t* ring_p = ring_w;
   const uint32_t ring_s = smem_addr(ring_p);
   const uint32_t bar_s = smem_addr(bars + w * (kStages + 1));
   const uint32_t qbar = bar_s + 8 * kStages;
@@ -1013,6 +1128,18 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     }
     if (has_next && !dead && !is_ul(nu)) q_fetch(nu);
     state_reset<G>(st);
+    // Fused append: the warp holding the unit's last tile rotates, quantises and stores the
+    // unit's new token, and patches it into that tile's slot once the slot has landed.
+    bool new_ok = false;
+    if constexpr (FUSED) {
+      const int xl = x + kWarps * (nt - 1);  // this warp's last tile of the unit
+      uint8_t* patch = reinterpret_cast<uint8_t*>(frag);  // free until the next unit's q
+      if (xl == cu.U + cu.n - 1 && !dead) {
+        new_ok = fused_append(cu.b, cu.h, lane, patch, p);
+        if (lane == 0) *reinterpret_cast<int*>(patch + 132) = cu.L - 1 - (xl - cu.U) * kTileTokens;
+        __syncwarp();
+      }
+    }
 
     auto ntok_of = [&](int xx) { return min(kTileTokens, cu.L - (xx - cu.U) * kTileTokens); };
     // Release a consumed slot and refill it with the warp's tile kStages ahead.
@@ -1030,6 +1157,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       if (!mbar_wait_bounded(bar_s + 8 * slot_i, parity, kWaitLimitNs)) {
         dead = true;
       } else {
+        if constexpr (FUSED) {
+          if (new_ok && nt == 1)
+            patch_slot<SEFF>(ring_w + slot_i * kSlotBytes, lane, reinterpret_cast<const uint8_t*>(frag));
+        }
         tile_qk<G, SEFF>(qf, ring_p + slot_i * kSlotBytes, ntok_of(x), lane, sc);
         float alpha[NQ];
         if (tile_softmax_stats<G>(st, sc, alpha)) tile_rescale<G>(st, alpha);
@@ -1048,6 +1179,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
         break;
       }
       float sn[2][NQ][2], alpha[NQ];
+      if constexpr (FUSED) {
+        if (new_ok && i + 2 == nt)
+          patch_slot<SEFF>(ring_w + nslot * kSlotBytes, lane, reinterpret_cast<const uint8_t*>(frag));
+      }
       tile_qk<G, SEFF>(qf, ring_p + nslot * kSlotBytes, ntok_of(xi + kWarps), lane, sn);
       const bool rescale = tile_softmax_stats<G>(st, sn, alpha);
       tile_pv<G, SEFF>(st, ring_p + cur * kSlotBytes, ntok_of(xi), lane, sc);
@@ -1161,15 +1296,16 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 }
 
 template <int G, int SEFF>
-void* kernel_ptr() {
-  return reinterpret_cast<void*>(&decode_kernel<G, SEFF>);
+void* kernel_ptr(bool fused) {
+  return fused ? reinterpret_cast<void*>(&decode_kernel<G, SEFF, true>)
+               : reinterpret_cast<void*>(&decode_kernel<G, SEFF, false>);
 }
 
-void* pick_kernel(int group, int seff) {
-#define KVQ_PICK(GG)                               \
-  if (group == GG) {                               \
-    if (seff == 16) return kernel_ptr<GG, 16>();   \
-    if (seff == 32) return kernel_ptr<GG, 32>();   \
+void* pick_kernel(int group, int seff, bool fused) {
+#define KVQ_PICK(GG)                                    \
+  if (group == GG) {                                    \
+    if (seff == 16) return kernel_ptr<GG, 16>(fused);   \
+    if (seff == 32) return kernel_ptr<GG, 32>(fused);   \
   }
   KVQ_PICK(1)
   KVQ_PICK(2)
@@ -1195,17 +1331,24 @@ size_t smem_bytes(int group, int max_batch) {
 
 int plan_decode(int group, int page_size, int max_batch, int num_sms, DecodeLaunch* out) {
   const int seff = page_size < kTileTokens ? page_size : kTileTokens;
-  void* fn = pick_kernel(group, seff);
-  if (!fn) return -1;
   const size_t smem = smem_bytes(group, max_batch);
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return -2;
-  int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kThreads, smem) != cudaSuccess)
-    return -2;
+  // The dynamic shared memory cap of both variants is set to the most any call of this
+  // library uses (max_batch 4096), so plans made for several caches never shrink it
+  // under one another; the grid is the smaller occupancy of the two.
+  const size_t cap_bytes = smem_bytes(group, 4096);
+  int occ = 3;
+  for (int fused = 0; fused < 2; fused++) {
+    void* fn = pick_kernel(group, seff, fused != 0);
+    if (!fn) return -1;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(cap_bytes)) != cudaSuccess)
+      return -2;
+    int o = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, kThreads, smem) != cudaSuccess)
+      return -2;
+    if (o < occ) occ = o;
+  }
   if (occ < 1) return -1;
-  if (occ > 3) occ = 3;
   out->grid = num_sms * occ;
   out->smem = smem;
   return 0;
@@ -1213,7 +1356,7 @@ int plan_decode(int group, int page_size, int max_batch, int num_sms, DecodeLaun
 
 int launch_decode(const DecodeParams& p, const DecodeLaunch& L, cudaStream_t stream) {
   const int seff = p.page_size < kTileTokens ? p.page_size : kTileTokens;
-  void* fn = pick_kernel(p.group, seff);
+  void* fn = pick_kernel(p.group, seff, p.k_new != nullptr);
   if (!fn) return -1;
   DecodeParams q = p;
   q.total_ctas = L.grid;

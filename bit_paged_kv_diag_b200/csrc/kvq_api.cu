@@ -223,9 +223,12 @@ int kvq_rotate_quant_append(kvq_cache* c, int32_t layer, const void* k, const vo
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;
 }
 
-int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, const int32_t* seq_lens,
-                         const int32_t* page_table, int32_t batch, float softmax_scale, void* out,
-                         void* stream) {
+namespace {
+
+// Shared by the decode and the fused append + decode calls.
+int decode_common(kvq_cache* c, int32_t layer, const void* k_new, const void* v_new, const void* q,
+                  const int32_t* seq_lens, const int32_t* page_table, int32_t batch,
+                  float softmax_scale, void* out, void* stream) {
   if (!c) return KVQ_EINVAL;
   if (layer < 0 || layer >= c->d.num_layers) return KVQ_EINVAL;
   if (batch < 0 || batch > c->d.max_batch) return KVQ_EINVAL;
@@ -256,9 +259,29 @@ int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, const int32
   p.q_scale = static_cast<float>(sm * 1.4426950408889634);  // log2(e)
   p.cb = c->cb;
   p.total_ctas = c->launch.grid;
+  p.k_new = static_cast<const __half*>(k_new);
+  p.v_new = static_cast<const __half*>(v_new);
   const int rc = kvq::launch_decode(p, c->launch, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;
+}
+
+}  // namespace
+
+int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, const int32_t* seq_lens,
+                         const int32_t* page_table, int32_t batch, float softmax_scale, void* out,
+                         void* stream) {
+  return decode_common(c, layer, nullptr, nullptr, q, seq_lens, page_table, batch, softmax_scale,
+                       out, stream);
+}
+
+int kvq_append_decode_attention(kvq_cache* c, int32_t layer, const void* k_new, const void* v_new,
+                                const void* q, const int32_t* seq_lens, const int32_t* page_table,
+                                int32_t batch, float softmax_scale, void* out, void* stream) {
+  if (c && batch > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)))
+    return KVQ_EINVAL;
+  return decode_common(c, layer, k_new, v_new, q, seq_lens, page_table, batch, softmax_scale, out,
+                       stream);
 }
 
 void* kvq_pool_ptr(const kvq_cache* c) { return c ? c->pool : nullptr; }

@@ -56,6 +56,11 @@ struct DecodeParams {
   float q_scale;                  // softmax_scale * log2(e)
   float cb;                       // fp32 nearest 1/sqrt(hadamard_block)
   int total_ctas;                 // C: CTAs in the grid
+  // Fused one-token append (null for a plain decode): the new K and V rows [batch][Hkv][128]
+  // are rotated, quantised and stored at position seq_lens[b], and the decode runs over
+  // seq_lens[b] + 1 tokens (the pool is then written through pool_layer).
+  const __half* k_new;
+  const __half* v_new;
 };
 
 // Host-side launchers (return 0 on success, <0 on an unsupported shape or a launch

@@ -132,6 +132,8 @@ int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, int32_t la
   p.q_scale = static_cast<float>(sm * 1.4426950408889634);  // log2(e)
   p.cb = static_cast<float>(1.0 / sqrt(static_cast<double>(d->hadamard_block)));
   p.total_ctas = L.grid;
+  p.k_new = nullptr;
+  p.v_new = nullptr;
   const int lrc = kvq::launch_decode(p, L, static_cast<cudaStream_t>(stream));
   if (lrc == -1) return KVQ_EUNSUPPORTED;
   return lrc == 0 ? KVQ_OK : KVQ_ECUDA;

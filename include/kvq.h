@@ -182,6 +182,27 @@ KVQ_API int kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, con
                          const int32_t* page_table, int32_t batch, float softmax_scale,
                          void* out, void* stream);
 
+/* Append one token per sequence and decode over it, in one launch: the fused form of
+ * kvq_rotate_quant_append (one new token per sequence, cu_new_tokens = 0, 1, ..., batch)
+ * followed by kvq_decode_attention.  It follows the pages' fused kernel that rotates,
+ * quantises and appends as the token is produced ("KVキャッシュを4ビットへ", section
+ * "システムこそが設計である — 融合カーネル"), and also saves the second launch per
+ * layer in a decode step.  The pool receives exactly the bytes the separate append would
+ * write.
+ *   k_new, v_new   device fp16 [batch][num_kv_heads][128], 16-byte aligned: the new
+ *                  token's K and V rows
+ *   seq_lens       device int32 [batch], lengths BEFORE the append: the new token goes to
+ *                  position seq_lens[b] and the decode attends seq_lens[b] + 1 tokens
+ *   q, page_table, batch, softmax_scale, out, stream: as for kvq_decode_attention
+ * A position beyond the sequence's page budget or a bad page id is flagged in the status
+ * word (KVQ_DEV_BAD_POS / KVQ_DEV_BAD_PAGE) and that row is not stored.
+ * Returns KVQ_OK or a negative status (before any launch). */
+KVQ_API int kvq_append_decode_attention(kvq_cache* c, int32_t layer, const void* k_new,
+                                        const void* v_new, const void* q,
+                                        const int32_t* seq_lens, const int32_t* page_table,
+                                        int32_t batch, float softmax_scale, void* out,
+                                        void* stream);
+
 /* Decode attention that allocates nothing.  The pages have no counterpart of this call;
  * it exists for callers that cannot call cudaMalloc: an inference runtime that has
  * reserved all of device memory for its own pool and forbids stray allocations, a plugin

@@ -76,9 +76,11 @@ def host_inputs(case: Case):
 
 
 class GpuRun:
-    """The CUDA path through the C ABI: alloc, prefill append, step append, decode."""
+    """The CUDA path through the C ABI: alloc, prefill append, step append, decode (or,
+    with fused=True and one new token per sequence, the step's append and the decode in
+    one kvq_append_decode_attention call)."""
 
-    def __init__(self, case: Case, kp, vp, kn, vn, q, softmax_scale=0.0):
+    def __init__(self, case: Case, kp, vp, kn, vn, q, softmax_scale=0.0, fused=False):
         import torch
         import bit_paged_kv_diag_b200 as kvq
         self.case = case
@@ -94,12 +96,17 @@ class GpuRun:
         if kp.shape[0] > 0:
             kvq.rotate_quant_append(self.cache, case.layer, t(kp), t(vp),
                                     t(workloads.cu_seqlens(case.lengths)), zeros, pt)
-        if kn.shape[0] > 0:
-            kvq.rotate_quant_append(self.cache, case.layer, t(kn), t(vn),
-                                    t(workloads.cu_seqlens(case.new)), lens, pt)
         self.lens_after = case.lengths + case.new
-        self.out = kvq.decode_attention(self.cache, case.layer, t(q), t(self.lens_after), pt,
-                                        softmax_scale=softmax_scale)
+        if fused:
+            assert np.all(case.new == 1), "the fused call appends one token per sequence"
+            self.out = kvq.append_decode_attention(self.cache, case.layer, t(kn), t(vn), t(q),
+                                                   lens, pt, softmax_scale=softmax_scale)
+        else:
+            if kn.shape[0] > 0:
+                kvq.rotate_quant_append(self.cache, case.layer, t(kn), t(vn),
+                                        t(workloads.cu_seqlens(case.new)), lens, pt)
+            self.out = kvq.decode_attention(self.cache, case.layer, t(q), t(self.lens_after), pt,
+                                            softmax_scale=softmax_scale)
         torch.cuda.synchronize()
         self.status = kvq.get_device_status(self.cache)
         self.host_pool = self.pool.cpu().numpy()
@@ -158,10 +165,10 @@ def check_outputs(gpu_out, ref_out, what=""):
     return worst
 
 
-def full_parity(case: Case, softmax_scale=0.0):
+def full_parity(case: Case, softmax_scale=0.0, fused=False):
     """Run everything at a size the oracle finishes in seconds; assert all bars."""
     kp, vp, kn, vn, q = host_inputs(case)
-    run = GpuRun(case, kp, vp, kn, vn, q, softmax_scale)
+    run = GpuRun(case, kp, vp, kn, vn, q, softmax_scale, fused=fused)
     try:
         assert run.status == 0, f"device status {run.status}"
         pt_ref = oracle.assign_pages(case.capacity, case.w.page_size, case.num_pages,

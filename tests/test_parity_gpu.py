@@ -64,6 +64,31 @@ def test_plain_int4_prefill_student_t():
     full_parity(make_case(w, [0, 0, 0, 0], [300, 257, 64, 1], block=1))
 
 
+@pytest.mark.parametrize("name,lengths,block", [
+    ("tiny", [256], None),
+    ("qwen3_4b_decode", [517, 300, 64, 1, 0, 129, 63, 65, 31, 32, 33, 4095], None),
+    ("long_context", [1000, 2049, 64, 777], None),
+    ("ragged", [130, 700, 129, 1024, 0, 2, 350, 64, 191, 1500, 17, 33], None),
+    ("ragged", [130, 700, 0, 95], 1),
+])
+def test_fused_append_decode(name, lengths, block):
+    """kvq_append_decode_attention: the pool gets exactly the oracle's append of the new
+    token (bit-exact, whole pool) and the outputs match the oracle's decode over it; the
+    new token lands on tile and page boundaries and in empty sequences."""
+    w = W[name]
+    r = full_parity(make_case(w, lengths, [1] * len(lengths), block=block), fused=True)
+    assert r["flips"] == 0
+
+
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+@pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])
+def test_fused_group_and_page_size_grid(group, page_size):
+    w = dataclasses.replace(W["qwen3_4b_decode"], num_kv_heads=2, num_q_heads=2 * group,
+                            page_size=page_size, block=64)
+    full_parity(make_case(w, [300, 0, 513, 31, 64], [1] * 5, permute=True, pool_factor=1.3),
+                fused=True)
+
+
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])
 def test_group_and_page_size_grid(group, page_size):
