@@ -6,16 +6,19 @@
 One step = one decode step of the Qwen3-4B-shaped workload (36 layers, 8 KV heads, 32
 query heads, head_dim 128, Hadamard block 128, page 16, 16 sequences of 4096 cached
 tokens): for every layer, the fused rotate-quant-append of the step's token of each
-sequence, then paged GQA decode attention over 4097 tokens.  The step is captured once
-as a CUDA graph and replayed.  ``value`` is effective HBM GB/s: the step's algorithmic
+sequence and paged GQA decode attention over 4097 tokens, in one launch per layer
+(kvq_append_decode_attention).  The step is captured once as a CUDA graph and replayed.
+The same step as two calls per layer (kvq_rotate_quant_append, kvq_decode_attention) is
+reported beside it (``step_separate_calls``).  ``value`` is effective HBM GB/s: the step's algorithmic
 bytes (132 B per cached (token, KV head) + page-table, q and out bytes for decode; 2 x 256
 B read + 132 B written per appended (token, KV head)) over the device time per step, all
 ranks summed.  The cache (2.5 GB) is far larger than the 126 MB L2, so nothing is reused
 across steps.
 
 Also reported: the roofline of the decode-attention call, the prefill-append throughput
-(8 x 8192 new tokens in one call, b = 32/64/128), end-to-end throughput through the C ABI
-with host buffers, and the CPU oracle timed on a bounded sample of the same workload.
+(8 x 8192 new tokens in one call, b = 32/64/128, and b = 1: plain INT4 without rotation),
+rotated against plain INT4 decode, end-to-end throughput through the C ABI with host
+buffers, and the CPU oracle timed on a bounded sample of the same workload.
 
 Multi-GPU: replicas only (each rank runs the whole workload on its own GPU; the path has
 no exchange step), timing = max over ranks.
@@ -157,13 +160,21 @@ def run_kvq(args, rank, world, local_rank):
            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(NL)]
 
     def step(instrument):
+        """One decode step: per layer, the token's append and decode attention in one
+        fused launch (kvq_append_decode_attention)."""
         for l in range(NL):
-            kvq.rotate_quant_append(cache, l, kn[l], vn[l], cu_new, lens_before, ptd)
             if instrument:
                 ev[l][0].record()
-            kvq.decode_attention(cache, l, q[l], lens_after, ptd, out=out[l])
+            kvq.append_decode_attention(cache, l, kn[l], vn[l], q[l], lens_before, ptd, out=out[l])
             if instrument:
                 ev[l][1].record()
+
+    def step_separate():
+        """The same step as two calls per layer: kvq_rotate_quant_append, then
+        kvq_decode_attention."""
+        for l in range(NL):
+            kvq.rotate_quant_append(cache, l, kn[l], vn[l], cu_new, lens_before, ptd)
+            kvq.decode_attention(cache, l, q[l], lens_after, ptd, out=out[l])
 
     # Eager warm-up (also initialises the library's launch state), then graph capture.
     # The timed graph has no event nodes between kernels, so consecutive launches keep
@@ -201,9 +212,25 @@ def run_kvq(args, rank, world, local_rank):
         dist.all_reduce(tms, op=dist.ReduceOp.MAX)
         ms = float(tms.item())
 
+    # The same step as separate append and decode calls (2 launches per layer).
+    sgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(sgraph, stream=side):
+        step_separate()
+    for _ in range(3):
+        sgraph.replay()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s0.record()
+    for _ in range(max(3, args.steps // 2)):
+        sgraph.replay()
+    s1.record()
+    torch.cuda.synchronize()
+    sep_ms = s0.elapsed_time(s1) / max(3, args.steps // 2)
+    del sgraph
+
     # Decode-attention launches: a graph of the 36 decode calls back to back, timed with
     # events around its replays (mean device time per launch, launch overlap included),
-    # and each launch alone between event nodes of the step graph.
+    # and each fused launch alone between event nodes of the step graph.
     dgraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(dgraph, stream=side):
         for l in range(NL):
@@ -284,8 +311,12 @@ def run_kvq(args, rank, world, local_rank):
                    "page_size": S, "global_batch": B * world, "seq_len": int(cap[0]),
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: 2.5 GB cache per step vs 126 MB L2",
-                   "graph": "one CUDA graph per step"},
-        "gpu_launches": args.steps * NL * 2,  # per layer: one append, one decode launch
+                   "graph": "one CUDA graph per step",
+                   "step": "per layer one kvq_append_decode_attention (fused 1-token append + decode)"},
+        "step_separate_calls": {"ms_per_step": round(sep_ms, 5),
+                                "value": round(world * step_bytes / (sep_ms * 1e-3) / 1e9, 1),
+                                "how": "per layer kvq_rotate_quant_append then kvq_decode_attention"},
+        "gpu_launches": args.steps * NL,  # per layer: one fused append + decode launch
         "device_status": status,
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -297,7 +328,7 @@ def run_kvq(args, rank, world, local_rank):
         "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
         "frac": round(ach / peak, 4), "peak_kind": peak_kind,
         "traffic": _traffic("decode", dec_b), "us_per_launch": round(dec_ms * 1e3, 3),
-        "us_per_launch_alone": round(iso_ms * 1e3, 3),
+        "fused_us_per_launch_alone": round(iso_ms * 1e3, 3),
         "bytes_per_launch": dec_b, "timing": dec_how}
     line["append"] = append
     line["plain_int4"] = plain

@@ -818,8 +818,11 @@ struct NewRow {
   uint32_t scale;    // fp16 bits, same in every lane
 };
 
-__device__ __forceinline__ NewRow quantise_new_row(const __half* row, int lane, const DecodeParams& p) {
-  const uint2 raw = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+__device__ __forceinline__ uint2 load_new_row(const __half* row, int lane) {
+  return __ldg(reinterpret_cast<const uint2*>(row) + lane);  // channels 4*lane..4*lane+3
+}
+
+__device__ __forceinline__ NewRow quantise_new_row(uint2 raw, int lane, const DecodeParams& p) {
   const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
   const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
   float x[4] = {lo.x, lo.y, hi.x, hi.y};
@@ -865,16 +868,16 @@ __device__ __forceinline__ NewRow quantise_new_row(const __half* row, int lane, 
   return r;
 }
 
-// The new token of unit (b, h): rotate and quantise its K and V rows, store them at
+// The new token of unit (b, h) (its raw K and V rows kraw, vraw as loaded by
+// load_new_row): rotate and quantise the rows, store them at
 // position seq_lens[b] of the pool (skipped, with the status flagged, when the position or
 // its page is out of range) and, in the block layout of one token, into the warp's patch
 // buffer (shared memory): [K codes 64 B][V codes 64 B][K scale][V scale].  Returns
 // whether the rows are stored and belong in the decode.
-__device__ __forceinline__ bool fused_append(int b, int h, int lane, uint8_t* patch,
-                                             const DecodeParams& p) {
-  const size_t row = (static_cast<size_t>(b) * p.num_kv_heads + h) * kD;
-  const NewRow kr = quantise_new_row(p.k_new + row, lane, p);
-  const NewRow vr = quantise_new_row(p.v_new + row, lane, p);
+__device__ __forceinline__ bool fused_append(int b, int h, int lane, uint8_t* patch, uint2 kraw,
+                                             uint2 vraw, const DecodeParams& p) {
+  const NewRow kr = quantise_new_row(kraw, lane, p);
+  const NewRow vr = quantise_new_row(vraw, lane, p);
   *reinterpret_cast<uint16_t*>(patch + 2 * lane) = static_cast<uint16_t>(kr.codes16);
   *reinterpret_cast<uint16_t*>(patch + 64 + 2 * lane) = static_cast<uint16_t>(vr.codes16);
   if (lane == 0) {
@@ -1050,6 +1053,22 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   auto is_ul = [&](const Unit& u) { return u.b == ul.b && u.h == ul.h; };
   const bool two_edges = has_tiles && !is_uf(ul);
 
+  // Fused append: the new K/V rows of the first unit, if this warp holds its last tile,
+  // are loaded before the wait (the inputs of an append are complete when the previous
+  // kernel lets this one start); later units load theirs at their segment's start.
+  uint2 kraw0 = make_uint2(0u, 0u), vraw0 = make_uint2(0u, 0u);
+  if constexpr (FUSED) {
+    if (x < X1) {
+      const int seg_end0 = min(X1, cu.U + cu.n);
+      const int xl0 = x + kWarps * ((seg_end0 - x + kWarps - 1) / kWarps - 1);
+      if (xl0 == cu.U + cu.n - 1) {
+        const size_t row = (static_cast<size_t>(cu.b) * p.num_kv_heads + cu.h) * kD;
+        kraw0 = load_new_row(p.k_new + row, lane);
+        vraw0 = load_new_row(p.v_new + row, lane);
+      }
+    }
+  }
+
   griddep_wait();
 
   // q goes ahead of the tile copies, so that it is not queued behind them; then the first
@@ -1135,7 +1154,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       const int xl = x + kWarps * (nt - 1);  // this warp's last tile of the unit
       uint8_t* patch = reinterpret_cast<uint8_t*>(frag);  // free until the next unit's q
       if (xl == cu.U + cu.n - 1 && !dead) {
-        new_ok = fused_append(cu.b, cu.h, lane, patch, p);
+        uint2 kraw = kraw0, vraw = vraw0;
+        if (x != X0 + w) {  // not the warp's first unit: load now
+          const size_t row = (static_cast<size_t>(cu.b) * p.num_kv_heads + cu.h) * kD;
+          kraw = load_new_row(p.k_new + row, lane);
+          vraw = load_new_row(p.v_new + row, lane);
+        }
+        new_ok = fused_append(cu.b, cu.h, lane, patch, kraw, vraw, p);
         if (lane == 0) *reinterpret_cast<int*>(patch + 132) = cu.L - 1 - (xl - cu.U) * kTileTokens;
         __syncwarp();
       }

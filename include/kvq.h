@@ -58,8 +58,9 @@
  *   * Launch overlap: both kernels use programmatic dependent launch.  Each lets the next
  *     kernel on the stream start at its own entry, and waits for the previous kernel to
  *     complete before it touches the pool, q, out or the handle's scratch.  Before that
- *     wait, decode already reads seq_lens and page_table, and append reads k, v,
- *     cu_new_tokens, seq_lens and page_table.  These arrays must therefore be complete
+ *     wait, decode already reads seq_lens and page_table, append reads k, v,
+ *     cu_new_tokens, seq_lens and page_table, and the fused append + decode reads k_new,
+ *     v_new, seq_lens and page_table.  These arrays must therefore be complete
  *     when the previous kernel on the stream lets its dependents start.  Kernels that do
  *     not use programmatic launch (PyTorch's, cuBLAS's, copies) only do so by completing,
  *     and this library's own kernels never write these arrays.
