@@ -61,6 +61,9 @@ def lib():
                                                 ctypes.c_double, f64p]),
             "oracle_attention_dense": (c_int, [f64p, f64p, f64p, c_int, c_int, c_int, c_int,
                                                ctypes.c_double, f64p]),
+            "oracle_prefill_attention": (c_int, [u8p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                 c_int, c_int, u16p, i32p, i32p, i32p, c_int,
+                                                 ctypes.c_double, f64p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -256,6 +259,26 @@ def decode_attention(g: Geometry, pool, layer, q16, seq_lens, page_table,
                                        sl.shape[0], float(softmax_scale),
                                        _p(out, ctypes.c_double))
     _check(rc, "decode_attention")
+    return out
+
+
+def prefill_attention(g: Geometry, pool, layer, q16, cu_q, seq_lens, page_table,
+                      softmax_scale=0.0) -> np.ndarray:
+    """Causal chunked-prefill attention, fp64 outputs [cu_q[-1]][Hq][D]: the chunk of
+    sequence b is its last cu_q[b+1] - cu_q[b] tokens of seq_lens[b]."""
+    pool = _c(pool, np.uint8)
+    q = _c(np.asarray(q16).view(np.uint16), np.uint16)
+    cu = _c(cu_q, np.int32)
+    sl = _c(seq_lens, np.int32)
+    pt = _c(page_table, np.int32)
+    out = np.zeros((int(cu[-1]), g.num_q_heads, g.head_dim), np.float64)
+    rc = lib().oracle_prefill_attention(_p(pool, ctypes.c_uint8), layer, g.num_pages,
+                                        g.num_kv_heads, g.num_q_heads, g.head_dim, g.block,
+                                        g.page_size, g.max_pages_per_seq, _p(q, ctypes.c_uint16),
+                                        _p(cu, ctypes.c_int32), _p(sl, ctypes.c_int32),
+                                        _p(pt, ctypes.c_int32), sl.shape[0], float(softmax_scale),
+                                        _p(out, ctypes.c_double))
+    _check(rc, "prefill_attention")
     return out
 
 

@@ -268,16 +268,13 @@ int oracle_read_row(const uint8_t* pool, int layer, int num_pages, int num_kv_he
  *   p = exp(score - max) / sum exp;  o' = sum_t p_t vhat_t;
  *   o = Hadamard(o')  (the orthonormal Sylvester matrix is its own inverse).
  * An empty sequence gives zeros.  out: [head_dim] fp64.  Returns 0 or <0. */
-int oracle_decode_one(const uint8_t* pool, int layer, int num_pages, int num_kv_heads,
-                      int num_q_heads, int head_dim, int block, int page_size,
-                      int max_pages_per_seq, const uint16_t* q, const int32_t* seq_lens,
-                      const int32_t* page_table, int b, int hq, double softmax_scale,
-                      double* out) {
+/* Attention of one query row qrow (fp16 bits, [head_dim]) of sequence b over its
+ * first L cached tokens of KV head h; the steps of oracle_decode_one below. */
+static int attend_row(const uint8_t* pool, int layer, int num_pages, int num_kv_heads,
+                      int head_dim, int block, int page_size, int max_pages_per_seq,
+                      const uint16_t* qrow, const int32_t* page_table, int b, int L, int h,
+                      double softmax_scale, double* out) {
   const int D = head_dim, S = page_size;
-  if (num_kv_heads <= 0 || num_q_heads % num_kv_heads) return -1;
-  const int G = num_q_heads / num_kv_heads;
-  const int h = hq / G;
-  const int L = seq_lens[b];
   if (softmax_scale == 0.0) softmax_scale = 1.0 / sqrt((double)D);
   for (int d = 0; d < D; d++) out[d] = 0.0;
   if (L <= 0) return 0;
@@ -289,8 +286,7 @@ int oracle_decode_one(const uint8_t* pool, int layer, int num_pages, int num_kv_
   if (!qr || !sc || !row) { free(qr); free(sc); free(row); return -1; }
   int rc = 0;
 
-  const uint16_t* qs = q + ((size_t)b * num_q_heads + hq) * D;
-  for (int d = 0; d < D; d++) qr[d] = (double)oracle_half_to_float(qs[d]);
+  for (int d = 0; d < D; d++) qr[d] = (double)oracle_half_to_float(qrow[d]);
   oracle_fwht_f64(qr, D, block);
 
   double mx = -INFINITY;
@@ -323,6 +319,18 @@ int oracle_decode_one(const uint8_t* pool, int layer, int num_pages, int num_kv_
   return rc;
 }
 
+int oracle_decode_one(const uint8_t* pool, int layer, int num_pages, int num_kv_heads,
+                      int num_q_heads, int head_dim, int block, int page_size,
+                      int max_pages_per_seq, const uint16_t* q, const int32_t* seq_lens,
+                      const int32_t* page_table, int b, int hq, double softmax_scale,
+                      double* out) {
+  if (num_kv_heads <= 0 || num_q_heads % num_kv_heads) return -1;
+  const int G = num_q_heads / num_kv_heads;
+  return attend_row(pool, layer, num_pages, num_kv_heads, head_dim, block, page_size,
+                    max_pages_per_seq, q + ((size_t)b * num_q_heads + hq) * head_dim,
+                    page_table, b, seq_lens[b], hq / G, softmax_scale, out);
+}
+
 /* All (b, hq) pairs: out [batch][num_q_heads][head_dim] fp64. */
 int oracle_decode_attention(const uint8_t* pool, int layer, int num_pages, int num_kv_heads,
                             int num_q_heads, int head_dim, int block, int page_size,
@@ -337,6 +345,39 @@ int oracle_decode_attention(const uint8_t* pool, int layer, int num_pages, int n
                                  out + ((size_t)b * num_q_heads + hq) * head_dim);
       if (rc) return rc;
     }
+  return 0;
+}
+
+/* Chunked-prefill attention over the paged cache, causal.  Sequence b holds
+ * L_b = seq_lens[b] tokens, the last C_b = cu_q[b+1] - cu_q[b] of which are the chunk's
+ * queries (already appended); query i of the chunk sits at position p = L_b - C_b + i and
+ * attends positions 0..p.  [P1, "KVキャッシュこそが本当のボトルネックである理由": serving
+ * engines run attention over the paged cache; a chunk of prompt tokens attending the
+ * cache causally is the many-query case of the same attention (a stated reading).]
+ * Each (query token, query head) is oracle_decode_one's computation over its causal
+ * prefix.  q, out: [cu_q[batch]][num_q_heads][head_dim] (fp16 bits in, fp64 out). */
+int oracle_prefill_attention(const uint8_t* pool, int layer, int num_pages, int num_kv_heads,
+                             int num_q_heads, int head_dim, int block, int page_size,
+                             int max_pages_per_seq, const uint16_t* q, const int32_t* cu_q,
+                             const int32_t* seq_lens, const int32_t* page_table, int batch,
+                             double softmax_scale, double* out) {
+  if (num_kv_heads <= 0 || num_q_heads % num_kv_heads) return -1;
+  const int G = num_q_heads / num_kv_heads, D = head_dim;
+  for (int b = 0; b < batch; b++) {
+    const int C = cu_q[b + 1] - cu_q[b], L = seq_lens[b];
+    if (C < 0 || C > L) return -1;
+    for (int i = 0; i < C; i++) {
+      const size_t tok = (size_t)cu_q[b] + i;
+      const int pos = L - C + i;
+      for (int hq = 0; hq < num_q_heads; hq++) {
+        const int rc = attend_row(pool, layer, num_pages, num_kv_heads, D, block, page_size,
+                                  max_pages_per_seq, q + (tok * num_q_heads + hq) * D,
+                                  page_table, b, pos + 1, hq / G, softmax_scale,
+                                  out + (tok * num_q_heads + hq) * D);
+        if (rc) return rc;
+      }
+    }
+  }
   return 0;
 }
 

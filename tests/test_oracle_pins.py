@@ -441,3 +441,75 @@ def test_cache_decode_equals_dense_attention_on_dequantised_rows():
     vhat = oracle.read_row(g, pool, 0, pt[1, 0], 0, 0, 1).astype(np.float64)
     Hn = scipy.linalg.block_diag(*[scipy.linalg.hadamard(64) / 8.0] * 2)
     assert np.max(np.abs(out[1, 0] - Hn @ vhat)) < 1e-12
+
+
+def _numpy_rows(pool, g, layer, page, head, slot, kv):
+    """Dequantised cache row read straight from the pool bytes (independent of the oracle's
+    reader): nibbles low = even channel, two's complement, times the fp16 scale."""
+    S, D = g.page_size, g.head_dim
+    blk = S * (D + 4)
+    base = ((layer * g.num_pages + page) * g.num_kv_heads + head) * blk
+    b = pool[base + kv * S * (D // 2) + slot * (D // 2):][:D // 2].astype(np.int16)
+    codes = np.empty(D, np.int16)
+    codes[0::2] = b & 0xF
+    codes[1::2] = b >> 4
+    codes = np.where(codes >= 8, codes - 16, codes)
+    s = pool[base + S * D + kv * S * 2 + slot * 2:][:2].view(np.float16)[0]
+    return codes.astype(np.float64) * float(s)
+
+
+def test_prefill_attention_is_causal_attention_on_the_cache():
+    """Chunked prefill: query i of sequence b's chunk (position L_b - C_b + i) attends
+    exactly cache positions 0..p.  Brute force in numpy (rows read from the pool bytes,
+    scipy's Hadamard, explicit softmax) on a tiny ragged case with a chunk of the whole
+    sequence, a partial chunk, one query, and an empty chunk."""
+    g = _tiny_geometry(block=32, S=16, hkv=2, hq=4, P=16, mp=4, layers=1)
+    rng = np.random.default_rng(21)
+    cap = np.array([37, 20, 9, 5], np.int32)
+    pt = oracle.assign_pages(cap, 16, 16, 4, rng.permutation(16).astype(np.int32))
+    pool = g.new_pool()
+    n = int(cap.sum())
+    k = rng.standard_normal((n, 2, 128)).astype(np.float16)
+    v = rng.standard_normal((n, 2, 128)).astype(np.float16)
+    oracle.rotate_quant_append(g, pool, 0, k, v, np.concatenate([[0], np.cumsum(cap)]).astype(np.int32),
+                               np.zeros(4, np.int32), pt)
+    chunks = np.array([37, 7, 1, 0], np.int32)
+    cu = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    q = rng.standard_normal((int(cu[-1]), 4, 128)).astype(np.float16)
+    out = oracle.prefill_attention(g, pool, 0, q, cu, cap, pt, softmax_scale=0.07)
+    Hn = scipy.linalg.block_diag(*[scipy.linalg.hadamard(32) / np.sqrt(32.0)] * 4)
+    for b in range(4):
+        for i in range(chunks[b]):
+            pos = cap[b] - chunks[b] + i
+            for hq in range(4):
+                h = hq // 2
+                K = np.stack([_numpy_rows(pool, g, 0, pt[b, t // 16], h, t % 16, 0) for t in range(pos + 1)])
+                V = np.stack([_numpy_rows(pool, g, 0, pt[b, t // 16], h, t % 16, 1) for t in range(pos + 1)])
+                qr = Hn @ q[cu[b] + i, hq].astype(np.float64)
+                sc = 0.07 * (K @ qr)
+                p = np.exp(sc - sc.max())
+                p /= p.sum()
+                ref = Hn @ (p @ V)
+                assert np.max(np.abs(out[cu[b] + i, hq] - ref)) < 1e-10, (b, i, hq)
+
+
+def test_prefill_attention_reduces_to_decode():
+    """A chunk of one query is decode over L_b; the last query of a longer chunk too."""
+    g = _tiny_geometry(block=64, S=16, hkv=2, hq=8, P=8, mp=4, layers=1)
+    rng = np.random.default_rng(22)
+    cap = np.array([50, 3], np.int32)
+    pt = oracle.assign_pages(cap, 16, 8, 4)
+    pool = g.new_pool()
+    k = rng.standard_normal((53, 2, 128)).astype(np.float16)
+    v = rng.standard_normal((53, 2, 128)).astype(np.float16)
+    oracle.rotate_quant_append(g, pool, 0, k, v, np.array([0, 50, 53], np.int32),
+                               np.zeros(2, np.int32), pt)
+    qd = rng.standard_normal((2, 8, 128)).astype(np.float16)
+    dec = oracle.decode_attention(g, pool, 0, qd, cap, pt)
+    one = oracle.prefill_attention(g, pool, 0, qd, np.array([0, 1, 2], np.int32), cap, pt)
+    assert np.array_equal(one, dec)
+    qc = rng.standard_normal((9, 8, 128)).astype(np.float16)
+    qc[5] = qd[0]
+    qc[8] = qd[1]
+    chunk = oracle.prefill_attention(g, pool, 0, qc, np.array([0, 6, 9], np.int32), cap, pt)
+    assert np.array_equal(chunk[5], dec[0]) and np.array_equal(chunk[8], dec[1])
