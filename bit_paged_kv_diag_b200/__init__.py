@@ -7,6 +7,7 @@ The names mirror the C ABI in ``include/kvq.h``:
 * ``kvq_rotate_quant_append``  -> :func:`rotate_quant_append`
 * ``kvq_decode_attention``     -> :func:`decode_attention`
 * ``kvq_append_decode_attention`` -> :func:`append_decode_attention`
+* ``kvq_prefill_attention``    -> :func:`prefill_attention`
 * ``kvq_free``                 -> :func:`free`
 * ``kvq_assign_pages``, ``kvq_pool_bytes``, ``kvq_get_device_status`` likewise.
 
@@ -23,7 +24,7 @@ from . import build as _build
 
 __all__ = [
     "KVQError", "Desc", "Cache", "lib", "pool_bytes", "assign_pages", "alloc_pages",
-    "rotate_quant_append", "decode_attention", "append_decode_attention",
+    "rotate_quant_append", "decode_attention", "append_decode_attention", "prefill_attention",
     "decode_attention_noalloc", "free",
     "get_device_status", "status_string",
     "EXPORTED",
@@ -36,6 +37,7 @@ EXPORTED = (
     "kvq_pool_bytes", "kvq_assign_pages", "kvq_alloc_pages", "kvq_rotate_quant_append",
     "kvq_decode_attention", "kvq_pool_ptr", "kvq_get_device_status", "kvq_free",
     "kvq_status_string", "kvq_decode_attention_noalloc", "kvq_append_decode_attention",
+    "kvq_prefill_attention",
 )
 
 
@@ -82,6 +84,8 @@ def lib() -> ctypes.CDLL:
                                                             ctypes.c_float, vp, vp]),
             "kvq_append_decode_attention": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, i32,
                                                            ctypes.c_float, vp, vp]),
+            "kvq_prefill_attention": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, i32, i32,
+                                                     ctypes.c_float, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -232,6 +236,24 @@ def append_decode_attention(cache: Cache, layer: int, k_new, v_new, q, seq_lens,
         _dev_ptr(seq_lens, "seq_lens", torch.int32), _dev_ptr(page_table, "page_table", torch.int32),
         batch, float(softmax_scale), _dev_ptr(out, "out", torch.float16), _stream_ptr(stream))
     _check(rc, "kvq_append_decode_attention")
+    return out
+
+
+def prefill_attention(cache: Cache, layer: int, q, cu_q, seq_lens, page_table, softmax_scale=0.0,
+                      out=None, stream=None, total_q=None):
+    """Causal chunked-prefill attention: q fp16 [total_q][Hq][128] (chunks concatenated),
+    cu_q int32 [batch+1], seq_lens int32 [batch] (lengths with the chunk appended)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    batch = int(seq_lens.shape[0])
+    tq = int(q.shape[0]) if total_q is None else int(total_q)
+    rc = lib().kvq_prefill_attention(
+        cache.handle, int(layer), _dev_ptr(q, "q", torch.float16),
+        _dev_ptr(cu_q, "cu_q", torch.int32), _dev_ptr(seq_lens, "seq_lens", torch.int32),
+        _dev_ptr(page_table, "page_table", torch.int32), batch, tq, float(softmax_scale),
+        _dev_ptr(out, "out", torch.float16), _stream_ptr(stream))
+    _check(rc, "kvq_prefill_attention")
     return out
 
 

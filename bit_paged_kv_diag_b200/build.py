@@ -13,7 +13,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkvq.so")
-SOURCES = ["kvq_api.cu", "append_kernel.cu", "decode_kernel.cu", "kvq_noalloc.cu"]
+SOURCES = ["kvq_api.cu", "append_kernel.cu", "decode_kernel.cu", "kvq_noalloc.cu",
+           "prefill_kernel.cu"]
 HEADERS = ["kvq_internal.h", "kvq_ptx.cuh"]
 
 NVCC_FLAGS = [

@@ -284,6 +284,42 @@ int kvq_append_decode_attention(kvq_cache* c, int32_t layer, const void* k_new, 
                        stream);
 }
 
+int kvq_prefill_attention(kvq_cache* c, int32_t layer, const void* q, const int32_t* cu_q,
+                          const int32_t* seq_lens, const int32_t* page_table, int32_t batch,
+                          int32_t total_q, float softmax_scale, void* out, void* stream) {
+  if (!c) return KVQ_EINVAL;
+  if (layer < 0 || layer >= c->d.num_layers) return KVQ_EINVAL;
+  if (batch < 0 || batch > c->d.max_batch || total_q < 0) return KVQ_EINVAL;
+  if (!(softmax_scale >= 0.0f) || isinf(softmax_scale)) return KVQ_EINVAL;
+  if (batch == 0 || total_q == 0) return KVQ_OK;
+  if (!q || !cu_q || !seq_lens || !page_table || !out) return KVQ_EINVAL;
+  if (!aligned16(q) || !aligned16(out)) return KVQ_EINVAL;
+  kvq::PrefillParams p;
+  const size_t layer_bytes = pool_bytes_of(&c->d) / c->d.num_layers;
+  p.pool_layer = c->pool + static_cast<size_t>(layer) * layer_bytes;
+  p.q = static_cast<const __half*>(q);
+  p.cu_q = cu_q;
+  p.seq_lens = seq_lens;
+  p.page_table = page_table;
+  p.out = static_cast<__half*>(out);
+  p.status = c->status;
+  p.batch = batch;
+  p.num_kv_heads = c->d.num_kv_heads;
+  p.group = c->d.num_q_heads / c->d.num_kv_heads;
+  p.num_pages = c->d.num_pages;
+  p.page_size = c->d.page_size;
+  p.page_shift = __builtin_ctz(static_cast<unsigned>(c->d.page_size));
+  p.max_pages_per_seq = c->d.max_pages_per_seq;
+  p.hadamard_block = c->d.hadamard_block;
+  const double sm = softmax_scale == 0.0f ? 1.0 / sqrt(static_cast<double>(c->d.head_dim))
+                                          : static_cast<double>(softmax_scale);
+  p.q_scale = static_cast<float>(sm * 1.4426950408889634);  // log2(e)
+  p.cb = c->cb;
+  const int rc = kvq::launch_prefill(p, total_q, static_cast<cudaStream_t>(stream));
+  if (rc == -1) return KVQ_EUNSUPPORTED;
+  return rc == 0 ? KVQ_OK : KVQ_ECUDA;
+}
+
 void* kvq_pool_ptr(const kvq_cache* c) { return c ? c->pool : nullptr; }
 
 int kvq_get_device_status(kvq_cache* c, int32_t* status, void* stream) {

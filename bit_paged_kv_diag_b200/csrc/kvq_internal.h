@@ -63,9 +63,31 @@ struct DecodeParams {
   const __half* v_new;
 };
 
+struct PrefillParams {
+  const uint8_t* pool_layer;      // block(0, 0) of the layer
+  const __half* q;                // [total_q][Hq][128], chunks concatenated by sequence
+  const int32_t* cu_q;            // [batch+1] chunk offsets
+  const int32_t* seq_lens;        // [batch] tokens cached, the chunk included
+  const int32_t* page_table;      // [batch][max_pages_per_seq]
+  __half* out;                    // [total_q][Hq][128]
+  int32_t* status;
+  int batch;
+  int num_kv_heads;
+  int group;
+  int num_pages;
+  int page_size;
+  int page_shift;
+  int max_pages_per_seq;
+  int hadamard_block;
+  float q_scale;                  // softmax_scale * log2(e)
+  float cb;
+  int total_q;                    // rows of q and out
+};
+
 // Host-side launchers (return 0 on success, <0 on an unsupported shape or a launch
 // error).
 int launch_append(const AppendParams& p, int block, int num_sms, cudaStream_t stream);
+int launch_prefill(const PrefillParams& p, int total_q, cudaStream_t stream);
 
 struct DecodeLaunch {
   int grid;          // CTAs (a multiple of the SM count)

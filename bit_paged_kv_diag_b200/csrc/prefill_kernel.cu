@@ -1,0 +1,572 @@
+// prefill_kernel.cu -- causal chunked-prefill attention over the rotated-INT4 paged KV
+// cache, for sm_100a.
+//
+// Method: "KVキャッシュを4ビットへ — SAW-INT4とシステムを踏まえたINT4量子化"
+// (youngju.dev): section "KVキャッシュこそが本当のボトルネックである理由" (attention runs
+// over the paged cache in serving engines) and "回転のトリック — ブロック対角アダマール"
+// (the orthonormal rotation keeps q.k, so attention runs in the rotated domain and the
+// output is rotated back).  A chunk of C prompt tokens of a sequence, already appended,
+// attends the cache causally: query i of the chunk (position L - C + i) sees positions
+// 0..L - C + i.
+//
+// Work decomposition.  A CTA (4 warps) takes 64 query rows of one (sequence, KV head):
+// QB = 64 / G consecutive chunk tokens times the G query heads of the KV head; warp w owns
+// rows 16w..16w+15 end to end (its own online softmax, no cross-warp merge).  The CTA
+// streams the causal KV range of its rows in tiles of 32 tokens through one shared ring of
+// 3 slots filled by bulk copies (cp.async.bulk, issued by warp 0; every warp releases a
+// slot by one arrival on the slot's "empty" barrier).  Per tile and warp:
+//   QK^T  int8 mma m16n8k32, A = q' cut into three int8 slices (as in decode; read from
+//         shared memory with ldmatrix), B = K codes as int8 (nibble moved to the byte's
+//         top), 4 n-tiles of 8 tokens; scores in the log2 domain with the K scale and the
+//         row's slice scale; causal mask on positions.
+//   softmax  online, per row; the row sum stays lane-partial until the end.
+//   PV    fp16 mma m16n8k16, A = P' = p * s_v as fp16 hi + lo (the score accumulators are
+//         the A fragments, no shuffles), B = V codes as exact fp16 (byte gather + magic
+//         conversion), 16 n-tiles of 8 channels.
+// The end: o'/l, the inverse block Hadamard across a row's channels (bits 1-2 of the
+// channel across lanes, the others in registers), times c_b, fp16 store.
+#include <cuda_fp16.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+#include "kvq_internal.h"
+#include "kvq_ptx.cuh"
+
+namespace kvq {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kRows = 64;        // query rows per CTA
+constexpr int kWarpsP = 4;
+constexpr int kThreadsP = 128;
+constexpr int kStagesP = 3;
+constexpr int kSlotBytesP = kTileTokens * (kD + 4);  // 4224
+constexpr unsigned kFullMask = 0xffffffffu;
+constexpr float kMagicP = 12582912.0f;  // 1.5 * 2^23
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+__device__ __forceinline__ void split_hi_lo_p(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(p0, p1);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(p0 - f.x, p1 - f.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Byte offset of token tau (0..31) of a ring slot: the slot holds pages of SEFF token
+// slots in the pool's block layout [K codes][V codes][K scales][V scales].
+template <int SEFF>
+__device__ __forceinline__ int tok_base(int tau) {
+  return (tau / SEFF) * (SEFF * 132);
+}
+
+// Issue the bulk copies of tile t (tokens 32t..) of sequence b, KV head h into a slot
+// (warp 0 calls; lane j < pages-needed copies page j).
+template <int SEFF>
+__device__ __forceinline__ void issue_tile(int t, int b, int h, int L, uint32_t slot, uint32_t bar,
+                                           int lane, uint64_t pol, const PrefillParams& p) {
+  const int S = p.page_size, sh = p.page_shift;
+  const uint32_t blk_bytes = static_cast<uint32_t>(S) * (kD + 4);
+  const int t0 = t * kTileTokens;
+  const int t1 = min(t0 + kTileTokens, L);  // > t0
+  if (SEFF < kTileTokens || S == kTileTokens) {
+    const int npg = ((t1 - 1) >> sh) - (t0 >> sh) + 1;
+    int pid = 0;
+    bool bad = false;
+    if (lane < npg) {
+      pid = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + (t0 >> sh) + lane);
+      bad = pid < 0 || pid >= p.num_pages;
+      if (bad) pid = 0;
+    }
+    if (__any_sync(kFullMask, bad) && lane == 0) atomicOr(p.status, KVQ_DEV_BAD_PAGE_BIT);
+    if (lane == 0) mbar_arrive_expect_tx(bar, npg * blk_bytes);
+    __syncwarp();
+    if (lane < npg)
+      bulk_copy_g2s(slot + lane * blk_bytes,
+                    p.pool_layer + (static_cast<size_t>(pid) * p.num_kv_heads + h) * blk_bytes,
+                    blk_bytes, bar, pol);
+  } else {
+    int pid = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + (t0 >> sh));
+    const bool bad = pid < 0 || pid >= p.num_pages;
+    if (bad) pid = 0;
+    if (bad && lane == 0) atomicOr(p.status, KVQ_DEV_BAD_PAGE_BIT);
+    const size_t o = static_cast<size_t>(t0 & (S - 1));
+    const uint8_t* blk = p.pool_layer + (static_cast<size_t>(pid) * p.num_kv_heads + h) * blk_bytes;
+    const uint8_t* src = blk + o * 64;
+    uint32_t dst = slot, bytes = 2048;
+    if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + 2048; }
+    if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 2; dst = slot + 4096; bytes = 64; }
+    if (lane == 3) { src = blk + static_cast<size_t>(S) * 130 + o * 2; dst = slot + 4160; bytes = 64; }
+    if (lane == 0) mbar_arrive_expect_tx(bar, kSlotBytesP);
+    __syncwarp();
+    if (lane < 4) bulk_copy_g2s(dst, src, bytes, bar, pol);
+  }
+}
+
+// Rotate one q row (lane: channels 4L..4L+3; the fixed butterfly, then x c_b x q_scale),
+// cut it into three int8 slices q' = M/64 (q1 + q2/128 + q3/16384), M the power of two >=
+// max |q'|, and store the slices in A-fragment order: qs[s][jj][row][kappa] with, inside
+// k-step jj, kappa = 4c + e <-> channel 32c + 8jj + 2e and kappa = 16 + 4c + e <-> channel
+// 32c + 8jj + 2e + 1.  Returns M / 1024 (the score scale of the row; K codes enter the MMA
+// times 16).
+__device__ __forceinline__ float prep_q_row(const __half* qrow, bool valid, uint8_t* qs, int row,
+                                            int lane, const PrefillParams& p) {
+  float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (valid) {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qrow) + lane);
+    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+    x[0] = lo.x; x[1] = lo.y; x[2] = hi.x; x[3] = hi.y;
+  }
+  if (p.hadamard_block > 1) {
+    const float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
+    x[0] = a0 + a2; x[2] = a0 - a2; x[1] = a1 + a3; x[3] = a1 - a3;
+#pragma unroll
+    for (int st = 0; st < 5; st++) {
+      if ((4 << st) < p.hadamard_block) {
+        const float sgn = ((lane >> st) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int e = 0; e < 4; e++) x[e] = __fmaf_rn(x[e], sgn, __shfl_xor_sync(kFullMask, x[e], 1 << st));
+      }
+    }
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; e++) {
+    x[e] = x[e] * p.cb * p.q_scale;
+    amax = fmaxf(amax, fabsf(x[e]));
+  }
+#pragma unroll
+  for (int d = 1; d < 32; d *= 2) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
+  float M = 1.0f;
+  if (amax > 1e-30f) {
+    const uint32_t bits = __float_as_uint(amax);
+    M = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax;
+  }
+  const float inv = 64.0f / M;
+  uint32_t ms[3][4];
+#pragma unroll
+  for (int e = 0; e < 4; e++) {
+    const float t = x[e] * inv;
+    const float m1 = t + kMagicP;
+    const float r1 = (t - (m1 - kMagicP)) * 128.0f;
+    const float m2 = r1 + kMagicP;
+    const float r2 = (r1 - (m2 - kMagicP)) * 128.0f;
+    const float m3 = r2 + kMagicP;
+    ms[0][e] = __float_as_uint(m1);
+    ms[1][e] = __float_as_uint(m2);
+    ms[2][e] = __float_as_uint(m3);
+  }
+  // Channels 4L + i: c = L/8, jj = (L%8)/2, e = 2(L%2) + i/2, odd = i%2.
+  const int c = lane >> 3, jj = (lane & 7) >> 1, e0 = 2 * (lane & 1);
+#pragma unroll
+  for (int s = 0; s < 3; s++) {
+    uint8_t* r = qs + ((s * 4 + jj) * kRows + row) * 32;
+    const uint16_t ev = static_cast<uint16_t>((ms[s][0] & 0xFFu) | ((ms[s][2] & 0xFFu) << 8));
+    const uint16_t od = static_cast<uint16_t>((ms[s][1] & 0xFFu) | ((ms[s][3] & 0xFFu) << 8));
+    *reinterpret_cast<uint16_t*>(r + 4 * c + e0) = ev;
+    *reinterpret_cast<uint16_t*>(r + 16 + 4 * c + e0) = od;
+  }
+  return M * (1.0f / 1024.0f);
+}
+
+template <int G, int SEFF>
+__global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) {
+  constexpr int QB = kRows / G;  // chunk tokens per CTA
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
+  uint8_t* ring = smem;                                        // [3][4224]
+  uint8_t* qs = ring + kStagesP * kSlotBytesP;                 // [3][4][64][32] int8
+  float* sfr = reinterpret_cast<float*>(qs + 3 * 4 * kRows * 32);  // [64] row scales
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sfr + kRows);   // full[3], empty[3]
+  int32_t* preq = reinterpret_cast<int32_t*>(bars + 2 * kStagesP);  // [batch + 1]
+  __shared__ int warp_sum[kWarpsP];
+  __shared__ int running;
+
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, c = lane & 3;
+  // Before griddep_wait only cu_q, seq_lens and the page table are read (inputs of this
+  // call); q, the pool and out are touched after it.
+  griddep_launch_dependents();
+  const uint32_t full_s = smem_addr(bars), empty_s = smem_addr(bars + kStagesP);
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < kStagesP; s++) {
+      mbar_init(full_s + 8 * s, 1);
+      mbar_init(empty_s + 8 * s, kWarpsP);
+    }
+    fence_mbar_init();
+    running = 0;
+  }
+  __syncthreads();
+
+  // Query blocks per sequence -> exclusive prefix preq[0..batch].
+  for (int base = 0; base < p.batch; base += kThreadsP) {
+    const int i = base + tid;
+    int n = 0;
+    if (i < p.batch) {
+      const int C = __ldg(p.cu_q + i + 1) - __ldg(p.cu_q + i);
+      n = C > 0 ? (C + QB - 1) / QB : 0;
+    }
+    int incl = n;
+#pragma unroll
+    for (int d = 1; d < 32; d *= 2) {
+      const int y = __shfl_up_sync(kFullMask, incl, d);
+      if (lane >= d) incl += y;
+    }
+    if (lane == 31) warp_sum[w] = incl;
+    __syncthreads();
+    int before = running;
+    for (int w2 = 0; w2 < w; w2++) before += warp_sum[w2];
+    if (i < p.batch) preq[i] = before + incl - n;
+    __syncthreads();
+    if (tid == kThreadsP - 1) running = before + incl;
+    __syncthreads();
+  }
+  if (tid == 0) preq[p.batch] = running;
+  __syncthreads();
+
+  const int nblk = preq[p.batch];
+  const int qbg = blockIdx.x / p.num_kv_heads, h = blockIdx.x - qbg * p.num_kv_heads;
+  if (qbg >= nblk) return;  // the whole CTA
+  int lo = 0, hi = p.batch;  // preq[lo] <= qbg < preq[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (preq[mid] <= qbg) lo = mid; else hi = mid;
+  }
+  const int b = lo, qb = qbg - preq[b];
+  const int cq0 = __ldg(p.cu_q + b);
+  const int C = __ldg(p.cu_q + b + 1) - cq0;
+  const int cap = p.max_pages_per_seq * p.page_size;
+  int L = __ldg(p.seq_lens + b);
+  if (L > cap || C > L || cq0 < 0 || cq0 + C > p.total_q) {
+    if (tid == 0) atomicOr(p.status, KVQ_DEV_BAD_POS_BIT);
+    return;
+  }
+  const int tok_first = qb * QB;                       // first chunk token of the CTA
+  const int tok_last = min(C, tok_first + QB) - 1;     // last valid one
+  const int pos_last = L - C + tok_last;
+  const int ntile = pos_last / kTileTokens + 1;
+  const uint64_t pol = l2_policy_evict_first();
+
+  griddep_wait();
+
+  // The first kStagesP tiles (warp 0), then every warp prepares its 16 q rows.
+  int issued = 0, done0 = 0;  // warp 0: tiles issued / tiles whose copy it waited for
+  if (w == 0)
+    for (; issued < kStagesP && issued < ntile; issued++)
+      issue_tile<SEFF>(issued, b, h, L, smem_addr(ring) + issued * kSlotBytesP,
+                       full_s + 8 * issued, lane, pol, p);
+  for (int rr = 0; rr < 16; rr++) {
+    const int row = 16 * w + rr;
+    const int ti = tok_first + row / G, gq = row % G;
+    const bool valid = ti < C;
+    const __half* qrow = p.q + ((static_cast<size_t>(cq0) + (valid ? ti : 0)) * p.num_kv_heads * G +
+                                h * G + gq) * kD;
+    const float sf = prep_q_row(qrow, valid, qs, row, lane, p);
+    if (lane == 0) sfr[row] = sf;
+  }
+  __syncwarp();
+
+  // This lane's rows: g and g + 8 of the warp's 16.
+  const int r0 = 16 * w + g, r1 = r0 + 8;
+  const float sf0 = sfr[r0], sf1 = sfr[r1];
+  const int pos0 = L - C + tok_first + r0 / G, pos1 = L - C + tok_first + r1 / G;
+  float o[16][4];
+#pragma unroll
+  for (int i = 0; i < 16; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+  float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.0f, l1 = 0.0f;
+  // V conversion constants of this lane's channel parity (channel 8cn + g).
+  const uint32_t vsel = static_cast<uint32_t>(g >> 1) | ((4u + static_cast<uint32_t>(g >> 1)) << 8);
+  const uint32_t vmask = (g & 1) ? 0x00F000F0u : 0x000F000Fu;
+  const uint32_t vxor = (g & 1) ? 0x64806480u : 0x64086408u;
+  const uint32_t vmul = (g & 1) ? 0x2C002C00u : 0x3C003C00u;  // 1/16 or 1
+  const uint32_t vadd = (g & 1) ? 0xD480D480u : 0xE408E408u;  // -72 or -1032
+  const uint32_t qs_s = smem_addr(qs);
+  // ldmatrix row address of this lane inside a [64][32] slice block: matrix L/8.
+  const int lm = lane >> 3, lr = lane & 7;
+  const uint32_t a_off = static_cast<uint32_t>((16 * w + lr + (lm & 1) * 8) * 32 + (lm >> 1) * 16);
+  bool dead = false;
+
+  for (int t = 0; t < ntile; t++) {
+    const int slot = t % kStagesP;
+    const uint32_t par = static_cast<uint32_t>((t / kStagesP) & 1);
+    if (!dead) {
+      if (mbar_wait_bounded(full_s + 8 * slot, par, kWaitNs)) done0++;
+      else dead = true;
+    }
+    const uint8_t* base = ring + slot * kSlotBytesP;
+    if (!dead) {
+      // K codes of tokens 8nt + g (bytes 16c..16c+15 of the row) and the K/V scales of
+      // tokens 8nt + 2c, 8nt + 2c + 1.
+      uint4 kr[4];
+      float sk[4][2], sv[4][2];
+#pragma unroll
+      for (int nt = 0; nt < 4; nt++) {
+        const int tau = 8 * nt + g;
+        kr[nt] = *reinterpret_cast<const uint4*>(base + tok_base<SEFF>(tau) + (tau % SEFF) * 64 + 16 * c);
+        const int tk = 8 * nt + 2 * c;
+        const uint8_t* pb = base + tok_base<SEFF>(tk);
+        const __half2 k2 = *reinterpret_cast<const __half2*>(pb + SEFF * 128 + (tk % SEFF) * 2);
+        const __half2 v2 = *reinterpret_cast<const __half2*>(pb + SEFF * 130 + (tk % SEFF) * 2);
+        const float2 kf = __half22float2(k2), vf = __half22float2(v2);
+        // Slots past the sequence's end hold stale bytes: their V scale must not reach P'.
+        const int tpos = t * kTileTokens + tk;
+        sk[nt][0] = kf.x; sk[nt][1] = kf.y;
+        sv[nt][0] = tpos < L ? vf.x : 0.0f;
+        sv[nt][1] = tpos + 1 < L ? vf.y : 0.0f;
+      }
+      // Scores: three int8 slices, accumulated in fp32 with weights 1, 2^-7, 2^-14.
+      float sc[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; nt++) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
+#pragma unroll
+      for (int s = 0; s < 3; s++) {
+        int acc[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; nt++) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+#pragma unroll
+        for (int jj = 0; jj < 4; jj++) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(qs_s + static_cast<uint32_t>((s * 4 + jj) * kRows * 32) + a_off, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < 4; nt++) {
+            const uint32_t wv = jj == 0 ? kr[nt].x : jj == 1 ? kr[nt].y : jj == 2 ? kr[nt].z : kr[nt].w;
+            mma_16832_s8(acc[nt], a0, a1, a2, a3, (wv << 4) & 0xF0F0F0F0u, wv & 0xF0F0F0F0u);
+          }
+        }
+        const float ws = s == 0 ? 1.0f : (s == 1 ? 1.0f / 128.0f : 1.0f / 16384.0f);
+#pragma unroll
+        for (int nt = 0; nt < 4; nt++)
+#pragma unroll
+          for (int e = 0; e < 4; e++) sc[nt][e] += static_cast<float>(acc[nt][e]) * ws;
+      }
+      // Scale, causal mask, row maxima.
+      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
+#pragma unroll
+      for (int nt = 0; nt < 4; nt++)
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+          const int tpos = t * kTileTokens + 8 * nt + 2 * c + e;
+          sc[nt][e] = tpos <= pos0 ? sc[nt][e] * (sf0 * sk[nt][e]) : -CUDART_INF_F;
+          sc[nt][2 + e] = tpos <= pos1 ? sc[nt][2 + e] * (sf1 * sk[nt][e]) : -CUDART_INF_F;
+          mx0 = fmaxf(mx0, sc[nt][e]);
+          mx1 = fmaxf(mx1, sc[nt][2 + e]);
+        }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, 2));
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      // A row with no visible token yet keeps m = -inf and p = 0.
+      const float al0 = mn0 == -CUDART_INF_F ? 1.0f : ex2_approx(m0 - mn0);
+      const float al1 = mn1 == -CUDART_INF_F ? 1.0f : ex2_approx(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      float ps0 = 0.0f, ps1 = 0.0f;
+#pragma unroll
+      for (int nt = 0; nt < 4; nt++)
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+          sc[nt][e] = mn0 == -CUDART_INF_F ? 0.0f : ex2_approx(sc[nt][e] - mn0);
+          sc[nt][2 + e] = mn1 == -CUDART_INF_F ? 0.0f : ex2_approx(sc[nt][2 + e] - mn1);
+          ps0 += sc[nt][e];
+          ps1 += sc[nt][2 + e];
+        }
+      l0 = l0 * al0 + ps0;
+      l1 = l1 * al1 + ps1;
+#pragma unroll
+      for (int cn = 0; cn < 16; cn++) {
+        o[cn][0] *= al0;
+        o[cn][1] *= al0;
+        o[cn][2] *= al1;
+        o[cn][3] *= al1;
+      }
+      // PV: two k-steps of 16 tokens.
+#pragma unroll
+      for (int kk = 0; kk < 2; kk++) {
+        uint32_t ah[4], al[4];
+        split_hi_lo_p(sc[2 * kk][0] * sv[2 * kk][0], sc[2 * kk][1] * sv[2 * kk][1], ah[0], al[0]);
+        split_hi_lo_p(sc[2 * kk][2] * sv[2 * kk][0], sc[2 * kk][3] * sv[2 * kk][1], ah[1], al[1]);
+        split_hi_lo_p(sc[2 * kk + 1][0] * sv[2 * kk + 1][0], sc[2 * kk + 1][1] * sv[2 * kk + 1][1],
+                      ah[2], al[2]);
+        split_hi_lo_p(sc[2 * kk + 1][2] * sv[2 * kk + 1][0], sc[2 * kk + 1][3] * sv[2 * kk + 1][1],
+                      ah[3], al[3]);
+        // V rows of tokens 16kk + 2c, +1 (b0) and 16kk + 8 + 2c, +1 (b1).
+        const int ta = 16 * kk + 2 * c, tb = ta + 8;
+        const uint8_t* va0 = base + tok_base<SEFF>(ta) + SEFF * 64 + (ta % SEFF) * 64;
+        const uint8_t* va1 = base + tok_base<SEFF>(ta + 1) + SEFF * 64 + ((ta + 1) % SEFF) * 64;
+        const uint8_t* vb0 = base + tok_base<SEFF>(tb) + SEFF * 64 + (tb % SEFF) * 64;
+        const uint8_t* vb1 = base + tok_base<SEFF>(tb + 1) + SEFF * 64 + ((tb + 1) % SEFF) * 64;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; q4++) {  // channel n-tiles 4q4 .. 4q4 + 3
+          const uint4 wa0 = *reinterpret_cast<const uint4*>(va0 + 16 * q4);
+          const uint4 wa1 = *reinterpret_cast<const uint4*>(va1 + 16 * q4);
+          const uint4 wb0 = *reinterpret_cast<const uint4*>(vb0 + 16 * q4);
+          const uint4 wb1 = *reinterpret_cast<const uint4*>(vb1 + 16 * q4);
+          const uint32_t xa0[4] = {wa0.x, wa0.y, wa0.z, wa0.w}, xa1[4] = {wa1.x, wa1.y, wa1.z, wa1.w};
+          const uint32_t xb0[4] = {wb0.x, wb0.y, wb0.z, wb0.w}, xb1[4] = {wb1.x, wb1.y, wb1.z, wb1.w};
+#pragma unroll
+          for (int k4 = 0; k4 < 4; k4++) {
+            const int cn = 4 * q4 + k4;  // channels 8cn..8cn+7; this lane's is 8cn + g
+            uint32_t b0 = lop3_and_xor(prmt(xa0[k4], xa1[k4], vsel), vmask, vxor);
+            uint32_t b1 = lop3_and_xor(prmt(xb0[k4], xb1[k4], vsel), vmask, vxor);
+            asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(b0) : "r"(b0), "r"(vmul), "r"(vadd));
+            asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(b1) : "r"(b1), "r"(vmul), "r"(vadd));
+            mma_16816(o[cn], ah[0], ah[1], ah[2], ah[3], b0, b1);
+            mma_16816(o[cn], al[0], al[1], al[2], al[3], b0, b1);
+          }
+        }
+      }
+    }
+    // Release the slot; warp 0 refills it with tile t + kStagesP once every warp is done.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_s + 8 * slot);
+    if (w == 0 && !dead && t + kStagesP < ntile) {
+      if (!mbar_wait_bounded(empty_s + 8 * slot, par, kWaitNs)) {
+        dead = true;
+      } else {
+        fence_proxy_async_smem();
+        issue_tile<SEFF>(t + kStagesP, b, h, L, smem_addr(ring) + slot * kSlotBytesP,
+                         full_s + 8 * slot, lane, pol, p);
+        issued++;
+      }
+    }
+  }
+  if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
+
+  // Row sums across the 4 lanes of a row; o'/l; inverse rotation; fp16 store.
+  l0 += __shfl_xor_sync(kFullMask, l0, 1);
+  l0 += __shfl_xor_sync(kFullMask, l0, 2);
+  l1 += __shfl_xor_sync(kFullMask, l1, 1);
+  l1 += __shfl_xor_sync(kFullMask, l1, 2);
+  const float i0 = l0 > 0.0f ? __frcp_rn(l0) : 0.0f, i1 = l1 > 0.0f ? __frcp_rn(l1) : 0.0f;
+#pragma unroll
+  for (int cn = 0; cn < 16; cn++) {
+    o[cn][0] *= i0;
+    o[cn][1] *= i0;
+    o[cn][2] *= i1;
+    o[cn][3] *= i1;
+  }
+  // Channel 8cn + 2c + e: bit 0 = e (in register pair), bits 1-2 = c (lanes ^1, ^2),
+  // bits 3-6 = cn (registers).  Stages h = 1, 2, ..., b/2 in this order.
+  const int block = p.hadamard_block;
+  if (block > 1) {
+#pragma unroll
+    for (int cn = 0; cn < 16; cn++) {
+      float a = o[cn][0], d = o[cn][1];
+      o[cn][0] = a + d; o[cn][1] = a - d;
+      a = o[cn][2]; d = o[cn][3];
+      o[cn][2] = a + d; o[cn][3] = a - d;
+    }
+#pragma unroll
+    for (int st = 0; st < 2; st++) {
+      if ((2 << st) < block) {
+        const float sgn = ((c >> st) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int cn = 0; cn < 16; cn++)
+#pragma unroll
+          for (int e = 0; e < 4; e++)
+            o[cn][e] = __fmaf_rn(o[cn][e], sgn, __shfl_xor_sync(kFullMask, o[cn][e], 1 << st));
+      }
+    }
+#pragma unroll
+    for (int hh = 1; hh < 16; hh *= 2) {
+      if (8 * hh < block) {
+#pragma unroll
+        for (int cn = 0; cn < 16; cn++)
+          if (!(cn & hh))
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+              const float a = o[cn][e], d = o[cn + hh][e];
+              o[cn][e] = a + d;
+              o[cn + hh][e] = a - d;
+            }
+      }
+    }
+  }
+  const int ta = tok_first + r0 / G, tb = tok_first + r1 / G;
+  __half* out0 = p.out + ((static_cast<size_t>(cq0) + ta) * p.num_kv_heads * G + h * G + r0 % G) * kD;
+  __half* out1 = p.out + ((static_cast<size_t>(cq0) + tb) * p.num_kv_heads * G + h * G + r1 % G) * kD;
+#pragma unroll
+  for (int cn = 0; cn < 16; cn++) {
+    if (ta < C)
+      *reinterpret_cast<__half2*>(out0 + 8 * cn + 2 * c) =
+          __floats2half2_rn(o[cn][0] * p.cb, o[cn][1] * p.cb);
+    if (tb < C)
+      *reinterpret_cast<__half2*>(out1 + 8 * cn + 2 * c) =
+          __floats2half2_rn(o[cn][2] * p.cb, o[cn][3] * p.cb);
+  }
+  if (dead && w == 0) {
+    // Let copies still in flight (issued by this warp, never waited for) land before the
+    // CTA's shared memory is released; warp 0 stopped issuing when it gave up.
+    for (int j = done0; j < issued; j++)
+      mbar_wait_bounded(full_s + 8 * (j % kStagesP), static_cast<uint32_t>((j / kStagesP) & 1),
+                        kWaitNs);
+  }
+}
+
+template <int G, int SEFF>
+void* prefill_ptr() {
+  return reinterpret_cast<void*>(&prefill_kernel<G, SEFF>);
+}
+
+void* pick_prefill(int group, int seff) {
+#define KVQ_PICKP(GG)                                  \
+  if (group == GG) {                                   \
+    if (seff == 16) return prefill_ptr<GG, 16>();      \
+    if (seff == 32) return prefill_ptr<GG, 32>();      \
+  }
+  KVQ_PICKP(1)
+  KVQ_PICKP(2)
+  KVQ_PICKP(4)
+  KVQ_PICKP(8)
+#undef KVQ_PICKP
+  return nullptr;
+}
+
+size_t prefill_smem(int max_batch) {
+  size_t s = static_cast<size_t>(kStagesP) * kSlotBytesP;  // ring
+  s += 3 * 4 * kRows * 32;                                  // q slices
+  s += sizeof(float) * kRows;                               // row scales
+  s += sizeof(uint64_t) * 2 * kStagesP;                     // barriers
+  s += static_cast<size_t>(max_batch + 1) * sizeof(int32_t);  // query-block prefix
+  s += 128;                                                  // alignment slack
+  return (s + 15) & ~static_cast<size_t>(15);
+}
+
+}  // namespace
+
+int launch_prefill(const PrefillParams& p, int total_q, cudaStream_t stream) {
+  const int seff = p.page_size < kTileTokens ? p.page_size : kTileTokens;
+  void* fn = pick_prefill(p.group, seff);
+  if (!fn) return -1;
+  if (p.batch == 0 || total_q == 0) return 0;
+  const int QB = kRows / p.group;
+  const long long blocks = (static_cast<long long>(total_q) + QB - 1) / QB + p.batch;
+  const long long grid = blocks * p.num_kv_heads;
+  if (grid > 0x7fffffffLL) return -1;
+  const size_t smem = prefill_smem(p.batch);
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(prefill_smem(4096))) != cudaSuccess)
+    return -2;
+  PrefillParams q = p;
+  q.total_q = total_q;
+  void* args[] = {&q};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreadsP);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelExC(&cfg, fn, args) != cudaSuccess) return -2;
+  return 0;
+}
+
+}  // namespace kvq

@@ -60,7 +60,8 @@
  *     complete before it touches the pool, q, out or the handle's scratch.  Before that
  *     wait, decode already reads seq_lens and page_table, append reads k, v,
  *     cu_new_tokens, seq_lens and page_table, and the fused append + decode reads k_new,
- *     v_new, seq_lens and page_table.  These arrays must therefore be complete
+ *     v_new, seq_lens and page_table, and prefill attention reads cu_q, seq_lens and
+ *     page_table.  These arrays must therefore be complete
  *     when the previous kernel on the stream lets its dependents start.  Kernels that do
  *     not use programmatic launch (PyTorch's, cuBLAS's, copies) only do so by completing,
  *     and this library's own kernels never write these arrays.
@@ -203,6 +204,31 @@ KVQ_API int kvq_append_decode_attention(kvq_cache* c, int32_t layer, const void*
                                         const int32_t* seq_lens, const int32_t* page_table,
                                         int32_t batch, float softmax_scale, void* out,
                                         void* stream);
+
+/* Causal chunked-prefill attention over the INT4 cache of one layer: many query tokens
+ * per sequence.  A chunk of C_b = cu_q[b+1] - cu_q[b] prompt tokens of sequence b, already
+ * appended (kvq_rotate_quant_append), attends the cache causally: query i of the chunk,
+ * at position seq_lens[b] - C_b + i, attends positions 0 .. seq_lens[b] - C_b + i.  The
+ * pages' attention over the paged cache ("KVキャッシュを4ビットへ", section
+ * "KVキャッシュこそが本当のボトルネックである理由") for the many-query case a serving
+ * engine runs on the same cache; decode is the case C_b = 1.
+ *   q              device fp16 [total_q][num_q_heads][128], the chunks concatenated in
+ *                  order of b, 16-byte aligned
+ *   cu_q           device int32 [batch+1], chunk offsets into q (cu_q[0] = 0)
+ *   seq_lens       device int32 [batch], tokens cached, the chunk included (C_b <=
+ *                  seq_lens[b] <= max_pages_per_seq * page_size)
+ *   page_table     device int32 [batch][max_pages_per_seq]
+ *   total_q        host int32, cu_q[batch] (sizes the launch)
+ *   softmax_scale  multiplier of q.k; 0 means 1/sqrt(128)
+ *   out            device fp16 [total_q][num_q_heads][128], 16-byte aligned
+ * A chunk longer than its sequence, or a length beyond the page budget, is flagged
+ * (KVQ_DEV_BAD_POS) and its rows are not written.  Uses no scratch; calls on one handle
+ * may run on any stream ordering the caller chooses.  Returns KVQ_OK or a negative status
+ * (before any launch). */
+KVQ_API int kvq_prefill_attention(kvq_cache* c, int32_t layer, const void* q,
+                                  const int32_t* cu_q, const int32_t* seq_lens,
+                                  const int32_t* page_table, int32_t batch, int32_t total_q,
+                                  float softmax_scale, void* out, void* stream);
 
 /* Decode attention that allocates nothing.  The pages have no counterpart of this call;
  * it exists for callers that cannot call cudaMalloc: an inference runtime that has

@@ -185,3 +185,48 @@ def full_parity(case: Case, softmax_scale=0.0, fused=False):
         return dict(flips=flips, total_codes=total, worst=worst)
     finally:
         run.close()
+
+
+def prefill_parity(case: Case, softmax_scale=0.0):
+    """Chunked prefill: the cache holds case.lengths tokens, the chunk of case.new tokens per
+    sequence is appended, then kvq_prefill_attention runs the chunk's queries causally.
+    Bars: page table and pool as for full_parity, outputs against the oracle's causal
+    attention on the GPU-written cache."""
+    import torch
+    import bit_paged_kv_diag_b200 as kvq
+    kp, vp, kn, vn, _ = host_inputs(case)
+    cu_q = workloads.cu_seqlens(case.new)
+    q = workloads.q_rows_chunk(case.w, case.layer, int(cu_q[-1]))
+    dev = torch.device("cuda")
+    d = case.desc()
+    pool = torch.zeros(kvq.pool_bytes(d), dtype=torch.uint8, device=dev)
+    cache, page_table = kvq.alloc_pages(d, case.capacity, case.page_order, pool=pool)
+    try:
+        pt = torch.from_numpy(page_table).to(dev)
+        t = lambda a: torch.as_tensor(a).to(dev)  # noqa: E731
+        zeros = torch.zeros(len(case.lengths), dtype=torch.int32, device=dev)
+        if kp.shape[0] > 0:
+            kvq.rotate_quant_append(cache, case.layer, t(kp), t(vp),
+                                    t(workloads.cu_seqlens(case.lengths)), zeros, pt)
+        if kn.shape[0] > 0:
+            kvq.rotate_quant_append(cache, case.layer, t(kn), t(vn), t(cu_q), t(case.lengths), pt)
+        lens_after = case.lengths + case.new
+        out = kvq.prefill_attention(cache, case.layer, t(q), t(cu_q), t(lens_after), pt,
+                                    softmax_scale=softmax_scale)
+        torch.cuda.synchronize()
+        status = kvq.get_device_status(cache)
+        assert status == 0, f"device status {status}"
+        host_pool = pool.cpu().numpy()
+        host_out = out.float().cpu().numpy()
+    finally:
+        cache.close()
+    pt_ref = oracle.assign_pages(case.capacity, case.w.page_size, case.num_pages,
+                                 case.max_pages_per_seq, case.page_order)
+    assert np.array_equal(page_table, pt_ref), "page table differs from the oracle's"
+    ref_pool = oracle_pool(case, kp, vp, kn, vn, pt_ref)
+    scale_mis, flips, other, total = compare_pools(case, host_pool, ref_pool)
+    assert scale_mis == 0 and other == 0 and flips <= MAX_FLIP_FRACTION * total
+    ref = oracle.prefill_attention(case.geometry(), host_pool, case.layer, q, cu_q, lens_after,
+                                   pt_ref, softmax_scale)
+    worst = check_outputs(host_out, ref, case.w.name + " prefill")
+    return dict(worst=worst, total_q=int(cu_q[-1]))

@@ -107,6 +107,8 @@ def test_calls_reject_bad_arguments_before_any_cuda_call():
     assert L.kvq_decode_attention(None, 0, None, None, None, 0, 0.0, None, None) == kvq.KVQ_EINVAL
     assert L.kvq_append_decode_attention(None, 0, None, None, None, None, None, 0, 0.0, None,
                                          None) == kvq.KVQ_EINVAL
+    assert L.kvq_prefill_attention(None, 0, None, None, None, None, 0, 0, 0.0, None,
+                                   None) == kvq.KVQ_EINVAL
     assert L.kvq_free(None) == kvq.KVQ_OK
     assert L.kvq_pool_ptr(None) is None
     assert kvq.status_string(kvq.KVQ_ENOPAGES) == "not enough pages"

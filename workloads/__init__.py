@@ -159,6 +159,13 @@ def q_rows(w: Workload, layer: int, stream: int = 0) -> np.ndarray:
     return to_fp16(r.standard_normal((w.batch, w.num_q_heads, w.head_dim)))
 
 
+def q_rows_chunk(w: Workload, layer: int, n_tokens: int, stream: int = 0) -> np.ndarray:
+    """q of n_tokens query tokens (chunks of several sequences concatenated), N(0,1), fp16
+    [n_tokens][Hq][D]."""
+    rng = rng_for(w, _S_Q, layer, 100 + stream)
+    return to_fp16(rng.standard_normal((n_tokens, w.num_q_heads, w.head_dim)))
+
+
 def cu_seqlens(counts) -> np.ndarray:
     counts = np.asarray(counts, np.int64)
     out = np.zeros(len(counts) + 1, np.int32)
