@@ -300,6 +300,7 @@ def run_kvq(args, rank, world, local_rank):
     cache.close()
     append = run_append_bench(dev) if rank == 0 else None
     plain = run_plain_decode_bench(dev) if rank == 0 else None
+    prefill = run_prefill_bench(dev) if rank == 0 else None
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -332,6 +333,7 @@ def run_kvq(args, rank, world, local_rank):
         "bytes_per_launch": dec_b, "timing": dec_how}
     line["append"] = append
     line["plain_int4"] = plain
+    line["prefill"] = prefill
     line["clocks"] = clk.result
     return line
 
@@ -445,6 +447,81 @@ def run_plain_decode_bench(dev, reps=10):
     res["how"] = ("graph of 36 decode calls over 4 layer pools of the qwen3_4b_decode shape, "
                   "b = 128 (rotated) and b = 1 (plain INT4)")
     return res
+
+
+def prefill_flops(lengths_after, chunks, num_q_heads):
+    """Algorithmic FLOPs of causal chunked prefill: 4 * 128 per (query row, visible token)
+    (q.k and p.v, a multiply and an add per channel each)."""
+    total = 0
+    for L, C in zip(lengths_after, chunks):
+        first = int(L) - int(C) + 1          # visible tokens of the chunk's first query
+        total += (first + first + int(C) - 1) * int(C) // 2
+    return total * num_q_heads * 4 * 128
+
+
+def run_prefill_bench(dev, reps=5):
+    """Chunked prefill (kvq_prefill_attention) on the chunked_prefill workload: 16 x 512
+    chunk tokens over 3584 cached ones, alternating two layer pools; device time per call
+    from events around a graph of the calls."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    w = workloads.WORKLOADS["chunked_prefill"]
+    L0 = np.asarray(w.context, np.int32)
+    B, H, HQ, S, NL = w.batch, w.num_kv_heads, w.num_q_heads, w.page_size, w.num_layers
+    chunk = np.full(B, w.new_tokens, np.int32)
+    cap = L0 + chunk
+    P = workloads.pool_pages(w, cap)
+    mp = int((cap.max() + S - 1) // S)
+    desc = kvq.Desc(NL, H, HQ, 128, w.block, S, P, B, mp)
+    cache, pt = kvq.alloc_pages(desc, cap, None)
+    ptd = torch.from_numpy(pt).to(dev)
+    zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+    cu_all = torch.from_numpy(workloads.cu_seqlens(cap)).to(dev)
+    for layer in range(NL):
+        kp = workloads.kv_rows_torch(w, layer, 0, int(cap.sum()), stream=1, device=dev)
+        vp = workloads.kv_rows_torch(w, layer, 1, int(cap.sum()), stream=1, device=dev)
+        kvq.rotate_quant_append(cache, layer, kp, vp, cu_all, zeros, ptd)
+        del kp, vp
+    T = int(chunk.sum())
+    q = torch.stack([torch.from_numpy(workloads.q_rows_chunk(w, layer, T)) for layer in range(NL)]).to(dev)
+    out = torch.empty_like(q)
+    cu_q = torch.from_numpy(workloads.cu_seqlens(chunk)).to(dev)
+    lens = torch.from_numpy(cap).to(dev)
+    calls = 4
+    side = torch.cuda.Stream(device=dev)
+    kvq.prefill_attention(cache, 0, q[0], cu_q, lens, ptd, out=out[0])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(calls):
+            kvq.prefill_attention(cache, i % NL, q[i % NL], cu_q, lens, ptd, out=out[i % NL])
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / (reps * calls)
+    assert kvq.get_device_status(cache) == 0
+    del g
+    cache.close()
+    fl = prefill_flops(cap, chunk, HQ)
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+        kind = "measured bf16 dense (burst)"
+    except Exception:
+        peak, kind = 1590.0, "fallback bf16 dense"
+    tf = fl / (us * 1e-6) / 1e12
+    return {"us_per_call": round(us, 2), "tflops": round(tf, 1), "peak_tflops": peak,
+            "frac": round(tf / peak, 4), "peak_kind": kind, "flops_per_call": fl,
+            "workload": "chunked_prefill: 16 sequences x 512-token chunk after 3584 cached "
+                        "tokens, Qwen3-4B heads (8 KV / 32 q), b = 128, page 16",
+            "note": "algorithmic FLOPs 4*128 per (query row, visible token); the kernel runs "
+                    "QK^T as three int8 slices and PV as fp16 hi+lo on mma.sync"}
 
 
 # ------------------------------------------------------------- CPU oracle arm --

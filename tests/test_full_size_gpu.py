@@ -138,3 +138,46 @@ def test_prefill_append_full_size(block):
     """8 x 8192 new tokens in one append call, then decode over them (b = 1 is plain INT4)."""
     w = W["prefill_append"]
     _full_size_parity(w, block, 103 + block)
+
+
+def test_chunked_prefill_full_size():
+    """16 sequences x a 512-token chunk after 3584 cached tokens (one layer): sampled query
+    rows of the chunk against the oracle (query i of a chunk is the one query of a chunk of
+    length 1 over the first L - C + i + 1 tokens)."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    w = W["chunked_prefill"]
+    dev = torch.device("cuda")
+    L0 = workloads.context_lengths(w)
+    chunk = np.full(w.batch, w.new_tokens, np.int32)
+    cap = L0 + chunk
+    S, H = w.page_size, w.num_kv_heads
+    P = workloads.pool_pages(w, cap)
+    mp = int((cap.max() + S - 1) // S)
+    desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, w.batch, mp)
+    pool = torch.zeros(kvq.pool_bytes(desc), dtype=torch.uint8, device=dev)
+    cache, pt = kvq.alloc_pages(desc, cap, None, pool=pool)
+    ptd = torch.from_numpy(pt).to(dev)
+    k = workloads.kv_rows_torch(w, 0, 0, int(cap.sum()), stream=1, device=dev)
+    v = workloads.kv_rows_torch(w, 0, 1, int(cap.sum()), stream=1, device=dev)
+    kvq.rotate_quant_append(cache, 0, k, v, torch.from_numpy(workloads.cu_seqlens(cap)).to(dev),
+                            torch.zeros(w.batch, dtype=torch.int32, device=dev), ptd)
+    cu_q = workloads.cu_seqlens(chunk)
+    q = workloads.q_rows_chunk(w, 0, int(cu_q[-1]))
+    out = kvq.prefill_attention(cache, 0, torch.from_numpy(q).to(dev),
+                                torch.from_numpy(cu_q).to(dev), torch.from_numpy(cap).to(dev), ptd)
+    torch.cuda.synchronize()
+    assert kvq.get_device_status(cache) == 0
+    host_pool = pool.cpu().numpy()
+    host_out = out.float().cpu().numpy()
+    cache.close()
+    g = oracle.Geometry(1, H, w.num_q_heads, 128, w.block, S, P, mp)
+    rng = np.random.default_rng(104)
+    for b in rng.choice(w.batch, 3, replace=False):
+        for i in sorted({0, int(chunk[b]) - 1, *rng.integers(0, int(chunk[b]), 4).tolist()}):
+            row = int(cu_q[b]) + i
+            pos = int(cap[b] - chunk[b]) + i
+            ref = oracle.prefill_attention(g, host_pool, 0, q[row:row + 1], np.array([0, 1], np.int32),
+                                           np.array([pos + 1], np.int32), pt[b:b + 1])
+            check_outputs(host_out[row:row + 1], ref, f"chunked prefill b={b} i={i}")

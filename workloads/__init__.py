@@ -70,6 +70,12 @@ WORKLOADS = {
     "ragged": Workload("ragged", num_layers=1, batch=256, num_kv_heads=8, num_q_heads=32,
                        block=128, page_size=16, dist="lognormal_outliers", seed=3,
                        ragged=(128, 8192), new_tokens=1, pool_factor=1.2, permute_pages=True),
+    # Chunked prefill on the Qwen3-4B shape: 16 sequences, a 512-token chunk appended after
+    # 3584 cached tokens, the chunk's queries attending causally.
+    "chunked_prefill": Workload("chunked_prefill", num_layers=2, batch=16, num_kv_heads=8,
+                                num_q_heads=32, block=128, page_size=16,
+                                dist="lognormal_outliers", seed=5, context=[3584] * 16,
+                                new_tokens=512),
     # Prefill-append stress: 8 x 8192 new tokens in one call, b swept over 32/64/128.
     "prefill_append": Workload("prefill_append", num_layers=1, batch=8, num_kv_heads=8,
                                num_q_heads=32, block=128, page_size=16, dist="student_t3",
