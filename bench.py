@@ -603,6 +603,31 @@ def run_kernel_case(which, calls):
 
     import bit_paged_kv_diag_b200 as kvq
     dev = torch.device("cuda", 0)
+    if which == "prefill":
+        # 16 sequences, a 128-token chunk after 896 cached tokens (chunked_prefill's heads).
+        w = workloads.WORKLOADS["chunked_prefill"]
+        B, H, S = w.batch, w.num_kv_heads, w.page_size
+        chunk = np.full(B, 128, np.int32)
+        cap = np.full(B, 1024, np.int32)
+        P = workloads.pool_pages(w, cap)
+        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S))
+        cache, pt = kvq.alloc_pages(desc, cap, None)
+        ptd = torch.from_numpy(pt).to(dev)
+        k = workloads.kv_rows_torch(w, 0, 0, int(cap.sum()), stream=1, device=dev)
+        v = workloads.kv_rows_torch(w, 0, 1, int(cap.sum()), stream=1, device=dev)
+        kvq.rotate_quant_append(cache, 0, k, v, torch.from_numpy(workloads.cu_seqlens(cap)).to(dev),
+                                torch.zeros(B, dtype=torch.int32, device=dev), ptd)
+        cu_q = torch.from_numpy(workloads.cu_seqlens(chunk)).to(dev)
+        q = torch.from_numpy(workloads.q_rows_chunk(w, 0, int(chunk.sum()))).to(dev)
+        lens = torch.from_numpy(cap).to(dev)
+        torch.cuda.synchronize()
+        for _ in range(calls):
+            kvq.prefill_attention(cache, 0, q, cu_q, lens, ptd)
+        torch.cuda.synchronize()
+        assert kvq.get_device_status(cache) == 0
+        cache.close()
+        print(json.dumps({"kernel_case": which, "calls": calls, "ok": True}))
+        return
     if which == "append":
         w = workloads.WORKLOADS["prefill_append"]
         B, H, S, T = w.batch, w.num_kv_heads, w.page_size, w.batch * w.new_tokens
@@ -651,7 +676,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["decode", "append"], default=None,
+    ap.add_argument("--kernel-case", choices=["decode", "append", "prefill"], default=None,
                     help="run one small case of one kernel (for ncu captures) and exit")
     ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()

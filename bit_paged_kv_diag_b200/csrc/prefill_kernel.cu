@@ -109,7 +109,8 @@ __device__ __forceinline__ void issue_tile(int t, int b, int h, int L, uint32_t 
 // cut it into three int8 slices q' = M/64 (q1 + q2/128 + q3/16384), M the power of two >=
 // max |q'|, and store the slices in A-fragment order: qs[s][jj][row][kappa] with, inside
 // k-step jj, kappa = 4c + e <-> channel 32c + 8jj + 2e and kappa = 16 + 4c + e <-> channel
-// 32c + 8jj + 2e + 1.  Returns M / 1024 (the score scale of the row; K codes enter the MMA
+// 32c + 8jj + 2e + 1.  The two 16-byte halves of a 32-byte row swap places on rows with
+// bit 2 set, so that ldmatrix's 8 rows fall in distinct banks.  Returns M / 1024 (the score scale of the row; K codes enter the MMA
 // times 16).
 __device__ __forceinline__ float prep_q_row(const __half* qrow, bool valid, uint8_t* qs, int row,
                                             int lane, const PrefillParams& p) {
@@ -164,10 +165,11 @@ __device__ __forceinline__ float prep_q_row(const __half* qrow, bool valid, uint
 #pragma unroll
   for (int s = 0; s < 3; s++) {
     uint8_t* r = qs + ((s * 4 + jj) * kRows + row) * 32;
+    const int sw = ((row >> 2) & 1) * 16;  // swizzle of the 16-byte halves
     const uint16_t ev = static_cast<uint16_t>((ms[s][0] & 0xFFu) | ((ms[s][2] & 0xFFu) << 8));
     const uint16_t od = static_cast<uint16_t>((ms[s][1] & 0xFFu) | ((ms[s][3] & 0xFFu) << 8));
-    *reinterpret_cast<uint16_t*>(r + 4 * c + e0) = ev;
-    *reinterpret_cast<uint16_t*>(r + 16 + 4 * c + e0) = od;
+    *reinterpret_cast<uint16_t*>(r + (0 ^ sw) + 4 * c + e0) = ev;
+    *reinterpret_cast<uint16_t*>(r + (16 ^ sw) + 4 * c + e0) = od;
   }
   return M * (1.0f / 1024.0f);
 }
@@ -180,7 +182,8 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
   uint8_t* ring = smem;                                        // [3][4224]
   uint8_t* qs = ring + kStagesP * kSlotBytesP;                 // [3][4][64][32] int8
   float* sfr = reinterpret_cast<float*>(qs + 3 * 4 * kRows * 32);  // [64] row scales
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sfr + kRows);   // full[3], empty[3]
+  uint8_t* vst = reinterpret_cast<uint8_t*>(sfr + kRows);      // [2][32 tokens][256 B] fp16 V
+  uint64_t* bars = reinterpret_cast<uint64_t*>(vst + 2 * kTileTokens * 256);  // full[3], empty[3]
   int32_t* preq = reinterpret_cast<int32_t*>(bars + 2 * kStagesP);  // [batch + 1]
   __shared__ int warp_sum[kWarpsP];
   __shared__ int running;
@@ -278,16 +281,11 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
 #pragma unroll
   for (int i = 0; i < 16; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
   float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.0f, l1 = 0.0f;
-  // V conversion constants of this lane's channel parity (channel 8cn + g).
-  const uint32_t vsel = static_cast<uint32_t>(g >> 1) | ((4u + static_cast<uint32_t>(g >> 1)) << 8);
-  const uint32_t vmask = (g & 1) ? 0x00F000F0u : 0x000F000Fu;
-  const uint32_t vxor = (g & 1) ? 0x64806480u : 0x64086408u;
-  const uint32_t vmul = (g & 1) ? 0x2C002C00u : 0x3C003C00u;  // 1/16 or 1
-  const uint32_t vadd = (g & 1) ? 0xD480D480u : 0xE408E408u;  // -72 or -1032
   const uint32_t qs_s = smem_addr(qs);
   // ldmatrix row address of this lane inside a [64][32] slice block: matrix L/8.
   const int lm = lane >> 3, lr = lane & 7;
-  const uint32_t a_off = static_cast<uint32_t>((16 * w + lr + (lm & 1) * 8) * 32 + (lm >> 1) * 16);
+  const int a_row = 16 * w + lr + (lm & 1) * 8;
+  const uint32_t a_off = static_cast<uint32_t>(a_row * 32 + (((lm >> 1) ^ ((a_row >> 2) & 1)) * 16));
   bool dead = false;
 
   for (int t = 0; t < ntile; t++) {
@@ -298,6 +296,35 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
       else dead = true;
     }
     const uint8_t* base = ring + slot * kSlotBytesP;
+    // The tile's V codes as fp16, once per CTA: warp w converts tokens 8w..8w+7 into the
+    // stage t % 2 ([token][channel], the 16-byte chunk index XOR (token & 7), so ldmatrix's
+    // 8 rows fall in distinct banks).  The barrier below also tells every warp that all
+    // warps are done with the stage's previous tile.
+    uint8_t* vs = vst + (t & 1) * (kTileTokens * 256);
+    if (!dead) {
+      const int tau = 8 * w + (lane >> 2), part = lane & 3;  // channels 32part .. 32part+31
+      const uint4 cw = *reinterpret_cast<const uint4*>(base + tok_base<SEFF>(tau) + SEFF * 64 +
+                                                       (tau % SEFF) * 64 + 16 * part);
+      const uint32_t wds[4] = {cw.x, cw.y, cw.z, cw.w};
+      uint32_t hv[16];
+#pragma unroll
+      for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          // byte k of word i: channels 32part + 8i + 2k (low nibble), +1 (high nibble)
+          uint32_t x = prmt(wds[i], 0u, static_cast<uint32_t>(k) | (static_cast<uint32_t>(k) << 8) | 0x4040u);
+          x = lop3_and_xor(x, 0x00F0000Fu, 0x64806408u);
+          asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(x) : "r"(x), "r"(0x2C003C00u), "r"(0xD480E408u));
+          hv[4 * i + k] = x;
+        }
+#pragma unroll
+      for (int i = 0; i < 4; i++) {  // 16-byte chunk 4part + i = channels 8(4part + i) ..
+        const int chunk = (4 * part + i) ^ (tau & 7);
+        *reinterpret_cast<uint4*>(vs + tau * 256 + chunk * 16) =
+            make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+      }
+    }
+    __syncthreads();
     if (!dead) {
       // K codes of tokens 8nt + g (bytes 16c..16c+15 of the row) and the K/V scales of
       // tokens 8nt + 2c, 8nt + 2c + 1.
@@ -394,30 +421,19 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
                       ah[2], al[2]);
         split_hi_lo_p(sc[2 * kk + 1][2] * sv[2 * kk + 1][0], sc[2 * kk + 1][3] * sv[2 * kk + 1][1],
                       ah[3], al[3]);
-        // V rows of tokens 16kk + 2c, +1 (b0) and 16kk + 8 + 2c, +1 (b1).
-        const int ta = 16 * kk + 2 * c, tb = ta + 8;
-        const uint8_t* va0 = base + tok_base<SEFF>(ta) + SEFF * 64 + (ta % SEFF) * 64;
-        const uint8_t* va1 = base + tok_base<SEFF>(ta + 1) + SEFF * 64 + ((ta + 1) % SEFF) * 64;
-        const uint8_t* vb0 = base + tok_base<SEFF>(tb) + SEFF * 64 + (tb % SEFF) * 64;
-        const uint8_t* vb1 = base + tok_base<SEFF>(tb + 1) + SEFF * 64 + ((tb + 1) % SEFF) * 64;
+        // B fragments of 2 channel n-tiles per ldmatrix: matrices (tokens 16kk..+7 |
+        // 16kk+8..+15) x (n-tile cp | cp + 1), transposed.
 #pragma unroll
-        for (int q4 = 0; q4 < 4; q4++) {  // channel n-tiles 4q4 .. 4q4 + 3
-          const uint4 wa0 = *reinterpret_cast<const uint4*>(va0 + 16 * q4);
-          const uint4 wa1 = *reinterpret_cast<const uint4*>(va1 + 16 * q4);
-          const uint4 wb0 = *reinterpret_cast<const uint4*>(vb0 + 16 * q4);
-          const uint4 wb1 = *reinterpret_cast<const uint4*>(vb1 + 16 * q4);
-          const uint32_t xa0[4] = {wa0.x, wa0.y, wa0.z, wa0.w}, xa1[4] = {wa1.x, wa1.y, wa1.z, wa1.w};
-          const uint32_t xb0[4] = {wb0.x, wb0.y, wb0.z, wb0.w}, xb1[4] = {wb1.x, wb1.y, wb1.z, wb1.w};
-#pragma unroll
-          for (int k4 = 0; k4 < 4; k4++) {
-            const int cn = 4 * q4 + k4;  // channels 8cn..8cn+7; this lane's is 8cn + g
-            uint32_t b0 = lop3_and_xor(prmt(xa0[k4], xa1[k4], vsel), vmask, vxor);
-            uint32_t b1 = lop3_and_xor(prmt(xb0[k4], xb1[k4], vsel), vmask, vxor);
-            asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(b0) : "r"(b0), "r"(vmul), "r"(vadd));
-            asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(b1) : "r"(b1), "r"(vmul), "r"(vadd));
-            mma_16816(o[cn], ah[0], ah[1], ah[2], ah[3], b0, b1);
-            mma_16816(o[cn], al[0], al[1], al[2], al[3], b0, b1);
-          }
+        for (int cp = 0; cp < 16; cp += 2) {
+          const int vtok = 16 * kk + (lm & 1) * 8 + lr;
+          const int vch = cp + (lm >> 1);  // 16-byte chunk = channel n-tile
+          uint32_t b0a, b1a, b0b, b1b;
+          ldsm_x4_trans(smem_addr(vs) + static_cast<uint32_t>(vtok * 256 + ((vch ^ (vtok & 7)) * 16)),
+                        b0a, b1a, b0b, b1b);
+          mma_16816(o[cp], ah[0], ah[1], ah[2], ah[3], b0a, b1a);
+          mma_16816(o[cp], al[0], al[1], al[2], al[3], b0a, b1a);
+          mma_16816(o[cp + 1], ah[0], ah[1], ah[2], ah[3], b0b, b1b);
+          mma_16816(o[cp + 1], al[0], al[1], al[2], al[3], b0b, b1b);
         }
       }
     }
@@ -531,6 +547,7 @@ size_t prefill_smem(int max_batch) {
   size_t s = static_cast<size_t>(kStagesP) * kSlotBytesP;  // ring
   s += 3 * 4 * kRows * 32;                                  // q slices
   s += sizeof(float) * kRows;                               // row scales
+  s += 2 * kTileTokens * 256;                               // fp16 V stages
   s += sizeof(uint64_t) * 2 * kStagesP;                     // barriers
   s += static_cast<size_t>(max_batch + 1) * sizeof(int32_t);  // query-block prefix
   s += 128;                                                  // alignment slack
