@@ -868,14 +868,11 @@ __device__ __forceinline__ NewRow quantise_new_row(uint2 raw, int lane, const De
   return r;
 }
 
-// The new token of unit (b, h) (its raw K and V rows kraw, vraw as loaded by
-// load_new_row): rotate and quantise the rows, store them at
-// position seq_lens[b] of the pool (skipped, with the status flagged, when the position or
-// its page is out of range) and, in the block layout of one token, into the warp's patch
-// buffer (shared memory): [K codes 64 B][V codes 64 B][K scale][V scale].  Returns
-// whether the rows are stored and belong in the decode.
-__device__ __forceinline__ bool fused_append(int b, int h, int lane, uint8_t* patch, uint2 kraw,
-                                             uint2 vraw, const DecodeParams& p) {
+// The new token of a unit (its raw K and V rows kraw, vraw as loaded by load_new_row):
+// rotate and quantise the rows into the warp's patch buffer (shared memory), in the block
+// layout of one token: [K codes 64 B][V codes 64 B][K scale][V scale].
+__device__ __forceinline__ void fused_quantise(uint2 kraw, uint2 vraw, int lane, uint8_t* patch,
+                                               const DecodeParams& p) {
   const NewRow kr = quantise_new_row(kraw, lane, p);
   const NewRow vr = quantise_new_row(vraw, lane, p);
   *reinterpret_cast<uint16_t*>(patch + 2 * lane) = static_cast<uint16_t>(kr.codes16);
@@ -885,6 +882,13 @@ __device__ __forceinline__ bool fused_append(int b, int h, int lane, uint8_t* pa
     *reinterpret_cast<uint16_t*>(patch + 130) = static_cast<uint16_t>(vr.scale);
   }
   __syncwarp();
+}
+
+// Store the patch buffer's token of unit (b, h) at position seq_lens[b] of the pool
+// (skipped, with the status flagged, when the position or its page is out of range).
+// Returns whether it is stored and belongs in the decode.
+__device__ __forceinline__ bool fused_store(int b, int h, int lane, const uint8_t* patch,
+                                            const DecodeParams& p) {
   const int pos = __ldg(p.seq_lens + b);
   const int S = p.page_size;
   const int lp = pos >> p.page_shift;
@@ -894,11 +898,13 @@ __device__ __forceinline__ bool fused_append(int b, int h, int lane, uint8_t* pa
   const int slot = pos & (S - 1);
   uint8_t* blk = const_cast<uint8_t*>(p.pool_layer) + (static_cast<size_t>(page) * p.num_kv_heads + h) *
                                       (static_cast<size_t>(S) * (kD + 4));
-  *reinterpret_cast<uint16_t*>(blk + slot * 64 + 2 * lane) = static_cast<uint16_t>(kr.codes16);
-  *reinterpret_cast<uint16_t*>(blk + S * 64 + slot * 64 + 2 * lane) = static_cast<uint16_t>(vr.codes16);
+  const uint16_t kc = *reinterpret_cast<const uint16_t*>(patch + 2 * lane);
+  const uint16_t vc = *reinterpret_cast<const uint16_t*>(patch + 64 + 2 * lane);
+  *reinterpret_cast<uint16_t*>(blk + slot * 64 + 2 * lane) = kc;
+  *reinterpret_cast<uint16_t*>(blk + S * 64 + slot * 64 + 2 * lane) = vc;
   if (lane == 0) {
-    *reinterpret_cast<uint16_t*>(blk + S * 128 + slot * 2) = static_cast<uint16_t>(kr.scale);
-    *reinterpret_cast<uint16_t*>(blk + S * 130 + slot * 2) = static_cast<uint16_t>(vr.scale);
+    *reinterpret_cast<uint16_t*>(blk + S * 128 + slot * 2) = *reinterpret_cast<const uint16_t*>(patch + 128);
+    *reinterpret_cast<uint16_t*>(blk + S * 130 + slot * 2) = *reinterpret_cast<const uint16_t*>(patch + 130);
   }
   return true;
 }
@@ -1053,18 +1059,22 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   auto is_ul = [&](const Unit& u) { return u.b == ul.b && u.h == ul.h; };
   const bool two_edges = has_tiles && !is_uf(ul);
 
-  // Fused append: the new K/V rows of the first unit, if this warp holds its last tile,
-  // are loaded before the wait (the inputs of an append are complete when the previous
-  // kernel lets this one start); later units load theirs at their segment's start.
-  uint2 kraw0 = make_uint2(0u, 0u), vraw0 = make_uint2(0u, 0u);
+  // Fused append: if this warp holds the last tile of its first unit and that unit's q
+  // comes from a CTA table (its own fragment table is then free as the patch buffer), the
+  // unit's new K/V rows are loaded, rotated and quantised before the wait -- the inputs
+  // of an append are complete when the previous kernel lets this one start, and this is
+  // pure arithmetic into shared memory; the pool store waits.  Other units do it at their
+  // segment's start.
+  bool pre_quantised = false;
   if constexpr (FUSED) {
-    if (x < X1) {
+    if (x < X1 && (is_uf(cu) || is_ul(cu))) {
       const int seg_end0 = min(X1, cu.U + cu.n);
       const int xl0 = x + kWarps * ((seg_end0 - x + kWarps - 1) / kWarps - 1);
       if (xl0 == cu.U + cu.n - 1) {
         const size_t row = (static_cast<size_t>(cu.b) * p.num_kv_heads + cu.h) * kD;
-        kraw0 = load_new_row(p.k_new + row, lane);
-        vraw0 = load_new_row(p.v_new + row, lane);
+        fused_quantise(load_new_row(p.k_new + row, lane), load_new_row(p.v_new + row, lane), lane,
+                       reinterpret_cast<uint8_t*>(frag), p);
+        pre_quantised = true;
       }
     }
   }
@@ -1154,13 +1164,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       const int xl = x + kWarps * (nt - 1);  // this warp's last tile of the unit
       uint8_t* patch = reinterpret_cast<uint8_t*>(frag);  // free until the next unit's q
       if (xl == cu.U + cu.n - 1 && !dead) {
-        uint2 kraw = kraw0, vraw = vraw0;
-        if (x != X0 + w) {  // not the warp's first unit: load now
+        if (!(pre_quantised && x == X0 + w)) {
           const size_t row = (static_cast<size_t>(cu.b) * p.num_kv_heads + cu.h) * kD;
-          kraw = load_new_row(p.k_new + row, lane);
-          vraw = load_new_row(p.v_new + row, lane);
+          fused_quantise(load_new_row(p.k_new + row, lane), load_new_row(p.v_new + row, lane), lane,
+                         patch, p);
         }
-        new_ok = fused_append(cu.b, cu.h, lane, patch, kraw, vraw, p);
+        new_ok = fused_store(cu.b, cu.h, lane, patch, p);
         if (lane == 0) *reinterpret_cast<int*>(patch + 132) = cu.L - 1 - (xl - cu.U) * kTileTokens;
         __syncwarp();
       }
