@@ -596,9 +596,11 @@ def run_reference(args, rank, world):
 # ------------------------------------------------------------ profiling cases --
 def run_kernel_case(which, calls):
     """A small case of one kernel for ncu captures: ``decode`` = decode attention on one
-    layer of the Qwen3-4B-shaped workload (69 MB of cache); ``append`` = the prefill-append
-    call (8 x 8192 tokens, b = 128; 268 MB read, 69 MB written).  The kernel is launched
-    ``calls`` times after the setup."""
+    layer of the Qwen3-4B-shaped workload (69 MB of cache); ``fused`` = the same with the
+    step's one-token append fused in; ``append`` = the prefill-append call (8 x 8192
+    tokens, b = 128; 268 MB read, 69 MB written); ``prefill`` = chunked-prefill attention
+    (16 x 128-token chunks after 896 cached tokens).  The kernel is launched ``calls``
+    times after the setup."""
     import torch
 
     import bit_paged_kv_diag_b200 as kvq
@@ -659,9 +661,15 @@ def run_kernel_case(which, calls):
         del kp, vp
         q = workloads.q_rows_torch(w, 0, device=dev)
         lens = torch.from_numpy(cap).to(dev)
+        kn = workloads.kv_rows_torch(w, 0, 0, B, stream=2, device=dev)
+        vn = workloads.kv_rows_torch(w, 0, 1, B, stream=2, device=dev)
+        lens_before = torch.from_numpy(L).to(dev)
         torch.cuda.synchronize()
         for _ in range(calls):
-            kvq.decode_attention(cache, 0, q, lens, ptd)
+            if which == "fused":
+                kvq.append_decode_attention(cache, 0, kn, vn, q, lens_before, ptd)
+            else:
+                kvq.decode_attention(cache, 0, q, lens, ptd)
     torch.cuda.synchronize()
     assert kvq.get_device_status(cache) == 0
     cache.close()
@@ -676,7 +684,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["decode", "append", "prefill"], default=None,
+    ap.add_argument("--kernel-case", choices=["decode", "fused", "append", "prefill"], default=None,
                     help="run one small case of one kernel (for ncu captures) and exit")
     ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()
