@@ -117,6 +117,25 @@ class ClockSampler:
         return False
 
 
+# ------------------------------------------------------------ rank plumbing --
+def max_over_ranks(value, world, device=None):
+    """The largest of a per-rank value (a device time) over all ranks; every rank calls it
+    with the same world and gets the max back.  NCCL (CUDA device) or gloo (CPU)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world, bytes_per_rank_step, ms_per_step):
+    """Weak scaling: every rank runs the whole workload; the job's throughput is all ranks'
+    bytes over the slowest rank's time."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------- GPU arm --
 def run_kvq(args, rank, world, local_rank):
     import torch
@@ -205,12 +224,7 @@ def run_kvq(args, rank, world, local_rank):
         t1.record()
         torch.cuda.synchronize()
     barrier()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        import torch.distributed as dist
-        tms = torch.tensor([ms], device=dev)
-        dist.all_reduce(tms, op=dist.ReduceOp.MAX)
-        ms = float(tms.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
 
     # The same step as separate append and decode calls (2 launches per layer).
     sgraph = torch.cuda.CUDAGraph()
@@ -225,7 +239,7 @@ def run_kvq(args, rank, world, local_rank):
         sgraph.replay()
     s1.record()
     torch.cuda.synchronize()
-    sep_ms = s0.elapsed_time(s1) / max(3, args.steps // 2)
+    sep_ms = max_over_ranks(s0.elapsed_time(s1) / max(3, args.steps // 2), world, dev)
     del sgraph
 
     # Decode-attention launches: a graph of the 36 decode calls back to back, timed with
@@ -261,7 +275,7 @@ def run_kvq(args, rank, world, local_rank):
     dec_b = decode_bytes(cap, H, HQ, S)
     app_b = append_bytes(B, H)
     step_bytes = NL * (dec_b + app_b)
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, ms_step)
     peak, peak_kind = _peaks()
 
     # End to end through the C ABI with host buffers: per step, H2D of q and the step's
@@ -287,12 +301,7 @@ def run_kvq(args, rank, world, local_rank):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        import torch.distributed as dist
-        tms = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tms, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tms.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
     d2h = hout.numel() * 2
 
@@ -315,11 +324,11 @@ def run_kvq(args, rank, world, local_rank):
                    "graph": "one CUDA graph per step",
                    "step": "per layer one kvq_append_decode_attention (fused 1-token append + decode)"},
         "step_separate_calls": {"ms_per_step": round(sep_ms, 5),
-                                "value": round(world * step_bytes / (sep_ms * 1e-3) / 1e9, 1),
+                                "value": round(whole_job_gbs(world, step_bytes, sep_ms), 1),
                                 "how": "per layer kvq_rotate_quant_append then kvq_decode_attention"},
         "gpu_launches": args.steps * NL,  # per layer: one fused append + decode launch
         "device_status": status,
-        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "e2e": {"value": round(whole_job_gbs(world, step_bytes, e2e_ms), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": round(e2e_ms, 5)},
     }
