@@ -75,7 +75,7 @@ def host_inputs(case: Case):
     return kp, vp, kn, vn, q
 
 
-class GpuRun:
+class CudaRun:
     """The CUDA path through the C ABI: alloc, prefill append, step append, decode (or,
     with fused=True and one new token per sequence, the step's append and the decode in
     one kvq_append_decode_attention call)."""
@@ -168,7 +168,7 @@ def check_outputs(gpu_out, ref_out, what=""):
 def full_parity(case: Case, softmax_scale=0.0, fused=False):
     """Run everything at a size the oracle finishes in seconds; assert all bars."""
     kp, vp, kn, vn, q = host_inputs(case)
-    run = GpuRun(case, kp, vp, kn, vn, q, softmax_scale, fused=fused)
+    run = CudaRun(case, kp, vp, kn, vn, q, softmax_scale, fused=fused)
     try:
         assert run.status == 0, f"device status {run.status}"
         pt_ref = oracle.assign_pages(case.capacity, case.w.page_size, case.num_pages,

@@ -165,9 +165,9 @@ def test_repeated_decode_is_bit_identical():
     import bit_paged_kv_diag_b200 as kvq
     w = W["long_context"]
     case = make_case(w, [5000, 31, 1, 2600], [1, 1, 1, 1])
-    from harness import GpuRun, host_inputs
+    from harness import CudaRun, host_inputs
     kp, vp, kn, vn, q = host_inputs(case)
-    run = GpuRun(case, kp, vp, kn, vn, q)
+    run = CudaRun(case, kp, vp, kn, vn, q)
     try:
         pt = torch.from_numpy(run.page_table).cuda()
         lens = torch.as_tensor(run.lens_after).cuda()

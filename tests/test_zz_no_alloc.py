@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 import workloads
-from harness import ATOL, RTOL, GpuRun, host_inputs, make_case
+from harness import ATOL, RTOL, CudaRun, host_inputs, make_case
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +28,7 @@ def test_noalloc_decode_matches_handle_decode_twice(name, lengths):
     w = workloads.WORKLOADS[name]
     case = make_case(w, lengths, [1] * len(lengths))
     kp, vp, kn, vn, q = host_inputs(case)
-    run = GpuRun(case, kp, vp, kn, vn, q)
+    run = CudaRun(case, kp, vp, kn, vn, q)
     try:
         d = case.desc()
         qd = torch.as_tensor(q).cuda()
