@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
   const int r0 = 16 * w + g, r1 = r0 + 8;
   const float sf0 = sfr[r0], sf1 = sfr[r1];
   const int pos0 = L - C + tok_first + r0 / G, pos1 = L - C + tok_first + r1 / G;
+  const int pos_min = L - C + tok_first + (16 * w) / G;  // the warp's first row's position
   float o[16][4];
 #pragma unroll
   for (int i = 0; i < 16; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
@@ -345,15 +346,17 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
         sv[nt][0] = tpos < L ? vf.x : 0.0f;
         sv[nt][1] = tpos + 1 < L ? vf.y : 0.0f;
       }
-      // Scores: three int8 slices, accumulated in fp32 with weights 1, 2^-7, 2^-14.
+      // Scores: three int8 slices.  Slice 2's accumulators are multiplied by 128 and slice
+      // 3's MMAs accumulate on top of them, so acc = acc2 * 128 + acc3 exactly (|acc_s| <=
+      // 2^20 fits); then s = s1 + acc * 2^-14.
       float sc[4][4];
-#pragma unroll
-      for (int nt = 0; nt < 4; nt++) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
+      int acc[4][4];
 #pragma unroll
       for (int s = 0; s < 3; s++) {
-        int acc[4][4];
+        if (s < 2) {
 #pragma unroll
-        for (int nt = 0; nt < 4; nt++) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+          for (int nt = 0; nt < 4; nt++) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+        }
 #pragma unroll
         for (int jj = 0; jj < 4; jj++) {
           uint32_t a0, a1, a2, a3;
@@ -364,24 +367,39 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
             mma_16832_s8(acc[nt], a0, a1, a2, a3, (wv << 4) & 0xF0F0F0F0u, wv & 0xF0F0F0F0u);
           }
         }
-        const float ws = s == 0 ? 1.0f : (s == 1 ? 1.0f / 128.0f : 1.0f / 16384.0f);
 #pragma unroll
         for (int nt = 0; nt < 4; nt++)
 #pragma unroll
-          for (int e = 0; e < 4; e++) sc[nt][e] += static_cast<float>(acc[nt][e]) * ws;
+          for (int e = 0; e < 4; e++) {
+            if (s == 0) sc[nt][e] = static_cast<float>(acc[nt][e]);
+            else if (s == 1) acc[nt][e] *= 128;
+            else sc[nt][e] += static_cast<float>(acc[nt][e]) * (1.0f / 16384.0f);
+          }
       }
-      // Scale, causal mask, row maxima.
+      // Scale, causal mask (only on tiles reaching past the warp's first row), row maxima.
       float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
+      if (t * kTileTokens + kTileTokens - 1 <= pos_min) {
 #pragma unroll
-      for (int nt = 0; nt < 4; nt++)
+        for (int nt = 0; nt < 4; nt++)
 #pragma unroll
-        for (int e = 0; e < 2; e++) {
-          const int tpos = t * kTileTokens + 8 * nt + 2 * c + e;
-          sc[nt][e] = tpos <= pos0 ? sc[nt][e] * (sf0 * sk[nt][e]) : -CUDART_INF_F;
-          sc[nt][2 + e] = tpos <= pos1 ? sc[nt][2 + e] * (sf1 * sk[nt][e]) : -CUDART_INF_F;
-          mx0 = fmaxf(mx0, sc[nt][e]);
-          mx1 = fmaxf(mx1, sc[nt][2 + e]);
-        }
+          for (int e = 0; e < 2; e++) {
+            sc[nt][e] *= sf0 * sk[nt][e];
+            sc[nt][2 + e] *= sf1 * sk[nt][e];
+            mx0 = fmaxf(mx0, sc[nt][e]);
+            mx1 = fmaxf(mx1, sc[nt][2 + e]);
+          }
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < 4; nt++)
+#pragma unroll
+          for (int e = 0; e < 2; e++) {
+            const int tpos = t * kTileTokens + 8 * nt + 2 * c + e;
+            sc[nt][e] = tpos <= pos0 ? sc[nt][e] * (sf0 * sk[nt][e]) : -CUDART_INF_F;
+            sc[nt][2 + e] = tpos <= pos1 ? sc[nt][2 + e] * (sf1 * sk[nt][e]) : -CUDART_INF_F;
+            mx0 = fmaxf(mx0, sc[nt][e]);
+            mx1 = fmaxf(mx1, sc[nt][2 + e]);
+          }
+      }
       mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, 1));
       mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, 1));
@@ -404,12 +422,14 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
         }
       l0 = l0 * al0 + ps0;
       l1 = l1 * al1 + ps1;
+      if (__any_sync(kFullMask, al0 != 1.0f || al1 != 1.0f)) {
 #pragma unroll
-      for (int cn = 0; cn < 16; cn++) {
-        o[cn][0] *= al0;
-        o[cn][1] *= al0;
-        o[cn][2] *= al1;
-        o[cn][3] *= al1;
+        for (int cn = 0; cn < 16; cn++) {
+          o[cn][0] *= al0;
+          o[cn][1] *= al0;
+          o[cn][2] *= al1;
+          o[cn][3] *= al1;
+        }
       }
       // PV: two k-steps of 16 tokens.
 #pragma unroll
