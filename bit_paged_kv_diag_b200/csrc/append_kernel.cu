@@ -8,27 +8,43 @@
 // kernel that rotates, quantises and appends into paged KV blocks without revisiting
 // past tokens).
 //
-// Work decomposition.  Two lanes handle one row (the K row or the V row of one
-// (token, KV head) pair, 128 fp16 channels); a warp handles the K and V rows of 8 pairs.
-// Lane l of a row holds the 16-channel chunks 2j + l (j = 0..3), read with 256-bit loads:
-// channel index bits 0-3 and 5-6 are inside the lane and bit 4 is across the lane pair.
-// So the butterfly stages h = 1, 2, 4, 8, 32, 64 are register-only and stage h = 16 is one
-// warp shuffle.  Stages run in the fixed order h = 1, 2, ..., b/2, each pair (i, i+h) with
-// bit h of i clear becoming (a + c, a - c) as one IEEE fp32 add and one subtract, then one
-// multiply by the fp32 constant nearest 1/sqrt(b): rotated values are bit-exact with any
+// Work decomposition.  Every warp runs its own pipeline: a warp stage is 8 consecutive
+// (token, KV head) pairs, their K rows (2 KB, contiguous in the token-packed input) and V
+// rows (2 KB), brought into a ring of 3 shared-memory slots by two 1-D bulk copies (TMA
+// engine, no multicast) that complete on the slot's mbarrier.  Warps take warp stages
+// gw, gw + W, ... (gw = the global warp index, W = all warps of the persistent grid) and
+// never wait for one another, so their serial parts (the row's scale, the stores) spread
+// out in time; no register holds prefetched data.  Two lanes handle one row (the K or V
+// row of one pair, 128 fp16 channels): lane l holds channels [64l, 64l + 64) as 8 chunks
+// of 8 channels.
+//
+// Bank-conflict-free reads.  A lane reads its chunks in the order c = t ^ rho (t = 0..7,
+// rho = lane & 7): the 8 lanes of a quarter warp then touch 8 different 16-byte bank
+// groups.  Register slot t holds chunk t ^ rho, so the butterfly stages that pair chunks
+// (h = 8, 16, 32: chunk bits 0-2) pair slots t and t ^ k as well; whether slot t holds the
+// lower or the upper chunk of the pair depends on rho, and each output is one fma with a
+// +-1 multiplier (fma(a, 1, c) = a + c and fma(c, -1, a) = a - c, rounded once: the IEEE
+// sum and difference).  Stages h = 1, 2, 4 are inside a chunk.  Only b = 128 has a stage
+// across the lane pair (h = 64): lane 1's slot t ^ 1 holds the partner of lane 0's slot t
+// (their rho differ in bit 0); after one exchange lane 0 keeps the sums (channels
+// [0, 64)) and lane 1 the differences (channels [64, 128)), in the same slot order.
+//
+// Stages run in the fixed order h = 1, 2, ..., b/2, each pair (i, i + h) with bit h of i
+// clear becoming (a + c, a - c) as one IEEE fp32 add and one subtract, then one multiply
+// by the fp32 constant nearest 1/sqrt(b): rotated values are bit-exact with any
 // implementation of that fixed-order butterfly.  Pairs of channels go through the packed
-// fp32x2 add/sub/mul of sm_100 (each lane of the pair is still one IEEE operation), and
-// fp16 -> fp32 conversion rides in the first stage's mixed-precision adds.
+// fp32x2 arithmetic of sm_100 (each half is still one IEEE operation) held in 64-bit
+// registers; fp16 -> fp32 conversion rides in the first stage's mixed-precision adds.
 //
 // Quantisation: m = max |y| (lane-pair shuffle), s = fp16_rn(m / 7) (IEEE division, once
 // per row).  Codes are round-half-even of y / s, clamped to [-8, 7], computed without
 // dividing: a fast multiply-by-reciprocal path, and an exact half-point comparison for
 // groups with a near-tie (see quantise()); codes stay bit-exact with division by the
-// stored fp16 scale.  Codes are packed two per byte (low nibble = even channel) and
-// written with 64-bit stores; lane 0 of the row stores the fp16 scale.
-//
-// The CTAs are persistent (one wave, two per SM): each takes row blocks i, i + grid, ...
-// and issues the loads of its next rows before computing the current ones.
+// stored fp16 scale.  Codes are packed two per byte (low nibble = even channel).  A
+// lane's 8 code words (one per chunk, in slot order) go through a per-warp staging area
+// in shared memory, written at their chunk's place and read back in channel order, so
+// that the row's 64 code bytes leave as two 16-byte stores per lane (one L2 request per
+// row and store); lane 0 of the row stores the scale.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -40,157 +56,237 @@ namespace kvq {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kRowsPerBlock = 128;           // rows (K or V) per CTA
-constexpr int kThreads = kRowsPerBlock * 2;  // 2 lanes per row
-constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23
+constexpr int kPairs = 8;                      // (token, KV head) pairs per warp stage
+constexpr int kWarps = 8;                      // warps per CTA
+constexpr int kThreads = 32 * kWarps;
+constexpr int kHalfBytes = kPairs * kD * 2;    // one tensor's rows of a warp stage: 2 KB
+constexpr int kSlotBytes = 2 * kHalfBytes;     // K rows, then V rows
+constexpr int kStages = 3;                     // ring slots per warp
+constexpr int kStgStride = 80;                 // staging bytes per row (64 used)
+// A warp's region: ring slots | staging lines | barriers, rounded to 128 bytes so that
+// every region (and so every copy destination) stays 16-byte aligned.
+constexpr int kWarpBytes = (kStages * kSlotBytes + 2 * kPairs * kStgStride + 8 * kStages + 127) / 128 * 128;
+constexpr int kSmemBytes = kWarps * kWarpBytes;
+constexpr int kCtasPerSm = 2;
+static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM must fit");
+constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
-__device__ __forceinline__ float cvt_f16(uint16_t h) {
-  // Exact fp16 -> fp32 through the mixed-precision add (h + -0.0 keeps signed zeros).
+// Two fp32 values in one 64-bit register (low half = the even channel).
+typedef unsigned long long f2;
+
+__device__ __forceinline__ f2 pk(float a, float b) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk(f2 v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+  f2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// a * b + c per half, one rounding each.
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// fp16 bits -> fp32, exact (h + -0.0 keeps signed zeros).
+__device__ __forceinline__ float cvt_f16(uint32_t h) {
   float d;
-  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(h), "f"(-0.0f));
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(static_cast<uint16_t>(h)), "f"(-0.0f));
   return d;
 }
 
-// Butterfly on two pairs at once: (a0,a1),(c0,c1) -> (a+c, a-c) per lane, IEEE fp32.
-__device__ __forceinline__ void bfly2(float& a0, float& a1, float& c0, float& c1) {
-  asm("{\n\t.reg .b64 pa, pc, ps, pd;\n\t"
-      "mov.b64 pa, {%0, %1};\n\tmov.b64 pc, {%2, %3};\n\t"
-      "add.rn.f32x2 ps, pa, pc;\n\tsub.rn.f32x2 pd, pa, pc;\n\t"
-      "mov.b64 {%0, %1}, ps;\n\tmov.b64 {%2, %3}, pd;\n\t}"
-      : "+f"(a0), "+f"(a1), "+f"(c0), "+f"(c1));
-}
-
-// (x0, x1) <- (x0 * s + o0, x1 * s + o1), one rounding each: with s = +-1 this is the
-// IEEE sum or difference of the two operands.
-__device__ __forceinline__ void fma2(float& x0, float& x1, float s, float o0, float o1) {
-  asm("{\n\t.reg .b64 px, ps, po, pd;\n\t"
-      "mov.b64 px, {%0, %1};\n\tmov.b64 ps, {%2, %2};\n\tmov.b64 po, {%3, %4};\n\t"
-      "fma.rn.f32x2 pd, px, ps, po;\n\tmov.b64 {%0, %1}, pd;\n\t}"
-      : "+f"(x0), "+f"(x1)
-      : "f"(s), "f"(o0), "f"(o1));
-}
-
-__device__ __forceinline__ void mul2(float& x0, float& x1, float s) {
-  asm("{\n\t.reg .b64 px, ps, pd;\n\t"
-      "mov.b64 px, {%0, %1};\n\tmov.b64 ps, {%2, %2};\n\t"
-      "mul.rn.f32x2 pd, px, ps;\n\tmov.b64 {%0, %1}, pd;\n\t}"
-      : "+f"(x0), "+f"(x1)
-      : "f"(s));
-}
-
-// This lane's half of a row: the 16-channel chunks 2j + l (j = 0..3), 256-bit loads.
-__device__ __forceinline__ void load_row(const __half* row, int l, u32x8 (&raw)[4]) {
-#pragma unroll
-  for (int j = 0; j < 4; j++) raw[j] = ldg_256_stream(row + 16 * (2 * j + l));
-}
-
-// x[16j + e] = channel 16(2j + l) + e.  b = 1 (plain INT4): the transform of size 1 is
-// the identity and c_b = 1, so the row is only converted.
-__device__ __forceinline__ void convert_plain(const u32x8 (&raw)[4], float (&x)[64]) {
-#pragma unroll
-  for (int j = 0; j < 4; j++)
-#pragma unroll
-    for (int w = 0; w < 8; w++) {
-      x[16 * j + 2 * w] = cvt_f16(static_cast<uint16_t>(raw[j].w[w] & 0xffffu));
-      x[16 * j + 2 * w + 1] = cvt_f16(static_cast<uint16_t>(raw[j].w[w] >> 16));
-    }
-}
-
-// The butterfly without its final scale: x = z, the rotated row being y = fl(c_b * z),
-// which quantise() applies where it needs y itself.
-template <int BLOCK>
-__device__ __forceinline__ void rotate_row(const u32x8 (&raw)[4], int l, unsigned pmask,
-                                           float (&x)[64]) {
-  if constexpr (BLOCK == 1) {
-    convert_plain(raw, x);
-    return;
-  } else {
-  // Stage h = 1 fused with the conversion: (a, c) -> (a + c, a - c).
-#pragma unroll
-  for (int j = 0; j < 4; j++)
-#pragma unroll
-    for (int w = 0; w < 8; w++) {
-      const uint16_t lo = static_cast<uint16_t>(raw[j].w[w] & 0xffffu);
-      const uint16_t hi = static_cast<uint16_t>(raw[j].w[w] >> 16);
-      const float c = cvt_f16(hi);
-      float s, d;
-      asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(s) : "h"(lo), "f"(c));
-      asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(lo), "f"(c));
-      x[16 * j + 2 * w] = s;
-      x[16 * j + 2 * w + 1] = d;
-    }
-  // In-lane stages h = 2, 4, 8 (bits 1-3 of the chunk-local index).
-#pragma unroll
-  for (int h = 2; h <= 8; h *= 2)
-#pragma unroll
-    for (int j = 0; j < 4; j++)
-#pragma unroll
-      for (int e = 0; e < 16; e += 2)
-        if (!(e & h)) bfly2(x[16 * j + e], x[16 * j + e + 1], x[16 * j + e + h], x[16 * j + e + h + 1]);
-  // Cross-lane stage h = 16: the lane holding the lower index computes own + other, the
-  // upper one other - own (fma with a +-1 multiplier rounds once: bit-identical).
-  if (16 < BLOCK) {
-    const float sgn = l ? -1.0f : 1.0f;
-#pragma unroll
-    for (int i = 0; i < 64; i += 2) {
-      const float o0 = __shfl_xor_sync(pmask, x[i], 1);
-      const float o1 = __shfl_xor_sync(pmask, x[i + 1], 1);
-      fma2(x[i], x[i + 1], sgn, o0, o1);
-    }
-  }
-  // In-lane stages h = 32 (chunk j with j ^ 1) and h = 64 (chunk j with j ^ 2).
-  if (32 < BLOCK) {
-#pragma unroll
-    for (int j = 0; j < 4; j += 2)
-#pragma unroll
-      for (int e = 0; e < 16; e += 2)
-        bfly2(x[16 * j + e], x[16 * j + e + 1], x[16 * (j + 1) + e], x[16 * (j + 1) + e + 1]);
-  }
-  if (64 < BLOCK) {
-#pragma unroll
-    for (int j = 0; j < 2; j++)
-#pragma unroll
-      for (int e = 0; e < 16; e += 2)
-        bfly2(x[16 * j + e], x[16 * j + e + 1], x[16 * (j + 2) + e], x[16 * (j + 2) + e + 1]);
-  }
-  }
-}
-
-// Codes of 8 channels from their magic-rounded sums (low nibble = code & 0xF).
-__device__ __forceinline__ uint32_t pack8_magic(const float (&m)[8]) {
-  uint32_t b[4];
-#pragma unroll
-  for (int k = 0; k < 4; k++)
-    b[k] = (__float_as_uint(m[2 * k]) & 0xFu) | ((__float_as_uint(m[2 * k + 1]) & 0xFu) << 4);
-  return prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
-}
-
-// Quantise this lane's 64 rotated values of a row; q[2j], q[2j+1] = packed codes of
-// chunk j.  Returns the fp16 scale bits (identical on both lanes of the row).
-//
-// Codes are round-half-even of y / s with s the stored fp16 scale.  Fast path (a normal,
-// unsaturated s, so |y/s| <= 7.004): multiply the unscaled butterfly output z by
-// fl(c_b * fl(1/s)) and round with the magic addend; the product is within 2^-19 of y/s,
-// so the result is exact unless the fraction is within 2^-19 of one half.  A group of 8 values with such a near-tie -- frequent for rows that are
-// not rotated, whose fp16 values meet exact ties -- and every group when s is subnormal
-// or saturated is recomputed exactly without dividing: k = floor(y*r) is within one of
-// the true floor, and (k + 1/2)*s is exact in fp32 (an fp16 scale times a number of 5
-// bits), so comparing y with it chooses between k and k + 1, an exact tie going to the
-// even one.  (If y*r fell on the wrong side of an integer n, y/s is within 2^-16 of n
-// and both candidates' half points place it at n.)  Codes are clamped to [-8, 7].
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 
-__device__ __forceinline__ uint16_t quantise(const float (&z)[64], float cb, unsigned pmask,
+// Issue the two bulk copies of warp stage j (pairs [8j, 8j + n)) into the slot at dst.
+__device__ __forceinline__ void issue_stage(const AppendParams& p, int j, int npairs,
+                                            uint32_t dst, uint32_t bar, uint64_t pol) {
+  const int g0 = j * kPairs;
+  const int left = npairs - g0;
+  const uint32_t bytes = static_cast<uint32_t>(left < kPairs ? left : kPairs) * (kD * 2);
+  mbar_arrive_expect_tx(bar, 2 * bytes);
+  bulk_copy_g2s(dst, p.k + static_cast<size_t>(g0) * kD, bytes, bar, pol);
+  bulk_copy_g2s(dst + kHalfBytes, p.v + static_cast<size_t>(g0) * kD, bytes, bar, pol);
+}
+
+// Where pair gp goes: its sequence b (the b with cu[b] <= t < cu[b+1]), position pos =
+// seq_lens[b] + t - cu[b], the raw page-table entry of page pos / S (checked at use, so
+// that the load is in flight meanwhile) and the slot pos % S, or slot -1 for a position
+// outside the page table.
+struct Dest {
+  int page;
+  int slot;
+  int h;
+};
+
+__device__ __forceinline__ Dest pair_dest(const AppendParams& p, int gp) {
+  Dest d;
+  const int t = static_cast<int>(static_cast<unsigned>(gp) / static_cast<unsigned>(p.num_kv_heads));
+  d.h = gp - t * p.num_kv_heads;
+  int lo = 0, hi = p.batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(p.cu_new_tokens + mid) <= t) lo = mid; else hi = mid;
+  }
+  const int pos = __ldg(p.seq_lens + lo) + (t - __ldg(p.cu_new_tokens + lo));
+  const int lp = pos >= 0 ? pos / p.page_size : 0;
+  if (pos < 0 || lp >= p.max_pages_per_seq) {
+    d.page = -1;
+    d.slot = -1;
+  } else {
+    d.page = __ldg(p.page_table + static_cast<size_t>(lo) * p.max_pages_per_seq + lp);
+    d.slot = pos - lp * p.page_size;
+  }
+  return d;
+}
+
+// The butterfly without its final scale: x = z, the rotated row being y = fl(c_b * z),
+// which quantise() applies where it needs y itself.  raw[t] = chunk t ^ rho of this lane's
+// half row (4 words = 8 fp16 channels); x[4t + e] = channels 2e, 2e + 1 of that chunk.
+template <int BLOCK>
+__device__ __forceinline__ void rotate_row(const uint4 (&raw)[8], int rho, int l, unsigned pmask,
+                                           f2 (&x)[32]) {
+#pragma unroll
+  for (int t = 0; t < 8; t++) {
+    const uint32_t w[4] = {raw[t].x, raw[t].y, raw[t].z, raw[t].w};
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      if constexpr (BLOCK == 1) {
+        // b = 1 (plain INT4): the transform of size 1 is the identity and c_b = 1.
+        x[4 * t + e] = pk(cvt_f16(w[e] & 0xffffu), cvt_f16(w[e] >> 16));
+      } else {
+        // Stage h = 1 fused with the conversion: (a, c) -> (a + c, a - c).
+        const float c = cvt_f16(w[e] >> 16);
+        const uint16_t lo = static_cast<uint16_t>(w[e] & 0xffffu);
+        float s, d;
+        asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(s) : "h"(lo), "f"(c));
+        asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(lo), "f"(c));
+        x[4 * t + e] = pk(s, d);
+      }
+    }
+  }
+  if constexpr (BLOCK > 1) {
+    // Stages h = 2 (pair index e <-> e + 1) and h = 4 (e <-> e + 2) inside each chunk.
+#pragma unroll
+    for (int t = 0; t < 8; t++)
+#pragma unroll
+      for (int e = 0; e < 4; e += 2) {
+        const f2 a = x[4 * t + e], c = x[4 * t + e + 1];
+        x[4 * t + e] = add2(a, c);
+        x[4 * t + e + 1] = sub2(a, c);
+      }
+#pragma unroll
+    for (int t = 0; t < 8; t++)
+#pragma unroll
+      for (int e = 0; e < 2; e++) {
+        const f2 a = x[4 * t + e], c = x[4 * t + e + 2];
+        x[4 * t + e] = add2(a, c);
+        x[4 * t + e + 2] = sub2(a, c);
+      }
+    // Stages h = 8, 16, 32: chunk bit k, slots t and t ^ (1 << k).  With bit k of rho
+    // clear slot t holds the lower chunk: (t, u) <- (t + u, t - u); set: (u, t) <- (u + t,
+    // u - t).  Both as fma(own, sg, other), sg = +-1.
+#pragma unroll
+    for (int k = 0; k < 3; k++) {
+      if ((8 << k) < BLOCK) {
+        const float sg = ((rho >> k) & 1) ? -1.0f : 1.0f;
+        const f2 SG = pk(sg, sg), NSG = pk(-sg, -sg);
+#pragma unroll
+        for (int t = 0; t < 8; t++) {
+          if (t & (1 << k)) continue;
+          const int u = t | (1 << k);
+#pragma unroll
+          for (int e = 0; e < 4; e++) {
+            const f2 a = x[4 * t + e], c = x[4 * u + e];
+            x[4 * t + e] = fma2(a, SG, c);
+            x[4 * u + e] = fma2(c, NSG, a);
+          }
+        }
+      }
+    }
+    if constexpr (BLOCK == 128) {
+      // Stage h = 64 across the lane pair.  Lane 0's slot t and lane 1's slot t ^ 1 hold
+      // the same chunk of their halves (rho differs in bit 0 between them), so every lane
+      // receives its partner's slot t ^ 1 for its slot t.  Lane 0 (the lower channel)
+      // keeps own + other, lane 1 (the upper) other - own: fma(own, +-1, other).
+      const float sg = l ? -1.0f : 1.0f;
+      const f2 SG = pk(sg, sg);
+#pragma unroll
+      for (int t = 0; t < 8; t += 2)
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          float a0, a1, c0, c1;
+          upk(x[4 * t + e], a0, a1);
+          upk(x[4 * (t + 1) + e], c0, c1);
+          const f2 ra = pk(__shfl_xor_sync(pmask, c0, 1), __shfl_xor_sync(pmask, c1, 1));
+          const f2 rc = pk(__shfl_xor_sync(pmask, a0, 1), __shfl_xor_sync(pmask, a1, 1));
+          x[4 * t + e] = fma2(x[4 * t + e], SG, ra);
+          x[4 * (t + 1) + e] = fma2(x[4 * (t + 1) + e], SG, rc);
+        }
+    }
+  }
+}
+
+// The 8 codes of one chunk from their magic-rounded values (code = low nibble of the
+// bits), packed low nibble = even channel.
+__device__ __forceinline__ uint32_t pack_chunk(const f2 (&m)[4]) {
+  float v[8];
+#pragma unroll
+  for (int e = 0; e < 4; e++) upk(m[e], v[2 * e], v[2 * e + 1]);
+  const uint32_t ev = prmt(prmt(__float_as_uint(v[0]), __float_as_uint(v[2]), 0x0040u),
+                           prmt(__float_as_uint(v[4]), __float_as_uint(v[6]), 0x0040u), 0x5410u);
+  const uint32_t od = prmt(prmt(__float_as_uint(v[1]), __float_as_uint(v[3]), 0x0040u),
+                           prmt(__float_as_uint(v[5]), __float_as_uint(v[7]), 0x0040u), 0x5410u);
+  uint32_t r;
+  // (ev & 0x0F0F0F0F) | ((od << 4) & 0xF0F0F0F0)
+  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(r) : "r"(ev), "r"(od << 4), "r"(0x0F0F0F0Fu));
+  return r;
+}
+
+// Quantise this lane's 64 values of a row; q[t] = packed codes of slot t's chunk.
+// Returns the fp16 scale bits (identical on both lanes of the row).
+//
+// Codes are round-half-even of y / s with s the stored fp16 scale.  Fast path (a normal,
+// unsaturated s, so |y/s| <= 7.004): t = z * fl(c_b * fl(1/s)) (exact product) is within
+// 4 roundings (< 2^-19) of y / s; fma(z, r_z, 1.5 * 2^23) rounds it to the nearest integer
+// (ties to even) in one step, and fma(z, r_z, -rint) gives t - rint with one rounding, so
+// the result is exact unless the fraction is within 2^-19 of one half.  A chunk with such
+// a near-tie -- frequent for rows that are not rotated, whose fp16 values meet exact ties
+// -- and every chunk when s is subnormal or saturated is recomputed exactly without
+// dividing: k = floor(y*r) is within one of the true floor, and (k + 1/2)*s is exact in
+// fp32 (an fp16 scale times a number of 5 bits), so comparing y with it chooses between k
+// and k + 1, an exact tie going to the even one.  (If y*r fell on the wrong side of an
+// integer n, y/s is within 2^-16 of n and both candidates' half points place it at n.)
+// Codes are clamped to [-8, 7].
+__device__ __forceinline__ uint16_t quantise(const f2 (&x)[32], float cb, unsigned pmask,
                                              uint32_t (&q)[8]) {
   // m = max |y| = fl(c_b * max |z|): rounding is monotonic, so scaling after the max gives
   // the max of the scaled values.
-  float zmax = 0.0f;
+  float cm[8];  // per chunk, then a tree: short dependency chains
 #pragma unroll
-  for (int i = 0; i < 64; i += 2) zmax = max3(zmax, fabsf(z[i]), fabsf(z[i + 1]));
+  for (int t = 0; t < 8; t++) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 4; e++) upk(x[4 * t + e], v[2 * e], v[2 * e + 1]);
+    cm[t] = max3(max3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])),
+                 max3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7])));
+  }
+  float zmax = max3(max3(cm[0], cm[1], cm[2]), max3(cm[3], cm[4], cm[5]), fmaxf(cm[6], cm[7]));
   zmax = fmaxf(zmax, __shfl_xor_sync(pmask, zmax, 1));
   const float m = __fmul_rn(cb, zmax);
   const float s32 = __fdiv_rn(m, 7.0f);
@@ -199,162 +295,217 @@ __device__ __forceinline__ uint16_t quantise(const float (&z)[64], float cb, uns
   const float s = __half2float(sh);
   if (s == 0.0f) {  // an all-zero row (or a scale that underflows): every code is 0
 #pragma unroll
-    for (int w = 0; w < 8; w++) q[w] = 0u;
+    for (int t = 0; t < 8; t++) q[t] = 0u;
     return __half_as_ushort(sh);
   }
   const bool normal = !sat && s >= 6.103515625e-05f;
   const float r = __frcp_rn(s);
-  // Fast path on z directly: t = z * fl(c_b * r) is within 4 roundings (< 2^-19 for
-  // |y/s| <= 7.004) of y / s.
   const float rz = __fmul_rn(cb, r);
   const float hs = 0.5f * s;
+  const f2 MM = pk(kMagic, kMagic);
+  const f2 RZ = pk(rz, rz);
+  // Fast path for 4 chunks at a time, without branches; chunks with a near-tie are marked
+  // and then recomputed exactly (rare for rotated rows).
 #pragma unroll
-  for (int c8 = 0; c8 < 8; c8++) {
-    float mg[8];
-    float dmax = 0.0f;
+  for (int g = 0; g < 8; g += 4) {
+    uint32_t redo = normal ? 0u : 0xFFu;
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      float t0 = z[8 * c8 + e], t1 = z[8 * c8 + e + 1];
-      mul2(t0, t1, rz);
-      float m0 = t0, m1 = t1;
-      fma2(m0, m1, 1.0f, kMagic, kMagic);           // t + 1.5*2^23, rounded: rint
-      float r0 = m0, r1 = m1;
-      fma2(r0, r1, 1.0f, -kMagic, -kMagic);         // the integer, exactly
-      float d0 = r0, d1 = r1;
-      fma2(d0, d1, -1.0f, t0, t1);                  // t - rint(t), exactly
-      dmax = max3(dmax, fabsf(d0), fabsf(d1));
-      mg[e] = m0;
-      mg[e + 1] = m1;
+    for (int t = g; t < g + 4; t++) {
+      f2 mg[4];
+      float d[8];
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        mg[e] = fma2(x[4 * t + e], RZ, MM);   // 1.5*2^23 + rint(t)
+        const f2 nr = sub2(MM, mg[e]);        // -rint(t), exactly
+        upk(fma2(x[4 * t + e], RZ, nr), d[2 * e], d[2 * e + 1]);  // t - rint(t)
+      }
+      const float dmax = max3(max3(fabsf(d[0]), fabsf(d[1]), fabsf(d[2])),
+                              max3(fabsf(d[3]), fabsf(d[4]), fabsf(d[5])), fmaxf(fabsf(d[6]), fabsf(d[7])));
+      if (!(dmax < 0.5f - 0x1p-19f)) redo |= 1u << t;
+      q[t] = pack_chunk(mg);
     }
-    if (!normal || !(dmax < 0.5f - 0x1p-19f)) {
+    if (redo) {
 #pragma unroll
-      for (int e = 0; e < 8; e++) {
-        const float y = __fmul_rn(z[8 * c8 + e], cb);  // the rotated value
-        const float k = floorf(__fmul_rn(y, r));
-        const float h = __fmaf_rn(k, s, hs);  // (k + 1/2) * s, exact
-        const bool odd = (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) != 0u;
-        const bool up = y > h || (y == h && odd);
-        const float t = fminf(fmaxf(up ? k + 1.0f : k, -8.0f), 7.0f);
-        mg[e] = __fadd_rn(t, kMagic);
+      for (int t = g; t < g + 4; t++) {
+        if (!((redo >> t) & 1u)) continue;
+        f2 mg[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          float z[2], o[2];
+          upk(x[4 * t + e], z[0], z[1]);
+#pragma unroll
+          for (int i = 0; i < 2; i++) {
+            const float y = __fmul_rn(z[i], cb);  // the rotated value
+            const float k = floorf(__fmul_rn(y, r));
+            const float h = __fmaf_rn(k, s, hs);  // (k + 1/2) * s, exact
+            const bool odd = (__float_as_uint(__fadd_rn(k, kMagic)) & 1u) != 0u;
+            const bool up = y > h || (y == h && odd);
+            const float c = fminf(fmaxf(up ? k + 1.0f : k, -8.0f), 7.0f);
+            o[i] = __fadd_rn(c, kMagic);
+          }
+          mg[e] = pk(o[0], o[1]);
+        }
+        q[t] = pack_chunk(mg);
       }
     }
-    q[c8] = pack8_magic(mg);
   }
   return __half_as_ushort(sh);
 }
 
-// The K or V row r of the call: (token, head) pair r / 2, tensor r % 2.
-__device__ __forceinline__ const __half* row_src(const AppendParams& p, long long r) {
-  return ((r & 1) ? p.v : p.k) + static_cast<size_t>(r >> 1) * kD;
-}
-
-// Persistent: CTA i takes row blocks i, i + grid, ...; the loads of a lane's next row are
-// issued before the current row is rotated, quantised and stored, so they are in flight
-// while it computes.
 template <int BLOCK>
-__global__ void __launch_bounds__(kThreads, 2) append_kernel(AppendParams p) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) append_kernel(AppendParams p) {
   // The next kernel may start its own prologue; the pool stores below wait for every
   // earlier kernel (griddep_wait), so they never race with a decode still reading.
   griddep_launch_dependents();
-  const int l = threadIdx.x & 1;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  // This warp's ring, staging lines and barriers.
+  const uint32_t ring = smem_addr(smem) + w * kWarpBytes;
+  const uint32_t stg = ring + kStages * kSlotBytes;
+  const uint32_t bar0 = stg + 2 * kPairs * kStgStride;
+  const int l = lane & 1, rho = lane & 7;
+  const int pr = lane >> 2;         // pair within the warp stage
+  const int kv = (lane >> 1) & 1;   // 0 = K row, 1 = V row
   // Shuffles never leave the lane pair of a row, so they name only those two lanes.
-  const unsigned pmask = 0x3u << (threadIdx.x & 30);
-  const long long nrows = 2LL * p.total_new_tokens * p.num_kv_heads;
-  const long long nblk = (nrows + kRowsPerBlock - 1) / kRowsPerBlock;
-  const int r_in = threadIdx.x >> 1;
-  long long rb = blockIdx.x;
-  u32x8 raw[4];
-  {
-    const long long row = rb * kRowsPerBlock + r_in;
-    if (row < nrows) load_row(row_src(p, row), l, raw);
+  const unsigned pmask = 0x3u << (lane & 30);
+  const int npairs = p.total_new_tokens * p.num_kv_heads;  // < 2^31 (host-checked)
+  const int nws = (npairs + kPairs - 1) / kPairs;
+  const int W = gridDim.x * kWarps;
+  const int gw = blockIdx.x * kWarps + w;
+  // This row's 80-byte staging line; the lane's half is at +32l.
+  const uint32_t stg_row = stg + (lane >> 1) * kStgStride + 32 * l;
+  const uint64_t pol = l2_policy_evict_first();
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; s++) mbar_init(bar0 + 8 * s, 1);
+    fence_mbar_init();
+#pragma unroll
+    for (int s = 0; s < kStages; s++) {
+      const int j = gw + s * W;
+      if (j < nws) issue_stage(p, j, npairs, ring + s * kSlotBytes, bar0 + 8 * s, pol);
+    }
   }
+  __syncwarp();
+
+  Dest dcur = {-1, -1, 0};
+  if (gw * kPairs + pr < npairs) dcur = pair_dest(p, gw * kPairs + pr);
   bool waited = false;
-  for (; rb < nblk; rb += gridDim.x) {
-    const long long row = rb * kRowsPerBlock + r_in;
-    const long long row_next = (rb + gridDim.x) * kRowsPerBlock + r_in;
-    u32x8 nxt[4];
-    if (rb + gridDim.x < nblk && row_next < nrows) load_row(row_src(p, row_next), l, nxt);
-    if (row < nrows) {  // both lanes of a row take the same branch
-      const long long pair = row >> 1;
-      const int kv = static_cast<int>(row & 1);
-      const int t = static_cast<int>(pair / p.num_kv_heads);
-      const int h = static_cast<int>(pair % p.num_kv_heads);
+  int s = 0;
+  uint32_t phase = 0;
+  for (int j = gw; j < nws; j += W) {
+    const uint32_t slot = ring + s * kSlotBytes;
+    const int gp = j * kPairs + pr;
+    const bool active = gp < npairs;
+    // The next warp stage's destination: its page-table load is in flight meanwhile.
+    Dest dnext = {-1, -1, 0};
+    if (j + W < nws && gp + W * kPairs < npairs) dnext = pair_dest(p, gp + W * kPairs);
 
-      float x[64];
-      rotate_row<BLOCK>(raw, l, pmask, x);
-
-      // Sequence of token t: the b with cu[b] <= t < cu[b+1] (binary search).
-      int lo = 0, hi = p.batch;
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(p.cu_new_tokens + mid) <= t) lo = mid; else hi = mid;
+    if (!mbar_wait_bounded(bar0 + 8 * s, phase, kWaitLimitNs)) {
+      // A copy did not land in time: flag it, let this warp's other copies finish
+      // (bounded) so nothing lands in shared memory after the CTA exits, and stop.
+      if (lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
+#pragma unroll
+      for (int k = 1; k < kStages; k++) {
+        const int sk = (s + k) % kStages;
+        if (j + k * W < nws)
+          mbar_wait_bounded(bar0 + 8 * sk, sk > s ? phase : phase ^ 1u, kWaitLimitNs);
       }
-      const int b = lo;
-      const int pos = __ldg(p.seq_lens + b) + (t - __ldg(p.cu_new_tokens + b));
-      const int lp = pos / p.page_size;
-      int page = -1;
-      if (pos >= 0 && lp < p.max_pages_per_seq)
-        page = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + lp);
-      const bool ok = pos >= 0 && lp < p.max_pages_per_seq && page >= 0 && page < p.num_pages;
+      return;
+    }
+    uint4 raw[8];
+    if (active) {
+      const uint32_t row = slot + kv * kHalfBytes + pr * (kD * 2) + l * kD;
+#pragma unroll
+      for (int t = 0; t < 8; t++) raw[t] = lds_128(row + 16 * (t ^ rho));
+    }
+    // Every read of this slot is done: it can take warp stage j + kStages * W.
+    __syncwarp();
+    if (lane == 0 && j + kStages * W < nws) {
+      fence_proxy_async_smem();
+      issue_stage(p, j + kStages * W, npairs, slot, bar0 + 8 * s, pol);
+    }
+    if (++s == kStages) {
+      s = 0;
+      phase ^= 1u;
+    }
 
+    if (active) {  // both lanes of a row, and both rows of a pair, take the same branch
+      f2 x[32];
+      rotate_row<BLOCK>(raw, rho, l, pmask, x);
       uint32_t q[8];
       const uint16_t sbits = quantise(x, p.cb, pmask, q);
+      // Slot t's word is word t ^ rho of the lane's half: through the staging line into
+      // channel order (the lane reads back only what it wrote).
+#pragma unroll
+      for (int t = 0; t < 8; t++) sts_32(stg_row + 4 * (t ^ rho), q[t]);
+      const uint4 c0 = lds_128(stg_row), c1 = lds_128(stg_row + 16);
       if (!waited) {
         griddep_wait();
         waited = true;
       }
-      if (!ok) {
+      const bool bad_pos = dcur.slot < 0;
+      if (bad_pos || dcur.page < 0 || dcur.page >= p.num_pages) {
         if (l == 0 && kv == 0)
-          atomicOr(p.status, (pos < 0 || lp >= p.max_pages_per_seq) ? KVQ_DEV_BAD_POS_BIT
-                                                                      : KVQ_DEV_BAD_PAGE_BIT);
+          atomicOr(p.status, bad_pos ? KVQ_DEV_BAD_POS_BIT : KVQ_DEV_BAD_PAGE_BIT);
       } else {
         const int S = p.page_size;
-        const int slot = pos - lp * S;
-        uint8_t* blk = p.pool_layer + (static_cast<size_t>(page) * p.num_kv_heads + h) *
+        uint8_t* blk = p.pool_layer + (static_cast<size_t>(dcur.page) * p.num_kv_heads + dcur.h) *
                                           (static_cast<size_t>(S) * (kD + 4));
-        uint8_t* crow =
-            blk + static_cast<size_t>(kv) * S * (kD / 2) + static_cast<size_t>(slot) * (kD / 2);
-#pragma unroll
-        for (int j = 0; j < 4; j++)
-          *reinterpret_cast<uint2*>(crow + 8 * (2 * j + l)) = make_uint2(q[2 * j], q[2 * j + 1]);
+        uint4* crow = reinterpret_cast<uint4*>(blk + static_cast<size_t>(kv) * S * (kD / 2) +
+                                               static_cast<size_t>(dcur.slot) * (kD / 2) + 32 * l);
+        crow[0] = c0;
+        crow[1] = c1;
         if (l == 0)
           *reinterpret_cast<uint16_t*>(blk + static_cast<size_t>(S) * kD +
-                                       static_cast<size_t>(kv) * S * 2 + static_cast<size_t>(slot) * 2) =
-              sbits;
+                                       static_cast<size_t>(kv) * S * 2 +
+                                       static_cast<size_t>(dcur.slot) * 2) = sbits;
       }
     }
-#pragma unroll
-    for (int j = 0; j < 4; j++) raw[j] = nxt[j];
+    dcur = dnext;
   }
+}
+
+template <int BLOCK>
+int launch_block(const cudaLaunchConfig_t& cfg, const AppendParams& p) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(append_kernel<BLOCK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return -2;
+    attr_set = true;
+  }
+  return cudaLaunchKernelEx(&cfg, append_kernel<BLOCK>, p) == cudaSuccess ? 0 : -2;
 }
 
 }  // namespace
 
 int launch_append(const AppendParams& p, int block, int num_sms, cudaStream_t stream) {
-  const long long nrows = 2LL * p.total_new_tokens * p.num_kv_heads;
-  if (nrows == 0) return 0;
-  const long long nblk = (nrows + kRowsPerBlock - 1) / kRowsPerBlock;
-  if (nblk > 0x7fffffffLL) return -1;
-  // One wave of persistent CTAs (2 per SM), or fewer for a small call.
-  const long long grid = nblk < 2LL * num_sms ? nblk : 2LL * num_sms;
+  const long long npairs = static_cast<long long>(p.total_new_tokens) * p.num_kv_heads;
+  if (npairs == 0) return 0;
+  if (npairs > 0x7fffffffLL - (64LL << 20)) return -1;  // int indexing in the kernel
+  const long long nws = (npairs + kPairs - 1) / kPairs;
+  // One wave of persistent CTAs, or fewer for a small call.
+  const long long full = static_cast<long long>(kCtasPerSm) * num_sms;
+  const long long need = (nws + kWarps - 1) / kWarps;
+  const long long grid = need < full ? need : full;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e;
   switch (block) {
-    case 1: e = cudaLaunchKernelEx(&cfg, append_kernel<1>, p); break;
-    case 32: e = cudaLaunchKernelEx(&cfg, append_kernel<32>, p); break;
-    case 64: e = cudaLaunchKernelEx(&cfg, append_kernel<64>, p); break;
-    case 128: e = cudaLaunchKernelEx(&cfg, append_kernel<128>, p); break;
+    case 1: return launch_block<1>(cfg, p);
+    case 32: return launch_block<32>(cfg, p);
+    case 64: return launch_block<64>(cfg, p);
+    case 128: return launch_block<128>(cfg, p);
     default: return -1;
   }
-  return e == cudaSuccess ? 0 : -2;
 }
 
 }  // namespace kvq

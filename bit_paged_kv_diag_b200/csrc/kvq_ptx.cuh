@@ -170,6 +170,10 @@ __device__ __forceinline__ uint2 lds_64(uint32_t addr) {
   return r;
 }
 
+__device__ __forceinline__ void sts_32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
   uint16_t r;
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
