@@ -11,6 +11,8 @@ attention).  Sources, cited by page title and section:
 * [P1] "KVキャッシュを4ビットへ — SAW-INT4とシステムを踏まえたINT4量子化" (youngju.dev)
 * [P2] "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving"
   (gist.science)
+* [P3] "BitDecoding-FP4:FP4 KVキャッシュのネイティブ復号" (sns.style): the NVFP4 cache
+  format (``fmt = 1``: E2M1 codes, one E4M3 scale per 16 channels)
 
 Every function is pinned by a ``-m "not gpu"`` test against something other than
 itself (explicit matrices, closed forms, invariants, brute force).
@@ -48,22 +50,28 @@ def lib():
             "oracle_pack_codes": (None, [i8p, c_int, u8p]),
             "oracle_unpack_codes": (None, [u8p, c_int, i8p]),
             "oracle_assign_pages": (c_int, [c_int, i32p, c_int, c_int, c_int, i32p, i32p]),
-            "oracle_block_bytes": (ctypes.c_size_t, [c_int, c_int]),
+            "oracle_block_bytes": (ctypes.c_size_t, [c_int, c_int, c_int]),
             "oracle_rotate_quant_append": (c_int, [u8p, c_int, c_int, c_int, c_int, c_int, c_int,
-                                                   c_int, u16p, u16p, i32p, i32p, i32p, c_int]),
+                                                   c_int, u16p, u16p, i32p, i32p, i32p, c_int,
+                                                   c_int]),
             "oracle_read_row": (c_int, [u8p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
-                                        c_int, c_int, f32p]),
+                                        c_int, c_int, f32p, c_int]),
             "oracle_decode_one": (c_int, [u8p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                           c_int, u16p, i32p, i32p, c_int, c_int, ctypes.c_double,
-                                          f64p]),
+                                          f64p, c_int]),
             "oracle_decode_attention": (c_int, [u8p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                 c_int, c_int, u16p, i32p, i32p, c_int,
-                                                ctypes.c_double, f64p]),
+                                                ctypes.c_double, f64p, c_int]),
+            "oracle_e4m3_to_float": (ctypes.c_float, [ctypes.c_uint8]),
+            "oracle_float_to_e4m3": (ctypes.c_uint8, [ctypes.c_float]),
+            "oracle_e2m1_to_float": (ctypes.c_float, [ctypes.c_uint8]),
+            "oracle_float_to_e2m1": (ctypes.c_uint8, [ctypes.c_float]),
+            "oracle_quant_row_nvfp4": (None, [f32p, c_int, u8p, u8p]),
             "oracle_attention_dense": (c_int, [f64p, f64p, f64p, c_int, c_int, c_int, c_int,
                                                ctypes.c_double, f64p]),
             "oracle_prefill_attention": (c_int, [u8p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                  c_int, c_int, u16p, i32p, i32p, i32p, c_int,
-                                                 ctypes.c_double, f64p]),
+                                                 ctypes.c_double, f64p, c_int]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -173,15 +181,45 @@ def assign_pages(capacity, page_size: int, num_pages: int, max_pages_per_seq: in
     return pt
 
 
-def block_bytes(page_size: int, head_dim: int) -> int:
-    return int(lib().oracle_block_bytes(page_size, head_dim))
+def block_bytes(page_size: int, head_dim: int, fmt: int = 0) -> int:
+    return int(lib().oracle_block_bytes(page_size, head_dim, fmt))
+
+
+# ---------------------------------------------------------------- NVFP4 ----
+def e4m3_to_float(b: int) -> float:
+    return float(lib().oracle_e4m3_to_float(int(b)))
+
+
+def float_to_e4m3(x: float) -> int:
+    """Nearest E4M3 code (ties to even, saturating at 448)."""
+    return int(lib().oracle_float_to_e4m3(float(x)))
+
+
+def e2m1_to_float(c: int) -> float:
+    return float(lib().oracle_e2m1_to_float(int(c)))
+
+
+def float_to_e2m1(x: float) -> int:
+    """Nearest E2M1 code (ties to even, saturating at 6, sign kept)."""
+    return int(lib().oracle_float_to_e2m1(float(x)))
+
+
+def quant_row_nvfp4(y):
+    """NVFP4 codes (one per channel, 0..15) and E4M3 block scales of a rotated fp32 row."""
+    y = _c(y, np.float32)
+    codes = np.zeros(y.shape[0], np.uint8)
+    scales = np.zeros(y.shape[0] // 16, np.uint8)
+    lib().oracle_quant_row_nvfp4(_p(y, ctypes.c_float), y.shape[0], _p(codes, ctypes.c_uint8),
+                                 _p(scales, ctypes.c_uint8))
+    return codes, scales
 
 
 class Geometry:
-    """Cache geometry shared by the oracle entry points (plain record)."""
+    """Cache geometry shared by the oracle entry points (plain record); fmt 0 = rotated
+    INT4 with one fp16 scale per token, 1 = NVFP4 (E2M1 codes, E4M3 scale per 16)."""
 
     def __init__(self, num_layers, num_kv_heads, num_q_heads, head_dim, block, page_size,
-                 num_pages, max_pages_per_seq):
+                 num_pages, max_pages_per_seq, fmt=0):
         self.num_layers = int(num_layers)
         self.num_kv_heads = int(num_kv_heads)
         self.num_q_heads = int(num_q_heads)
@@ -190,11 +228,12 @@ class Geometry:
         self.page_size = int(page_size)
         self.num_pages = int(num_pages)
         self.max_pages_per_seq = int(max_pages_per_seq)
+        self.fmt = int(fmt)
 
     @property
     def pool_bytes(self) -> int:
         return (self.num_layers * self.num_pages * self.num_kv_heads
-                * block_bytes(self.page_size, self.head_dim))
+                * block_bytes(self.page_size, self.head_dim, self.fmt))
 
     def new_pool(self) -> np.ndarray:
         return np.zeros(self.pool_bytes, np.uint8)
@@ -213,7 +252,8 @@ def rotate_quant_append(g: Geometry, pool: np.ndarray, layer: int, k16, v16, cu_
     rc = lib().oracle_rotate_quant_append(
         _p(pool, ctypes.c_uint8), layer, g.num_pages, g.num_kv_heads, g.head_dim, g.block,
         g.page_size, g.max_pages_per_seq, _p(k, ctypes.c_uint16), _p(v, ctypes.c_uint16),
-        _p(cu, ctypes.c_int32), _p(sl, ctypes.c_int32), _p(pt, ctypes.c_int32), cu.shape[0] - 1)
+        _p(cu, ctypes.c_int32), _p(sl, ctypes.c_int32), _p(pt, ctypes.c_int32), cu.shape[0] - 1,
+        g.fmt)
     _check(rc, "rotate_quant_append")
 
 
@@ -222,7 +262,7 @@ def read_row(g: Geometry, pool, layer, page, head, slot, kv) -> np.ndarray:
     pool = _c(pool, np.uint8)
     rc = lib().oracle_read_row(_p(pool, ctypes.c_uint8), layer, g.num_pages, g.num_kv_heads,
                                g.head_dim, g.page_size, page, head, slot, kv,
-                               _p(out, ctypes.c_float))
+                               _p(out, ctypes.c_float), g.fmt)
     _check(rc, "read_row")
     return out
 
@@ -239,7 +279,7 @@ def decode_one(g: Geometry, pool, layer, q16, seq_lens, page_table, b, hq,
                                  g.num_q_heads, g.head_dim, g.block, g.page_size,
                                  g.max_pages_per_seq, _p(q, ctypes.c_uint16),
                                  _p(sl, ctypes.c_int32), _p(pt, ctypes.c_int32), int(b), int(hq),
-                                 float(softmax_scale), _p(out, ctypes.c_double))
+                                 float(softmax_scale), _p(out, ctypes.c_double), g.fmt)
     _check(rc, "decode_one")
     return out
 
@@ -257,7 +297,7 @@ def decode_attention(g: Geometry, pool, layer, q16, seq_lens, page_table,
                                        g.page_size, g.max_pages_per_seq, _p(q, ctypes.c_uint16),
                                        _p(sl, ctypes.c_int32), _p(pt, ctypes.c_int32),
                                        sl.shape[0], float(softmax_scale),
-                                       _p(out, ctypes.c_double))
+                                       _p(out, ctypes.c_double), g.fmt)
     _check(rc, "decode_attention")
     return out
 
@@ -277,7 +317,7 @@ def prefill_attention(g: Geometry, pool, layer, q16, cu_q, seq_lens, page_table,
                                         g.page_size, g.max_pages_per_seq, _p(q, ctypes.c_uint16),
                                         _p(cu, ctypes.c_int32), _p(sl, ctypes.c_int32),
                                         _p(pt, ctypes.c_int32), sl.shape[0], float(softmax_scale),
-                                        _p(out, ctypes.c_double))
+                                        _p(out, ctypes.c_double), g.fmt)
     _check(rc, "prefill_attention")
     return out
 

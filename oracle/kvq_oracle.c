@@ -10,6 +10,8 @@
  *        (youngju.dev blog, explaining the SAW-INT4 preprint)
  *   [P2] "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World
  *        LLM Serving" (gist.science explainer of the same preprint)
+ *   [P3] "BitDecoding-FP4:FP4 KVキャッシュのネイティブ復号" (sns.style), for the
+ *        NVFP4 cache format (fmt = 1): E2M1 codes with E4M3 block scales.
  *
  * Where the pages leave a step open, the reading taken is stated beside the
  * step and collected in the design notes.  Every floating-point step below is
@@ -149,6 +151,85 @@ void oracle_unpack_codes(const uint8_t* in, int d, int8_t* codes) {
   }
 }
 
+/* --------------------------------------------------------------- NVFP4 ---- */
+/* [P3, "背景と概要": NVFP4 is a 4-bit microscaling format -- 4-bit elements sharing a
+ * block scale -- and "深掘り分析": its block scales are E4M3.]  The pages give no
+ * formulas; the readings, for the cache format fmt = 1:
+ *   element  E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; magnitudes
+ *            {0, 0.5, 1, 1.5, 2, 3, 4, 6} for codes 0..7, bit 3 the sign;
+ *   block    16 consecutive channels of one rotated row share one scale;
+ *   scale    E4M3 (bias 7, 3 mantissa bits, no infinity, largest 448), the value
+ *            amax / 6 (one fp32 division) rounded to nearest, ties to even, and
+ *            saturated to 448; no second, per-tensor scale;
+ *   codes    t = y * r with r = 1 / s (both fp32 operations), rounded to the nearest
+ *            E2M1 magnitude (ties to the even code), saturated to 6, the sign of t
+ *            kept (so -0 is code 8); every code 0 when s == 0.
+ * Both roundings are written out as a search over the format's finite values, the
+ * plainest statement of round-to-nearest-even. */
+float oracle_e4m3_to_float(uint8_t b) {
+  const int sgn = (b >> 7) & 1, e = (b >> 3) & 0xF, m = b & 7;
+  double v = e == 0 ? (double)m / 8.0 * ldexp(1.0, -6) : (1.0 + (double)m / 8.0) * ldexp(1.0, e - 7);
+  return (float)(sgn ? -v : v);
+}
+
+/* Nearest E4M3 code to x (x >= 0 or negative: the sign is kept), ties to the even code,
+ * saturating at 448.  Codes 0..126 are the non-negative finite values in order. */
+uint8_t oracle_float_to_e4m3(float x) {
+  const int sgn = signbit(x) ? 1 : 0;
+  const double a = fabs((double)x);
+  int best = 0;
+  double bestd = INFINITY;
+  for (int c = 0; c <= 126; c++) {
+    const double d = fabs(a - (double)oracle_e4m3_to_float((uint8_t)c));
+    if (d < bestd || (d == bestd && (c & 1) == 0)) { best = c; bestd = d; }
+  }
+  return (uint8_t)((sgn << 7) | best);
+}
+
+float oracle_e2m1_to_float(uint8_t c) {
+  static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  const float v = mag[c & 7];
+  return (c & 8) ? -v : v;
+}
+
+/* Nearest E2M1 code to x, ties to the even code, saturating at 6, sign of x kept. */
+uint8_t oracle_float_to_e2m1(float x) {
+  const int sgn = signbit(x) ? 1 : 0;
+  const double a = fabs((double)x);
+  int best = 0;
+  double bestd = INFINITY;
+  for (int c = 0; c < 8; c++) {
+    const double d = fabs(a - (double)oracle_e2m1_to_float((uint8_t)c));
+    if (d < bestd || (d == bestd && (c & 1) == 0)) { best = c; bestd = d; }
+  }
+  return (uint8_t)((sgn << 3) | best);
+}
+
+/* NVFP4 quantisation of one rotated row y[0..d) (d a multiple of 16): codes[0..d) (one
+ * E2M1 code per byte, 0..15) and scales[0..d/16) (E4M3 bytes). */
+void oracle_quant_row_nvfp4(const float* y, int d, uint8_t* codes, uint8_t* scales) {
+  for (int b0 = 0; b0 < d; b0 += 16) {
+    float m = 0.0f;
+    for (int i = b0; i < b0 + 16; i++) {
+      const float a = fabsf(y[i]);
+      if (a > m) m = a;
+    }
+    const float s32 = m / 6.0f;
+    const uint8_t sb = oracle_float_to_e4m3(s32);
+    const float s = oracle_e4m3_to_float(sb);
+    scales[b0 / 16] = sb;
+    if (s == 0.0f) {
+      for (int i = b0; i < b0 + 16; i++) codes[i] = 0;
+      continue;
+    }
+    const float r = 1.0f / s;
+    for (int i = b0; i < b0 + 16; i++) {
+      const float t = y[i] * r;
+      codes[i] = oracle_float_to_e2m1(t);
+    }
+  }
+}
+
 /* ------------------------------------------------------------- paging ---- */
 /* Deterministic page assignment (a stated reading; the pages only fix
  * "fixed-size blocks plus a page table" [P1, "KVキャッシュこそが本当の
@@ -178,18 +259,22 @@ int oracle_assign_pages(int batch, const int32_t* capacity, int page_size, int n
 }
 
 /* Byte size of one (page, head) block: K codes, V codes, K scales, V scales,
- * each for page_size tokens (a stated reading of the block layout). */
-size_t oracle_block_bytes(int page_size, int head_dim) {
-  return (size_t)page_size * (size_t)(head_dim + 4);
+ * each for page_size tokens (a stated reading of the block layout).  A token row's
+ * scales take 2 bytes (fmt 0: one fp16) or head_dim / 16 bytes (fmt 1: E4M3 per block). */
+static size_t row_scale_bytes(int head_dim, int fmt) { return fmt ? (size_t)head_dim / 16 : 2; }
+
+size_t oracle_block_bytes(int page_size, int head_dim, int fmt) {
+  return (size_t)page_size * ((size_t)head_dim + 2 * row_scale_bytes(head_dim, fmt));
 }
 
 /* Offset of block (layer, page, head) in the pool.  Pool layout, outermost
  * first: layer, page, KV head; inside a block:
- *   [K codes  S x D/2 bytes][V codes  S x D/2 bytes][K scales S x fp16][V scales S x fp16]. */
+ *   [K codes  S x D/2 bytes][V codes  S x D/2 bytes][K scales S x sb][V scales S x sb]
+ * with sb = row_scale_bytes (one fp16, or D/16 E4M3 bytes). */
 static size_t block_offset(int layer, int page, int head, int num_pages, int num_kv_heads,
-                           int page_size, int head_dim) {
+                           int page_size, int head_dim, int fmt) {
   return (((size_t)layer * num_pages + (size_t)page) * num_kv_heads + (size_t)head) *
-         oracle_block_bytes(page_size, head_dim);
+         oracle_block_bytes(page_size, head_dim, fmt);
 }
 
 /* Rotate, quantise and append new tokens into the paged pool.
@@ -207,12 +292,20 @@ static size_t block_offset(int layer, int page, int head, int num_pages, int num
 int oracle_rotate_quant_append(uint8_t* pool, int layer, int num_pages, int num_kv_heads,
                                int head_dim, int block, int page_size, int max_pages_per_seq,
                                const uint16_t* k, const uint16_t* v, const int32_t* cu_new_tokens,
-                               const int32_t* seq_lens, const int32_t* page_table, int batch) {
+                               const int32_t* seq_lens, const int32_t* page_table, int batch,
+                               int fmt) {
   const int D = head_dim, S = page_size;
   if (D <= 0 || D % 2 || D % block || S <= 0 || batch < 0) return -1;
+  if (fmt && D % 16) return -1;
+  const size_t sb = row_scale_bytes(D, fmt);
   float* row = (float*)malloc(sizeof(float) * (size_t)D);
   int8_t* codes = (int8_t*)malloc((size_t)D);
-  if (!row || !codes) { free(row); free(codes); return -1; }
+  uint8_t* fcodes = (uint8_t*)malloc((size_t)D);
+  uint8_t* fscales = (uint8_t*)malloc((size_t)D / 16 + 1);
+  if (!row || !codes || !fcodes || !fscales) {
+    free(row); free(codes); free(fcodes); free(fscales);
+    return -1;
+  }
   int rc = 0;
   for (int b = 0; b < batch && rc == 0; b++) {
     for (int t = cu_new_tokens[b]; t < cu_new_tokens[b + 1] && rc == 0; t++) {
@@ -222,36 +315,56 @@ int oracle_rotate_quant_append(uint8_t* pool, int layer, int num_pages, int num_
       const int page = page_table[(size_t)b * max_pages_per_seq + lp];
       if (page < 0 || page >= num_pages) { rc = -4; break; }
       for (int h = 0; h < num_kv_heads; h++) {
-        uint8_t* blk = pool + block_offset(layer, page, h, num_pages, num_kv_heads, S, D);
+        uint8_t* blk = pool + block_offset(layer, page, h, num_pages, num_kv_heads, S, D, fmt);
         for (int kv = 0; kv < 2; kv++) {
           const uint16_t* src = (kv == 0 ? k : v) + ((size_t)t * num_kv_heads + h) * D;
           for (int d = 0; d < D; d++) row[d] = oracle_half_to_float(src[d]);
           oracle_fwht_f32(row, D, block);
-          uint16_t sbits = oracle_quant_row(row, D, codes);
-          oracle_pack_codes(codes, D, blk + (size_t)kv * S * (D / 2) + (size_t)slot * (D / 2));
-          uint8_t* sp = blk + (size_t)S * D + (size_t)kv * S * 2 + (size_t)slot * 2;
-          memcpy(sp, &sbits, 2);
+          uint8_t* cp = blk + (size_t)kv * S * (D / 2) + (size_t)slot * (D / 2);
+          uint8_t* sp = blk + (size_t)S * D + (size_t)kv * S * sb + (size_t)slot * sb;
+          if (fmt) {
+            oracle_quant_row_nvfp4(row, D, fcodes, fscales);
+            for (int j = 0; j < D / 2; j++) cp[j] = (uint8_t)(fcodes[2 * j] | (fcodes[2 * j + 1] << 4));
+            memcpy(sp, fscales, sb);
+          } else {
+            uint16_t sbits = oracle_quant_row(row, D, codes);
+            oracle_pack_codes(codes, D, cp);
+            memcpy(sp, &sbits, 2);
+          }
         }
       }
     }
   }
   free(row);
   free(codes);
+  free(fcodes);
+  free(fscales);
   return rc;
 }
 
 /* Dequantised row of the cache: code * scale in fp32 (exact: a 4-bit integer
- * times an 11-bit significand).  kv = 0 for K, 1 for V. */
+ * times an 11-bit significand, or an E2M1 value times an E4M3 scale, 2 + 4
+ * significant bits).  kv = 0 for K, 1 for V. */
 int oracle_read_row(const uint8_t* pool, int layer, int num_pages, int num_kv_heads, int head_dim,
-                    int page_size, int page, int head, int slot, int kv, float* out) {
+                    int page_size, int page, int head, int slot, int kv, float* out, int fmt) {
   const int D = head_dim, S = page_size;
   if (page < 0 || page >= num_pages || slot < 0 || slot >= S) return -1;
-  const uint8_t* blk = pool + block_offset(layer, page, head, num_pages, num_kv_heads, S, D);
-  int8_t codes[1024];
+  const uint8_t* blk = pool + block_offset(layer, page, head, num_pages, num_kv_heads, S, D, fmt);
+  const size_t sb = row_scale_bytes(D, fmt);
+  const uint8_t* cp = blk + (size_t)kv * S * (D / 2) + (size_t)slot * (D / 2);
+  const uint8_t* sp = blk + (size_t)S * D + (size_t)kv * S * sb + (size_t)slot * sb;
   if (D > 1024) return -1;
-  oracle_unpack_codes(blk + (size_t)kv * S * (D / 2) + (size_t)slot * (D / 2), D, codes);
+  if (fmt) {
+    for (int d = 0; d < D; d++) {
+      const uint8_t c = (uint8_t)((cp[d / 2] >> (4 * (d & 1))) & 0xF);
+      out[d] = oracle_e2m1_to_float(c) * oracle_e4m3_to_float(sp[d / 16]);
+    }
+    return 0;
+  }
+  int8_t codes[1024];
+  oracle_unpack_codes(cp, D, codes);
   uint16_t sbits;
-  memcpy(&sbits, blk + (size_t)S * D + (size_t)kv * S * 2 + (size_t)slot * 2, 2);
+  memcpy(&sbits, sp, 2);
   const float s = oracle_half_to_float(sbits);
   for (int d = 0; d < D; d++) out[d] = (float)codes[d] * s;
   return 0;
@@ -273,7 +386,7 @@ int oracle_read_row(const uint8_t* pool, int layer, int num_pages, int num_kv_he
 static int attend_row(const uint8_t* pool, int layer, int num_pages, int num_kv_heads,
                       int head_dim, int block, int page_size, int max_pages_per_seq,
                       const uint16_t* qrow, const int32_t* page_table, int b, int L, int h,
-                      double softmax_scale, double* out) {
+                      double softmax_scale, double* out, int fmt) {
   const int D = head_dim, S = page_size;
   if (softmax_scale == 0.0) softmax_scale = 1.0 / sqrt((double)D);
   for (int d = 0; d < D; d++) out[d] = 0.0;
@@ -292,7 +405,7 @@ static int attend_row(const uint8_t* pool, int layer, int num_pages, int num_kv_
   double mx = -INFINITY;
   for (int t = 0; t < L && rc == 0; t++) {
     const int page = page_table[(size_t)b * max_pages_per_seq + t / S];
-    if (oracle_read_row(pool, layer, num_pages, num_kv_heads, D, S, page, h, t % S, 0, row)) {
+    if (oracle_read_row(pool, layer, num_pages, num_kv_heads, D, S, page, h, t % S, 0, row, fmt)) {
       rc = -4;
       break;
     }
@@ -308,7 +421,7 @@ static int attend_row(const uint8_t* pool, int layer, int num_pages, int num_kv_
   }
   for (int t = 0; t < L && rc == 0; t++) {
     const int page = page_table[(size_t)b * max_pages_per_seq + t / S];
-    oracle_read_row(pool, layer, num_pages, num_kv_heads, D, S, page, h, t % S, 1, row);
+    oracle_read_row(pool, layer, num_pages, num_kv_heads, D, S, page, h, t % S, 1, row, fmt);
     const double p = sc[t] / den;
     for (int d = 0; d < D; d++) out[d] += p * (double)row[d];
   }
@@ -323,12 +436,12 @@ int oracle_decode_one(const uint8_t* pool, int layer, int num_pages, int num_kv_
                       int num_q_heads, int head_dim, int block, int page_size,
                       int max_pages_per_seq, const uint16_t* q, const int32_t* seq_lens,
                       const int32_t* page_table, int b, int hq, double softmax_scale,
-                      double* out) {
+                      double* out, int fmt) {
   if (num_kv_heads <= 0 || num_q_heads % num_kv_heads) return -1;
   const int G = num_q_heads / num_kv_heads;
   return attend_row(pool, layer, num_pages, num_kv_heads, head_dim, block, page_size,
                     max_pages_per_seq, q + ((size_t)b * num_q_heads + hq) * head_dim,
-                    page_table, b, seq_lens[b], hq / G, softmax_scale, out);
+                    page_table, b, seq_lens[b], hq / G, softmax_scale, out, fmt);
 }
 
 /* All (b, hq) pairs: out [batch][num_q_heads][head_dim] fp64. */
@@ -336,13 +449,13 @@ int oracle_decode_attention(const uint8_t* pool, int layer, int num_pages, int n
                             int num_q_heads, int head_dim, int block, int page_size,
                             int max_pages_per_seq, const uint16_t* q, const int32_t* seq_lens,
                             const int32_t* page_table, int batch, double softmax_scale,
-                            double* out) {
+                            double* out, int fmt) {
   for (int b = 0; b < batch; b++)
     for (int hq = 0; hq < num_q_heads; hq++) {
       int rc = oracle_decode_one(pool, layer, num_pages, num_kv_heads, num_q_heads, head_dim,
                                  block, page_size, max_pages_per_seq, q, seq_lens, page_table, b,
                                  hq, softmax_scale,
-                                 out + ((size_t)b * num_q_heads + hq) * head_dim);
+                                 out + ((size_t)b * num_q_heads + hq) * head_dim, fmt);
       if (rc) return rc;
     }
   return 0;
@@ -360,7 +473,7 @@ int oracle_prefill_attention(const uint8_t* pool, int layer, int num_pages, int 
                              int num_q_heads, int head_dim, int block, int page_size,
                              int max_pages_per_seq, const uint16_t* q, const int32_t* cu_q,
                              const int32_t* seq_lens, const int32_t* page_table, int batch,
-                             double softmax_scale, double* out) {
+                             double softmax_scale, double* out, int fmt) {
   if (num_kv_heads <= 0 || num_q_heads % num_kv_heads) return -1;
   const int G = num_q_heads / num_kv_heads, D = head_dim;
   for (int b = 0; b < batch; b++) {
@@ -373,7 +486,7 @@ int oracle_prefill_attention(const uint8_t* pool, int layer, int num_pages, int 
         const int rc = attend_row(pool, layer, num_pages, num_kv_heads, D, block, page_size,
                                   max_pages_per_seq, q + (tok * num_q_heads + hq) * D,
                                   page_table, b, pos + 1, hq / G, softmax_scale,
-                                  out + (tok * num_q_heads + hq) * D);
+                                  out + (tok * num_q_heads + hq) * D, fmt);
         if (rc) return rc;
       }
     }
