@@ -47,11 +47,16 @@ class KVQError(RuntimeError):
         self.status = status
 
 
+FORMAT_INT4 = 0
+FORMAT_NVFP4 = 1
+
+
 class Desc(ctypes.Structure):
-    """``kvq_desc``: cache geometry (host integers)."""
+    """``kvq_desc``: cache geometry (host integers); ``kv_format`` 0 = rotated INT4,
+    1 = NVFP4 (``FORMAT_NVFP4``); omitted trailing fields are 0."""
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_layers", "num_kv_heads", "num_q_heads", "head_dim", "hadamard_block",
-        "page_size", "num_pages", "max_batch", "max_pages_per_seq")]
+        "page_size", "num_pages", "max_batch", "max_pages_per_seq", "kv_format")]
 
     def __repr__(self):
         return "Desc(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"

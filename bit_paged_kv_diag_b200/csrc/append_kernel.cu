@@ -45,6 +45,14 @@
 // in shared memory, written at their chunk's place and read back in channel order, so
 // that the row's 64 code bytes leave as two 16-byte stores per lane (one L2 request per
 // row and store); lane 0 of the row stores the scale.
+//
+// NVFP4 rows ("BitDecoding-FP4:FP4 KVキャッシュのネイティブ復号" (sns.style), sections
+// "背景と概要", "深掘り分析": 4-bit microscaling elements with E4M3 block scales): after
+// the same rotation, each block of 16 channels -- slots t and t ^ 1 of a lane, since the
+// rotation of the read order keeps chunk pairs together -- gets s = E4M3(fl(max|y| / 6))
+// (round to nearest even, saturated at 448) and codes E2M1(fl(y * fl(1/s))) (nearest
+// even, saturated at 6, sign kept), both by the hardware conversions cvt.rn.satfinite;
+// all codes 0 when s == 0.  A lane's 4 scale bytes are stored as one word.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -91,6 +99,11 @@ __device__ __forceinline__ f2 add2(f2 a, f2 b) {
 __device__ __forceinline__ f2 sub2(f2 a, f2 b) {
   f2 r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
 // a * b + c per half, one rounding each.
@@ -352,7 +365,79 @@ __device__ __forceinline__ uint16_t quantise(const f2 (&x)[32], float cb, unsign
   return __half_as_ushort(sh);
 }
 
-template <int BLOCK>
+// Two fp32 values -> one byte of E2M1 codes (lo -> low nibble), nearest even, saturating.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u32.u8 %0, q;\n\t}"
+      : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two fp32 values -> two E4M3 bytes (lo -> low byte), nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 bytes (low 16 bits) -> their values (exact).
+__device__ __forceinline__ float2 e4m3x2_value(uint32_t b) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(b)));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// NVFP4 quantisation of this lane's 64 values: q[t] = the 4 code bytes of slot t's chunk;
+// returns the lane's 4 scale bytes in block order (byte m = block 4l + m of the row).
+__device__ __forceinline__ uint32_t quantise_fp4(const f2 (&x)[32], float cb, int rho,
+                                                uint32_t (&q)[8]) {
+  const f2 CB = pk(cb, cb);
+  float sv[4];
+  uint32_t sb[4];
+#pragma unroll
+  for (int u = 0; u < 4; u++) {  // slot pair (2u, 2u + 1) = one block of 16 channels
+    float v[16];
+#pragma unroll
+    for (int e = 0; e < 8; e++) upk(x[8 * u + e], v[2 * e], v[2 * e + 1]);
+    const float m8a = max3(max3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])),
+                           max3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7])));
+    const float m8b = max3(max3(fabsf(v[8]), fabsf(v[9]), fabsf(v[10])),
+                           max3(fabsf(v[11]), fabsf(v[12]), fabsf(v[13])), fmaxf(fabsf(v[14]), fabsf(v[15])));
+    // max |y| = fl(c_b * max |z|) (rounding is monotonic)
+    sv[u] = __fdiv_rn(__fmul_rn(cb, fmaxf(m8a, m8b)), 6.0f);
+  }
+  const uint32_t s01 = e4m3x2(sv[0], sv[1]), s23 = e4m3x2(sv[2], sv[3]);
+  sb[0] = s01 & 0xFFu;
+  sb[1] = s01 >> 8;
+  sb[2] = s23 & 0xFFu;
+  sb[3] = s23 >> 8;
+  const float2 f01 = e4m3x2_value(s01), f23 = e4m3x2_value(s23);
+  const float sf[4] = {f01.x, f01.y, f23.x, f23.y};
+#pragma unroll
+  for (int u = 0; u < 4; u++) {
+    const float r = sf[u] != 0.0f ? __frcp_rn(sf[u]) : 0.0f;
+    const f2 R = pk(r, r);
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      const int t = 2 * u + h;
+      uint32_t w = 0;
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        float a, b;
+        upk(mul2(mul2(x[4 * t + e], CB), R), a, b);  // t = fl(fl(z * c_b) * r)
+        w |= e2m1x2(a, b) << (8 * e);
+      }
+      q[t] = sf[u] != 0.0f ? w : 0u;  // a zero scale: every code 0
+    }
+  }
+  // Byte u of the word belongs to block (2u ^ rho) >> 1 = u ^ (rho >> 1) of the lane's half.
+  const uint32_t words = sb[0] | (sb[1] << 8) | (sb[2] << 16) | (sb[3] << 24);
+  const uint32_t r2 = static_cast<uint32_t>(rho >> 1);
+  const uint32_t sel = (0u ^ r2) | ((1u ^ r2) << 4) | ((2u ^ r2) << 8) | ((3u ^ r2) << 12);
+  return prmt(words, 0u, sel);
+}
+
+template <int BLOCK, bool FP4>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) append_kernel(AppendParams p) {
   // The next kernel may start its own prologue; the pool stores below wait for every
   // earlier kernel (griddep_wait), so they never race with a decode still reading.
@@ -434,7 +519,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) append_kernel(AppendPara
       f2 x[32];
       rotate_row<BLOCK>(raw, rho, l, pmask, x);
       uint32_t q[8];
-      const uint16_t sbits = quantise(x, p.cb, pmask, q);
+      uint32_t sbits;
+      if constexpr (FP4) sbits = quantise_fp4(x, p.cb, rho, q);
+      else sbits = quantise(x, p.cb, pmask, q);
       // Slot t's word is word t ^ rho of the lane's half: through the staging line into
       // channel order (the lane reads back only what it wrote).
 #pragma unroll
@@ -450,32 +537,47 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) append_kernel(AppendPara
           atomicOr(p.status, bad_pos ? KVQ_DEV_BAD_POS_BIT : KVQ_DEV_BAD_PAGE_BIT);
       } else {
         const int S = p.page_size;
+        constexpr int kScaleBytes = FP4 ? kD / 16 : 2;  // per token row
         uint8_t* blk = p.pool_layer + (static_cast<size_t>(dcur.page) * p.num_kv_heads + dcur.h) *
-                                          (static_cast<size_t>(S) * (kD + 4));
+                                          (static_cast<size_t>(S) * (kD + 2 * kScaleBytes));
         uint4* crow = reinterpret_cast<uint4*>(blk + static_cast<size_t>(kv) * S * (kD / 2) +
                                                static_cast<size_t>(dcur.slot) * (kD / 2) + 32 * l);
         crow[0] = c0;
         crow[1] = c1;
-        if (l == 0)
-          *reinterpret_cast<uint16_t*>(blk + static_cast<size_t>(S) * kD +
-                                       static_cast<size_t>(kv) * S * 2 +
-                                       static_cast<size_t>(dcur.slot) * 2) = sbits;
+        uint8_t* srow = blk + static_cast<size_t>(S) * kD + static_cast<size_t>(kv) * S * kScaleBytes +
+                        static_cast<size_t>(dcur.slot) * kScaleBytes;
+        if constexpr (FP4) {
+          *reinterpret_cast<uint32_t*>(srow + 4 * l) = sbits;
+        } else {
+          if (l == 0) *reinterpret_cast<uint16_t*>(srow) = static_cast<uint16_t>(sbits);
+        }
       }
     }
     dcur = dnext;
   }
 }
 
-template <int BLOCK>
+template <int BLOCK, bool FP4>
 int launch_block(const cudaLaunchConfig_t& cfg, const AppendParams& p) {
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(append_kernel<BLOCK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(append_kernel<BLOCK, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBytes) != cudaSuccess)
       return -2;
     attr_set = true;
   }
-  return cudaLaunchKernelEx(&cfg, append_kernel<BLOCK>, p) == cudaSuccess ? 0 : -2;
+  return cudaLaunchKernelEx(&cfg, append_kernel<BLOCK, FP4>, p) == cudaSuccess ? 0 : -2;
+}
+
+template <bool FP4>
+int launch_format(const cudaLaunchConfig_t& cfg, const AppendParams& p, int block) {
+  switch (block) {
+    case 1: return launch_block<1, FP4>(cfg, p);
+    case 32: return launch_block<32, FP4>(cfg, p);
+    case 64: return launch_block<64, FP4>(cfg, p);
+    case 128: return launch_block<128, FP4>(cfg, p);
+    default: return -1;
+  }
 }
 
 }  // namespace
@@ -499,13 +601,7 @@ int launch_append(const AppendParams& p, int block, int num_sms, cudaStream_t st
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  switch (block) {
-    case 1: return launch_block<1>(cfg, p);
-    case 32: return launch_block<32>(cfg, p);
-    case 64: return launch_block<64>(cfg, p);
-    case 128: return launch_block<128>(cfg, p);
-    default: return -1;
-  }
+  return p.fp4 ? launch_format<true>(cfg, p, block) : launch_format<false>(cfg, p, block);
 }
 
 }  // namespace kvq

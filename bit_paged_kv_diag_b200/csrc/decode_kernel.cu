@@ -54,7 +54,10 @@ namespace kvq {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kSlotBytes = kTileTokens * (kD + 4);  // 4224: one tile of codes + scales
+// Token row of a (page, head) block: codes, then scales (INT4: one fp16 per K/V row;
+// NVFP4: one E4M3 per 16 channels), and the ring slot of one tile.
+constexpr int row_bytes(bool fp4) { return fp4 ? kD + kD / 8 : kD + 4; }
+constexpr int slot_bytes(bool fp4) { return kTileTokens * row_bytes(fp4); }
 constexpr int kWarps = kDecodeWarps;                // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 3;                          // ring slots per warp
@@ -123,7 +126,7 @@ struct PageBatch {
 
 constexpr uint64_t kEntryBad = 8u;
 
-template <int SEFF>
+template <int SEFF, bool FP4>
 __device__ __forceinline__ uint64_t load_page_batch(int tb, int X0, int X1, int w, int lane,
                                                     const int32_t* pre, const int32_t* lens,
                                                     const DecodeParams& p) {
@@ -142,7 +145,7 @@ __device__ __forceinline__ uint64_t load_page_batch(int tb, int X0, int X1, int 
         pid = 0;
         flags = kEntryBad;
       }
-      const size_t blk_bytes = static_cast<size_t>(p.page_size) * (kD + 4);
+      const size_t blk_bytes = static_cast<size_t>(p.page_size) * row_bytes(FP4);
       e = reinterpret_cast<uint64_t>(p.pool_layer +
                                      (static_cast<size_t>(pid) * p.num_kv_heads + u.h) * blk_bytes);
       if (SEFF == kTileTokens) e |= static_cast<uint64_t>((t0 & (p.page_size - 1)) / kTileTokens);
@@ -156,7 +159,7 @@ __device__ __forceinline__ uint64_t load_page_batch(int tb, int X0, int X1, int 
 // kPPT holds the tile's page entry j).  The slot holds a virtual page of SEFF = min(S, 32)
 // token slots per copied page, [K codes][V codes][K scales][V scales], the pool's own
 // block layout.
-template <int SEFF>
+template <int SEFF, bool FP4>
 __device__ __forceinline__ void tile_issue(uint64_t e, uint32_t slot, uint32_t bar, int lane,
                                            uint64_t pol, const DecodeParams& p) {
   constexpr int kPPT = PageBatch<SEFF>::kPPT;
@@ -165,7 +168,7 @@ __device__ __forceinline__ void tile_issue(uint64_t e, uint32_t slot, uint32_t b
   const int S = p.page_size;
   if (SEFF < kTileTokens || S == kTileTokens) {
     const uint8_t* blk = reinterpret_cast<const uint8_t*>(e & ~static_cast<uint64_t>(15));
-    const uint32_t blk_bytes = static_cast<uint32_t>(S) * (kD + 4);
+    const uint32_t blk_bytes = static_cast<uint32_t>(S) * row_bytes(FP4);
     const int npg = __popc(__ballot_sync(kFull, have));
     if (lane == 0) mbar_arrive_expect_tx(bar, npg * blk_bytes);
     __syncwarp();
@@ -177,10 +180,16 @@ __device__ __forceinline__ void tile_issue(uint64_t e, uint32_t slot, uint32_t b
     const size_t o = static_cast<size_t>(e0 & 7u) * kTileTokens;  // tile's first token in the page
     const uint8_t* src = blk + o * 64;
     uint32_t dst = slot, bytes = 2048;
-    if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + 2048; }
-    if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 2; dst = slot + 4096; bytes = 64; }
-    if (lane == 3) { src = blk + static_cast<size_t>(S) * 130 + o * 2; dst = slot + 4160; bytes = 64; }
-    if (lane == 0) mbar_arrive_expect_tx(bar, kSlotBytes);
+    if constexpr (FP4) {  // scales: 8 E4M3 bytes per token row
+      if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + 2048; }
+      if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 8; dst = slot + 4096; bytes = 256; }
+      if (lane == 3) { src = blk + static_cast<size_t>(S) * 136 + o * 8; dst = slot + 4352; bytes = 256; }
+    } else {
+      if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + 2048; }
+      if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 2; dst = slot + 4096; bytes = 64; }
+      if (lane == 3) { src = blk + static_cast<size_t>(S) * 130 + o * 2; dst = slot + 4160; bytes = 64; }
+    }
+    if (lane == 0) mbar_arrive_expect_tx(bar, slot_bytes(FP4));
     __syncwarp();
     if (lane < 4) bulk_copy_g2s(dst, src, bytes, bar, pol);
   }
@@ -189,7 +198,7 @@ __device__ __forceinline__ void tile_issue(uint64_t e, uint32_t slot, uint32_t b
 // A warp's producer: issues its tiles t = 0, 1, ... (CTA tile X0 + w + kWarps*t) in
 // order into its ring, slot t % kStages; page entries come from batches loaded one
 // batch ahead.
-template <int SEFF>
+template <int SEFF, bool FP4>
 struct Producer {
   int t;         // next tile to issue
   int nT;        // tiles of this warp
@@ -198,8 +207,8 @@ struct Producer {
   uint64_t nxt;  // ... of the next batch
 };
 
-template <int SEFF>
-__device__ __forceinline__ void producer_issue(Producer<SEFF>& pr, int X0, int X1, int w, int lane,
+template <int SEFF, bool FP4>
+__device__ __forceinline__ void producer_issue(Producer<SEFF, FP4>& pr, int X0, int X1, int w, int lane,
                                                uint32_t ring_s, uint32_t bar_s, uint64_t pol,
                                                const int32_t* pre, const int32_t* lens,
                                                const DecodeParams& p) {
@@ -207,12 +216,12 @@ __device__ __forceinline__ void producer_issue(Producer<SEFF>& pr, int X0, int X
   if (pr.t >= pr.tb + kBatch) {
     pr.tb += kBatch;
     pr.cur = pr.nxt;
-    pr.nxt = pr.tb + kBatch < pr.nT ? load_page_batch<SEFF>(pr.tb + kBatch, X0, X1, w, lane, pre, lens, p) : 0;
+    pr.nxt = pr.tb + kBatch < pr.nT ? load_page_batch<SEFF, FP4>(pr.tb + kBatch, X0, X1, w, lane, pre, lens, p) : 0;
   }
   const int src = (pr.t - pr.tb) * kPPT + lane;
   const uint64_t e = __shfl_sync(kFull, pr.cur, src & 31);
   const int s = pr.t % kStages;
-  tile_issue<SEFF>(e, ring_s + s * kSlotBytes, bar_s + 8 * s, lane, pol, p);
+  tile_issue<SEFF, FP4>(e, ring_s + s * slot_bytes(FP4), bar_s + 8 * s, lane, pol, p);
   pr.t++;
 }
 
@@ -237,6 +246,62 @@ struct QFrag {
 //   frag word ((qi*3 + s)*4 + c)*8 + 2*jj + half, byte e  <->  channel 32c + 8jj + 2e + half.
 // The warp prepares queries q0, q0 + QSTEP, ... < G (all of them for QSTEP = 1; a
 // quarter each when the CTA's warps share one unit's rows).
+// Rotated, scaled queries qb, qb + QSTEP, ... (QB of them; indices past G repeat the last
+// one and are not stored by the callers): x[b][e] = channel 4*lane + e, and the power of
+// two M[b] >= max |q'| (1 for a zero row).
+template <int G, int QSTEP, int QB>
+__device__ __forceinline__ void rotate_q(const uint8_t* qraw, int qb, int lane, const DecodeParams& p,
+                                       float (&x)[QB][4], float (&M)[QB]) {
+#pragma unroll
+  for (int b = 0; b < QB; b++) {
+    const int qi = min(qb + b * QSTEP, G - 1);  // a clamped duplicate is computed, not stored
+    const uint2 raw = *reinterpret_cast<const uint2*>(qraw + qi * kD * 2 + 8 * lane);
+    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+    const float t0 = lo.x, t1 = lo.y, t2 = hi.x, t3 = hi.y;
+    const float a0 = __fadd_rn(t0, t1), a1 = __fsub_rn(t0, t1);
+    const float a2 = __fadd_rn(t2, t3), a3 = __fsub_rn(t2, t3);
+    const bool rot = p.hadamard_block > 1;  // b = 1 (plain INT4): no rotation
+    x[b][0] = rot ? __fadd_rn(a0, a2) : t0;
+    x[b][2] = rot ? __fsub_rn(a0, a2) : t2;
+    x[b][1] = rot ? __fadd_rn(a1, a3) : t1;
+    x[b][3] = rot ? __fsub_rn(a1, a3) : t3;
+  }
+#pragma unroll
+  for (int s = 0; s < 5; s++) {
+    if ((4 << s) < p.hadamard_block) {
+      const float sgn = ((lane >> s) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+      for (int b = 0; b < QB; b++)
+#pragma unroll
+        for (int e = 0; e < 4; e++)
+          x[b][e] = __fmaf_rn(x[b][e], sgn, __shfl_xor_sync(kFull, x[b][e], 1 << s));
+    }
+  }
+  float amax[QB];
+#pragma unroll
+  for (int b = 0; b < QB; b++) {
+    amax[b] = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      x[b][e] = __fmul_rn(__fmul_rn(x[b][e], p.cb), p.q_scale);
+      amax[b] = fmaxf(amax[b], fabsf(x[b][e]));
+    }
+  }
+#pragma unroll
+  for (int d = 1; d < 32; d *= 2)
+#pragma unroll
+    for (int b = 0; b < QB; b++) amax[b] = fmaxf(amax[b], __shfl_xor_sync(kFull, amax[b], d));
+#pragma unroll
+  for (int b = 0; b < QB; b++) {
+    M[b] = 1.0f;
+    if (amax[b] > 1e-30f) {
+      const uint32_t bits = __float_as_uint(amax[b]);
+      M[b] = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax[b];
+    }
+  }
+}
+
 template <int G, int QSTEP>
 __device__ __forceinline__ void prep_q_warp(const uint8_t* qraw, uint32_t* frag, float* sf, int lane,
                                             const DecodeParams& p, int q0 = 0) {
@@ -369,6 +434,171 @@ __device__ __forceinline__ void qfrag_load(QFrag<G>& f, const uint32_t* qfb, con
     f.sf[QFrag<G>::NQ - 1] = sfb[2 * c + 1];
   } else {
     f.sf[0] = c < G ? sfb[c] : 1.0f;
+  }
+}
+
+// ---------------------------------------------------------------- NVFP4 q --
+// NVFP4 cache ("BitDecoding-FP4:FP4 KVキャッシュのネイティブ復号" (sns.style): E2M1 codes
+// with an E4M3 scale per 16 channels).  K and V are dequantised to fp16 exactly (an E2M1
+// value times an E4M3 scale has at most 6 significant bits and lies in [2^-10, 2688]);
+// QK^T and PV run as mma.sync m16n8k16 f16 x f16 -> f32.  q' is normalised by M (the
+// power of two >= max |q'|) to |q~| <= 2^14 and carried as fp16 hi + lo parts (about
+// 2^-22 relative).  Fragment table row (qi, part) = 128 fp16 in channel order.
+template <int G, int QSTEP>
+__device__ __forceinline__ void prep_q4_warp(const uint8_t* qraw, uint32_t* frag, float* sf, int lane,
+                                             const DecodeParams& p, int q0 = 0) {
+  constexpr int NQW = (G + QSTEP - 1) / QSTEP;
+  constexpr int QB = NQW < 4 ? NQW : 4;
+  __half* base = reinterpret_cast<__half*>(frag);
+#pragma unroll 1
+  for (int qb = q0; qb < G; qb += QB * QSTEP) {
+    float x[QB][4], Mq[QB];
+    rotate_q<G, QSTEP, QB>(qraw, qb, lane, p, x, Mq);
+#pragma unroll
+    for (int b = 0; b < QB; b++) {
+      const int qi = qb + b * QSTEP;
+      if (qi >= G) continue;
+      const float inv = __fdiv_rn(16384.0f, Mq[b]);  // exact: powers of two
+      __half hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        const float t = x[b][e] * inv;
+        hi[e] = __float2half_rn(t);
+        lo[e] = __float2half_rn(t - __half2float(hi[e]));
+      }
+      *reinterpret_cast<uint2*>(base + (qi * 2) * kD + 4 * lane) =
+          make_uint2(pack_half2(hi[0], hi[1]), pack_half2(hi[2], hi[3]));
+      *reinterpret_cast<uint2*>(base + (qi * 2 + 1) * kD + 4 * lane) =
+          make_uint2(pack_half2(lo[0], lo[1]), pack_half2(lo[2], lo[3]));
+      if (lane == 0) sf[qi] = Mq[b] * (1.0f / 16384.0f);
+    }
+  }
+  __syncwarp();
+}
+
+// f16 B fragments of q~ per k-step kk (16 channels: k rows 2c + e <-> channel
+// 32c + 4kk + e, k rows 2c + 8 + e <-> channel 32c + 4kk + 2 + e), column g.
+// G <= 4: column g holds part g & 1 (hi, lo) of query g / 2 in H; G == 8: H and L are the
+// hi and lo parts of query g.
+template <int G>
+struct QFrag4 {
+  static constexpr int NQ = (G == 8) ? 2 : 1;
+  uint32_t H[8][2];
+  uint32_t L[G == 8 ? 8 : 1][2];
+  float sf[NQ];
+};
+
+template <int G>
+__device__ __forceinline__ void qfrag4_load(QFrag4<G>& f, const uint32_t* qfb, const float* sfb,
+                                            int lane) {
+  const int g = lane >> 2, c = lane & 3;
+  const int qi = (G == 8) ? g : (g >> 1);
+  const bool ok = qi < G;
+  const int row_h = (G == 8) ? 2 * g : 2 * qi + (g & 1);
+#pragma unroll
+  for (int part = 0; part < (G == 8 ? 2 : 1); part++) {
+    uint4 w[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      w[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (ok) w[i] = reinterpret_cast<const uint4*>(qfb + (row_h + part) * (kD / 2) + 16 * c)[i];
+    }
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++) {
+      const uint4 q4 = w[kk >> 1];
+      const uint32_t a = (kk & 1) ? q4.z : q4.x, b = (kk & 1) ? q4.w : q4.y;
+      if (part == 0) {
+        f.H[kk][0] = a;
+        f.H[kk][1] = b;
+      } else {
+        f.L[G == 8 ? kk : 0][0] = a;
+        f.L[G == 8 ? kk : 0][1] = b;
+      }
+    }
+  }
+  if (G == 8) {
+    f.sf[0] = sfb[2 * c];
+    f.sf[QFrag4<G>::NQ - 1] = sfb[2 * c + 1];
+  } else {
+    f.sf[0] = c < G ? sfb[c] : 1.0f;
+  }
+}
+
+// The 4 bytes of w, each two E2M1 codes (low nibble first) -> 4 x fp16x2, exact.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&d)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(w));
+}
+
+// Two E4M3 scale bytes (low 16 bits, low byte first) -> fp16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t b) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(b)));
+  return h;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Scores (log2 domain) of an NVFP4 tile, in tile_qk's layout: A row g <-> token tau0,
+// row g + 8 <-> tau1; the lane's 16 code bytes of a token row are channels 32c..32c+31
+// (blocks 2c, 2c + 1), byte 2kk <-> channels 32c + 4kk, +1 (k columns 2c, 2c + 1).
+template <int G, int SEFF>
+__device__ __forceinline__ void tile_qk4(const QFrag4<G>& qf, const uint8_t* slot, int ntok, int lane,
+                                         float (&sc)[2][QFrag4<G>::NQ][2]) {
+  constexpr int RB = row_bytes(true);
+  const int g = lane >> 2, c = lane & 3;
+  const int tau0 = (g < 4) ? g : g + 4;
+  const int tau1 = tau0 + 4;
+#pragma unroll
+  for (int j = 0; j < 2; j++) {
+    const uint8_t* pbase = slot + (16 * j / SEFF) * (SEFF * RB);
+    const int sl = (16 * j) % SEFF;
+    const uint4 ka = *reinterpret_cast<const uint4*>(pbase + (sl + tau0) * 64 + 16 * c);
+    const uint4 kc = *reinterpret_cast<const uint4*>(pbase + (sl + tau1) * 64 + 16 * c);
+    const uint32_t sa = *reinterpret_cast<const uint16_t*>(pbase + SEFF * 128 + (sl + tau0) * 8 + 2 * c);
+    const uint32_t sc2 = *reinterpret_cast<const uint16_t*>(pbase + SEFF * 128 + (sl + tau1) * 8 + 2 * c);
+    const uint32_t fa = e4m3x2_to_f16x2(sa), fc = e4m3x2_to_f16x2(sc2);
+    const uint32_t sA[2] = {prmt(fa, fa, 0x1010u), prmt(fa, fa, 0x3232u)};
+    const uint32_t sC[2] = {prmt(fc, fc, 0x1010u), prmt(fc, fc, 0x3232u)};
+    const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
+    const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
+    float accH[4] = {0.0f, 0.0f, 0.0f, 0.0f}, accL[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int wi = 0; wi < 4; wi++) {  // word wi = k-steps 2wi, 2wi + 1
+      uint32_t da[4], dc[4];
+      e2m1x8_to_f16x2(wa[wi], da);
+      e2m1x8_to_f16x2(wc[wi], dc);
+      const int blk = wi >> 1;  // k-steps 0-3: block 2c; 4-7: block 2c + 1
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int kk = 2 * wi + h;
+        const uint32_t a0 = hmul2(da[2 * h], sA[blk]), a2 = hmul2(da[2 * h + 1], sA[blk]);
+        const uint32_t a1 = hmul2(dc[2 * h], sC[blk]), a3 = hmul2(dc[2 * h + 1], sC[blk]);
+        mma_16816(accH, a0, a1, a2, a3, qf.H[kk][0], qf.H[kk][1]);
+        if (G == 8) mma_16816(accL, a0, a1, a2, a3, qf.L[G == 8 ? kk : 0][0], qf.L[G == 8 ? kk : 0][1]);
+      }
+    }
+    const bool v0 = 16 * j + tau0 < ntok, v1 = 16 * j + tau1 < ntok;
+    if (G == 8) {
+#pragma unroll
+      for (int qq = 0; qq < 2; qq++)
+#pragma unroll
+        for (int r = 0; r < 2; r++) {
+          const int e = 2 * r + qq;
+          sc[j][qq][r] = (r ? v1 : v0) ? (accH[e] + accL[e]) * qf.sf[qq] : -CUDART_INF_F;
+        }
+    } else {
+      // Column 2c = hi part, 2c + 1 = lo part of query c.
+      sc[j][0][0] = v0 ? (accH[0] + accH[1]) * qf.sf[0] : -CUDART_INF_F;
+      sc[j][0][1] = v1 ? (accH[2] + accH[3]) * qf.sf[0] : -CUDART_INF_F;
+    }
   }
 }
 
@@ -566,6 +796,102 @@ __device__ __forceinline__ void tile_pv(State<G>& st, const uint8_t* slot, int n
       const uint32_t a2 = nib_lo_to_half2(r23), a3 = nib_hi_to_half2(r23);
       mma_16816(st.o[i], a0, a1, a2, a3, bh0, bh1);
       if (G == 8) mma_16816(st.o[i], a0, a1, a2, a3, bl0, bl1);
+    }
+  }
+}
+
+// Bytes 0 and 2 of w, each two E2M1 codes (low nibble first) -> 2 x fp16x2, exact.
+__device__ __forceinline__ void e2m1x2_b02_to_f16x2(uint32_t w, uint32_t& d0, uint32_t& d2) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b2;\n\t}"
+      : "=r"(d0), "=r"(d2)
+      : "r"(w));
+}
+
+// (a & m) | (b & ~m)
+__device__ __forceinline__ uint32_t bitsel(uint32_t a, uint32_t b, uint32_t m) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(r) : "r"(a), "r"(b), "r"(m));
+  return r;
+}
+
+// PV of an NVFP4 tile with probabilities pr: as tile_pv, with P' = p; the V scales are
+// applied in the dequantised A operand (the lane's channels 16g..16g+15 are block g of
+// each token row, so a register's two tokens each take their own scale).
+template <int G, int SEFF>
+__device__ __forceinline__ void tile_pv4(State<G>& st, const uint8_t* slot, int ntok, int lane,
+                                         const float (&pr)[2][QFrag4<G>::NQ][2]) {
+  constexpr int RB = row_bytes(true);
+  const int g = lane >> 2, c = lane & 3;
+  const int tau0 = (g < 4) ? g : g + 4;
+  const int tau1 = tau0 + 4;
+  const int srcA = 4 * c + (g >> 1);
+  const int srcB = srcA + 16;
+#pragma unroll
+  for (int j = 0; j < 2; j++) {
+    const uint8_t* pbase = slot + (16 * j / SEFF) * (SEFF * RB);
+    const int sl = (16 * j) % SEFF;
+    const uint8_t* vb = pbase + SEFF * 64 + sl * 64;
+    const uint8_t* vs = pbase + SEFF * 128 + SEFF * 8 + sl * 8;  // V scales [token][8]
+    const bool v0 = 16 * j + tau0 < ntok, v1 = 16 * j + tau1 < ntok;
+    uint32_t bh0, bh1, bl0 = 0u, bl1 = 0u;
+    if (G == 8) {
+      uint32_t xh[2], xl[2];
+#pragma unroll
+      for (int qq = 0; qq < 2; qq++) {
+        const float p0 = v0 ? pr[j][qq][0] : 0.0f, p1 = v1 ? pr[j][qq][1] : 0.0f;
+        split_hi_lo(p0, p1, xh[qq], xl[qq]);
+      }
+      const uint32_t aE = __shfl_sync(kFull, xh[0], srcA), aO = __shfl_sync(kFull, xh[1], srcA);
+      const uint32_t cE = __shfl_sync(kFull, xh[0], srcB), cO = __shfl_sync(kFull, xh[1], srcB);
+      const uint32_t dE = __shfl_sync(kFull, xl[0], srcA), dO = __shfl_sync(kFull, xl[1], srcA);
+      const uint32_t eE = __shfl_sync(kFull, xl[0], srcB), eO = __shfl_sync(kFull, xl[1], srcB);
+      bh0 = (g & 1) ? aO : aE;
+      bh1 = (g & 1) ? cO : cE;
+      bl0 = (g & 1) ? dO : dE;
+      bl1 = (g & 1) ? eO : eE;
+    } else {
+      const float p0 = v0 ? pr[j][0][0] : 0.0f, p1 = v1 ? pr[j][0][1] : 0.0f;
+      uint32_t xh, xl;
+      split_hi_lo(p0, p1, xh, xl);
+      const uint32_t aH = __shfl_sync(kFull, xh, srcA), aL = __shfl_sync(kFull, xl, srcA);
+      const uint32_t cH = __shfl_sync(kFull, xh, srcB), cL = __shfl_sync(kFull, xl, srcB);
+      bh0 = (g & 1) ? aL : aH;
+      bh1 = (g & 1) ? cL : cH;
+      if ((g >> 1) >= G) bh0 = bh1 = 0u;
+    }
+    // V rows of tokens c, c+4, c+8, c+12; this thread's channels [16g, 16g+16) = block g.
+    const uint2 t0 = *reinterpret_cast<const uint2*>(vb + (c + 0) * 64 + 8 * g);
+    const uint2 t1 = *reinterpret_cast<const uint2*>(vb + (c + 4) * 64 + 8 * g);
+    const uint2 t2 = *reinterpret_cast<const uint2*>(vb + (c + 8) * 64 + 8 * g);
+    const uint2 t3 = *reinterpret_cast<const uint2*>(vb + (c + 12) * 64 + 8 * g);
+    const uint32_t s01 = static_cast<uint32_t>(vs[(c + 0) * 8 + g]) | (static_cast<uint32_t>(vs[(c + 4) * 8 + g]) << 8);
+    const uint32_t s23 = static_cast<uint32_t>(vs[(c + 8) * 8 + g]) | (static_cast<uint32_t>(vs[(c + 12) * 8 + g]) << 8);
+    const uint32_t S01 = e4m3x2_to_f16x2(s01), S23 = e4m3x2_to_f16x2(s23);
+    const uint32_t w0[2] = {t0.x, t0.y}, w1[2] = {t1.x, t1.y};
+    const uint32_t w2[2] = {t2.x, t2.y}, w3[2] = {t3.x, t3.y};
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {  // m-tiles i, i + 1: bytes e, e + 1 of word i / 4
+      const uint32_t e = i & 3;
+      // bytes: [row0 byte e, row1 byte e, row0 byte e+1, row1 byte e+1]
+      const uint32_t sel = e | ((4 + e) << 4) | ((e + 1) << 8) | ((5 + e) << 12);
+      const uint32_t X01 = prmt(w0[i >> 2], w1[i >> 2], sel);
+      const uint32_t X23 = prmt(w2[i >> 2], w3[i >> 2], sel);
+      // even channels: low nibbles of the two tokens; odd: high nibbles (bytes 0 and 2)
+      const uint32_t ev01 = bitsel(X01, X01 >> 4, 0x000F000Fu), od01 = bitsel(X01 >> 4, X01 >> 8, 0x000F000Fu);
+      const uint32_t ev23 = bitsel(X23, X23 >> 4, 0x000F000Fu), od23 = bitsel(X23 >> 4, X23 >> 8, 0x000F000Fu);
+      uint32_t a0[2], a1[2], a2[2], a3[2];
+      e2m1x2_b02_to_f16x2(ev01, a0[0], a0[1]);
+      e2m1x2_b02_to_f16x2(od01, a1[0], a1[1]);
+      e2m1x2_b02_to_f16x2(ev23, a2[0], a2[1]);
+      e2m1x2_b02_to_f16x2(od23, a3[0], a3[1]);
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const uint32_t A0 = hmul2(a0[h], S01), A1 = hmul2(a1[h], S01);
+        const uint32_t A2 = hmul2(a2[h], S23), A3 = hmul2(a3[h], S23);
+        mma_16816(st.o[i + h], A0, A1, A2, A3, bh0, bh1);
+        if (G == 8) mma_16816(st.o[i + h], A0, A1, A2, A3, bl0, bl1);
+      }
     }
   }
 }
@@ -928,12 +1254,62 @@ __device__ __forceinline__ void patch_slot(uint8_t* slot, int lane, const uint8_
 }
 
 // Per-warp fragment table: G queries x 96 words, at least one staging record.
-constexpr int frag_words(int g) { return g * 96 > kPartStride ? g * 96 : kPartStride; }
+// (NVFP4: G queries x 2 fp16 parts x 128 channels = G x 128 words.)
+constexpr int frag_words(int g, bool fp4) {
+  return (fp4 ? g * 128 : g * 96) > kPartStride ? (fp4 ? g * 128 : g * 96) : kPartStride;
+}
 
-// FUSED: the one-token append runs inside (p.k_new, p.v_new set).
-template <int G, int SEFF, bool FUSED>
+// The format's q preparation, fragments and tile steps.
+template <int G, int QSTEP, bool FP4>
+__device__ __forceinline__ void prep_q(const uint8_t* qraw, uint32_t* frag, float* sf, int lane,
+                                       const DecodeParams& p, int q0 = 0) {
+  if constexpr (FP4) prep_q4_warp<G, QSTEP>(qraw, frag, sf, lane, p, q0);
+  else prep_q_warp<G, QSTEP>(qraw, frag, sf, lane, p, q0);
+}
+
+template <int G, bool FP4>
+struct QF {
+  using type = QFrag<G>;
+};
+template <int G>
+struct QF<G, true> {
+  using type = QFrag4<G>;
+};
+
+template <int G>
+__device__ __forceinline__ void qfrag_get(QFrag<G>& f, const uint32_t* qfb, const float* sfb, int lane) {
+  qfrag_load<G>(f, qfb, sfb, lane);
+}
+template <int G>
+__device__ __forceinline__ void qfrag_get(QFrag4<G>& f, const uint32_t* qfb, const float* sfb, int lane) {
+  qfrag4_load<G>(f, qfb, sfb, lane);
+}
+
+template <int G, int SEFF>
+__device__ __forceinline__ void tile_qk_any(const QFrag<G>& qf, const uint8_t* slot, int ntok, int lane,
+                                            float (&sc)[2][QFrag<G>::NQ][2]) {
+  tile_qk<G, SEFF>(qf, slot, ntok, lane, sc);
+}
+template <int G, int SEFF>
+__device__ __forceinline__ void tile_qk_any(const QFrag4<G>& qf, const uint8_t* slot, int ntok, int lane,
+                                            float (&sc)[2][QFrag4<G>::NQ][2]) {
+  tile_qk4<G, SEFF>(qf, slot, ntok, lane, sc);
+}
+
+template <int G, int SEFF, bool FP4>
+__device__ __forceinline__ void tile_pv_any(State<G>& st, const uint8_t* slot, int ntok, int lane,
+                                            const float (&pr)[2][QFrag<G>::NQ][2]) {
+  if constexpr (FP4) tile_pv4<G, SEFF>(st, slot, ntok, lane, pr);
+  else tile_pv<G, SEFF>(st, slot, ntok, lane, pr);
+}
+
+// FUSED: the one-token append runs inside (p.k_new, p.v_new set; INT4 only).
+// FP4: the cache holds NVFP4 rows.
+template <int G, int SEFF, bool FUSED, bool FP4>
 __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
-  constexpr int kFragWords = frag_words(G);
+  static_assert(!(FUSED && FP4), "the fused append is INT4 only");
+  constexpr int kFragWords = frag_words(G, FP4);
+  constexpr int kSlot = slot_bytes(FP4);
   extern __shared__ __align__(128) uint8_t smem_raw[];
   // Bulk copies need 16-byte aligned destinations; align to 128 bytes (the allocation
   // carries 128 spare bytes for this).
@@ -942,7 +1318,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   // Per warp (index w) and two more for the CTA's first and last unit (indices kWarps,
   // kWarps + 1): raw q rows, fragment table, M factors.
   constexpr int kQT = kWarps + 2;
-  uint8_t* qraw_all = ring + kWarps * kStages * kSlotBytes;                  // [kQT][G][128] fp16
+  uint8_t* qraw_all = ring + kWarps * kStages * kSlot;                       // [kQT][G][128] fp16
   uint32_t* frag_all = reinterpret_cast<uint32_t*>(qraw_all + kQT * G * kD * 2);  // [kQT][kFragWords]
   float* sf_all = reinterpret_cast<float*>(frag_all + kQT * kFragWords);     // [kQT][8]
   float* mbuf = sf_all + kQT * 8;                                            // [w][G][132]
@@ -1008,7 +1384,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   uint8_t* qraw = qraw_all + w * G * kD * 2;
   uint32_t* frag = frag_all + w * kFragWords;
   float* sf = sf_all + w * 8;
-  uint8_t* ring_w = ring + w * kStages * kSlotBytes;
+  uint8_t* ring_w = ring + w * kStages * kSlot;
   const uint8_t* ring_p = ring_w;
   const uint32_t ring_s = smem_addr(ring_p);
   const uint32_t bar_s = smem_addr(bars + w * (kStages + 1));
@@ -1023,12 +1399,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 
   // Producer: page-id batches 0 and 1 (page table only: before the wait).
   constexpr int kBatch = PageBatch<SEFF>::kBatch;
-  Producer<SEFF> pr;
+  Producer<SEFF, FP4> pr;
   pr.t = 0;
   pr.nT = has_tiles ? max(0, (X1 - X0 - w + kWarps - 1) / kWarps) : 0;
   pr.tb = 0;
-  pr.cur = has_tiles ? load_page_batch<SEFF>(0, X0, X1, w, lane, pre, lens, p) : 0;
-  pr.nxt = pr.nT > kBatch ? load_page_batch<SEFF>(kBatch, X0, X1, w, lane, pre, lens, p) : 0;
+  pr.cur = has_tiles ? load_page_batch<SEFF, FP4>(0, X0, X1, w, lane, pre, lens, p) : 0;
+  pr.nxt = pr.nT > kBatch ? load_page_batch<SEFF, FP4>(kBatch, X0, X1, w, lane, pre, lens, p) : 0;
 
   // This warp's q rows of a unit: one bulk copy into its raw-q buffer, completing on qbar.
   int q_issued = 0, q_done = 0;  // q copies issued / waited for (one in flight at most)
@@ -1095,7 +1471,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   }
   if (x < X1 && !is_uf(cu) && !is_ul(cu)) q_fetch(cu);
   while (pr.t < pr.nT && pr.t < kStages)
-    producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
+    producer_issue<SEFF, FP4>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
 
   // An empty sequence has no tiles: its output rows are zeros (CTAs share the writes).
   const int row_words = p.num_kv_heads * G * kD / 8;  // 16-byte words per sequence
@@ -1119,7 +1495,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     return p.part + (static_cast<size_t>(unit + kc) * kWarps + ww) * G * kPartStride;
   };
   float* const rec_f = mbuf;                             // [kWarps][G][kPartStride]
-  float* const rec_l = reinterpret_cast<float*>(ring);   // warp ww's: + ww*kStages*kSlotBytes
+  float* const rec_l = reinterpret_cast<float*>(ring);   // warp ww's: + ww*kStages*kSlot
 
   int consumed = 0;   // tiles of this warp consumed (tile t uses slot t % kStages)
   bool dead = false;  // a bounded wait gave up: stop touching the ring
@@ -1127,13 +1503,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
   if (!mbar_wait_bounded(qbar_cta, 0u, kWaitLimitNs)) dead = true;
   if (!dead)
     for (int t = 0; t < (two_edges ? 2 : 1); t++)
-      prep_q_warp<G, kWarps>(qraw_all + (kWarps + t) * G * kD * 2, frag_all + (kWarps + t) * kFragWords,
+      prep_q<G, kWarps, FP4>(qraw_all + (kWarps + t) * G * kD * 2, frag_all + (kWarps + t) * kFragWords,
                              sf_all + (kWarps + t) * 8, lane, p, w);
   if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
   __syncthreads();
   State<G> st;
   state_reset<G>(st);
-  QFrag<G> qf;
+  typename QF<G, FP4>::type qf;
   constexpr int NQ = QFrag<G>::NQ;
   while (x < X1) {
     const int seg_end = min(X1, cu.U + cu.n);
@@ -1146,14 +1522,14 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     // next unit's rows into the freed buffer.
     const int table = is_uf(cu) ? kWarps : (is_ul(cu) ? kWarps + 1 : -1);
     if (table >= 0) {
-      qfrag_load<G>(qf, frag_all + table * kFragWords, sf_all + table * 8, lane);
+      qfrag_get<G>(qf, frag_all + table * kFragWords, sf_all + table * 8, lane);
     } else {
       if (!dead) {
         if (mbar_wait_bounded(qbar, static_cast<uint32_t>(q_done & 1), kWaitLimitNs)) q_done++;
         else dead = true;
       }
-      if (!dead) prep_q_warp<G, 1>(qraw, frag, sf, lane, p);
-      qfrag_load<G>(qf, frag, sf, lane);
+      if (!dead) prep_q<G, 1, FP4>(qraw, frag, sf, lane, p);
+      qfrag_get<G>(qf, frag, sf, lane);
     }
     if (has_next && !dead && !is_ul(nu)) q_fetch(nu);
     state_reset<G>(st);
@@ -1181,7 +1557,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       __syncwarp();
       if (pr.t < pr.nT) {
         fence_proxy_async_smem();
-        producer_issue<SEFF>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
+        producer_issue<SEFF, FP4>(pr, X0, X1, w, lane, ring_s, bar_s, pol, pre, lens, p);
       }
     };
     float sc[2][NQ][2];
@@ -1193,9 +1569,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       } else {
         if constexpr (FUSED) {
           if (new_ok && nt == 1)
-            patch_slot<SEFF>(ring_w + slot_i * kSlotBytes, lane, reinterpret_cast<const uint8_t*>(frag));
+            patch_slot<SEFF>(ring_w + slot_i * kSlot, lane, reinterpret_cast<const uint8_t*>(frag));
         }
-        tile_qk<G, SEFF>(qf, ring_p + slot_i * kSlotBytes, ntok_of(x), lane, sc);
+        tile_qk_any<G, SEFF>(qf, ring_p + slot_i * kSlot, ntok_of(x), lane, sc);
         float alpha[NQ];
         if (tile_softmax_stats<G>(st, sc, alpha)) tile_rescale<G>(st, alpha);
       }
@@ -1215,11 +1591,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       float sn[2][NQ][2], alpha[NQ];
       if constexpr (FUSED) {
         if (new_ok && i + 2 == nt)
-          patch_slot<SEFF>(ring_w + nslot * kSlotBytes, lane, reinterpret_cast<const uint8_t*>(frag));
+          patch_slot<SEFF>(ring_w + nslot * kSlot, lane, reinterpret_cast<const uint8_t*>(frag));
       }
-      tile_qk<G, SEFF>(qf, ring_p + nslot * kSlotBytes, ntok_of(xi + kWarps), lane, sn);
+      tile_qk_any<G, SEFF>(qf, ring_p + nslot * kSlot, ntok_of(xi + kWarps), lane, sn);
       const bool rescale = tile_softmax_stats<G>(st, sn, alpha);
-      tile_pv<G, SEFF>(st, ring_p + cur * kSlotBytes, ntok_of(xi), lane, sc);
+      tile_pv_any<G, SEFF, FP4>(st, ring_p + cur * kSlot, ntok_of(xi), lane, sc);
       consumed++;
       slot_i = nslot;
       parity = npar;
@@ -1233,7 +1609,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
           for (int r = 0; r < 2; r++) sc[j][qq][r] = sn[j][qq][r];
     }
     if (!dead) {  // last tile of the unit for this warp
-      tile_pv<G, SEFF>(st, ring_p + slot_i * kSlotBytes, ntok_of(x + kWarps * (nt - 1)), lane, sc);
+      tile_pv_any<G, SEFF, FP4>(st, ring_p + slot_i * kSlot, ntok_of(x + kWarps * (nt - 1)), lane, sc);
       consumed++;
       refill();
     }
@@ -1247,7 +1623,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     } else if (unit == unit_f) {
       state_write<G>(st, rec_f + w * G * kPartStride, lane);
     } else if (unit == unit_l) {
-      state_write<G>(st, rec_l + w * (kStages * kSlotBytes / 4), lane);
+      state_write<G>(st, rec_l + w * (kStages * kSlot / 4), lane);
     } else {
       state_write<G>(st, warp_slot(unit, w), lane);
     }
@@ -1271,7 +1647,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
     shared_edge[e] = !(u.U >= X0 && u.U + u.n <= X1);
     if (u.n == 1) continue;  // already finished by its warp
     float* base = e == 0 ? rec_f : rec_l;
-    const int wstride = e == 0 ? G * kPartStride : kStages * kSlotBytes / 4;
+    const int wstride = e == 0 ? G * kPartStride : kStages * kSlot / 4;
     auto rec = [&](int j) -> const float* { return base + ((a - X0 + j) & (kWarps - 1)) * wstride; };
     merge_few<G, kWarps, false, kWarps>(min(kWarps, c), rec, w, out_row(u.b, u.h),
                                         shared_edge[e] ? warp_slot(unit, 0) : nullptr, lane, p);
@@ -1330,16 +1706,17 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 }
 
 template <int G, int SEFF>
-void* kernel_ptr(bool fused) {
-  return fused ? reinterpret_cast<void*>(&decode_kernel<G, SEFF, true>)
-               : reinterpret_cast<void*>(&decode_kernel<G, SEFF, false>);
+void* kernel_ptr(bool fused, bool fp4) {
+  if (fp4) return fused ? nullptr : reinterpret_cast<void*>(&decode_kernel<G, SEFF, false, true>);
+  return fused ? reinterpret_cast<void*>(&decode_kernel<G, SEFF, true, false>)
+               : reinterpret_cast<void*>(&decode_kernel<G, SEFF, false, false>);
 }
 
-void* pick_kernel(int group, int seff, bool fused) {
-#define KVQ_PICK(GG)                                    \
-  if (group == GG) {                                    \
-    if (seff == 16) return kernel_ptr<GG, 16>(fused);   \
-    if (seff == 32) return kernel_ptr<GG, 32>(fused);   \
+void* pick_kernel(int group, int seff, bool fused, bool fp4) {
+#define KVQ_PICK(GG)                                         \
+  if (group == GG) {                                         \
+    if (seff == 16) return kernel_ptr<GG, 16>(fused, fp4);   \
+    if (seff == 32) return kernel_ptr<GG, 32>(fused, fp4);   \
   }
   KVQ_PICK(1)
   KVQ_PICK(2)
@@ -1349,10 +1726,10 @@ void* pick_kernel(int group, int seff, bool fused) {
   return nullptr;
 }
 
-size_t smem_bytes(int group, int max_batch) {
-  size_t s = static_cast<size_t>(kWarps) * kStages * kSlotBytes;      // rings
+size_t smem_bytes(int group, int max_batch, bool fp4) {
+  size_t s = static_cast<size_t>(kWarps) * kStages * slot_bytes(fp4);  // rings
   s += static_cast<size_t>(kWarps + 2) * group * kD * 2;             // raw q rows
-  s += sizeof(uint32_t) * (kWarps + 2) * frag_words(group);          // q fragment tables
+  s += sizeof(uint32_t) * (kWarps + 2) * frag_words(group, fp4);     // q fragment tables
   s += sizeof(float) * (kWarps + 2) * 8;                             // M factors
   s += sizeof(float) * kWarps * group * kPartStride;                 // CTA merge buffer
   s += sizeof(uint64_t) * (kWarps * (kStages + 1) + 1);              // mbarriers
@@ -1363,16 +1740,17 @@ size_t smem_bytes(int group, int max_batch) {
 
 }  // namespace
 
-int plan_decode(int group, int page_size, int max_batch, int num_sms, DecodeLaunch* out) {
+int plan_decode(int group, int page_size, int max_batch, int num_sms, int fp4, DecodeLaunch* out) {
   const int seff = page_size < kTileTokens ? page_size : kTileTokens;
-  const size_t smem = smem_bytes(group, max_batch);
-  // The dynamic shared memory cap of both variants is set to the most any call of this
+  const size_t smem = smem_bytes(group, max_batch, fp4 != 0);
+  // The dynamic shared memory cap of the variants is set to the most any call of this
   // library uses (max_batch 4096), so plans made for several caches never shrink it
-  // under one another; the grid is the smaller occupancy of the two.
-  const size_t cap_bytes = smem_bytes(group, 4096);
+  // under one another; the grid is the smaller occupancy of the variants (INT4: plain
+  // and fused; NVFP4: plain only).
+  const size_t cap_bytes = smem_bytes(group, 4096, fp4 != 0);
   int occ = 3;
-  for (int fused = 0; fused < 2; fused++) {
-    void* fn = pick_kernel(group, seff, fused != 0);
+  for (int fused = 0; fused < (fp4 ? 1 : 2); fused++) {
+    void* fn = pick_kernel(group, seff, fused != 0, fp4 != 0);
     if (!fn) return -1;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(cap_bytes)) != cudaSuccess)
@@ -1390,7 +1768,7 @@ int plan_decode(int group, int page_size, int max_batch, int num_sms, DecodeLaun
 
 int launch_decode(const DecodeParams& p, const DecodeLaunch& L, cudaStream_t stream) {
   const int seff = p.page_size < kTileTokens ? p.page_size : kTileTokens;
-  void* fn = pick_kernel(p.group, seff, p.k_new != nullptr);
+  void* fn = pick_kernel(p.group, seff, p.k_new != nullptr, p.fp4 != 0);
   if (!fn) return -1;
   DecodeParams q = p;
   q.total_ctas = L.grid;

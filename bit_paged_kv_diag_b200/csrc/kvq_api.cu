@@ -48,6 +48,7 @@ bool desc_ok(const kvq_desc* d, int* why) {
   if (hb != 1 && hb != 32 && hb != 64 && hb != 128) return false;  // 1: plain INT4, no rotation
   const int S = d->page_size;
   if (S != 16 && S != 32 && S != 64 && S != 128 && S != 256) return false;
+  if (d->kv_format != KVQ_FORMAT_INT4 && d->kv_format != KVQ_FORMAT_NVFP4) return false;
   if (d->max_batch > 4096) return false;
   if (static_cast<long long>(d->max_pages_per_seq) * S > (1LL << 30)) return false;
   if (static_cast<long long>(d->max_batch) * d->max_pages_per_seq > (1LL << 31) - 1) return false;
@@ -59,10 +60,16 @@ bool desc_ok(const kvq_desc* d, int* why) {
   return true;
 }
 
+// Bytes of one token row of a (page, head) block: K and V codes, then the scales (one
+// fp16 each for INT4; one E4M3 per 16 channels each for NVFP4).
+size_t row_bytes(const kvq_desc* d) {
+  return static_cast<size_t>(d->head_dim) +
+         (d->kv_format == KVQ_FORMAT_NVFP4 ? static_cast<size_t>(d->head_dim) / 8 : 4);
+}
+
 size_t pool_bytes_of(const kvq_desc* d) {
   return static_cast<size_t>(d->num_layers) * static_cast<size_t>(d->num_pages) *
-         static_cast<size_t>(d->num_kv_heads) * static_cast<size_t>(d->page_size) *
-         static_cast<size_t>(d->head_dim + 4);
+         static_cast<size_t>(d->num_kv_heads) * static_cast<size_t>(d->page_size) * row_bytes(d);
 }
 
 // fp32 value nearest 1/sqrt(b) (b = 32, 64, 128).
@@ -148,7 +155,8 @@ int kvq_alloc_pages(const kvq_desc* d, void* dev_pool, size_t pool_bytes, int32_
     return KVQ_ECUDA;
   }
   const int g = d->num_q_heads / d->num_kv_heads;
-  if (kvq::plan_decode(g, d->page_size, d->max_batch, c->num_sms, &c->launch) != 0) {
+  if (kvq::plan_decode(g, d->page_size, d->max_batch, c->num_sms,
+                       d->kv_format == KVQ_FORMAT_NVFP4, &c->launch) != 0) {
     delete c;
     return KVQ_ECUDA;
   }
@@ -218,6 +226,7 @@ int kvq_rotate_quant_append(kvq_cache* c, int32_t layer, const void* k, const vo
   p.page_size = c->d.page_size;
   p.max_pages_per_seq = c->d.max_pages_per_seq;
   p.cb = c->cb;
+  p.fp4 = c->d.kv_format == KVQ_FORMAT_NVFP4;
   const int rc = kvq::launch_append(p, c->d.hadamard_block, c->num_sms, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;
@@ -261,6 +270,8 @@ int decode_common(kvq_cache* c, int32_t layer, const void* k_new, const void* v_
   p.total_ctas = c->launch.grid;
   p.k_new = static_cast<const __half*>(k_new);
   p.v_new = static_cast<const __half*>(v_new);
+  p.fp4 = c->d.kv_format == KVQ_FORMAT_NVFP4;
+  if (p.fp4 && k_new) return KVQ_EUNSUPPORTED;  // the fused append is INT4 only
   const int rc = kvq::launch_decode(p, c->launch, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;
@@ -290,6 +301,7 @@ int kvq_prefill_attention(kvq_cache* c, int32_t layer, const void* q, const int3
   if (!c) return KVQ_EINVAL;
   if (layer < 0 || layer >= c->d.num_layers) return KVQ_EINVAL;
   if (batch < 0 || batch > c->d.max_batch || total_q < 0) return KVQ_EINVAL;
+  if (c->d.kv_format != KVQ_FORMAT_INT4) return KVQ_EUNSUPPORTED;
   if (!(softmax_scale >= 0.0f) || isinf(softmax_scale)) return KVQ_EINVAL;
   if (batch == 0 || total_q == 0) return KVQ_OK;
   if (!q || !cu_q || !seq_lens || !page_table || !out) return KVQ_EINVAL;

@@ -27,6 +27,7 @@ struct AppendParams {
   int page_size;
   int max_pages_per_seq;
   float cb;                       // fp32 nearest 1/sqrt(hadamard_block)
+  int fp4;                        // 1: NVFP4 rows (E2M1 codes, E4M3 scale per 16 channels)
 };
 
 // Tokens per decode tile (one shared-memory ring slot per tile).
@@ -61,6 +62,7 @@ struct DecodeParams {
   // seq_lens[b] + 1 tokens (the pool is then written through pool_layer).
   const __half* k_new;
   const __half* v_new;
+  int fp4;                        // 1: NVFP4 cache (host-side kernel choice)
 };
 
 struct PrefillParams {
@@ -94,7 +96,7 @@ struct DecodeLaunch {
   size_t smem;       // dynamic shared memory per CTA
 };
 // Shape of the decode pass for a batch capacity (grid sized to fill every SM).
-int plan_decode(int group, int page_size, int max_batch, int num_sms, DecodeLaunch* out);
+int plan_decode(int group, int page_size, int max_batch, int num_sms, int fp4, DecodeLaunch* out);
 int launch_decode(const DecodeParams& p, const DecodeLaunch& L, cudaStream_t stream);
 
 }  // namespace kvq

@@ -67,6 +67,7 @@ bool noalloc_desc_ok(const kvq_desc* d) {
   if (hb != 1 && hb != 32 && hb != 64 && hb != 128) return false;  // 1: plain INT4, no rotation
   const int S = d->page_size;
   if (S != 16 && S != 32 && S != 64 && S != 128 && S != 256) return false;
+  if (d->kv_format != KVQ_FORMAT_INT4 && d->kv_format != KVQ_FORMAT_NVFP4) return false;
   if (d->max_batch > 4096) return false;
   if (static_cast<long long>(d->max_pages_per_seq) * S > (1LL << 30)) return false;
   const long long tiles_per_seq = (static_cast<long long>(d->max_pages_per_seq) * S + 31) / 32;
@@ -105,12 +106,13 @@ int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, int32_t la
   if (rc != KVQ_OK) return rc;
 
   kvq::DecodeLaunch L;
-  if (kvq::plan_decode(g, d->page_size, batch, num_sms, &L) != 0) return KVQ_ECUDA;
+  const int fp4 = d->kv_format == KVQ_FORMAT_NVFP4;
+  if (kvq::plan_decode(g, d->page_size, batch, num_sms, fp4, &L) != 0) return KVQ_ECUDA;
   if ((units + L.grid) * g > kNoAllocMaxRecords) return KVQ_EUNSUPPORTED;
 
   kvq::DecodeParams p;
   const size_t layer_bytes = static_cast<size_t>(d->num_pages) * d->num_kv_heads *
-                             d->page_size * (d->head_dim + 4);
+                             d->page_size * (d->head_dim + (fp4 ? d->head_dim / 8 : 4));
   p.pool_layer = static_cast<const uint8_t*>(pool) + static_cast<size_t>(layer) * layer_bytes;
   p.q = static_cast<const __half*>(q);
   p.seq_lens = seq_lens;
@@ -134,6 +136,7 @@ int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, int32_t la
   p.total_ctas = L.grid;
   p.k_new = nullptr;
   p.v_new = nullptr;
+  p.fp4 = fp4;
   const int lrc = kvq::launch_decode(p, L, static_cast<cudaStream_t>(stream));
   if (lrc == -1) return KVQ_EUNSUPPORTED;
   return lrc == 0 ? KVQ_OK : KVQ_ECUDA;

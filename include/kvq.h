@@ -6,6 +6,8 @@
  *   [P1] "KVキャッシュを4ビットへ — SAW-INT4とシステムを踏まえたINT4量子化" (youngju.dev)
  *   [P2] "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving"
  *        (gist.science)
+ *   [P3] "BitDecoding-FP4:FP4 KVキャッシュのネイティブ復号" (sns.style): the NVFP4
+ *        cache format, kv_format = KVQ_FORMAT_NVFP4 below
  *
  *   * Every new K/V row (fp16, head_dim = 128 channels) is rotated by an orthonormal
  *     block-diagonal Hadamard transform (blocks of b = 32, 64 or 128 channels) [P1,
@@ -28,12 +30,22 @@
  *   GQA        query head hq reads KV head hq / (num_q_heads / num_kv_heads);
  *   softmax    scale 1/sqrt(head_dim) unless given; an empty sequence outputs zeros.
  *
+ * NVFP4 format (kv_format = KVQ_FORMAT_NVFP4) [P3, "背景と概要", "深掘り分析": a 4-bit
+ * microscaling format with E4M3 block scales; the pages give no formulas, the readings]:
+ *   the same rotation; then per block of 16 channels an E4M3 scale s = the fp32 value
+ *   max |y| / 6 rounded to nearest even and saturated at 448; codes = E2M1 (sign, 2
+ *   exponent bits, 1 mantissa bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6) nearest to y * (1/s)
+ *   (fp32 reciprocal and product), ties to the even code, saturated at 6, the sign kept;
+ *   all codes 0 when s == 0; no per-tensor scale.  Packing as for INT4.
+ *
  * Pool layout (device memory, bytes; one pool holds every layer):
  *   block(layer, page, kv_head) starts at
- *       ((layer * num_pages + page) * num_kv_heads + kv_head) * page_size * 132
- *   and holds, for the page_size token slots of that page:
+ *       ((layer * num_pages + page) * num_kv_heads + kv_head) * page_size * R
+ *   with R = 132 (INT4) or 144 (NVFP4), and holds, for the page_size token slots:
  *       [K codes  page_size x 64 B][V codes  page_size x 64 B]
- *       [K scales page_size x fp16][V scales page_size x fp16]
+ *       [K scales page_size x fp16][V scales page_size x fp16]           (INT4)
+ *       [K scales page_size x 8 E4M3][V scales page_size x 8 E4M3]       (NVFP4: block j
+ *                                                          of a row = channels 16j..16j+15)
  *   Token at position pos of sequence b lives in page page_table[b][pos / page_size],
  *   slot pos % page_size.  The page table is shared by all layers.
  *
@@ -106,7 +118,12 @@ typedef struct kvq_cache kvq_cache; /* opaque, library-owned handle */
  *   page_size          S tokens per page: 16, 32, 64, 128 or 256
  *   num_pages          pages per layer in the pool                            (>= 1)
  *   max_batch          largest batch any call will pass                (1 .. 4096)
- *   max_pages_per_seq  row length of the page table                          (>= 1) */
+ *   max_pages_per_seq  row length of the page table                          (>= 1)
+ *   kv_format          KVQ_FORMAT_INT4 (0) or KVQ_FORMAT_NVFP4 (1); NVFP4 caches support
+ *                      append and decode (fused append + decode and chunked prefill
+ *                      return KVQ_EUNSUPPORTED) */
+#define KVQ_FORMAT_INT4 0
+#define KVQ_FORMAT_NVFP4 1
 typedef struct {
   int32_t num_layers;
   int32_t num_kv_heads;
@@ -117,10 +134,11 @@ typedef struct {
   int32_t num_pages;
   int32_t max_batch;
   int32_t max_pages_per_seq;
+  int32_t kv_format;
 } kvq_desc;
 
 /* Bytes of the pool a descriptor needs:
- * num_layers * num_pages * num_kv_heads * page_size * (head_dim + 4).
+ * num_layers * num_pages * num_kv_heads * page_size * R (R = 132 INT4, 144 NVFP4).
  * Returns 0 for an invalid descriptor.  Host only. */
 KVQ_API size_t kvq_pool_bytes(const kvq_desc* d);
 

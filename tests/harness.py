@@ -2,8 +2,9 @@
 and through the CPU oracle on the same seeded inputs, and compare.
 
 Acceptance (the tolerance readings stated in the design notes):
-* page tables and fp16 scales bit-exact;
-* INT4 codes exact except +-1 flips, counted, fewer than 1e-5 of all codes;
+* page tables and fp16 scales bit-exact (NVFP4: E4M3 scales bit-exact);
+* INT4 codes exact except +-1 flips, counted, fewer than 1e-5 of all codes (NVFP4: E2M1
+  codes likewise, a flip being a step to the neighbouring magnitude with the same sign);
 * decode outputs |gpu - ref| <= 2e-3 + 1e-2 * |ref| elementwise, ref = fp64 oracle on the
   GPU-written (same dequantised) cache.
 """
@@ -30,6 +31,7 @@ class Case:
     layer: int = 0
     num_layers: int = 1
     max_batch: int = 0
+    fmt: int = 0                 # 0 = rotated INT4, 1 = NVFP4
 
     @property
     def capacity(self):
@@ -39,16 +41,16 @@ class Case:
         import bit_paged_kv_diag_b200 as kvq
         return kvq.Desc(self.num_layers, self.w.num_kv_heads, self.w.num_q_heads, 128,
                         self.block, self.w.page_size, self.num_pages,
-                        max(self.max_batch, len(self.lengths)), self.max_pages_per_seq)
+                        max(self.max_batch, len(self.lengths)), self.max_pages_per_seq, self.fmt)
 
     def geometry(self):
         return oracle.Geometry(self.num_layers, self.w.num_kv_heads, self.w.num_q_heads, 128,
                                self.block, self.w.page_size, self.num_pages,
-                               self.max_pages_per_seq)
+                               self.max_pages_per_seq, self.fmt)
 
 
 def make_case(w, lengths, new, block=None, pool_factor=None, permute=None, extra_pages_per_seq=0,
-              layer=0, num_layers=1, max_batch=0):
+              layer=0, num_layers=1, max_batch=0, fmt=0):
     lengths = np.asarray(lengths, np.int32)
     new = np.asarray(new, np.int32)
     S = w.page_size
@@ -59,7 +61,7 @@ def make_case(w, lengths, new, block=None, pool_factor=None, permute=None, extra
     perm = w.permute_pages if permute is None else permute
     order = workloads.rng_for(w, 2, len(lengths)).permutation(P).astype(np.int32) if perm else None
     mp = max(1, int(need_pages.max()) + extra_pages_per_seq)
-    return Case(w, lengths, new, block or w.block, P, order, mp, layer, num_layers, max_batch)
+    return Case(w, lengths, new, block or w.block, P, order, mp, layer, num_layers, max_batch, fmt)
 
 
 def host_inputs(case: Case):
@@ -120,7 +122,7 @@ def compare_pools(case: Case, gpu_pool: np.ndarray, ref_pool: np.ndarray):
     """(scale mismatches, code flips (+-1), other code mismatches, total codes)."""
     g = case.geometry()
     S = g.page_size
-    blk = S * 132
+    blk = oracle.block_bytes(S, 128, g.fmt)
     a = gpu_pool.reshape(-1, blk)
     b = ref_pool.reshape(-1, blk)
     scale_mis = int(np.count_nonzero(a[:, S * 128:] != b[:, S * 128:]))
@@ -133,9 +135,14 @@ def compare_pools(case: Case, gpu_pool: np.ndarray, ref_pool: np.ndarray):
         for sh in (0, 4):
             na = ((xa >> sh) & 0xF)
             nb = ((xb >> sh) & 0xF)
-            na = np.where(na >= 8, na - 16, na)
-            nb = np.where(nb >= 8, nb - 16, nb)
-            d = np.abs(na - nb)
+            if g.fmt == 1:  # E2M1: sign bit 3, magnitude index 0..7
+                same_sign = (na & 8) == (nb & 8)
+                d = np.where(same_sign, np.abs((na & 7) - (nb & 7)), 99)
+                d = np.where(na == nb, 0, d)
+            else:
+                na = np.where(na >= 8, na - 16, na)
+                nb = np.where(nb >= 8, nb - 16, nb)
+                d = np.abs(na - nb)
             flips += int(np.count_nonzero(d == 1))
             other += int(np.count_nonzero(d > 1))
     total_codes = int(ca.size) * 2

@@ -45,8 +45,12 @@ def test_pool_bytes_and_descriptor_validation():
     d = _desc()
     assert kvq.pool_bytes(d) == 2 * 100 * 8 * 16 * 132
     assert kvq.pool_bytes(_desc(hadamard_block=1)) == 2 * 100 * 8 * 16 * 132  # plain INT4
+    # NVFP4: 64 B codes + 8 E4M3 scale bytes per K and per V row
+    assert kvq.pool_bytes(_desc(kv_format=kvq.FORMAT_NVFP4)) == 2 * 100 * 8 * 16 * 144
+    import oracle
+    assert 144 * 16 == oracle.block_bytes(16, 128, 1)
     for bad in [dict(head_dim=64), dict(hadamard_block=16), dict(hadamard_block=2),
-                dict(page_size=24),
+                dict(page_size=24), dict(kv_format=2), dict(kv_format=-1),
                 dict(num_q_heads=24), dict(num_q_heads=48), dict(max_batch=5000),
                 dict(num_layers=0), dict(num_pages=0)]:
         assert kvq.pool_bytes(_desc(**bad)) == 0, bad
