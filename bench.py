@@ -51,16 +51,21 @@ def _peaks():
         return 6650.0, "fallback"
 
 
-def decode_bytes(lengths_after, num_kv_heads, num_q_heads, page_size):
+def decode_bytes(lengths_after, num_kv_heads, num_q_heads, page_size, per_token_head=None):
     lengths_after = np.asarray(lengths_after, np.int64)
-    cache = int(lengths_after.sum()) * num_kv_heads * BYTES_PER_TOKEN_HEAD
+    per = BYTES_PER_TOKEN_HEAD if per_token_head is None else per_token_head
+    cache = int(lengths_after.sum()) * num_kv_heads * per
     table = int(((lengths_after + page_size - 1) // page_size).sum()) * 4
     qo = 2 * len(lengths_after) * num_q_heads * 128 * 2
     return cache + table + qo
 
 
-def append_bytes(tokens, num_kv_heads):
-    return int(tokens) * num_kv_heads * (2 * 256 + 132)
+def append_bytes(tokens, num_kv_heads, row_bytes=132):
+    return int(tokens) * num_kv_heads * (2 * 256 + row_bytes)
+
+
+# NVFP4 rows: 64 B of E2M1 codes and 8 E4M3 scales for K and for V.
+BYTES_PER_TOKEN_HEAD_NVFP4 = 2 * 64 + 2 * 8
 
 
 # --------------------------------------------------------------------- clocks --
@@ -309,6 +314,7 @@ def run_kvq(args, rank, world, local_rank):
     cache.close()
     append = run_append_bench(dev) if rank == 0 else None
     plain = run_plain_decode_bench(dev) if rank == 0 else None
+    nvfp4 = run_nvfp4_bench(dev) if rank == 0 else None
     prefill = run_prefill_bench(dev) if rank == 0 else None
 
     line = {
@@ -342,6 +348,7 @@ def run_kvq(args, rank, world, local_rank):
         "bytes_per_launch": dec_b, "timing": dec_how}
     line["append"] = append
     line["plain_int4"] = plain
+    line["nvfp4"] = nvfp4
     line["prefill"] = prefill
     line["clocks"] = clk.result
     return line
@@ -455,6 +462,92 @@ def run_plain_decode_bench(dev, reps=10):
         cache.close()
     res["how"] = ("graph of 36 decode calls over 4 layer pools of the qwen3_4b_decode shape, "
                   "b = 128 (rotated) and b = 1 (plain INT4)")
+    return res
+
+
+def run_nvfp4_bench(dev, reps=10):
+    """The NVFP4 cache format (E2M1 codes, E4M3 scale per 16 channels, b = 128): decode on
+    the Qwen3-4B-shaped layer (a graph of 36 calls over 4 layer pools, as the plain-INT4
+    line) and the 8 x 8192-token prefill append."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    peak, peak_kind = _peaks()
+    res = {}
+    w = workloads.WORKLOADS[WORKLOAD]
+    L = np.asarray(w.context, np.int32)
+    B, H, HQ, S, NL = w.batch, w.num_kv_heads, w.num_q_heads, w.page_size, 4
+    cap = L + 1
+    P = workloads.pool_pages(w, cap)
+    mp = int((cap.max() + S - 1) // S)
+    desc = kvq.Desc(NL, H, HQ, 128, w.block, S, P, B, mp, kvq.FORMAT_NVFP4)
+    cache, pt = kvq.alloc_pages(desc, cap, None)
+    ptd = torch.from_numpy(pt).to(dev)
+    zeros = torch.zeros(B, dtype=torch.int32, device=dev)
+    cu = torch.from_numpy(workloads.cu_seqlens(cap)).to(dev)
+    for layer in range(NL):
+        kp = workloads.kv_rows_torch(w, layer, 0, int(cap.sum()), stream=1, device=dev)
+        vp = workloads.kv_rows_torch(w, layer, 1, int(cap.sum()), stream=1, device=dev)
+        kvq.rotate_quant_append(cache, layer, kp, vp, cu, zeros, ptd)
+        del kp, vp
+    q = torch.stack([workloads.q_rows_torch(w, l, device=dev) for l in range(NL)])
+    out = torch.empty_like(q)
+    lens = torch.from_numpy(cap).to(dev)
+    side = torch.cuda.Stream(device=dev)
+    kvq.decode_attention(cache, 0, q[0], lens, ptd, out=out[0])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(36):
+            kvq.decode_attention(cache, i % NL, q[i % NL], lens, ptd, out=out[i % NL])
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / (reps * 36)
+    nb = decode_bytes(cap, H, HQ, S, BYTES_PER_TOKEN_HEAD_NVFP4)
+    gbs = nb / (us * 1e-6) / 1e9
+    res["decode"] = {"us_per_launch": round(us, 3), "bytes_per_launch": nb, "gbs": round(gbs, 1),
+                     "frac": round(gbs / peak, 4), "peak": peak, "peak_kind": peak_kind,
+                     "traffic": _traffic("decode_nvfp4", nb),
+                     "how": "graph of 36 decode calls over 4 layer pools of the qwen3_4b_decode "
+                            "shape, b = 128, 144 B per (token, KV head)"}
+    assert kvq.get_device_status(cache) == 0
+    del g
+    cache.close()
+
+    wa = workloads.WORKLOADS["prefill_append"]
+    B, H, S, T = wa.batch, wa.num_kv_heads, wa.page_size, wa.batch * wa.new_tokens
+    cap = np.full(B, wa.new_tokens, np.int32)
+    P = workloads.pool_pages(wa, cap)
+    mp = int((cap.max() + S - 1) // S)
+    k = workloads.kv_rows_torch(wa, 0, 0, T, stream=1, device=dev)
+    v = workloads.kv_rows_torch(wa, 0, 1, T, stream=1, device=dev)
+    cu = torch.from_numpy(workloads.cu_seqlens(cap)).to(dev)
+    z = torch.zeros(B, dtype=torch.int32, device=dev)
+    desc = kvq.Desc(1, H, wa.num_q_heads, 128, 128, S, P, B, mp, kvq.FORMAT_NVFP4)
+    cache, pt = kvq.alloc_pages(desc, cap, None)
+    ptd = torch.from_numpy(pt).to(dev)
+    for _ in range(3):
+        kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(20):
+        kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / 20
+    gbs = append_bytes(T, H, BYTES_PER_TOKEN_HEAD_NVFP4) / (us * 1e-6) / 1e9
+    res["append_b128"] = {"us_per_call": round(us, 2), "tok_s": round(T / (us * 1e-6), 1),
+                          "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                          "workload": "prefill_append: 8 x 8192 tokens, 8 KV heads, page 16"}
+    assert kvq.get_device_status(cache) == 0
+    cache.close()
     return res
 
 
@@ -608,12 +701,15 @@ def run_kernel_case(which, calls):
     layer of the Qwen3-4B-shaped workload (69 MB of cache); ``fused`` = the same with the
     step's one-token append fused in; ``append`` = the prefill-append call (8 x 8192
     tokens, b = 128; 268 MB read, 69 MB written); ``prefill`` = chunked-prefill attention
-    (16 x 128-token chunks after 896 cached tokens).  The kernel is launched ``calls``
+    (16 x 128-token chunks after 896 cached tokens); ``decode_nvfp4`` and ``append_nvfp4``
+    are the decode and append cases on an NVFP4 cache.  The kernel is launched ``calls``
     times after the setup."""
     import torch
 
     import bit_paged_kv_diag_b200 as kvq
     dev = torch.device("cuda", 0)
+    fmt = kvq.FORMAT_NVFP4 if which.endswith("_nvfp4") else kvq.FORMAT_INT4
+    which = which.replace("_nvfp4", "")
     if which == "prefill":
         # 16 sequences, a 128-token chunk after 896 cached tokens (chunked_prefill's heads).
         w = workloads.WORKLOADS["chunked_prefill"]
@@ -644,7 +740,8 @@ def run_kernel_case(which, calls):
         B, H, S, T = w.batch, w.num_kv_heads, w.page_size, w.batch * w.new_tokens
         cap = np.full(B, w.new_tokens, np.int32)
         P = workloads.pool_pages(w, cap)
-        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S))
+        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S),
+                        fmt)
         cache, pt = kvq.alloc_pages(desc, cap, None)
         ptd = torch.from_numpy(pt).to(dev)
         k = workloads.kv_rows_torch(w, 0, 0, T, stream=1, device=dev)
@@ -660,7 +757,8 @@ def run_kernel_case(which, calls):
         B, H, S = w.batch, w.num_kv_heads, w.page_size
         cap = L + 1
         P = workloads.pool_pages(w, cap)
-        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S))
+        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S),
+                        fmt)
         cache, pt = kvq.alloc_pages(desc, cap, None)
         ptd = torch.from_numpy(pt).to(dev)
         kp = workloads.kv_rows_torch(w, 0, 0, int(cap.sum()), stream=1, device=dev)
@@ -693,7 +791,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["decode", "fused", "append", "prefill"], default=None,
+    ap.add_argument("--kernel-case", choices=["decode", "fused", "append", "prefill", "decode_nvfp4",
+                                              "append_nvfp4"], default=None,
                     help="run one small case of one kernel (for ncu captures) and exit")
     ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()
