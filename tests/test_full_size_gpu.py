@@ -8,7 +8,8 @@ at full size, with inputs drawn on the device by the seeded generators.  Checked
 * the page table, bit-exact against the oracle's allocator (whole table);
 * appended rows: for a seeded sample of (token, KV head, K|V) rows, the oracle's rotation,
   scale and codes of the same input row against the bytes the kernel wrote at the row's
-  page and slot (scale bit-exact, codes exact up to counted +-1 flips);
+  page and slot (scale bit-exact, codes exact up to counted +-1 flips; for the NVFP4
+  format the 8 E4M3 scales and the E2M1 codes);
 * decode outputs: for a few whole sequences (the longest, the shortest, one more), the
   fp64 oracle over the GPU-written cache against the kernel's fp16 output rows, within
   |d| <= 2e-3 + 1e-2 |ref|.
@@ -28,7 +29,7 @@ W = workloads.WORKLOADS
 ROW_SAMPLES = 1500
 
 
-def _run_full(w, block):
+def _run_full(w, block, fmt=0):
     """Prefill every cached token, append the step's tokens, decode; returns host views."""
     import torch
 
@@ -41,7 +42,7 @@ def _run_full(w, block):
     P = workloads.pool_pages(w, cap)
     order = workloads.page_order(w, P)
     mp = int((cap.max() + S - 1) // S)
-    desc = kvq.Desc(1, H, w.num_q_heads, 128, block, S, P, w.batch, mp)
+    desc = kvq.Desc(1, H, w.num_q_heads, 128, block, S, P, w.batch, mp, fmt)
     pool = torch.zeros(kvq.pool_bytes(desc), dtype=torch.uint8, device=dev)
     cache, pt = kvq.alloc_pages(desc, cap, order, pool=pool)
     ptd = torch.from_numpy(pt).to(dev)
@@ -68,10 +69,10 @@ def _run_full(w, block):
     return res
 
 
-def _check_rows(w, block, r, rng):
+def _check_rows(w, block, r, rng, fmt=0):
     """Sampled appended rows against the oracle's rotation + quantisation of the same row."""
     S, H = w.page_size, w.num_kv_heads
-    blk = S * 132
+    blk = oracle.block_bytes(S, 128, fmt)
     flips = total = 0
     for name, (k, v, cu, before) in r["rows"].items():
         n = k.shape[0]
@@ -88,11 +89,24 @@ def _check_rows(w, block, r, rng):
             slot = pos % S
             h, kv = int(heads[i]), int(kvs[i])
             x = (vs if kv else ks)[i, h].astype(np.float32)
-            bits, codes = oracle.quant_row(oracle.fwht_f32(x, block))
             base = (page * H + h) * blk
+            packed = r["pool"][base + kv * S * 64 + slot * 64:][:64]
+            if fmt == 1:
+                codes, scales = oracle.quant_row_nvfp4(oracle.fwht_f32(x, block))
+                got_scales = r["pool"][base + S * 128 + kv * S * 8 + slot * 8:][:8]
+                assert np.array_equal(got_scales, scales), (name, int(t), h, kv)
+                got = np.stack([packed & 0xF, packed >> 4], 1).reshape(-1)
+                same = (got & 8) == (codes & 8)
+                d = np.where(got == codes, 0, np.where(same, np.abs((got & 7).astype(np.int16) -
+                                                                   (codes & 7).astype(np.int16)), 99))
+                assert d.max() <= 1, (name, int(t), h, kv)
+                flips += int(np.count_nonzero(d))
+                total += 128
+                continue
+            bits, codes = oracle.quant_row(oracle.fwht_f32(x, block))
             got_scale = int(r["pool"][base + S * 128 + kv * S * 2 + slot * 2:][:2].view(np.uint16)[0])
             assert got_scale == bits, (name, int(t), h, kv, got_scale, bits)
-            got = oracle.unpack_codes(r["pool"][base + kv * S * 64 + slot * 64:][:64], 128)
+            got = oracle.unpack_codes(packed, 128)
             d = np.abs(got.astype(np.int16) - codes.astype(np.int16))
             assert d.max() <= 1, (name, int(t), h, kv)
             flips += int(np.count_nonzero(d))
@@ -100,25 +114,25 @@ def _check_rows(w, block, r, rng):
     assert flips <= max(1, 1e-5 * total), f"{flips} +-1 flips in {total} sampled codes"
 
 
-def _check_decode(w, block, r, seqs):
+def _check_decode(w, block, r, seqs, fmt=0):
     g = oracle.Geometry(1, w.num_kv_heads, w.num_q_heads, 128, block, w.page_size, r["P"],
-                        r["mp"])
+                        r["mp"], fmt)
     for b in seqs:
         ref = oracle.decode_attention(g, r["pool"], 0, r["q"][b:b + 1], r["cap"][b:b + 1],
                                       r["page_table"][b:b + 1])
         check_outputs(r["out"][b:b + 1], ref, f"{w.name} sequence {b}")
 
 
-def _full_size_parity(w, block, seed):
-    r = _run_full(w, block)
+def _full_size_parity(w, block, seed, fmt=0):
+    r = _run_full(w, block, fmt)
     assert r["status"] == 0, f"device status {r['status']}"
     pt_ref = oracle.assign_pages(r["cap"], w.page_size, r["P"], r["mp"], r["order"])
     assert np.array_equal(r["page_table"], pt_ref), "page table differs from the oracle's"
     rng = np.random.default_rng(seed)
-    _check_rows(w, block, r, rng)
+    _check_rows(w, block, r, rng, fmt)
     cap = r["cap"]
     seqs = sorted({int(np.argmax(cap)), int(np.argmin(cap)), int(rng.integers(0, len(cap)))})
-    _check_decode(w, block, r, seqs)
+    _check_decode(w, block, r, seqs, fmt)
 
 
 def test_long_context_full_size():
@@ -138,6 +152,17 @@ def test_prefill_append_full_size(block):
     """8 x 8192 new tokens in one append call, then decode over them (b = 1 is plain INT4)."""
     w = W["prefill_append"]
     _full_size_parity(w, block, 103 + block)
+
+
+def test_nvfp4_ragged_full_size():
+    """The NVFP4 cache on the ragged workload at full size (256 sequences, scattered pages)."""
+    w = W["ragged"]
+    _full_size_parity(w, w.block, 202, fmt=1)
+
+
+def test_nvfp4_prefill_append_full_size():
+    """8 x 8192 new tokens into an NVFP4 cache in one call, then decode (b = 128)."""
+    _full_size_parity(W["prefill_append"], 128, 203, fmt=1)
 
 
 def test_chunked_prefill_full_size():
