@@ -74,3 +74,76 @@ def test_nvfp4_unsupported_calls():
         assert e.value.status == kvq.KVQ_EUNSUPPORTED
     finally:
         cache.close()
+
+
+def _edge_rows(n, H, rng):
+    """fp16 rows [n][H][128] whose 16-channel blocks hit the format's edges: saturating
+    scales (max |y| / 6 > 448), scales that round to zero or to subnormal E4M3 values, exact
+    E2M1 ties (scale 0.5 so that y * (1/s) is exact), signed zeros, all-zero blocks, and
+    ordinary Gaussian blocks."""
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float64)
+    rows = np.zeros((n, H, 128), np.float64)
+    for t in range(n):
+        for h in range(H):
+            for blk in range(8):
+                kind = (t * 7 + h * 3 + blk) % 7
+                x = rng.standard_normal(16)
+                if kind == 0:      # saturating: up to 60000
+                    x = x / np.abs(x).max() * 60000.0
+                elif kind == 1:    # max / 6 below half the smallest E4M3 step: scale 0
+                    x = x / np.abs(x).max() * 4e-3
+                elif kind == 2:    # subnormal E4M3 scale
+                    x = x / np.abs(x).max() * 0.05
+                elif kind == 3:    # exact ties at scale 0.5 (max = 3)
+                    x = np.concatenate([mids * 0.5, -mids * 0.5, [3.0, -0.0]])
+                    rng.shuffle(x)
+                elif kind == 4:    # all zero, some negative zeros
+                    x = np.where(rng.integers(0, 2, 16) == 1, -0.0, 0.0)
+                elif kind == 5:    # ties at scale 0.5 plus tiny values rounding to +-0
+                    x = np.concatenate([mids * 0.5, [3.0, 0.01, -0.01, 0.1, -0.1, 0.2, -0.2, 0.12, -0.12]])
+                rows[t, h, 16 * blk:16 * blk + 16] = x
+    return rows.astype(np.float16)
+
+
+@pytest.mark.parametrize("block", [1, 32])
+def test_nvfp4_edge_rows(block):
+    """Constructed rows through append and decode: the pool must equal the oracle's byte for
+    byte (ties, saturation, zero and subnormal scales, signed zeros), outputs within the
+    tolerance of the fp64 oracle on that pool."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    import oracle
+    from harness import check_outputs
+    rng = np.random.default_rng(31)
+    H, HQ, S, L = 2, 8, 16, 77
+    k = _edge_rows(L, H, rng)
+    v = _edge_rows(L, H, rng)
+    P = 8
+    d = kvq.Desc(1, H, HQ, 128, block, S, P, 1, P, kvq.FORMAT_NVFP4)
+    dev = torch.device("cuda")
+    pool = torch.zeros(kvq.pool_bytes(d), dtype=torch.uint8, device=dev)
+    cap = np.array([L], np.int32)
+    cache, pt = kvq.alloc_pages(d, cap, None, pool=pool)
+    try:
+        ptd = torch.from_numpy(pt).to(dev)
+        kvq.rotate_quant_append(cache, 0, torch.from_numpy(k).to(dev), torch.from_numpy(v).to(dev),
+                                torch.tensor([0, L], dtype=torch.int32, device=dev),
+                                torch.zeros(1, dtype=torch.int32, device=dev), ptd)
+        q = rng.standard_normal((1, HQ, 128)).astype(np.float16)
+        out = kvq.decode_attention(cache, 0, torch.from_numpy(q).to(dev),
+                                   torch.from_numpy(cap).to(dev), ptd)
+        torch.cuda.synchronize()
+        assert kvq.get_device_status(cache) == 0
+        gpool = pool.cpu().numpy()
+        gout = out.float().cpu().numpy()
+    finally:
+        cache.close()
+    g = oracle.Geometry(1, H, HQ, 128, block, S, P, P, fmt=1)
+    ref_pool = g.new_pool()
+    oracle.rotate_quant_append(g, ref_pool, 0, k, v, np.array([0, L], np.int32),
+                               np.array([0], np.int32), pt)
+    diff = np.nonzero(gpool != ref_pool)[0]
+    assert diff.size == 0, f"{diff.size} pool bytes differ, first at {diff[:8]}"
+    ref = oracle.decode_attention(g, gpool, 0, q, cap, pt)
+    check_outputs(gout, ref, f"nvfp4 edge rows b={block}")
