@@ -42,6 +42,12 @@
 // sum is not precise enough to cancel a large offset afterwards.)  The GQA group is the N = 8
 // side of both products; the dequantised cache is the M side.  The K scale multiplies the
 // fp32 score of its token; softmax runs in the log2 domain with exp2.
+//
+// NVFP4 cache (template argument FP4; "BitDecoding-FP4:FP4 KVキャッシュのネイティブ復号"
+// (sns.style): E2M1 codes with an E4M3 scale per 16 channels, 144-byte token rows): the
+// same work split, rings and merges; K and V are dequantised exactly to fp16 (hardware
+// E2M1 / E4M3 conversions and one fp16 multiply), both products run as f16 mma.sync, and q
+// is carried as fp16 hi + lo parts (tile_qk4, tile_pv4, prep_q4_warp).
 #include <cuda_fp16.h>
 #include <math_constants.h>
 #include <stdint.h>
