@@ -51,6 +51,13 @@ def test_nvfp4_group_and_page_size_grid(group, page_size):
                           pool_factor=1.3, fmt=1))
 
 
+def test_nvfp4_multi_layer_pool_and_custom_softmax_scale():
+    """Layer offsets inside a multi-layer NVFP4 pool, and an explicit softmax scale."""
+    w = W["ragged"]
+    full_parity(make_case(w, [200, 90, 333], [1, 1, 1], layer=2, num_layers=3, fmt=1),
+                softmax_scale=0.05)
+
+
 def test_nvfp4_unsupported_calls():
     import torch
 

@@ -18,15 +18,16 @@ from harness import ATOL, RTOL, CudaRun, host_inputs, make_case
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name,lengths", [
-    ("long_context", [5000, 31, 1, 2600]),    # units split over many CTAs, and short ones
-    ("qwen3_4b_decode", [517, 300, 64, 1, 0, 129, 63, 65]),
+@pytest.mark.parametrize("name,lengths,fmt", [
+    ("long_context", [5000, 31, 1, 2600], 0),    # units split over many CTAs, and short ones
+    ("qwen3_4b_decode", [517, 300, 64, 1, 0, 129, 63, 65], 0),
+    ("qwen3_4b_decode", [517, 300, 64, 1, 0, 129, 63, 65], 1),   # NVFP4 cache
 ])
-def test_noalloc_decode_matches_handle_decode_twice(name, lengths):
+def test_noalloc_decode_matches_handle_decode_twice(name, lengths, fmt):
     import torch
     import bit_paged_kv_diag_b200 as kvq
     w = workloads.WORKLOADS[name]
-    case = make_case(w, lengths, [1] * len(lengths))
+    case = make_case(w, lengths, [1] * len(lengths), fmt=fmt)
     kp, vp, kn, vn, q = host_inputs(case)
     run = CudaRun(case, kp, vp, kn, vn, q)
     try:
