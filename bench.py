@@ -517,6 +517,31 @@ def run_nvfp4_bench(dev, reps=10):
                      "traffic": _traffic("decode_nvfp4", nb),
                      "how": "graph of 36 decode calls over 4 layer pools of the qwen3_4b_decode "
                             "shape, b = 128, 144 B per (token, KV head)"}
+    del g
+    # The fused step on the NVFP4 cache: per layer one kvq_append_decode_attention (the
+    # same token re-appended at position L every replay).
+    kn = torch.stack([workloads.kv_rows_torch(w, l, 0, B, stream=2, device=dev) for l in range(NL)])
+    vn = torch.stack([workloads.kv_rows_torch(w, l, 1, B, stream=2, device=dev) for l in range(NL)])
+    before = torch.from_numpy(L).to(dev)
+    kvq.append_decode_attention(cache, 0, kn[0], vn[0], q[0], before, ptd, out=out[0])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(36):
+            kvq.append_decode_attention(cache, i % NL, kn[i % NL], vn[i % NL], q[i % NL], before,
+                                        ptd, out=out[i % NL])
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    step_b = 36 * (nb + B * H * 2 * 256 + B * H * BYTES_PER_TOKEN_HEAD_NVFP4)
+    res["fused_step"] = {"ms_per_36_layers": round(ms, 5), "gbs": round(step_b / (ms * 1e-3) / 1e9, 1),
+                         "how": "graph of 36 kvq_append_decode_attention calls over 4 layer pools"}
     assert kvq.get_device_status(cache) == 0
     del g
     cache.close()

@@ -871,8 +871,12 @@ __device__ __forceinline__ void tile_pv4(State<G>& st, const uint8_t* slot, int 
     const uint2 t1 = *reinterpret_cast<const uint2*>(vb + (c + 4) * 64 + 8 * g);
     const uint2 t2 = *reinterpret_cast<const uint2*>(vb + (c + 8) * 64 + 8 * g);
     const uint2 t3 = *reinterpret_cast<const uint2*>(vb + (c + 12) * 64 + 8 * g);
-    const uint32_t s01 = static_cast<uint32_t>(vs[(c + 0) * 8 + g]) | (static_cast<uint32_t>(vs[(c + 4) * 8 + g]) << 8);
-    const uint32_t s23 = static_cast<uint32_t>(vs[(c + 8) * 8 + g]) | (static_cast<uint32_t>(vs[(c + 12) * 8 + g]) << 8);
+    // Tokens past the sequence's end take scale 0: their slot bytes are whatever the pool or
+    // an earlier tile left there, and an E4M3 NaN would survive the zero probability.
+    const int t0n = 16 * j + c;
+    const uint32_t s0 = t0n < ntok ? vs[(c + 0) * 8 + g] : 0u, s1 = t0n + 4 < ntok ? vs[(c + 4) * 8 + g] : 0u;
+    const uint32_t s2 = t0n + 8 < ntok ? vs[(c + 8) * 8 + g] : 0u, s3 = t0n + 12 < ntok ? vs[(c + 12) * 8 + g] : 0u;
+    const uint32_t s01 = s0 | (s1 << 8), s23 = s2 | (s3 << 8);
     const uint32_t S01 = e4m3x2_to_f16x2(s01), S23 = e4m3x2_to_f16x2(s23);
     const uint32_t w0[2] = {t0.x, t0.y}, w1[2] = {t1.x, t1.y};
     const uint32_t w2[2] = {t2.x, t2.y}, w3[2] = {t3.x, t3.y};
@@ -1154,10 +1158,14 @@ __device__ __forceinline__ uint2 load_new_row(const __half* row, int lane) {
   return __ldg(reinterpret_cast<const uint2*>(row) + lane);  // channels 4*lane..4*lane+3
 }
 
-__device__ __forceinline__ NewRow quantise_new_row(uint2 raw, int lane, const DecodeParams& p) {
+// The rotated row y = fl(c_b * butterfly(x)) of channels 4*lane..4*lane+3.
+__device__ __forceinline__ void rotate_new_row(uint2 raw, int lane, const DecodeParams& p, float (&x)[4]) {
   const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
   const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-  float x[4] = {lo.x, lo.y, hi.x, hi.y};
+  x[0] = lo.x;
+  x[1] = lo.y;
+  x[2] = hi.x;
+  x[3] = hi.y;
   if (p.hadamard_block > 1) {
     const float a0 = __fadd_rn(x[0], x[1]), a1 = __fsub_rn(x[0], x[1]);
     const float a2 = __fadd_rn(x[2], x[3]), a3 = __fsub_rn(x[2], x[3]);
@@ -1176,6 +1184,11 @@ __device__ __forceinline__ NewRow quantise_new_row(uint2 raw, int lane, const De
 #pragma unroll
     for (int e = 0; e < 4; e++) x[e] = __fmul_rn(x[e], p.cb);
   }
+}
+
+__device__ __forceinline__ NewRow quantise_new_row(uint2 raw, int lane, const DecodeParams& p) {
+  float x[4];
+  rotate_new_row(raw, lane, p, x);
   float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
   for (int d = 1; d < 32; d *= 2) m = fmaxf(m, __shfl_xor_sync(kFull, m, d));
@@ -1200,18 +1213,67 @@ __device__ __forceinline__ NewRow quantise_new_row(uint2 raw, int lane, const De
   return r;
 }
 
+// NVFP4 new row, bit-identical to the append kernel: lanes 4m..4m+3 hold block m (16
+// channels); s = E4M3(fl(max |y| / 6)) (nearest even, saturating), codes = E2M1(fl(y *
+// fl(1/s))) (nearest even, saturating, sign kept), 0 when s == 0.  codes16 = the lane's two
+// code bytes; scale = block m's E4M3 byte (the same in its 4 lanes).
+__device__ __forceinline__ NewRow quantise_new_row_fp4(uint2 raw, int lane, const DecodeParams& p) {
+  float x[4];
+  rotate_new_row(raw, lane, p, x);
+  float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+  m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+  uint16_t sb2;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sb2) : "f"(0.0f), "f"(__fdiv_rn(m, 6.0f)));
+  const uint32_t sh = e4m3x2_to_f16x2(sb2);
+  const float s = __half2float(__ushort_as_half(static_cast<uint16_t>(sh & 0xFFFFu)));
+  NewRow r;
+  r.scale = sb2 & 0xFFu;
+  r.codes16 = 0u;
+  if (s != 0.0f) {
+    const float rc = __frcp_rn(s);
+    uint32_t b0, b1;
+    asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u32.u8 %0, q;\n\t}"
+        : "=r"(b0) : "f"(__fmul_rn(x[1], rc)), "f"(__fmul_rn(x[0], rc)));
+    asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u32.u8 %0, q;\n\t}"
+        : "=r"(b1) : "f"(__fmul_rn(x[3], rc)), "f"(__fmul_rn(x[2], rc)));
+    r.codes16 = b0 | (b1 << 8);
+  }
+  return r;
+}
+
+// Bytes of a token's scales in a block row (K, then V) and the patch buffer's layout:
+// [K codes 64 B][V codes 64 B][K scales][V scales], then the token's place in its tile.
+template <bool FP4>
+struct PatchLayout {
+  static constexpr int kScale = FP4 ? kD / 16 : 2;   // per K or V row
+  static constexpr int kJ = 128 + 2 * kScale;          // 132 or 144
+};
+
 // The new token of a unit (its raw K and V rows kraw, vraw as loaded by load_new_row):
 // rotate and quantise the rows into the warp's patch buffer (shared memory), in the block
-// layout of one token: [K codes 64 B][V codes 64 B][K scale][V scale].
+// layout of one token.
+template <bool FP4>
 __device__ __forceinline__ void fused_quantise(uint2 kraw, uint2 vraw, int lane, uint8_t* patch,
                                                const DecodeParams& p) {
-  const NewRow kr = quantise_new_row(kraw, lane, p);
-  const NewRow vr = quantise_new_row(vraw, lane, p);
-  *reinterpret_cast<uint16_t*>(patch + 2 * lane) = static_cast<uint16_t>(kr.codes16);
-  *reinterpret_cast<uint16_t*>(patch + 64 + 2 * lane) = static_cast<uint16_t>(vr.codes16);
-  if (lane == 0) {
-    *reinterpret_cast<uint16_t*>(patch + 128) = static_cast<uint16_t>(kr.scale);
-    *reinterpret_cast<uint16_t*>(patch + 130) = static_cast<uint16_t>(vr.scale);
+  if constexpr (FP4) {
+    const NewRow kr = quantise_new_row_fp4(kraw, lane, p);
+    const NewRow vr = quantise_new_row_fp4(vraw, lane, p);
+    *reinterpret_cast<uint16_t*>(patch + 2 * lane) = static_cast<uint16_t>(kr.codes16);
+    *reinterpret_cast<uint16_t*>(patch + 64 + 2 * lane) = static_cast<uint16_t>(vr.codes16);
+    if ((lane & 3) == 0) {
+      patch[128 + (lane >> 2)] = static_cast<uint8_t>(kr.scale);
+      patch[136 + (lane >> 2)] = static_cast<uint8_t>(vr.scale);
+    }
+  } else {
+    const NewRow kr = quantise_new_row(kraw, lane, p);
+    const NewRow vr = quantise_new_row(vraw, lane, p);
+    *reinterpret_cast<uint16_t*>(patch + 2 * lane) = static_cast<uint16_t>(kr.codes16);
+    *reinterpret_cast<uint16_t*>(patch + 64 + 2 * lane) = static_cast<uint16_t>(vr.codes16);
+    if (lane == 0) {
+      *reinterpret_cast<uint16_t*>(patch + 128) = static_cast<uint16_t>(kr.scale);
+      *reinterpret_cast<uint16_t*>(patch + 130) = static_cast<uint16_t>(vr.scale);
+    }
   }
   __syncwarp();
 }
@@ -1219,8 +1281,10 @@ __device__ __forceinline__ void fused_quantise(uint2 kraw, uint2 vraw, int lane,
 // Store the patch buffer's token of unit (b, h) at position seq_lens[b] of the pool
 // (skipped, with the status flagged, when the position or its page is out of range).
 // Returns whether it is stored and belongs in the decode.
+template <bool FP4>
 __device__ __forceinline__ bool fused_store(int b, int h, int lane, const uint8_t* patch,
                                             const DecodeParams& p) {
+  constexpr int SC = PatchLayout<FP4>::kScale;
   const int pos = __ldg(p.seq_lens + b);
   const int S = p.page_size;
   const int lp = pos >> p.page_shift;
@@ -1229,32 +1293,43 @@ __device__ __forceinline__ bool fused_store(int b, int h, int lane, const uint8_
   if (page < 0 || page >= p.num_pages) return false;     // flagged when the tile is issued
   const int slot = pos & (S - 1);
   uint8_t* blk = const_cast<uint8_t*>(p.pool_layer) + (static_cast<size_t>(page) * p.num_kv_heads + h) *
-                                      (static_cast<size_t>(S) * (kD + 4));
+                                      (static_cast<size_t>(S) * (kD + 2 * SC));
   const uint16_t kc = *reinterpret_cast<const uint16_t*>(patch + 2 * lane);
   const uint16_t vc = *reinterpret_cast<const uint16_t*>(patch + 64 + 2 * lane);
   *reinterpret_cast<uint16_t*>(blk + slot * 64 + 2 * lane) = kc;
   *reinterpret_cast<uint16_t*>(blk + S * 64 + slot * 64 + 2 * lane) = vc;
   if (lane == 0) {
-    *reinterpret_cast<uint16_t*>(blk + S * 128 + slot * 2) = *reinterpret_cast<const uint16_t*>(patch + 128);
-    *reinterpret_cast<uint16_t*>(blk + S * 130 + slot * 2) = *reinterpret_cast<const uint16_t*>(patch + 130);
+    if constexpr (FP4) {
+      *reinterpret_cast<uint2*>(blk + S * 128 + slot * 8) = *reinterpret_cast<const uint2*>(patch + 128);
+      *reinterpret_cast<uint2*>(blk + S * 136 + slot * 8) = *reinterpret_cast<const uint2*>(patch + 136);
+    } else {
+      *reinterpret_cast<uint16_t*>(blk + S * 128 + slot * 2) = *reinterpret_cast<const uint16_t*>(patch + 128);
+      *reinterpret_cast<uint16_t*>(blk + S * 130 + slot * 2) = *reinterpret_cast<const uint16_t*>(patch + 130);
+    }
   }
   return true;
 }
 
-// Overwrite token j (0..31, kept at byte 132 of the patch buffer) of a landed ring slot
-// with the patch buffer's token (the slot's copy of the pool may predate the store above).  The warp syncs before the slot
-// is read.
-template <int SEFF>
+// Overwrite token j (0..31, kept at byte PatchLayout::kJ of the patch buffer) of a landed
+// ring slot with the patch buffer's token (the slot's copy of the pool may predate the
+// store above).  The warp syncs before the slot is read.
+template <int SEFF, bool FP4>
 __device__ __forceinline__ void patch_slot(uint8_t* slot, int lane, const uint8_t* patch) {
-  const int j = *reinterpret_cast<const int*>(patch + 132);  // the token's place in the tile
-  uint8_t* base = slot + (j / SEFF) * (SEFF * 132);
+  constexpr int SC = PatchLayout<FP4>::kScale;
+  const int j = *reinterpret_cast<const int*>(patch + PatchLayout<FP4>::kJ);  // place in the tile
+  uint8_t* base = slot + (j / SEFF) * (SEFF * row_bytes(FP4));
   const int jj = j % SEFF;
   const uint32_t wv = reinterpret_cast<const uint32_t*>(patch)[lane];  // bytes 4*lane..
   uint8_t* dst = lane < 16 ? base + jj * 64 + 4 * lane : base + SEFF * 64 + jj * 64 + 4 * (lane - 16);
   *reinterpret_cast<uint32_t*>(dst) = wv;
   if (lane == 0) {
-    *reinterpret_cast<uint16_t*>(base + SEFF * 128 + jj * 2) = *reinterpret_cast<const uint16_t*>(patch + 128);
-    *reinterpret_cast<uint16_t*>(base + SEFF * 130 + jj * 2) = *reinterpret_cast<const uint16_t*>(patch + 130);
+    if constexpr (FP4) {
+      *reinterpret_cast<uint2*>(base + SEFF * 128 + jj * SC) = *reinterpret_cast<const uint2*>(patch + 128);
+      *reinterpret_cast<uint2*>(base + SEFF * (128 + SC) + jj * SC) = *reinterpret_cast<const uint2*>(patch + 136);
+    } else {
+      *reinterpret_cast<uint16_t*>(base + SEFF * 128 + jj * 2) = *reinterpret_cast<const uint16_t*>(patch + 128);
+      *reinterpret_cast<uint16_t*>(base + SEFF * 130 + jj * 2) = *reinterpret_cast<const uint16_t*>(patch + 130);
+    }
   }
   __syncwarp();
 }
@@ -1309,11 +1384,10 @@ __device__ __forceinline__ void tile_pv_any(State<G>& st, const uint8_t* slot, i
   else tile_pv<G, SEFF>(st, slot, ntok, lane, pr);
 }
 
-// FUSED: the one-token append runs inside (p.k_new, p.v_new set; INT4 only).
+// FUSED: the one-token append runs inside (p.k_new, p.v_new set).
 // FP4: the cache holds NVFP4 rows.
 template <int G, int SEFF, bool FUSED, bool FP4>
 __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
-  static_assert(!(FUSED && FP4), "the fused append is INT4 only");
   constexpr int kFragWords = frag_words(G, FP4);
   constexpr int kSlot = slot_bytes(FP4);
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -1454,8 +1528,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       const int xl0 = x + kWarps * ((seg_end0 - x + kWarps - 1) / kWarps - 1);
       if (xl0 == cu.U + cu.n - 1) {
         const size_t row = (static_cast<size_t>(cu.b) * p.num_kv_heads + cu.h) * kD;
-        fused_quantise(load_new_row(p.k_new + row, lane), load_new_row(p.v_new + row, lane), lane,
-                       reinterpret_cast<uint8_t*>(frag), p);
+        fused_quantise<FP4>(load_new_row(p.k_new + row, lane), load_new_row(p.v_new + row, lane), lane,
+                            reinterpret_cast<uint8_t*>(frag), p);
         pre_quantised = true;
       }
     }
@@ -1548,11 +1622,12 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       if (xl == cu.U + cu.n - 1 && !dead) {
         if (!(pre_quantised && x == X0 + w)) {
           const size_t row = (static_cast<size_t>(cu.b) * p.num_kv_heads + cu.h) * kD;
-          fused_quantise(load_new_row(p.k_new + row, lane), load_new_row(p.v_new + row, lane), lane,
-                         patch, p);
+          fused_quantise<FP4>(load_new_row(p.k_new + row, lane), load_new_row(p.v_new + row, lane), lane,
+                              patch, p);
         }
-        new_ok = fused_store(cu.b, cu.h, lane, patch, p);
-        if (lane == 0) *reinterpret_cast<int*>(patch + 132) = cu.L - 1 - (xl - cu.U) * kTileTokens;
+        new_ok = fused_store<FP4>(cu.b, cu.h, lane, patch, p);
+        if (lane == 0)
+          *reinterpret_cast<int*>(patch + PatchLayout<FP4>::kJ) = cu.L - 1 - (xl - cu.U) * kTileTokens;
         __syncwarp();
       }
     }
@@ -1575,7 +1650,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       } else {
         if constexpr (FUSED) {
           if (new_ok && nt == 1)
-            patch_slot<SEFF>(ring_w + slot_i * kSlot, lane, reinterpret_cast<const uint8_t*>(frag));
+            patch_slot<SEFF, FP4>(ring_w + slot_i * kSlot, lane, reinterpret_cast<const uint8_t*>(frag));
         }
         tile_qk_any<G, SEFF>(qf, ring_p + slot_i * kSlot, ntok_of(x), lane, sc);
         float alpha[NQ];
@@ -1597,7 +1672,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
       float sn[2][NQ][2], alpha[NQ];
       if constexpr (FUSED) {
         if (new_ok && i + 2 == nt)
-          patch_slot<SEFF>(ring_w + nslot * kSlot, lane, reinterpret_cast<const uint8_t*>(frag));
+          patch_slot<SEFF, FP4>(ring_w + nslot * kSlot, lane, reinterpret_cast<const uint8_t*>(frag));
       }
       tile_qk_any<G, SEFF>(qf, ring_p + nslot * kSlot, ntok_of(xi + kWarps), lane, sn);
       const bool rescale = tile_softmax_stats<G>(st, sn, alpha);
@@ -1713,7 +1788,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(DecodeParams p) {
 
 template <int G, int SEFF>
 void* kernel_ptr(bool fused, bool fp4) {
-  if (fp4) return fused ? nullptr : reinterpret_cast<void*>(&decode_kernel<G, SEFF, false, true>);
+  if (fp4)
+    return fused ? reinterpret_cast<void*>(&decode_kernel<G, SEFF, true, true>)
+                 : reinterpret_cast<void*>(&decode_kernel<G, SEFF, false, true>);
   return fused ? reinterpret_cast<void*>(&decode_kernel<G, SEFF, true, false>)
                : reinterpret_cast<void*>(&decode_kernel<G, SEFF, false, false>);
 }
@@ -1751,11 +1828,11 @@ int plan_decode(int group, int page_size, int max_batch, int num_sms, int fp4, D
   const size_t smem = smem_bytes(group, max_batch, fp4 != 0);
   // The dynamic shared memory cap of the variants is set to the most any call of this
   // library uses (max_batch 4096), so plans made for several caches never shrink it
-  // under one another; the grid is the smaller occupancy of the variants (INT4: plain
-  // and fused; NVFP4: plain only).
+  // under one another; the grid is the smaller occupancy of the variants (plain and
+  // fused).
   const size_t cap_bytes = smem_bytes(group, 4096, fp4 != 0);
   int occ = 3;
-  for (int fused = 0; fused < (fp4 ? 1 : 2); fused++) {
+  for (int fused = 0; fused < 2; fused++) {
     void* fn = pick_kernel(group, seff, fused != 0, fp4 != 0);
     if (!fn) return -1;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,

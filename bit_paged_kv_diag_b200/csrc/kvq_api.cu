@@ -271,7 +271,6 @@ int decode_common(kvq_cache* c, int32_t layer, const void* k_new, const void* v_
   p.k_new = static_cast<const __half*>(k_new);
   p.v_new = static_cast<const __half*>(v_new);
   p.fp4 = c->d.kv_format == KVQ_FORMAT_NVFP4;
-  if (p.fp4 && k_new) return KVQ_EUNSUPPORTED;  // the fused append is INT4 only
   const int rc = kvq::launch_decode(p, c->launch, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;

@@ -120,8 +120,8 @@ typedef struct kvq_cache kvq_cache; /* opaque, library-owned handle */
  *   max_batch          largest batch any call will pass                (1 .. 4096)
  *   max_pages_per_seq  row length of the page table                          (>= 1)
  *   kv_format          KVQ_FORMAT_INT4 (0) or KVQ_FORMAT_NVFP4 (1); NVFP4 caches support
- *                      append and decode (fused append + decode and chunked prefill
- *                      return KVQ_EUNSUPPORTED) */
+ *                      append, decode and the fused append + decode (chunked prefill
+ *                      returns KVQ_EUNSUPPORTED) */
 #define KVQ_FORMAT_INT4 0
 #define KVQ_FORMAT_NVFP4 1
 typedef struct {

@@ -6,7 +6,8 @@ as the INT4 path: page tables and E4M3 scales bit-exact, E2M1 codes exact up to 
 neighbour flips (< 1e-5), decode outputs within |d| <= 2e-3 + 1e-2 |ref| of the fp64 oracle
 on the GPU-written cache.  Covered: every workload's heads and value distribution, every
 Hadamard block (1 = no rotation), every G and page size, ragged lengths and empty
-sequences; and the calls NVFP4 does not implement return KVQ_EUNSUPPORTED.
+sequences; the fused one-token append + decode; and chunked prefill, which NVFP4 does not
+implement, returns KVQ_EUNSUPPORTED.
 """
 import numpy as np
 import pytest
@@ -58,6 +59,27 @@ def test_nvfp4_multi_layer_pool_and_custom_softmax_scale():
                 softmax_scale=0.05)
 
 
+@pytest.mark.parametrize("name,lengths,block", [
+    ("tiny", [256], 32),
+    ("qwen3_4b_decode", [517, 300, 64, 1, 0, 129, 63, 65], 128),
+    ("ragged", [130, 700, 129, 1024, 0, 2, 350, 64, 191, 1500, 17, 33], 1),
+])
+def test_nvfp4_fused_append_decode(name, lengths, block):
+    """The step's one-token append inside the decode launch, on the NVFP4 cache."""
+    w = W[name]
+    full_parity(make_case(w, lengths, [1] * len(lengths), block=block, fmt=1), fused=True)
+
+
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+@pytest.mark.parametrize("page_size", [16, 32, 64, 256])
+def test_nvfp4_fused_group_and_page_size_grid(group, page_size):
+    import dataclasses
+    w = dataclasses.replace(W["qwen3_4b_decode"], num_kv_heads=2, num_q_heads=2 * group,
+                            page_size=page_size, block=64)
+    full_parity(make_case(w, [300, 0, 513, 31, 64], [1] * 5, permute=True, pool_factor=1.3,
+                          fmt=1), fused=True)
+
+
 def test_nvfp4_unsupported_calls():
     import torch
 
@@ -68,13 +90,9 @@ def test_nvfp4_unsupported_calls():
     cache, pt = kvq.alloc_pages(case.desc(), case.capacity, case.page_order)
     try:
         ptd = torch.from_numpy(pt).to(dev)
-        H, HQ = w.num_kv_heads, w.num_q_heads
-        kn = torch.zeros((1, H, 128), dtype=torch.float16, device=dev)
+        HQ = w.num_q_heads
         q = torch.zeros((1, HQ, 128), dtype=torch.float16, device=dev)
         lens = torch.tensor([256], dtype=torch.int32, device=dev)
-        with pytest.raises(kvq.KVQError) as e:
-            kvq.append_decode_attention(cache, 0, kn, kn, q, lens, ptd)
-        assert e.value.status == kvq.KVQ_EUNSUPPORTED
         with pytest.raises(kvq.KVQError) as e:
             kvq.prefill_attention(cache, 0, q, torch.tensor([0, 1], dtype=torch.int32, device=dev),
                                   lens, ptd)
@@ -154,3 +172,45 @@ def test_nvfp4_edge_rows(block):
     assert diff.size == 0, f"{diff.size} pool bytes differ, first at {diff[:8]}"
     ref = oracle.decode_attention(g, gpool, 0, q, cap, pt)
     check_outputs(gout, ref, f"nvfp4 edge rows b={block}")
+
+
+def test_nvfp4_nan_bytes_past_the_end_do_not_leak():
+    """A pool pre-filled with 0x7F bytes (E4M3 NaN): slots past each sequence's end keep
+    NaN scales, which must not reach the outputs (their probabilities are zero)."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    import oracle
+    from harness import check_outputs
+    w = W["qwen3_4b_decode"]
+    lengths = np.array([37, 1, 100, 16, 17], np.int32)
+    case = make_case(w, lengths, [0] * len(lengths), fmt=1)
+    dev = torch.device("cuda")
+    d = case.desc()
+    pool = torch.full((kvq.pool_bytes(d),), 0x7F, dtype=torch.uint8, device=dev)
+    cache, pt = kvq.alloc_pages(d, case.capacity, case.page_order, pool=pool)
+    try:
+        ptd = torch.from_numpy(pt).to(dev)
+        n = int(lengths.sum())
+        k = workloads.kv_rows(w, 0, 0, n, stream=1)
+        v = workloads.kv_rows(w, 0, 1, n, stream=1)
+        kvq.rotate_quant_append(cache, 0, torch.from_numpy(k).to(dev), torch.from_numpy(v).to(dev),
+                                torch.from_numpy(workloads.cu_seqlens(lengths)).to(dev),
+                                torch.zeros(len(lengths), dtype=torch.int32, device=dev), ptd)
+        q = workloads.q_rows(dataclasses_replace(w, batch=len(lengths)), 0)
+        out = kvq.decode_attention(cache, 0, torch.from_numpy(q).to(dev),
+                                   torch.from_numpy(lengths).to(dev), ptd)
+        torch.cuda.synchronize()
+        assert kvq.get_device_status(cache) == 0
+        host_pool = pool.cpu().numpy()
+        got = out.float().cpu().numpy()
+    finally:
+        cache.close()
+    assert np.isfinite(got).all()
+    ref = oracle.decode_attention(case.geometry(), host_pool, 0, q, lengths, pt)
+    check_outputs(got, ref, "nvfp4 with NaN bytes past the end")
+
+
+def dataclasses_replace(w, **kw):
+    import dataclasses
+    return dataclasses.replace(w, **kw)
