@@ -726,8 +726,8 @@ def run_kernel_case(which, calls):
     layer of the Qwen3-4B-shaped workload (69 MB of cache); ``fused`` = the same with the
     step's one-token append fused in; ``append`` = the prefill-append call (8 x 8192
     tokens, b = 128; 268 MB read, 69 MB written); ``prefill`` = chunked-prefill attention
-    (16 x 128-token chunks after 896 cached tokens); ``decode_nvfp4`` and ``append_nvfp4``
-    are the decode and append cases on an NVFP4 cache.  The kernel is launched ``calls``
+    (16 x 128-token chunks after 896 cached tokens); ``decode_nvfp4``, ``fused_nvfp4`` and
+    ``append_nvfp4`` are the same cases on an NVFP4 cache.  The kernel is launched ``calls``
     times after the setup."""
     import torch
 
@@ -817,7 +817,7 @@ def main():
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", choices=["decode", "fused", "append", "prefill", "decode_nvfp4",
-                                              "append_nvfp4"], default=None,
+                                              "fused_nvfp4", "append_nvfp4"], default=None,
                     help="run one small case of one kernel (for ncu captures) and exit")
     ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()
