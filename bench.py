@@ -322,10 +322,7 @@ def run_kvq(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4+fp16",
         "data": "synthetic (seeded K/V with lognormal outlier channels and RMS multipliers)",
-        "config": {"workload": WORKLOAD, "layers": NL, "batch": B, "context": int(L[0]),
-                   "kv_heads": H, "q_heads": HQ, "head_dim": 128, "hadamard_block": w.block,
-                   "page_size": S, "global_batch": B * world, "seq_len": int(cap[0]),
-                   "parallelism": f"replicas x{world}",
+        "config": {**workload_config(world),
                    "l2": "inputs larger than L2: 2.5 GB cache per step vs 126 MB L2",
                    "graph": "one CUDA graph per step",
                    "step": "per layer one kvq_append_decode_attention (fused 1-token append + decode)"},
@@ -690,6 +687,16 @@ def oracle_sample(budget_s, n_units_max=None):
                 return byt / el / 1e9, desc
 
 
+def workload_config(world):
+    """The bench workload's shape keys, shared by both arms' JSON lines."""
+    w = workloads.WORKLOADS[WORKLOAD]
+    L = np.asarray(w.context, np.int32)
+    return {"workload": WORKLOAD, "layers": w.num_layers, "batch": w.batch, "context": int(L[0]),
+            "kv_heads": w.num_kv_heads, "q_heads": w.num_q_heads, "head_dim": 128,
+            "hadamard_block": w.block, "page_size": w.page_size, "global_batch": w.batch * world,
+            "seq_len": int(L[0]) + 1, "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args, rank, world):
     """--impl reference: the CPU oracle as it stands, on host cores, same metric and
     workload; each step a bounded sample sized so the whole run ends in a few minutes."""
@@ -712,7 +719,8 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": "bounded per step"},
+        "config": {**workload_config(world),
+                   "sample": "bounded per step: the oracle on host cores"},
         "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": descs[-1] if descs else ""},
         "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
