@@ -570,6 +570,7 @@ def run_nvfp4_bench(dev, reps=10):
                           "workload": "prefill_append: 8 x 8192 tokens, 8 KV heads, page 16"}
     assert kvq.get_device_status(cache) == 0
     cache.close()
+    res["prefill"] = run_prefill_bench(dev, fmt=1)
     return res
 
 
@@ -583,10 +584,10 @@ def prefill_flops(lengths_after, chunks, num_q_heads):
     return total * num_q_heads * 4 * 128
 
 
-def run_prefill_bench(dev, reps=5):
+def run_prefill_bench(dev, reps=5, fmt=0):
     """Chunked prefill (kvq_prefill_attention) on the chunked_prefill workload: 16 x 512
     chunk tokens over 3584 cached ones, alternating two layer pools; device time per call
-    from events around a graph of the calls."""
+    from events around a graph of the calls.  fmt 1: the NVFP4 cache."""
     import torch
 
     import bit_paged_kv_diag_b200 as kvq
@@ -597,7 +598,7 @@ def run_prefill_bench(dev, reps=5):
     cap = L0 + chunk
     P = workloads.pool_pages(w, cap)
     mp = int((cap.max() + S - 1) // S)
-    desc = kvq.Desc(NL, H, HQ, 128, w.block, S, P, B, mp)
+    desc = kvq.Desc(NL, H, HQ, 128, w.block, S, P, B, mp, fmt)
     cache, pt = kvq.alloc_pages(desc, cap, None)
     ptd = torch.from_numpy(pt).to(dev)
     zeros = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -645,7 +646,9 @@ def run_prefill_bench(dev, reps=5):
             "workload": "chunked_prefill: 16 sequences x 512-token chunk after 3584 cached "
                         "tokens, Qwen3-4B heads (8 KV / 32 q), b = 128, page 16",
             "note": "algorithmic FLOPs 4*128 per (query row, visible token); the kernel runs "
-                    "QK^T as three int8 slices and PV as fp16 hi+lo on mma.sync"}
+                    + ("QK^T as fp16 q hi+lo against the dequantised fp16 K stage and PV as "
+                       "fp16 on mma.sync (NVFP4 cache)" if fmt else
+                       "QK^T as three int8 slices and PV as fp16 hi+lo on mma.sync")}
 
 
 # ------------------------------------------------------------- CPU oracle arm --

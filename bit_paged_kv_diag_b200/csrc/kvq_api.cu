@@ -300,7 +300,6 @@ int kvq_prefill_attention(kvq_cache* c, int32_t layer, const void* q, const int3
   if (!c) return KVQ_EINVAL;
   if (layer < 0 || layer >= c->d.num_layers) return KVQ_EINVAL;
   if (batch < 0 || batch > c->d.max_batch || total_q < 0) return KVQ_EINVAL;
-  if (c->d.kv_format != KVQ_FORMAT_INT4) return KVQ_EUNSUPPORTED;
   if (!(softmax_scale >= 0.0f) || isinf(softmax_scale)) return KVQ_EINVAL;
   if (batch == 0 || total_q == 0) return KVQ_OK;
   if (!q || !cu_q || !seq_lens || !page_table || !out) return KVQ_EINVAL;
@@ -326,6 +325,7 @@ int kvq_prefill_attention(kvq_cache* c, int32_t layer, const void* q, const int3
                                           : static_cast<double>(softmax_scale);
   p.q_scale = static_cast<float>(sm * 1.4426950408889634);  // log2(e)
   p.cb = c->cb;
+  p.fp4 = c->d.kv_format == KVQ_FORMAT_NVFP4;
   const int rc = kvq::launch_prefill(p, total_q, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;

@@ -84,6 +84,7 @@ struct PrefillParams {
   float q_scale;                  // softmax_scale * log2(e)
   float cb;
   int total_q;                    // rows of q and out
+  int fp4;                        // 1: NVFP4 cache
 };
 
 // Host-side launchers (return 0 on success, <0 on an unsupported shape or a launch

@@ -25,6 +25,13 @@
 //         conversion), 16 n-tiles of 8 channels.
 // The end: o'/l, the inverse block Hadamard across a row's channels (bits 1-2 of the
 // channel across lanes, the others in registers), times c_b, fp16 store.
+//
+// NVFP4 cache (template argument FP4; "BitDecoding-FP4:FP4 KVキャッシュのネイティブ復号"
+// (sns.style): E2M1 codes with an E4M3 scale per 16 channels, 144-byte token rows): K is
+// dequantised exactly to fp16 once per CTA and tile into a second swizzled stage, like V;
+// QK^T runs as fp16 mma m16n8k16 with q' carried as fp16 hi + lo parts (both accumulate into
+// one accumulator), B fragments read with ldmatrix; P' = p.  Scales of tokens past the
+// sequence's end are taken as 0 in both stages (their slot bytes are stale).
 #include <cuda_fp16.h>
 #include <math_constants.h>
 #include <stdint.h>
@@ -42,7 +49,10 @@ constexpr int kRows = 64;        // query rows per CTA
 constexpr int kWarpsP = 4;
 constexpr int kThreadsP = 128;
 constexpr int kStagesP = 3;
-constexpr int kSlotBytesP = kTileTokens * (kD + 4);  // 4224
+// Token row of a (page, head) block (INT4: codes + 2 fp16 scales; NVFP4: codes + 2 x 8 E4M3
+// scales) and the ring slot of one 32-token tile.
+constexpr int row_bytes_p(bool fp4) { return fp4 ? kD + kD / 8 : kD + 4; }
+constexpr int slot_bytes_p(bool fp4) { return kTileTokens * row_bytes_p(fp4); }
 constexpr unsigned kFullMask = 0xffffffffu;
 constexpr float kMagicP = 12582912.0f;  // 1.5 * 2^23
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -57,18 +67,18 @@ __device__ __forceinline__ void split_hi_lo_p(float p0, float p1, uint32_t& hi, 
 
 // Byte offset of token tau (0..31) of a ring slot: the slot holds pages of SEFF token
 // slots in the pool's block layout [K codes][V codes][K scales][V scales].
-template <int SEFF>
+template <int SEFF, bool FP4>
 __device__ __forceinline__ int tok_base(int tau) {
-  return (tau / SEFF) * (SEFF * 132);
+  return (tau / SEFF) * (SEFF * row_bytes_p(FP4));
 }
 
 // Issue the bulk copies of tile t (tokens 32t..) of sequence b, KV head h into a slot
 // (warp 0 calls; lane j < pages-needed copies page j).
-template <int SEFF>
+template <int SEFF, bool FP4>
 __device__ __forceinline__ void issue_tile(int t, int b, int h, int L, uint32_t slot, uint32_t bar,
                                            int lane, uint64_t pol, const PrefillParams& p) {
   const int S = p.page_size, sh = p.page_shift;
-  const uint32_t blk_bytes = static_cast<uint32_t>(S) * (kD + 4);
+  const uint32_t blk_bytes = static_cast<uint32_t>(S) * row_bytes_p(FP4);
   const int t0 = t * kTileTokens;
   const int t1 = min(t0 + kTileTokens, L);  // > t0
   if (SEFF < kTileTokens || S == kTileTokens) {
@@ -96,10 +106,16 @@ __device__ __forceinline__ void issue_tile(int t, int b, int h, int L, uint32_t 
     const uint8_t* blk = p.pool_layer + (static_cast<size_t>(pid) * p.num_kv_heads + h) * blk_bytes;
     const uint8_t* src = blk + o * 64;
     uint32_t dst = slot, bytes = 2048;
-    if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + 2048; }
-    if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 2; dst = slot + 4096; bytes = 64; }
-    if (lane == 3) { src = blk + static_cast<size_t>(S) * 130 + o * 2; dst = slot + 4160; bytes = 64; }
-    if (lane == 0) mbar_arrive_expect_tx(bar, kSlotBytesP);
+    if constexpr (FP4) {  // scales: 8 E4M3 bytes per token row
+      if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + 2048; }
+      if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 8; dst = slot + 4096; bytes = 256; }
+      if (lane == 3) { src = blk + static_cast<size_t>(S) * 136 + o * 8; dst = slot + 4352; bytes = 256; }
+    } else {
+      if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + 2048; }
+      if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 2; dst = slot + 4096; bytes = 64; }
+      if (lane == 3) { src = blk + static_cast<size_t>(S) * 130 + o * 2; dst = slot + 4160; bytes = 64; }
+    }
+    if (lane == 0) mbar_arrive_expect_tx(bar, slot_bytes_p(FP4));
     __syncwarp();
     if (lane < 4) bulk_copy_g2s(dst, src, bytes, bar, pol);
   }
@@ -174,16 +190,122 @@ __device__ __forceinline__ float prep_q_row(const __half* qrow, bool valid, uint
   return M * (1.0f / 1024.0f);
 }
 
-template <int G, int SEFF>
+// NVFP4 path: the same rotated, scaled row normalised to q~ = q' * 2^14 / M and stored as
+// fp16 hi + lo parts in A-fragment order: qs[part][kk][row][16 channels], k-step kk =
+// channels 16kk..16kk+15 in order, the same 16-byte swizzle as the int8 slices.  Returns
+// M / 2^14 (the score scale of the row).
+__device__ __forceinline__ float prep_q_row4(const __half* qrow, bool valid, uint8_t* qs, int row,
+                                             int lane, const PrefillParams& p) {
+  float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (valid) {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qrow) + lane);
+    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+    x[0] = lo.x; x[1] = lo.y; x[2] = hi.x; x[3] = hi.y;
+  }
+  if (p.hadamard_block > 1) {
+    const float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
+    x[0] = a0 + a2; x[2] = a0 - a2; x[1] = a1 + a3; x[3] = a1 - a3;
+#pragma unroll
+    for (int st = 0; st < 5; st++) {
+      if ((4 << st) < p.hadamard_block) {
+        const float sgn = ((lane >> st) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int e = 0; e < 4; e++) x[e] = __fmaf_rn(x[e], sgn, __shfl_xor_sync(kFullMask, x[e], 1 << st));
+      }
+    }
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; e++) {
+    x[e] = x[e] * p.cb * p.q_scale;
+    amax = fmaxf(amax, fabsf(x[e]));
+  }
+#pragma unroll
+  for (int d = 1; d < 32; d *= 2) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, d));
+  float M = 1.0f;
+  if (amax > 1e-30f) {
+    const uint32_t bits = __float_as_uint(amax);
+    M = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax;
+  }
+  const float inv = 16384.0f / M;  // exact: powers of two
+  __half hv[4], lv[4];
+#pragma unroll
+  for (int e = 0; e < 4; e++) {
+    const float t = x[e] * inv;
+    hv[e] = __float2half_rn(t);
+    lv[e] = __float2half_rn(t - __half2float(hv[e]));
+  }
+  // Channels 4L..4L+3: k-step L/4, bytes 8(L%4).. of the 32-byte row, halves swizzled.
+  const int kk = lane >> 2;
+  const int off = (8 * (lane & 3)) ^ (((row >> 2) & 1) * 16);
+  const uint2 wh = make_uint2(pack_half2(hv[0], hv[1]), pack_half2(hv[2], hv[3]));
+  const uint2 wl = make_uint2(pack_half2(lv[0], lv[1]), pack_half2(lv[2], lv[3]));
+  *reinterpret_cast<uint2*>(qs + ((0 * 8 + kk) * kRows + row) * 32 + off) = wh;
+  *reinterpret_cast<uint2*>(qs + ((1 * 8 + kk) * kRows + row) * 32 + off) = wl;
+  return M * (1.0f / 16384.0f);
+}
+
+// One byte of two E2M1 codes (low nibble first) -> fp16x2, exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2_p(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+      : "=r"(r)
+      : "r"(byte));
+  return r;
+}
+
+// Two E4M3 bytes (low 16 bits, low byte first) -> fp16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_p(uint32_t b) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(b)));
+  return h;
+}
+
+__device__ __forceinline__ uint32_t hmul2_p(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// NVFP4 stage: token tau's 32 channels 32part..32part+31 of K (kv = 0) or V (kv = 1),
+// dequantised to fp16 (E2M1 value x E4M3 scale, exact) into the swizzled [token][channel]
+// stage; scale 0 for a token past the sequence's end.
+template <int SEFF>
+__device__ __forceinline__ void stage_fp4(const uint8_t* base, int tau, int part, int kv, bool live,
+                                          uint8_t* stage) {
+  const uint8_t* row = base + tok_base<SEFF, true>(tau);
+  const uint4 cw = *reinterpret_cast<const uint4*>(row + kv * SEFF * 64 + (tau % SEFF) * 64 + 16 * part);
+  const uint32_t sb = live ? *reinterpret_cast<const uint16_t*>(row + SEFF * 128 + kv * SEFF * 8 +
+                                                                (tau % SEFF) * 8 + 2 * part)
+                           : 0u;
+  const uint32_t s2 = e4m3x2_to_f16x2_p(sb);
+  const uint32_t sdup[2] = {prmt(s2, s2, 0x1010u), prmt(s2, s2, 0x3232u)};  // blocks 2part, +1
+  const uint32_t wds[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+  for (int i = 0; i < 4; i++) {  // 16-byte chunk 4part + i = channels 8(4part + i) ..
+    uint32_t hv[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) hv[k] = hmul2_p(e2m1x2_to_f16x2_p(wds[i] >> (8 * k)), sdup[i >> 1]);
+    const int chunk = (4 * part + i) ^ (tau & 7);
+    *reinterpret_cast<uint4*>(stage + tau * 256 + chunk * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+  }
+}
+
+template <int G, int SEFF, bool FP4>
 __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) {
   constexpr int QB = kRows / G;  // chunk tokens per CTA
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
-  uint8_t* ring = smem;                                        // [3][4224]
-  uint8_t* qs = ring + kStagesP * kSlotBytesP;                 // [3][4][64][32] int8
-  float* sfr = reinterpret_cast<float*>(qs + 3 * 4 * kRows * 32);  // [64] row scales
+  constexpr int kSlotP = slot_bytes_p(FP4);
+  constexpr int kQsBytes = FP4 ? 2 * 8 * kRows * 32 : 3 * 4 * kRows * 32;
+  uint8_t* ring = smem;                                        // [3][slot]
+  uint8_t* qs = ring + kStagesP * kSlotP;                      // int8 slices or fp16 hi/lo
+  float* sfr = reinterpret_cast<float*>(qs + kQsBytes);        // [64] row scales
   uint8_t* vst = reinterpret_cast<uint8_t*>(sfr + kRows);      // [2][32 tokens][256 B] fp16 V
-  uint64_t* bars = reinterpret_cast<uint64_t*>(vst + 2 * kTileTokens * 256);  // full[3], empty[3]
+  uint8_t* kst = vst + 2 * kTileTokens * 256;                  // NVFP4: [2][32][256] fp16 K
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kst + (FP4 ? 2 * kTileTokens * 256 : 0));  // full[3], empty[3]
   int32_t* preq = reinterpret_cast<int32_t*>(bars + 2 * kStagesP);  // [batch + 1]
   __shared__ int warp_sum[kWarpsP];
   __shared__ int running;
@@ -260,15 +382,16 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
   int issued = 0, done0 = 0;  // warp 0: tiles issued / tiles whose copy it waited for
   if (w == 0)
     for (; issued < kStagesP && issued < ntile; issued++)
-      issue_tile<SEFF>(issued, b, h, L, smem_addr(ring) + issued * kSlotBytesP,
-                       full_s + 8 * issued, lane, pol, p);
+      issue_tile<SEFF, FP4>(issued, b, h, L, smem_addr(ring) + issued * kSlotP,
+                            full_s + 8 * issued, lane, pol, p);
   for (int rr = 0; rr < 16; rr++) {
     const int row = 16 * w + rr;
     const int ti = tok_first + row / G, gq = row % G;
     const bool valid = ti < C;
     const __half* qrow = p.q + ((static_cast<size_t>(cq0) + (valid ? ti : 0)) * p.num_kv_heads * G +
                                 h * G + gq) * kD;
-    const float sf = prep_q_row(qrow, valid, qs, row, lane, p);
+    const float sf = FP4 ? prep_q_row4(qrow, valid, qs, row, lane, p)
+                         : prep_q_row(qrow, valid, qs, row, lane, p);
     if (lane == 0) sfr[row] = sf;
   }
   __syncwarp();
@@ -296,15 +419,22 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
       if (mbar_wait_bounded(full_s + 8 * slot, par, kWaitNs)) done0++;
       else dead = true;
     }
-    const uint8_t* base = ring + slot * kSlotBytesP;
+    const uint8_t* base = ring + slot * kSlotP;
     // The tile's V codes as fp16, once per CTA: warp w converts tokens 8w..8w+7 into the
     // stage t % 2 ([token][channel], the 16-byte chunk index XOR (token & 7), so ldmatrix's
     // 8 rows fall in distinct banks).  The barrier below also tells every warp that all
     // warps are done with the stage's previous tile.
     uint8_t* vs = vst + (t & 1) * (kTileTokens * 256);
-    if (!dead) {
+    uint8_t* ks = kst + (t & 1) * (kTileTokens * 256);  // NVFP4 only
+    if (FP4 && !dead) {
       const int tau = 8 * w + (lane >> 2), part = lane & 3;  // channels 32part .. 32part+31
-      const uint4 cw = *reinterpret_cast<const uint4*>(base + tok_base<SEFF>(tau) + SEFF * 64 +
+      const bool live = t * kTileTokens + tau < L;
+      stage_fp4<SEFF>(base, tau, part, 0, live, ks);
+      stage_fp4<SEFF>(base, tau, part, 1, live, vs);
+    }
+    if (!FP4 && !dead) {
+      const int tau = 8 * w + (lane >> 2), part = lane & 3;  // channels 32part .. 32part+31
+      const uint4 cw = *reinterpret_cast<const uint4*>(base + tok_base<SEFF, FP4>(tau) + SEFF * 64 +
                                                        (tau % SEFF) * 64 + 16 * part);
       const uint32_t wds[4] = {cw.x, cw.y, cw.z, cw.w};
       uint32_t hv[16];
@@ -327,16 +457,52 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
     }
     __syncthreads();
     if (!dead) {
+      float sc[4][4];
+      float sk[4][2], sv[4][2];
+      if constexpr (FP4) {
+        // Scores: fp16 q~ hi and lo parts against the fp16 K stage (k-step kk = channels
+        // 16kk..16kk+15; ldmatrix of two n-tiles of 8 tokens at once), one accumulator.
+        float acc[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; nt++) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++) {
+          uint32_t h0, h1, h2, h3, l0_, l1_, l2_, l3_;
+          ldsm_x4(qs_s + static_cast<uint32_t>((0 * 8 + kk) * kRows * 32) + a_off, h0, h1, h2, h3);
+          ldsm_x4(qs_s + static_cast<uint32_t>((1 * 8 + kk) * kRows * 32) + a_off, l0_, l1_, l2_, l3_);
+#pragma unroll
+          for (int np = 0; np < 4; np += 2) {
+            const int ktok = 8 * (np + (lm >> 1)) + lr;
+            const int kch = 2 * kk + (lm & 1);
+            uint32_t b0a, b1a, b0b, b1b;
+            ldsm_x4(smem_addr(ks) + static_cast<uint32_t>(ktok * 256 + ((kch ^ (ktok & 7)) * 16)),
+                    b0a, b1a, b0b, b1b);
+            mma_16816(acc[np], h0, h1, h2, h3, b0a, b1a);
+            mma_16816(acc[np], l0_, l1_, l2_, l3_, b0a, b1a);
+            mma_16816(acc[np + 1], h0, h1, h2, h3, b0b, b1b);
+            mma_16816(acc[np + 1], l0_, l1_, l2_, l3_, b0b, b1b);
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 4; nt++) {
+#pragma unroll
+          for (int e = 0; e < 4; e++) sc[nt][e] = acc[nt][e];
+          // K scales are inside the stage; V scales inside the V stage (0 past the end).
+          const int tpos = t * kTileTokens + 8 * nt + 2 * c;
+          sk[nt][0] = sk[nt][1] = 1.0f;
+          sv[nt][0] = tpos < L ? 1.0f : 0.0f;
+          sv[nt][1] = tpos + 1 < L ? 1.0f : 0.0f;
+        }
+      } else {
       // K codes of tokens 8nt + g (bytes 16c..16c+15 of the row) and the K/V scales of
       // tokens 8nt + 2c, 8nt + 2c + 1.
       uint4 kr[4];
-      float sk[4][2], sv[4][2];
 #pragma unroll
       for (int nt = 0; nt < 4; nt++) {
         const int tau = 8 * nt + g;
-        kr[nt] = *reinterpret_cast<const uint4*>(base + tok_base<SEFF>(tau) + (tau % SEFF) * 64 + 16 * c);
+        kr[nt] = *reinterpret_cast<const uint4*>(base + tok_base<SEFF, FP4>(tau) + (tau % SEFF) * 64 + 16 * c);
         const int tk = 8 * nt + 2 * c;
-        const uint8_t* pb = base + tok_base<SEFF>(tk);
+        const uint8_t* pb = base + tok_base<SEFF, FP4>(tk);
         const __half2 k2 = *reinterpret_cast<const __half2*>(pb + SEFF * 128 + (tk % SEFF) * 2);
         const __half2 v2 = *reinterpret_cast<const __half2*>(pb + SEFF * 130 + (tk % SEFF) * 2);
         const float2 kf = __half22float2(k2), vf = __half22float2(v2);
@@ -349,7 +515,6 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
       // Scores: three int8 slices.  Slice 2's accumulators are multiplied by 128 and slice
       // 3's MMAs accumulate on top of them, so acc = acc2 * 128 + acc3 exactly (|acc_s| <=
       // 2^20 fits); then s = s1 + acc * 2^-14.
-      float sc[4][4];
       int acc[4][4];
 #pragma unroll
       for (int s = 0; s < 3; s++) {
@@ -376,6 +541,7 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
             else sc[nt][e] += static_cast<float>(acc[nt][e]) * (1.0f / 16384.0f);
           }
       }
+      }  // INT4 scores
       // Scale, causal mask (only on tiles reaching past the warp's first row), row maxima.
       float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
       if (t * kTileTokens + kTileTokens - 1 <= pos_min) {
@@ -465,7 +631,7 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
         dead = true;
       } else {
         fence_proxy_async_smem();
-        issue_tile<SEFF>(t + kStagesP, b, h, L, smem_addr(ring) + slot * kSlotBytesP,
+        issue_tile<SEFF, FP4>(t + kStagesP, b, h, L, smem_addr(ring) + slot * kSlotP,
                          full_s + 8 * slot, lane, pol, p);
         issued++;
       }
@@ -545,15 +711,16 @@ __global__ void __launch_bounds__(kThreadsP, 3) prefill_kernel(PrefillParams p) 
 }
 
 template <int G, int SEFF>
-void* prefill_ptr() {
-  return reinterpret_cast<void*>(&prefill_kernel<G, SEFF>);
+void* prefill_ptr(bool fp4) {
+  return fp4 ? reinterpret_cast<void*>(&prefill_kernel<G, SEFF, true>)
+             : reinterpret_cast<void*>(&prefill_kernel<G, SEFF, false>);
 }
 
-void* pick_prefill(int group, int seff) {
-#define KVQ_PICKP(GG)                                  \
-  if (group == GG) {                                   \
-    if (seff == 16) return prefill_ptr<GG, 16>();      \
-    if (seff == 32) return prefill_ptr<GG, 32>();      \
+void* pick_prefill(int group, int seff, bool fp4) {
+#define KVQ_PICKP(GG)                                      \
+  if (group == GG) {                                       \
+    if (seff == 16) return prefill_ptr<GG, 16>(fp4);       \
+    if (seff == 32) return prefill_ptr<GG, 32>(fp4);       \
   }
   KVQ_PICKP(1)
   KVQ_PICKP(2)
@@ -563,11 +730,11 @@ void* pick_prefill(int group, int seff) {
   return nullptr;
 }
 
-size_t prefill_smem(int max_batch) {
-  size_t s = static_cast<size_t>(kStagesP) * kSlotBytesP;  // ring
-  s += 3 * 4 * kRows * 32;                                  // q slices
+size_t prefill_smem(int max_batch, bool fp4) {
+  size_t s = static_cast<size_t>(kStagesP) * slot_bytes_p(fp4);  // ring
+  s += fp4 ? 2 * 8 * kRows * 32 : 3 * 4 * kRows * 32;      // q: fp16 hi/lo or int8 slices
   s += sizeof(float) * kRows;                               // row scales
-  s += 2 * kTileTokens * 256;                               // fp16 V stages
+  s += (fp4 ? 4 : 2) * kTileTokens * 256;                   // fp16 V (and K) stages
   s += sizeof(uint64_t) * 2 * kStagesP;                     // barriers
   s += static_cast<size_t>(max_batch + 1) * sizeof(int32_t);  // query-block prefix
   s += 128;                                                  // alignment slack
@@ -578,16 +745,16 @@ size_t prefill_smem(int max_batch) {
 
 int launch_prefill(const PrefillParams& p, int total_q, cudaStream_t stream) {
   const int seff = p.page_size < kTileTokens ? p.page_size : kTileTokens;
-  void* fn = pick_prefill(p.group, seff);
+  void* fn = pick_prefill(p.group, seff, p.fp4 != 0);
   if (!fn) return -1;
   if (p.batch == 0 || total_q == 0) return 0;
   const int QB = kRows / p.group;
   const long long blocks = (static_cast<long long>(total_q) + QB - 1) / QB + p.batch;
   const long long grid = blocks * p.num_kv_heads;
   if (grid > 0x7fffffffLL) return -1;
-  const size_t smem = prefill_smem(p.batch);
+  const size_t smem = prefill_smem(p.batch, p.fp4 != 0);
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(prefill_smem(4096))) != cudaSuccess)
+                           static_cast<int>(prefill_smem(4096, p.fp4 != 0))) != cudaSuccess)
     return -2;
   PrefillParams q = p;
   q.total_q = total_q;

@@ -119,9 +119,8 @@ typedef struct kvq_cache kvq_cache; /* opaque, library-owned handle */
  *   num_pages          pages per layer in the pool                            (>= 1)
  *   max_batch          largest batch any call will pass                (1 .. 4096)
  *   max_pages_per_seq  row length of the page table                          (>= 1)
- *   kv_format          KVQ_FORMAT_INT4 (0) or KVQ_FORMAT_NVFP4 (1); NVFP4 caches support
- *                      append, decode and the fused append + decode (chunked prefill
- *                      returns KVQ_EUNSUPPORTED) */
+ *   kv_format          KVQ_FORMAT_INT4 (0) or KVQ_FORMAT_NVFP4 (1); every call supports
+ *                      both formats */
 #define KVQ_FORMAT_INT4 0
 #define KVQ_FORMAT_NVFP4 1
 typedef struct {

@@ -6,8 +6,7 @@ as the INT4 path: page tables and E4M3 scales bit-exact, E2M1 codes exact up to 
 neighbour flips (< 1e-5), decode outputs within |d| <= 2e-3 + 1e-2 |ref| of the fp64 oracle
 on the GPU-written cache.  Covered: every workload's heads and value distribution, every
 Hadamard block (1 = no rotation), every G and page size, ragged lengths and empty
-sequences; the fused one-token append + decode; and chunked prefill, which NVFP4 does not
-implement, returns KVQ_EUNSUPPORTED.
+sequences; the fused one-token append + decode; and causal chunked prefill.
 """
 import numpy as np
 import pytest
@@ -80,25 +79,34 @@ def test_nvfp4_fused_group_and_page_size_grid(group, page_size):
                           fmt=1), fused=True)
 
 
-def test_nvfp4_unsupported_calls():
-    import torch
+@pytest.mark.parametrize("name,lengths,chunks", [
+    ("tiny", [0], [257]),
+    ("qwen3_4b_decode", [0, 300, 31, 64, 1000, 7], [100, 17, 1, 65, 16, 0]),
+    ("long_context", [2000, 0, 513], [40, 130, 7]),
+    ("ragged", [128, 700, 0, 95, 33], [64, 3, 80, 1, 31]),
+    ("prefill_append", [0, 0], [300, 129]),
+])
+def test_nvfp4_prefill_workloads(name, lengths, chunks):
+    """Causal chunked prefill over the NVFP4 cache."""
+    from harness import prefill_parity
+    prefill_parity(make_case(W[name], lengths, chunks, fmt=1))
 
-    import bit_paged_kv_diag_b200 as kvq
-    w = W["tiny"]
-    case = make_case(w, w.context, [1], fmt=1)
-    dev = torch.device("cuda")
-    cache, pt = kvq.alloc_pages(case.desc(), case.capacity, case.page_order)
-    try:
-        ptd = torch.from_numpy(pt).to(dev)
-        HQ = w.num_q_heads
-        q = torch.zeros((1, HQ, 128), dtype=torch.float16, device=dev)
-        lens = torch.tensor([256], dtype=torch.int32, device=dev)
-        with pytest.raises(kvq.KVQError) as e:
-            kvq.prefill_attention(cache, 0, q, torch.tensor([0, 1], dtype=torch.int32, device=dev),
-                                  lens, ptd)
-        assert e.value.status == kvq.KVQ_EUNSUPPORTED
-    finally:
-        cache.close()
+
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+@pytest.mark.parametrize("page_size", [16, 32, 64, 256])
+def test_nvfp4_prefill_group_and_page_size_grid(group, page_size):
+    import dataclasses
+    from harness import prefill_parity
+    w = dataclasses.replace(W["qwen3_4b_decode"], num_kv_heads=2, num_q_heads=2 * group,
+                            page_size=page_size, block=64)
+    prefill_parity(make_case(w, [300, 0, 47], [70, 65, 9], permute=True, pool_factor=1.3, fmt=1))
+
+
+@pytest.mark.parametrize("block", [1, 32])
+def test_nvfp4_prefill_blocks_and_softmax_scale(block):
+    from harness import prefill_parity
+    prefill_parity(make_case(W["ragged"], [200, 5], [33, 64], block=block, fmt=1),
+                   softmax_scale=0.05)
 
 
 def _edge_rows(n, H, rng):
