@@ -737,8 +737,8 @@ def run_kernel_case(which, calls):
     layer of the Qwen3-4B-shaped workload (69 MB of cache); ``fused`` = the same with the
     step's one-token append fused in; ``append`` = the prefill-append call (8 x 8192
     tokens, b = 128; 268 MB read, 69 MB written); ``prefill`` = chunked-prefill attention
-    (16 x 128-token chunks after 896 cached tokens); ``decode_nvfp4``, ``fused_nvfp4`` and
-    ``append_nvfp4`` are the same cases on an NVFP4 cache.  The kernel is launched ``calls``
+    (16 x 128-token chunks after 896 cached tokens); ``decode_nvfp4``, ``fused_nvfp4``,
+    ``append_nvfp4`` and ``prefill_nvfp4`` are the same cases on an NVFP4 cache.  The kernel is launched ``calls``
     times after the setup."""
     import torch
 
@@ -753,7 +753,8 @@ def run_kernel_case(which, calls):
         chunk = np.full(B, 128, np.int32)
         cap = np.full(B, 1024, np.int32)
         P = workloads.pool_pages(w, cap)
-        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S))
+        desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S),
+                        fmt)
         cache, pt = kvq.alloc_pages(desc, cap, None)
         ptd = torch.from_numpy(pt).to(dev)
         k = workloads.kv_rows_torch(w, 0, 0, int(cap.sum()), stream=1, device=dev)
@@ -828,7 +829,8 @@ def main():
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", choices=["decode", "fused", "append", "prefill", "decode_nvfp4",
-                                              "fused_nvfp4", "append_nvfp4"], default=None,
+                                              "fused_nvfp4", "append_nvfp4", "prefill_nvfp4"],
+                    default=None,
                     help="run one small case of one kernel (for ncu captures) and exit")
     ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()
