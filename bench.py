@@ -690,6 +690,43 @@ def oracle_sample(budget_s, n_units_max=None):
                 return byt / el / 1e9, desc
 
 
+def oracle_sample_threads(budget_s, threads):
+    """The same oracle decode on every host core: threads call the oracle's C decode of one
+    (sequence, query head) at a time (the C call releases the interpreter lock) over the
+    G query heads of the layer's units, on one cache written once.  Returns (GB/s,
+    threads, description)."""
+    import concurrent.futures
+    import oracle
+    w = workloads.WORKLOADS[WORKLOAD]
+    G, H, S = w.group, w.num_kv_heads, w.page_size
+    L = int(w.context[0])
+    g = oracle.Geometry(1, H, w.num_q_heads, 128, w.block, S, (L + 1 + S - 1) // S,
+                        (L + 1 + S - 1) // S)
+    cap = np.full(1, L + 1, np.int32)
+    pt = oracle.assign_pages(cap, S, g.num_pages, g.max_pages_per_seq)
+    pool = g.new_pool()
+    kp, vp = workloads.kv_rows(w, 0, 0, L + 1, 1), workloads.kv_rows(w, 0, 1, L + 1, 1)
+    oracle.rotate_quant_append(g, pool, 0, kp, vp, workloads.cu_seqlens([L + 1]),
+                               np.zeros(1, np.int32), pt)
+    q = workloads.q_rows(w, 0)[:1]
+    t0 = time.perf_counter()
+
+    def work(tid):
+        n = 0
+        while time.perf_counter() - t0 < budget_s:
+            oracle.decode_one(g, pool, 0, q, cap, pt, 0, (tid + n * threads) % (H * G))
+            n += 1
+        return n
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        calls = sum(ex.map(work, range(threads)))
+    el = time.perf_counter() - t0
+    byt = calls / G * ((L + 1) * BYTES_PER_TOKEN_HEAD + 2 * G * 256)
+    desc = (f"oracle (C, fp64 attention, {threads} threads): decode of {calls} (sequence, query "
+            f"head) rows at {L + 1} tokens, one layer of {WORKLOAD}; {el:.2f} s")
+    return byt / el / 1e9, threads, desc
+
+
 def workload_config(world):
     """The bench workload's shape keys, shared by both arms' JSON lines."""
     w = workloads.WORKLOADS[WORKLOAD]
@@ -865,6 +902,9 @@ def main():
                 v, d = oracle_sample(12.0)
                 line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": 1,
                                         "kind": "oracle", "sample": d}
+                v, n, d = oracle_sample_threads(8.0, os.cpu_count() or 1)
+                line["cpu_baseline_all_cores"] = {"value": round(v, 4), "unit": "GB/s", "cores": n,
+                                                  "kind": "oracle", "sample": d}
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:
