@@ -149,7 +149,9 @@ struct Dest {
 
 __device__ __forceinline__ Dest pair_dest(const AppendParams& p, int gp) {
   Dest d;
-  const int t = static_cast<int>(static_cast<unsigned>(gp) / static_cast<unsigned>(p.num_kv_heads));
+  // t = gp / num_kv_heads by the host's multiplier (gp < 2^31); pos / S and pos % S by
+  // the power-of-two page size.
+  const int t = static_cast<int>(__umulhi(static_cast<uint32_t>(gp) << 1, p.heads_magic) >> p.heads_shift);
   d.h = gp - t * p.num_kv_heads;
   int lo = 0, hi = p.batch;
   while (hi - lo > 1) {
@@ -157,13 +159,13 @@ __device__ __forceinline__ Dest pair_dest(const AppendParams& p, int gp) {
     if (__ldg(p.cu_new_tokens + mid) <= t) lo = mid; else hi = mid;
   }
   const int pos = __ldg(p.seq_lens + lo) + (t - __ldg(p.cu_new_tokens + lo));
-  const int lp = pos >= 0 ? pos / p.page_size : 0;
+  const int lp = pos >= 0 ? pos >> p.page_shift : 0;
   if (pos < 0 || lp >= p.max_pages_per_seq) {
     d.page = -1;
     d.slot = -1;
   } else {
     d.page = __ldg(p.page_table + static_cast<size_t>(lo) * p.max_pages_per_seq + lp);
-    d.slot = pos - lp * p.page_size;
+    d.slot = pos & (p.page_size - 1);
   }
   return d;
 }

@@ -227,6 +227,18 @@ int kvq_rotate_quant_append(kvq_cache* c, int32_t layer, const void* k, const vo
   p.max_pages_per_seq = c->d.max_pages_per_seq;
   p.cb = c->cb;
   p.fp4 = c->d.kv_format == KVQ_FORMAT_NVFP4;
+  p.page_shift = __builtin_ctz(static_cast<unsigned>(c->d.page_size));
+  // Division by an invariant integer (Granlund and Montgomery, "Division by invariant
+  // integers using multiplication", 1994, Theorem 4.2 with N = 31): for l = ceil(log2 d)
+  // and m = ceil(2^(31 + l) / d), floor(n * m / 2^(31 + l)) = floor(n / d) for every
+  // 0 <= n < 2^31, and m < 2^32.
+  {
+    const unsigned d = static_cast<unsigned>(c->d.num_kv_heads);
+    int l = 0;
+    while ((1ull << l) < d) l++;
+    p.heads_magic = static_cast<uint32_t>(((1ull << (31 + l)) + d - 1) / d);
+    p.heads_shift = l;
+  }
   const int rc = kvq::launch_append(p, c->d.hadamard_block, c->num_sms, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;

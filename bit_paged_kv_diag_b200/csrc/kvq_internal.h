@@ -28,6 +28,10 @@ struct AppendParams {
   int max_pages_per_seq;
   float cb;                       // fp32 nearest 1/sqrt(hadamard_block)
   int fp4;                        // 1: NVFP4 rows (E2M1 codes, E4M3 scale per 16 channels)
+  int page_shift;                 // log2(page_size)
+  // n / num_kv_heads for 0 <= n < 2^31 as umulhi(2n, heads_magic) >> heads_shift
+  uint32_t heads_magic;
+  int heads_shift;
 };
 
 // Tokens per decode tile (one shared-memory ring slot per tile).

@@ -89,6 +89,17 @@ def test_fused_group_and_page_size_grid(group, page_size):
                 fused=True)
 
 
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("kv_heads", [3, 5])
+def test_kv_heads_not_a_power_of_two(kv_heads, fmt):
+    """3 and 5 KV heads (G = 4): the append's split of its (token, KV head) pairs and the
+    decode's units, with multi-token appends after cached tokens, on both cache formats."""
+    w = dataclasses.replace(W["qwen3_4b_decode"], num_kv_heads=kv_heads,
+                            num_q_heads=4 * kv_heads)
+    full_parity(make_case(w, [300, 1, 513, 0, 64], [37, 1, 200, 3, 9], permute=True,
+                          pool_factor=1.3, fmt=fmt))
+
+
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])
 def test_group_and_page_size_grid(group, page_size):
