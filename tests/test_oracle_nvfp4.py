@@ -143,3 +143,55 @@ def test_nvfp4_decode_is_dense_attention_on_lossless_rows():
         ref = oracle.attention_dense(q[0, hq].astype(np.float64), k[:, hq // G].astype(np.float64),
                                      v[:, hq // G].astype(np.float64), 1, 0)
         np.testing.assert_allclose(out[0, hq], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_nvfp4_pool_bytes_follow_the_documented_layout():
+    """The oracle's NVFP4 append writes exactly what the header's pool layout says: an
+    expected pool built here byte by byte -- block ((layer*P + page)*Hkv + head)*S*144,
+    codes of slot s at kv*S*64 + s*64 (low nibble = even channel), the 8 E4M3 block scales
+    at S*128 + kv*S*8 + s*8 -- from the row quantiser applied to the rotated rows, equals
+    the oracle's pool (other layers and unused slots stay zero); and reading the bytes back
+    with a table of E2M1 values and torch's E4M3 gives the oracle's dequantised rows."""
+    rng = np.random.default_rng(11)
+    L, H, Hq, b, S, P, mp, layer = 2, 2, 8, 32, 16, 8, 4, 1
+    g = oracle.Geometry(L, H, Hq, 128, b, S, P, mp, fmt=1)
+    cap = np.array([37, 5], np.int32)
+    pt = oracle.assign_pages(cap, S, P, mp, rng.permutation(P).astype(np.int32))
+    n = int(cap.sum())
+    k = (rng.standard_t(3, (n, H, 128)) * 3).astype(np.float16)
+    v = rng.standard_normal((n, H, 128)).astype(np.float16)
+    cu = np.array([0, 37, 42], np.int32)
+    pool = g.new_pool()
+    oracle.rotate_quant_append(g, pool, layer, k, v, cu, np.zeros(2, np.int32), pt)
+
+    want = np.zeros_like(pool)
+    R = 144
+    for seq in range(2):
+        for pos in range(int(cap[seq])):
+            page, slot = int(pt[seq, pos // S]), pos % S
+            for h in range(H):
+                base = ((layer * P + page) * H + h) * S * R
+                for kv, src in ((0, k), (1, v)):
+                    y = oracle.fwht_f32(src[cu[seq] + pos, h].astype(np.float32), b)
+                    codes, sc = oracle.quant_row_nvfp4(y)
+                    codes = codes.astype(np.uint8)
+                    packed = (codes[0::2] & 0xF) | ((codes[1::2] & 0xF) << 4)
+                    o = base + kv * S * 64 + slot * 64
+                    want[o:o + 64] = packed
+                    o = base + S * 128 + kv * S * 8 + slot * 8
+                    want[o:o + 8] = sc
+    assert np.array_equal(pool, want)
+
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    for seq, pos, h, kv in ((0, 0, 0, 0), (0, 36, 1, 1), (1, 4, 1, 0), (0, 17, 0, 1)):
+        page, slot = int(pt[seq, pos // S]), pos % S
+        base = ((layer * P + page) * H + h) * S * R
+        byt = pool[base + kv * S * 64 + slot * 64:][:64]
+        c = np.empty(128, np.int64)
+        c[0::2] = byt & 0xF
+        c[1::2] = byt >> 4
+        vals = np.where(c & 8, -1.0, 1.0) * mags[c & 7]
+        sc = pool[base + S * 128 + kv * S * 8 + slot * 8:][:8].copy()
+        s = torch.from_numpy(sc).view(torch.float8_e4m3fn).double().numpy()
+        row = vals * np.repeat(s, 16)
+        assert np.array_equal(row, oracle.read_row(g, pool, layer, page, h, slot, kv).astype(np.float64))
