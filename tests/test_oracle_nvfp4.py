@@ -39,7 +39,8 @@ def test_e4m3_rounding_matches_torch():
     vals = np.array([oracle.e4m3_to_float(c) for c in range(127)], np.float64)
     mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
     x = np.concatenate([x, mids, np.float32([0.0, 448.0, 460.0, 464.0, 1e6])])
-    ref = torch.from_numpy(np.minimum(x, 448.0).astype(np.float32)).to(torch.float8_e4m3fn)
+    x = np.concatenate([x, -x])  # the sign is kept (-0 included)
+    ref = torch.from_numpy(np.clip(x, -448.0, 448.0).astype(np.float32)).to(torch.float8_e4m3fn)
     ref = ref.view(torch.uint8).numpy()
     got = np.array([oracle.float_to_e4m3(float(v)) for v in x], np.uint8)
     assert np.array_equal(got, ref), np.nonzero(got != ref)[0][:10]
