@@ -56,6 +56,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "kvq_internal.h"
 #include "kvq_ptx.cuh"
 
@@ -561,12 +563,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) append_kernel(AppendPara
 
 template <int BLOCK, bool FP4>
 int launch_block(const cudaLaunchConfig_t& cfg, const AppendParams& p) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The shared-memory opt-in is an attribute of the function in the current device's
+  // context: set it once per device (devices 64 and up set it on every launch).
+  static std::atomic<unsigned long long> attr_set{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -2;
+  const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+  if (bit == 0 || (attr_set.load(std::memory_order_acquire) & bit) == 0) {
     if (cudaFuncSetAttribute(append_kernel<BLOCK, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBytes) != cudaSuccess)
       return -2;
-    attr_set = true;
+    attr_set.fetch_or(bit, std::memory_order_release);
   }
   return cudaLaunchKernelEx(&cfg, append_kernel<BLOCK, FP4>, p) == cudaSuccess ? 0 : -2;
 }
