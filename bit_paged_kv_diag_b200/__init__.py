@@ -200,7 +200,10 @@ def alloc_pages(desc: Desc, capacity_tokens=None, page_order=None, pool=None):
 
 def rotate_quant_append(cache: Cache, layer: int, k, v, cu_new_tokens, seq_lens, page_table,
                         stream=None) -> None:
-    """Fused rotate + INT4 quantise + paged append of fp16 k, v [T][Hkv][128] (CUDA)."""
+    """Fused rotate + quantise + paged append of fp16 k, v [T][Hkv][128] (CUDA): INT4 rows,
+    or NVFP4 rows for a cache made with kv_format = FORMAT_NVFP4.  Token t of sequence b
+    (cu_new_tokens[b] <= t < cu_new_tokens[b+1]) lands at position seq_lens[b] + t -
+    cu_new_tokens[b]; seq_lens is not updated."""
     import torch
     T = int(k.shape[0])
     batch = int(seq_lens.shape[0])
