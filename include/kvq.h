@@ -66,8 +66,7 @@
  *     pool; the library owns the handle, its split-KV scratch, its status word and the
  *     pool when it allocated it.  One handle must not be used from two streams at once
  *     (decode calls share the handle's scratch).
-
- *   * Launch overlap: both kernels use programmatic dependent launch.  Each lets the next
+ *   * Launch overlap: every kernel of this library uses programmatic dependent launch.  Each lets the next
  *     kernel on the stream start at its own entry, and waits for the previous kernel to
  *     complete before it touches the pool, q, out or the handle's scratch.  Before that
  *     wait, decode already reads seq_lens and page_table, append reads k, v,
@@ -168,7 +167,8 @@ KVQ_API int kvq_alloc_pages(const kvq_desc* d, void* dev_pool, size_t pool_bytes
                     int32_t* page_table, kvq_cache** out);
 
 /* Fused block-diagonal Hadamard rotation + token-wise INT4 quantisation + paged append
- * for one layer [P1, "システムこそが設計である — 融合カーネル"].  One kernel launch.
+ * for one layer [P1, "システムこそが設計である — 融合カーネル"]; NVFP4 rows instead
+ * for a cache with kv_format = KVQ_FORMAT_NVFP4.  One kernel launch.
  *   layer             0 .. num_layers-1
  *   k, v              device fp16 [total_new_tokens][num_kv_heads][128], token-major,
  *                     32-byte aligned (rows are read with 256-bit loads)
@@ -185,8 +185,8 @@ KVQ_API int kvq_rotate_quant_append(kvq_cache* c, int32_t layer, const void* k, 
                             const int32_t* page_table, int32_t batch,
                             int32_t total_new_tokens, void* stream);
 
-/* Paged GQA decode attention over the INT4 cache of one layer: one query token per
- * sequence.  One kernel launch: a split-KV pass whose last-arriving CTA per (sequence,
+/* Paged GQA decode attention over the cache (INT4 or NVFP4) of one layer: one query
+ * token per sequence.  One kernel launch: a split-KV pass whose last-arriving CTA per (sequence,
  * KV head) merges the splits and applies the inverse rotation.
  *   q              device fp16 [batch][num_q_heads][128], 16-byte aligned
  *   seq_lens       device int32 [batch], lengths AFTER any append (tokens to attend)
@@ -222,8 +222,8 @@ KVQ_API int kvq_append_decode_attention(kvq_cache* c, int32_t layer, const void*
                                         int32_t batch, float softmax_scale, void* out,
                                         void* stream);
 
-/* Causal chunked-prefill attention over the INT4 cache of one layer: many query tokens
- * per sequence.  A chunk of C_b = cu_q[b+1] - cu_q[b] prompt tokens of sequence b, already
+/* Causal chunked-prefill attention over the cache (INT4 or NVFP4) of one layer: many
+ * query tokens per sequence.  A chunk of C_b = cu_q[b+1] - cu_q[b] prompt tokens of sequence b, already
  * appended (kvq_rotate_quant_append), attends the cache causally: query i of the chunk,
  * at position seq_lens[b] - C_b + i, attends positions 0 .. seq_lens[b] - C_b + i.  The
  * pages' attention over the paged cache ("KVキャッシュを4ビットへ", section
