@@ -116,3 +116,36 @@ def test_calls_reject_bad_arguments_before_any_cuda_call():
     assert L.kvq_free(None) == kvq.KVQ_OK
     assert L.kvq_pool_ptr(None) is None
     assert kvq.status_string(kvq.KVQ_ENOPAGES) == "not enough pages"
+
+
+def test_noalloc_decode_rejects_bad_arguments_before_any_cuda_call():
+    """The allocation-free decode checks its descriptor, layer, batch, scale, pointers,
+    alignment and the fixed scratch's unit limit before its first CUDA call."""
+    L = kvq.lib()
+    d = _desc()
+    ok = 0x10000  # 16-byte aligned stand-ins; nothing is dereferenced on these paths
+    args = lambda **kw: dict(dict(d=ctypes.byref(d), pool=ok, layer=0, q=ok, lens=ok, pt=ok,  # noqa: E731
+                                  batch=4, scale=0.0, out=ok), **kw)
+
+    def call(a):
+        return L.kvq_decode_attention_noalloc(a["d"], a["pool"], a["layer"], a["q"], a["lens"],
+                                              a["pt"], a["batch"], a["scale"], a["out"], None)
+
+    assert call(args(d=None)) == kvq.KVQ_EINVAL
+    for bad in (dict(head_dim=96), dict(num_q_heads=24), dict(hadamard_block=16),
+                dict(page_size=8), dict(kv_format=2), dict(max_batch=5000)):
+        assert call(args(d=ctypes.byref(_desc(**bad)))) == kvq.KVQ_EUNSUPPORTED, bad
+    assert call(args(layer=2)) == kvq.KVQ_EINVAL
+    assert call(args(layer=-1)) == kvq.KVQ_EINVAL
+    assert call(args(batch=17)) == kvq.KVQ_EINVAL
+    assert call(args(batch=-1)) == kvq.KVQ_EINVAL
+    assert call(args(scale=-1.0)) == kvq.KVQ_EINVAL
+    assert call(args(scale=float("inf"))) == kvq.KVQ_EINVAL
+    assert call(args(scale=float("nan"))) == kvq.KVQ_EINVAL
+    assert call(args(batch=0, q=None)) == kvq.KVQ_OK  # nothing to do
+    for name in ("pool", "q", "lens", "pt", "out"):
+        assert call(args(**{name: None})) == kvq.KVQ_EINVAL, name
+    for name in ("pool", "q", "out"):
+        assert call(args(**{name: ok + 8})) == kvq.KVQ_EINVAL, name
+    big = _desc(num_kv_heads=8, num_q_heads=8, max_batch=4096)
+    assert call(args(d=ctypes.byref(big), batch=513)) == kvq.KVQ_EUNSUPPORTED  # 513 * 8 > 4096
