@@ -17,8 +17,15 @@ across steps.
 
 Also reported: the roofline of the decode-attention call, the prefill-append throughput
 (8 x 8192 new tokens in one call, b = 32/64/128, and b = 1: plain INT4 without rotation),
-rotated against plain INT4 decode, end-to-end throughput through the C ABI with host
-buffers, and the CPU oracle timed on a bounded sample of the same workload.
+rotated against plain INT4 decode, the NVFP4 cache's decode, fused step and append, the
+chunked-prefill attention, end-to-end throughput through the C ABI with host buffers, and
+the CPU oracle timed on a bounded sample of the same workload on one host core
+(``cpu_baseline``) and on every host core (``cpu_baseline_all_cores``).
+
+    python bench.py --kernel-case decode|fused|append|prefill|decode_nvfp4|fused_nvfp4|
+                                  append_nvfp4|prefill_nvfp4 [--calls C]
+
+runs one case of one kernel (for profiler captures) and prints only its status.
 
 Multi-GPU: replicas only (each rank runs the whole workload on its own GPU; the path has
 no exchange step), timing = max over ranks.
