@@ -47,6 +47,7 @@ import workloads  # noqa: E402
 METRIC = ("INT4 paged decode-attn effective HBM GB/s (% of peak); fused quant-append tok/s")
 WORKLOAD = "qwen3_4b_decode"
 BYTES_PER_TOKEN_HEAD = 132
+NOMINAL_HBM_GBS = 8000.0  # the B200's nominal HBM3e bandwidth, for context beside the measured peak
 
 
 def _peaks():
@@ -347,6 +348,7 @@ def run_kvq(args, rank, world, local_rank):
         "kernel": "decode_kernel (decode attention of one layer, one launch)",
         "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
         "frac": round(ach / peak, 4), "peak_kind": peak_kind,
+        "frac_of_nominal": round(ach / NOMINAL_HBM_GBS, 4),
         "traffic": _traffic("decode", dec_b), "us_per_launch": round(dec_ms * 1e3, 3),
         "fused_us_per_launch_alone": round(iso_ms * 1e3, 3),
         "bytes_per_launch": dec_b, "timing": dec_how}
