@@ -15,12 +15,16 @@ B read + 132 B written per appended (token, KV head)) over the device time per s
 ranks summed.  The cache (2.5 GB) is far larger than the 126 MB L2, so nothing is reused
 across steps.
 
-Also reported: the roofline of the decode-attention call, the prefill-append throughput
-(8 x 8192 new tokens in one call, b = 32/64/128, and b = 1: plain INT4 without rotation),
-rotated against plain INT4 decode, the NVFP4 cache's decode, fused step and append, the
-chunked-prefill attention, end-to-end throughput through the C ABI with host buffers, and
-the CPU oracle timed on a bounded sample of the same workload on one host core
-(``cpu_baseline``) and on every host core (``cpu_baseline_all_cores``).
+Also reported: the roofline of the step's kernel (the fused append + decode launch, the only
+kernel of the timed step) and of the plain decode-attention call, the prefill-append
+throughput (8 x 8192 new tokens in one call, b = 32/64/128, and b = 1: plain INT4 without
+rotation; L2 flushed between calls), rotated against plain INT4 decode, the NVFP4 cache's
+decode, fused step and append, the chunked-prefill attention, the long-context (4 sequences
+up to 128K tokens, G = 8) and ragged (256 sequences, scattered pages) workloads' decode and
+decode step at full size, the tiny workload's step latency, end-to-end throughput through
+the C ABI with host buffers, and the CPU oracle timed on a bounded sample of the same
+workload on one host core (``cpu_baseline``) and on every host core
+(``cpu_baseline_all_cores``), and its append throughput (``cpu_baseline_append``).
 
     python bench.py --kernel-case decode|fused|append|prefill|decode_nvfp4|fused_nvfp4|
                                   append_nvfp4|prefill_nvfp4 [--calls C]
@@ -74,6 +78,25 @@ def append_bytes(tokens, num_kv_heads, row_bytes=132):
 
 # NVFP4 rows: 64 B of E2M1 codes and 8 E4M3 scales for K and for V.
 BYTES_PER_TOKEN_HEAD_NVFP4 = 2 * 64 + 2 * 8
+
+# A write larger than the 126 MB L2 between timed calls whose inputs and outputs would fit.
+FLUSH_BYTES = 256 << 20
+
+
+def _timed_calls(fn, reps, flush=None):
+    """Mean device time (ms) of fn() over reps calls, events around each call on the
+    current stream; with flush, a write of that buffer before every call (not timed)."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a, b in ev:
+        if flush is not None:
+            flush.zero_()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in ev]))
 
 
 # --------------------------------------------------------------------- clocks --
@@ -324,6 +347,7 @@ def run_kvq(args, rank, world, local_rank):
     plain = run_plain_decode_bench(dev) if rank == 0 else None
     nvfp4 = run_nvfp4_bench(dev) if rank == 0 else None
     prefill = run_prefill_bench(dev) if rank == 0 else None
+    configs = run_decode_configs(dev) if rank == 0 else {}
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -343,19 +367,37 @@ def run_kvq(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": round(e2e_ms, 5)},
     }
-    ach = dec_b / (dec_ms * 1e-3) / 1e9
+    # The timed step is 36 launches of one kernel (the fused append + decode), so that is
+    # the roofline kernel: its algorithmic bytes per launch over its mean launch time in
+    # the timed graph (events around the timed replays, on the replay stream).
+    fused_b = dec_b + app_b
+    fused_us = ms_step * 1e3 / NL
+    ach = fused_b / (fused_us * 1e-6) / 1e9
     line["roofline"] = {
-        "kernel": "decode_kernel (decode attention of one layer, one launch)",
+        "kernel": "decode_kernel<G, S, fused> (one-token append + decode attention of one "
+                  "layer, one launch; the only kernel of the timed step)",
         "bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
         "frac": round(ach / peak, 4), "peak_kind": peak_kind,
         "frac_of_nominal": round(ach / NOMINAL_HBM_GBS, 4),
+        "traffic": _traffic("fused", fused_b), "us_per_launch": round(fused_us, 3),
+        "us_per_launch_alone": round(iso_ms * 1e3, 3),
+        "bytes_per_launch": fused_b,
+        "timing": "timed step graph: mean device time per launch (36 launches per step, "
+                  "programmatic launch overlap included); 'alone' = between event nodes"}
+    dach = dec_b / (dec_ms * 1e-3) / 1e9
+    line["decode_attention"] = {
+        "kernel": "decode_kernel<G, S> (decode attention of one layer, one launch)",
+        "achieved": round(dach, 1), "unit": "GB/s", "frac": round(dach / peak, 4),
+        "frac_of_nominal": round(dach / NOMINAL_HBM_GBS, 4),
         "traffic": _traffic("decode", dec_b), "us_per_launch": round(dec_ms * 1e3, 3),
-        "fused_us_per_launch_alone": round(iso_ms * 1e3, 3),
         "bytes_per_launch": dec_b, "timing": dec_how}
     line["append"] = append
     line["plain_int4"] = plain
     line["nvfp4"] = nvfp4
     line["prefill"] = prefill
+    line["long_context"] = configs.get("long_context")
+    line["ragged"] = configs.get("ragged")
+    line["tiny"] = configs.get("tiny")
     line["clocks"] = clk.result
     return line
 
@@ -391,6 +433,7 @@ def run_append_bench(dev, reps=20):
     v = workloads.kv_rows_torch(w, 0, 1, T, stream=1, device=dev)
     cu = torch.from_numpy(workloads.cu_seqlens(cap)).to(dev)
     z = torch.zeros(B, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     res = {}
     peak, _ = _peaks()
     for block in [1] + list(w.blocks_sweep):
@@ -400,13 +443,8 @@ def run_append_bench(dev, reps=20):
         for _ in range(3):
             kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
-        b.record()
-        torch.cuda.synchronize()
-        us = a.elapsed_time(b) * 1e3 / reps
+        us = _timed_calls(lambda: kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd), reps,
+                          flush) * 1e3
         gbs = append_bytes(T, H) / (us * 1e-6) / 1e9
         res[f"b{block}"] = {"us_per_call": round(us, 2), "tok_s": round(T / (us * 1e-6), 1),
                             "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
@@ -414,6 +452,8 @@ def run_append_bench(dev, reps=20):
         cache.close()
     res["workload"] = ("prefill_append: 8 x 8192 tokens, 8 KV heads, page 16, Student-t(3); "
                        "b1 = plain INT4 (no rotation)")
+    res["timing"] = ("events around each call, a 256 MB write between calls (flushes the "
+                     "126 MB L2)")
     res["traffic"] = _traffic("append", append_bytes(T, H))
     return res
 
@@ -567,12 +607,8 @@ def run_nvfp4_bench(dev, reps=10):
     for _ in range(3):
         kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
     torch.cuda.synchronize()
-    a.record()
-    for _ in range(20):
-        kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
-    b.record()
-    torch.cuda.synchronize()
-    us = a.elapsed_time(b) * 1e3 / 20
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    us = _timed_calls(lambda: kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd), 20, flush) * 1e3
     gbs = append_bytes(T, H, BYTES_PER_TOKEN_HEAD_NVFP4) / (us * 1e-6) / 1e9
     res["append_b128"] = {"us_per_call": round(us, 2), "tok_s": round(T / (us * 1e-6), 1),
                           "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
@@ -580,6 +616,158 @@ def run_nvfp4_bench(dev, reps=10):
     assert kvq.get_device_status(cache) == 0
     cache.close()
     res["prefill"] = run_prefill_bench(dev, fmt=1)
+    return res
+
+
+def _fill_cache(cache, w, lens, ptd, layers, dev):
+    """Write lens[b] tokens of every sequence into each layer through the append kernel."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    zeros = torch.zeros(len(lens), dtype=torch.int32, device=dev)
+    cu = torch.from_numpy(workloads.cu_seqlens(lens)).to(dev)
+    for layer in range(layers):
+        kp = workloads.kv_rows_torch(w, layer, 0, int(np.sum(lens)), stream=1, device=dev)
+        vp = workloads.kv_rows_torch(w, layer, 1, int(np.sum(lens)), stream=1, device=dev)
+        kvq.rotate_quant_append(cache, layer, kp, vp, cu, zeros, ptd)
+        del kp, vp
+    torch.cuda.synchronize()
+
+
+def run_decode_config(dev, name, reps=5):
+    """Decode throughput on one decode workload at its full size: plain decode attention
+    (kvq_decode_attention) and the decode step (kvq_append_decode_attention: the step's
+    token of every sequence appended, then attention over it), each as a graph of calls
+    alternating over the workload's layer pools, mean device time per launch from events
+    around the replays.  long_context keeps two layer pools (2 x 190 MB), ragged one
+    (1.1 GB), both larger than the 126 MB L2."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    w = workloads.WORKLOADS[name]
+    L = workloads.context_lengths(w)
+    B, H, HQ, S = w.batch, w.num_kv_heads, w.num_q_heads, w.page_size
+    NL = 2 if name == "long_context" else 1
+    cap = L + 1
+    P = workloads.pool_pages(w, cap)
+    mp = int((cap.max() + S - 1) // S)
+    desc = kvq.Desc(NL, H, HQ, 128, w.block, S, P, B, mp)
+    cache, pt = kvq.alloc_pages(desc, cap, workloads.page_order(w, P))
+    ptd = torch.from_numpy(pt).to(dev)
+    _fill_cache(cache, w, L, ptd, NL, dev)
+    q = torch.stack([workloads.q_rows_torch(w, l, device=dev) for l in range(NL)])
+    kn = torch.stack([workloads.kv_rows_torch(w, l, 0, B, stream=2, device=dev) for l in range(NL)])
+    vn = torch.stack([workloads.kv_rows_torch(w, l, 1, B, stream=2, device=dev) for l in range(NL)])
+    out = torch.empty_like(q)
+    before = torch.from_numpy(L).to(dev)
+    after = torch.from_numpy(cap).to(dev)
+    side = torch.cuda.Stream(device=dev)
+    calls = 8
+    peak, peak_kind = _peaks()
+    dec_b = decode_bytes(cap, H, HQ, S)
+    fused_b = dec_b + append_bytes(B, H)
+    res = {"workload": f"{name}: batch {B}, {H} KV heads, {HQ} query heads, b = {w.block}, "
+                       f"page {S}, {int(cap.sum())} cached tokens after the step's append"
+                       + (", pages scattered through a 1.2x pool" if w.permute_pages else ""),
+           "bytes_per_launch": dec_b, "peak": peak, "peak_kind": peak_kind}
+    for key, fn, nb in (
+            ("decode", lambda l: kvq.decode_attention(cache, l, q[l], after, ptd, out=out[l]), dec_b),
+            ("fused", lambda l: kvq.append_decode_attention(cache, l, kn[l], vn[l], q[l], before, ptd,
+                                                            out=out[l]), fused_b)):
+        fn(0)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(calls):
+                fn(i % NL)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) * 1e3 / (reps * calls)
+        gbs = nb / (us * 1e-6) / 1e9
+        res[key] = {"us_per_launch": round(us, 3), "bytes_per_launch": nb, "gbs": round(gbs, 1),
+                    "frac": round(gbs / peak, 4), "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 4),
+                    "traffic": _traffic(f"{key}_{name}", nb)}
+        del g
+    res["how"] = (f"graph of {calls} calls alternating over {NL} layer pool(s), events around "
+                  f"{reps} replays; fused = the step's one-token append + decode in one launch")
+    if name == "long_context":
+        res["step_36_layers_ms_extrapolated"] = round(36 * res["fused"]["us_per_launch"] / 1e3, 4)
+    assert kvq.get_device_status(cache) == 0
+    cache.close()
+    return res
+
+
+def run_tiny_latency(dev, reps=200):
+    """The tiny workload's decode step (one fused append + decode launch over 257 tokens):
+    latency of one call alone (events around each eager call, median) and back to back in
+    a graph (mean per launch)."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    w = workloads.WORKLOADS["tiny"]
+    L = np.asarray(w.context, np.int32)
+    B, H, HQ, S = w.batch, w.num_kv_heads, w.num_q_heads, w.page_size
+    cap = L + 1
+    P = workloads.pool_pages(w, cap)
+    mp = int((cap.max() + S - 1) // S)
+    desc = kvq.Desc(1, H, HQ, 128, w.block, S, P, B, mp)
+    cache, pt = kvq.alloc_pages(desc, cap, None)
+    ptd = torch.from_numpy(pt).to(dev)
+    _fill_cache(cache, w, L, ptd, 1, dev)
+    q = workloads.q_rows_torch(w, 0, device=dev)
+    kn = workloads.kv_rows_torch(w, 0, 0, B, stream=2, device=dev)
+    vn = workloads.kv_rows_torch(w, 0, 1, B, stream=2, device=dev)
+    out = torch.empty_like(q)
+    before = torch.from_numpy(L).to(dev)
+    fn = lambda: kvq.append_decode_attention(cache, 0, kn, vn, q, before, ptd, out=out)  # noqa: E731
+    for _ in range(10):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(50)]
+    for a, b in ev:
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+    alone = float(np.median([a.elapsed_time(b) for a, b in ev])) * 1e3
+    side = torch.cuda.Stream(device=dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for _ in range(100):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps // 100 + 1):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    per = a.elapsed_time(b) * 1e3 / ((reps // 100 + 1) * 100)
+    assert kvq.get_device_status(cache) == 0
+    del g
+    cache.close()
+    return {"workload": "tiny: 1 sequence, 2 KV heads, 8 query heads, b = 32, page 16, "
+                        "256 cached tokens + the step's token",
+            "us_per_call_alone": round(alone, 3), "us_per_call_graph": round(per, 3),
+            "bytes_per_call": decode_bytes(cap, H, HQ, S) + append_bytes(B, H),
+            "how": "fused append + decode; alone = median of 50 eager calls with events around "
+                   "each; graph = mean over back-to-back launches in a graph of 100"}
+
+
+def run_decode_configs(dev):
+    res = {}
+    for name in ("long_context", "ragged"):
+        res[name] = run_decode_config(dev, name)
+    res["tiny"] = run_tiny_latency(dev)
     return res
 
 
@@ -736,6 +924,49 @@ def oracle_sample_threads(budget_s, threads):
     return byt / el / 1e9, threads, desc
 
 
+def cpu_model():
+    """The host CPU's model name (first 'model name' line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_append_sample(budget_s, threads=1):
+    """The oracle's rotate-quant-append on the prefill-append workload (b = 128, 8 KV heads,
+    Student-t(3) rows): calls of 64 tokens, each thread appending into its own one-sequence
+    pool (the C call releases the interpreter lock).  Returns (tokens/s, description)."""
+    import concurrent.futures
+    import oracle
+    w = workloads.WORKLOADS["prefill_append"]
+    H, S, n = w.num_kv_heads, w.page_size, 64
+    g = oracle.Geometry(1, H, w.num_q_heads, 128, 128, S, n // S, n // S)
+    pt = oracle.assign_pages(np.array([n], np.int32), S, n // S, n // S)
+    k, v = workloads.kv_rows(w, 0, 0, n, 1), workloads.kv_rows(w, 0, 1, n, 1)
+    cu, z = workloads.cu_seqlens([n]), np.zeros(1, np.int32)
+    t0 = time.perf_counter()
+
+    def work(tid):
+        pool = g.new_pool()
+        calls = 0
+        while time.perf_counter() - t0 < budget_s:
+            oracle.rotate_quant_append(g, pool, 0, k, v, cu, z, pt)
+            calls += 1
+        return calls
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        calls = sum(ex.map(work, range(threads)))
+    el = time.perf_counter() - t0
+    desc = (f"oracle (C, fp32 rotation, {threads} thread(s)): {calls} calls of {n} tokens x {H} "
+            f"KV heads, b = 128, prefill_append rows; {el:.2f} s")
+    return calls * n / el, desc
+
+
 def workload_config(world):
     """The bench workload's shape keys, shared by both arms' JSON lines."""
     w = workloads.WORKLOADS[WORKLOAD]
@@ -771,7 +1002,7 @@ def run_reference(args, rank, world):
         "config": {**workload_config(world),
                    "sample": "bounded per step: the oracle on host cores"},
         "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": descs[-1] if descs else ""},
+                         "sample": descs[-1] if descs else "", "cpu_model": cpu_model()},
         "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -784,8 +1015,10 @@ def run_kernel_case(which, calls):
     step's one-token append fused in; ``append`` = the prefill-append call (8 x 8192
     tokens, b = 128; 268 MB read, 69 MB written); ``prefill`` = chunked-prefill attention
     (16 x 128-token chunks after 896 cached tokens); ``decode_nvfp4``, ``fused_nvfp4``,
-    ``append_nvfp4`` and ``prefill_nvfp4`` are the same cases on an NVFP4 cache.  The kernel is launched ``calls``
-    times after the setup."""
+    ``append_nvfp4`` and ``prefill_nvfp4`` are the same cases on an NVFP4 cache;
+    ``decode_long`` / ``fused_long`` and ``decode_ragged`` / ``fused_ragged`` are the decode
+    and the fused step on one layer of the long-context (190 MB) and ragged (1.1 GB)
+    workloads.  The kernel is launched ``calls`` times after the setup."""
     import torch
 
     import bit_paged_kv_diag_b200 as kvq
@@ -835,20 +1068,21 @@ def run_kernel_case(which, calls):
         for _ in range(calls):
             kvq.rotate_quant_append(cache, 0, k, v, cu, z, ptd)
     else:
-        w = workloads.WORKLOADS[WORKLOAD]
-        L = np.asarray(w.context, np.int32)
+        # decode / fused on the Qwen3-4B-shaped layer; decode_long / fused_long on the
+        # long-context workload (one layer, 190 MB); decode_ragged / fused_ragged on the
+        # ragged workload (1.1 GB).
+        which, _, wl = which.partition("_")
+        w = workloads.WORKLOADS[{"": WORKLOAD, "long": "long_context", "ragged": "ragged"}[wl]]
+        L = workloads.context_lengths(w)
         B, H, S = w.batch, w.num_kv_heads, w.page_size
         cap = L + 1
         P = workloads.pool_pages(w, cap)
         desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, int((cap.max() + S - 1) // S),
                         fmt)
-        cache, pt = kvq.alloc_pages(desc, cap, None)
+        cache, pt = kvq.alloc_pages(desc, cap, workloads.page_order(w, P))
         ptd = torch.from_numpy(pt).to(dev)
-        kp = workloads.kv_rows_torch(w, 0, 0, int(cap.sum()), stream=1, device=dev)
-        vp = workloads.kv_rows_torch(w, 0, 1, int(cap.sum()), stream=1, device=dev)
-        kvq.rotate_quant_append(cache, 0, kp, vp, torch.from_numpy(workloads.cu_seqlens(cap)).to(dev),
-                                torch.zeros(B, dtype=torch.int32, device=dev), ptd)
-        del kp, vp
+        _fill_cache(cache, w, cap, ptd, 1, dev)
+        torch.cuda.empty_cache()
         q = workloads.q_rows_torch(w, 0, device=dev)
         lens = torch.from_numpy(cap).to(dev)
         kn = workloads.kv_rows_torch(w, 0, 0, B, stream=2, device=dev)
@@ -875,7 +1109,9 @@ def main():
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", choices=["decode", "fused", "append", "prefill", "decode_nvfp4",
-                                              "fused_nvfp4", "append_nvfp4", "prefill_nvfp4"],
+                                              "fused_nvfp4", "append_nvfp4", "prefill_nvfp4",
+                                              "decode_long", "fused_long", "decode_ragged",
+                                              "fused_ragged"],
                     default=None,
                     help="run one small case of one kernel (for ncu captures) and exit")
     ap.add_argument("--calls", type=int, default=3)
@@ -908,12 +1144,20 @@ def main():
         line = run_kvq(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                v, d = oracle_sample(12.0)
+                v, d = oracle_sample(10.0)
+                model = cpu_model()
                 line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": 1,
-                                        "kind": "oracle", "sample": d}
-                v, n, d = oracle_sample_threads(8.0, os.cpu_count() or 1)
+                                        "kind": "oracle", "sample": d, "cpu_model": model}
+                ncpu = os.cpu_count() or 1
+                v, n, d = oracle_sample_threads(6.0, ncpu)
                 line["cpu_baseline_all_cores"] = {"value": round(v, 4), "unit": "GB/s", "cores": n,
-                                                  "kind": "oracle", "sample": d}
+                                                  "kind": "oracle", "sample": d, "cpu_model": model}
+                a1, d1 = oracle_append_sample(4.0, 1)
+                an, dn = oracle_append_sample(4.0, ncpu)
+                line["cpu_baseline_append"] = {
+                    "unit": "tok/s", "kind": "oracle", "cpu_model": model,
+                    "one_core": {"value": round(a1, 1), "cores": 1, "sample": d1},
+                    "all_cores": {"value": round(an, 1), "cores": ncpu, "sample": dn}}
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

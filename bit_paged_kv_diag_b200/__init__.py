@@ -85,8 +85,8 @@ def lib() -> ctypes.CDLL:
             "kvq_get_device_status": (ctypes.c_int, [vp, i32p, vp]),
             "kvq_free": (ctypes.c_int, [vp]),
             "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
-            "kvq_decode_attention_noalloc": (ctypes.c_int, [dp, vp, i32, vp, vp, vp, i32,
-                                                            ctypes.c_float, vp, vp]),
+            "kvq_decode_attention_noalloc": (ctypes.c_int, [dp, vp, ctypes.c_size_t, i32, vp, vp,
+                                                            vp, i32, ctypes.c_float, vp, vp, vp]),
             "kvq_append_decode_attention": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, vp, i32,
                                                            ctypes.c_float, vp, vp]),
             "kvq_prefill_attention": (ctypes.c_int, [vp, i32, vp, vp, vp, vp, i32, i32,
@@ -266,18 +266,20 @@ def prefill_attention(cache: Cache, layer: int, q, cu_q, seq_lens, page_table, s
 
 
 def decode_attention_noalloc(desc: Desc, pool, layer: int, q, seq_lens, page_table,
-                             softmax_scale=0.0, out=None, stream=None):
+                             softmax_scale=0.0, out=None, status=None, stream=None):
     """Decode attention without a handle and without any device allocation by the library
-    (scratch lives in a fixed device array; see include/kvq.h for its limits)."""
+    (its scratch lives in a fixed device array; limits in include/kvq.h).  ``status``: an
+    optional int32 CUDA tensor of one element that receives the KVQ_DEV_* bits."""
     import torch
     if out is None:
         out = torch.empty_like(q)
     batch = int(seq_lens.shape[0])
+    st = None if status is None else _dev_ptr(status, "status", torch.int32)
     rc = lib().kvq_decode_attention_noalloc(
-        ctypes.byref(desc), _dev_ptr(pool, "pool", torch.uint8), int(layer),
+        ctypes.byref(desc), _dev_ptr(pool, "pool", torch.uint8), int(pool.numel()), int(layer),
         _dev_ptr(q, "q", torch.float16), _dev_ptr(seq_lens, "seq_lens", torch.int32),
         _dev_ptr(page_table, "page_table", torch.int32), batch, float(softmax_scale),
-        _dev_ptr(out, "out", torch.float16), _stream_ptr(stream))
+        _dev_ptr(out, "out", torch.float16), st, _stream_ptr(stream))
     _check(rc, "kvq_decode_attention_noalloc")
     return out
 

@@ -30,9 +30,9 @@ struct kvq_cache {
   float cb;
 };
 
-namespace {
+namespace kvq {
 
-bool desc_ok(const kvq_desc* d, int* why) {
+bool desc_valid(const kvq_desc* d, int* why) {
   *why = KVQ_EINVAL;
   if (!d) return false;
   if (d->num_layers < 1 || d->num_kv_heads < 1 || d->num_q_heads < 1 || d->num_pages < 1 ||
@@ -60,16 +60,26 @@ bool desc_ok(const kvq_desc* d, int* why) {
   return true;
 }
 
-// Bytes of one token row of a (page, head) block: K and V codes, then the scales (one
-// fp16 each for INT4; one E4M3 per 16 channels each for NVFP4).
-size_t row_bytes(const kvq_desc* d) {
+// K and V codes, then the scales (one fp16 each for INT4; one E4M3 per 16 channels each
+// for NVFP4).
+size_t desc_row_bytes(const kvq_desc* d) {
   return static_cast<size_t>(d->head_dim) +
          (d->kv_format == KVQ_FORMAT_NVFP4 ? static_cast<size_t>(d->head_dim) / 8 : 4);
 }
 
+size_t desc_layer_bytes(const kvq_desc* d) {
+  return static_cast<size_t>(d->num_pages) * static_cast<size_t>(d->num_kv_heads) *
+         static_cast<size_t>(d->page_size) * desc_row_bytes(d);
+}
+
+}  // namespace kvq
+
+namespace {
+
+bool desc_ok(const kvq_desc* d, int* why) { return kvq::desc_valid(d, why); }
+
 size_t pool_bytes_of(const kvq_desc* d) {
-  return static_cast<size_t>(d->num_layers) * static_cast<size_t>(d->num_pages) *
-         static_cast<size_t>(d->num_kv_heads) * static_cast<size_t>(d->page_size) * row_bytes(d);
+  return static_cast<size_t>(d->num_layers) * kvq::desc_layer_bytes(d);
 }
 
 // fp32 value nearest 1/sqrt(b) (b = 32, 64, 128).

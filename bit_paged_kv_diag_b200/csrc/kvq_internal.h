@@ -5,7 +5,18 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/kvq.h"
+
 namespace kvq {
+
+// Descriptor validation shared by every entry point that takes a kvq_desc: true when the
+// geometry is one the kernels implement; otherwise *why is KVQ_EINVAL (a null descriptor,
+// a non-positive size) or KVQ_EUNSUPPORTED (a shape outside the kernels).
+bool desc_valid(const kvq_desc* d, int* why);
+// Bytes of one token row of a (page, head) block (132 INT4, 144 NVFP4) and of one layer of
+// the pool; desc_valid(d) must hold.
+size_t desc_row_bytes(const kvq_desc* d);
+size_t desc_layer_bytes(const kvq_desc* d);
 
 // Device status bits (same values as KVQ_DEV_* in include/kvq.h).
 constexpr int KVQ_DEV_BAD_PAGE_BIT = 1;

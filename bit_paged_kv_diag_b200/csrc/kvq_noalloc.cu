@@ -5,8 +5,9 @@
 // of device memory for its own pool and forbids stray allocations, a plugin whose host
 // framework owns every device allocation, or a latency-critical path where cudaMalloc's
 // implicit device synchronisation is not acceptable.  kvq_decode_attention_noalloc runs the
-// same decode kernel with its scratch (status word, per-unit arrival counters, per-CTA
-// partials) in one file-scope __device__ array of fixed size, so it allocates nothing.
+// same decode kernel with its scratch (per-unit arrival counters, per-CTA partials, and a
+// status word for callers that pass none) in one file-scope __device__ array of fixed size,
+// so it allocates nothing.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -19,8 +20,11 @@
 namespace {
 
 // Static scratch: [status word, padded to 256 B][arrival counters][partial records].
-constexpr int kNoAllocMaxUnits = 4096;    // batch * num_kv_heads
-constexpr int kNoAllocMaxRecords = 4096;  // (batch * num_kv_heads + grid CTAs) * G
+// The records bound the call: (batch * num_kv_heads + grid CTAs) * G <= kNoAllocMaxRecords.
+// That bound also keeps batch * num_kv_heads below kNoAllocMaxUnits, the size of the
+// counter array (one counter per (sequence, KV head) unit).
+constexpr int kNoAllocMaxUnits = 4096;
+constexpr int kNoAllocMaxRecords = 4096;
 constexpr size_t kNoAllocCounterBytes = kNoAllocMaxUnits * sizeof(int32_t);
 constexpr size_t kNoAllocBytes =
     256 + kNoAllocCounterBytes + static_cast<size_t>(kNoAllocMaxRecords) * kvq::kDecodeWarps *
@@ -34,14 +38,28 @@ std::mutex g_setup_mu;
 unsigned char* g_scratch_addr[kMaxDevices];  // device address of the array, per device
 int g_num_sms[kMaxDevices];
 
-// Once per device, with that device current: the array's device address (its name in
-// host code is only a host-side stand-in) and zeroed counters.
-int setup_device(int dev, unsigned char** scratch, int* num_sms) {
+// Launch shapes already planned, so a call after the first for a given shape makes no
+// attribute or occupancy queries.  Keyed by device, G, page size, format and the batch
+// rounded up to a power of two (the plan's shared memory holds per-sequence arrays).
+struct PlanEntry {
+  int dev, g, page_size, fp4, batch_cap;
+  kvq::DecodeLaunch launch;
+};
+constexpr int kMaxPlans = 256;
+PlanEntry g_plans[kMaxPlans];
+int g_num_plans = 0;
+
+// The array's device address on the current device (its name in host code is only a
+// host-side stand-in), looked up on every call: the lookup is a host-side query that
+// allocates nothing, and it stays right if the context was reset since the last call.
+// The first time an address is seen on a device, the counters are zeroed (synchronising
+// the device); a module loaded anew after a reset starts zeroed as well.
+int scratch_for(int dev, unsigned char** scratch, int* num_sms) {
   if (dev < 0 || dev >= kMaxDevices) return KVQ_EUNSUPPORTED;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return KVQ_ECUDA;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_addr[dev]) {
-    void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return KVQ_ECUDA;
+  if (g_scratch_addr[dev] != addr) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return KVQ_ECUDA;
@@ -55,45 +73,46 @@ int setup_device(int dev, unsigned char** scratch, int* num_sms) {
   return KVQ_OK;
 }
 
-bool noalloc_desc_ok(const kvq_desc* d) {
-  if (!d || d->num_layers < 1 || d->num_kv_heads < 1 || d->num_q_heads < 1 ||
-      d->num_pages < 1 || d->max_batch < 1 || d->max_pages_per_seq < 1)
-    return false;
-  if (d->num_q_heads % d->num_kv_heads) return false;
-  const int g = d->num_q_heads / d->num_kv_heads;
-  if (g != 1 && g != 2 && g != 4 && g != 8) return false;
-  if (d->head_dim != 128) return false;
-  const int hb = d->hadamard_block;
-  if (hb != 1 && hb != 32 && hb != 64 && hb != 128) return false;  // 1: plain INT4, no rotation
-  const int S = d->page_size;
-  if (S != 16 && S != 32 && S != 64 && S != 128 && S != 256) return false;
-  if (d->kv_format != KVQ_FORMAT_INT4 && d->kv_format != KVQ_FORMAT_NVFP4) return false;
-  if (d->max_batch > 4096) return false;
-  if (static_cast<long long>(d->max_pages_per_seq) * S > (1LL << 30)) return false;
-  const long long tiles_per_seq = (static_cast<long long>(d->max_pages_per_seq) * S + 31) / 32;
-  if (static_cast<long long>(d->max_batch) * d->num_kv_heads * tiles_per_seq >= (1LL << 30))
-    return false;
-  return true;
+// Returns 0, -1 (shape the decode kernel does not implement) or -2 (CUDA error).
+int plan_for(int dev, int g, int page_size, int fp4, int batch, int num_sms, kvq::DecodeLaunch* L) {
+  int cap = 16;
+  while (cap < batch) cap *= 2;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  for (int i = 0; i < g_num_plans; i++) {
+    const PlanEntry& e = g_plans[i];
+    if (e.dev == dev && e.g == g && e.page_size == page_size && e.fp4 == fp4 && e.batch_cap == cap) {
+      *L = e.launch;
+      return 0;
+    }
+  }
+  const int rc = kvq::plan_decode(g, page_size, cap, num_sms, fp4, L);
+  if (rc != 0) return rc;
+  if (g_num_plans < kMaxPlans) g_plans[g_num_plans++] = PlanEntry{dev, g, page_size, fp4, cap, *L};
+  return 0;
 }
 
 }  // namespace
 
 extern "C" {
 
-int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, int32_t layer,
-                                 const void* q, const int32_t* seq_lens,
+int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, size_t pool_bytes,
+                                 int32_t layer, const void* q, const int32_t* seq_lens,
                                  const int32_t* page_table, int32_t batch, float softmax_scale,
-                                 void* out, void* stream) {
-  if (!noalloc_desc_ok(d)) return d ? KVQ_EUNSUPPORTED : KVQ_EINVAL;
+                                 void* out, int32_t* dev_status, void* stream) {
+  int why = KVQ_OK;
+  if (!kvq::desc_valid(d, &why)) return why;
   if (layer < 0 || layer >= d->num_layers) return KVQ_EINVAL;
   if (batch < 0 || batch > d->max_batch) return KVQ_EINVAL;
   if (!(softmax_scale >= 0.0f) || isinf(softmax_scale)) return KVQ_EINVAL;
   if (batch == 0) return KVQ_OK;
   if (!pool || !q || !seq_lens || !page_table || !out) return KVQ_EINVAL;
+  const size_t layer_bytes = kvq::desc_layer_bytes(d);
+  if (pool_bytes < static_cast<size_t>(d->num_layers) * layer_bytes) return KVQ_EINVAL;
   const uintptr_t a16 = 15u;
   if ((reinterpret_cast<uintptr_t>(pool) | reinterpret_cast<uintptr_t>(q) |
        reinterpret_cast<uintptr_t>(out)) & a16)
     return KVQ_EINVAL;
+  if (reinterpret_cast<uintptr_t>(dev_status) & 3u) return KVQ_EINVAL;
   const int g = d->num_q_heads / d->num_kv_heads;
   const long long units = static_cast<long long>(batch) * d->num_kv_heads;
   if (units > kNoAllocMaxUnits) return KVQ_EUNSUPPORTED;
@@ -102,23 +121,23 @@ int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, int32_t la
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ECUDA;
   unsigned char* scratch = nullptr;
   int num_sms = 0;
-  const int rc = setup_device(dev, &scratch, &num_sms);
+  const int rc = scratch_for(dev, &scratch, &num_sms);
   if (rc != KVQ_OK) return rc;
 
   kvq::DecodeLaunch L;
   const int fp4 = d->kv_format == KVQ_FORMAT_NVFP4;
-  if (kvq::plan_decode(g, d->page_size, batch, num_sms, fp4, &L) != 0) return KVQ_ECUDA;
+  const int prc = plan_for(dev, g, d->page_size, fp4, batch, num_sms, &L);
+  if (prc == -1) return KVQ_EUNSUPPORTED;
+  if (prc != 0) return KVQ_ECUDA;
   if ((units + L.grid) * g > kNoAllocMaxRecords) return KVQ_EUNSUPPORTED;
 
   kvq::DecodeParams p;
-  const size_t layer_bytes = static_cast<size_t>(d->num_pages) * d->num_kv_heads *
-                             d->page_size * (d->head_dim + (fp4 ? d->head_dim / 8 : 4));
   p.pool_layer = static_cast<const uint8_t*>(pool) + static_cast<size_t>(layer) * layer_bytes;
   p.q = static_cast<const __half*>(q);
   p.seq_lens = seq_lens;
   p.page_table = page_table;
   p.out = static_cast<__half*>(out);
-  p.status = reinterpret_cast<int32_t*>(scratch);
+  p.status = dev_status ? dev_status : reinterpret_cast<int32_t*>(scratch);
   p.counters = reinterpret_cast<int32_t*>(scratch + 256);
   p.part = reinterpret_cast<float*>(scratch + 256 + kNoAllocCounterBytes);
   p.batch = batch;

@@ -153,7 +153,8 @@ KVQ_API int kvq_assign_pages(const kvq_desc* d, int32_t batch, const int32_t* ca
                      const int32_t* page_order, int32_t* page_table);
 
 /* Create a cache handle, the split-KV scratch and (optionally) the pool, and assign
- * pages with kvq_assign_pages.
+ * pages with kvq_assign_pages: the pages' fixed-size KV blocks addressed through a page
+ * table ("KVキャッシュを4ビットへ", section "KVキャッシュこそが本当のボトルネックである理由").
  *   dev_pool    device buffer of >= kvq_pool_bytes(d) bytes, 16-byte aligned, owned by
  *               the caller; NULL = the library allocates (cudaMalloc) and owns the pool
  *   pool_bytes  size of dev_pool (ignored when dev_pool is NULL)
@@ -186,7 +187,10 @@ KVQ_API int kvq_rotate_quant_append(kvq_cache* c, int32_t layer, const void* k, 
                             int32_t total_new_tokens, void* stream);
 
 /* Paged GQA decode attention over the cache (INT4 or NVFP4) of one layer: one query
- * token per sequence.  One kernel launch: a split-KV pass whose last-arriving CTA per (sequence,
+ * token per sequence.  The pages' fused attention over the paged, quantised cache, q
+ * rotated with the cache's transform and the output rotated back ("KVキャッシュを4ビットへ",
+ * sections "KVキャッシュこそが本当のボトルネックである理由" and "回転のトリック —
+ * ブロック対角アダマール").  One kernel launch: a split-KV pass whose last-arriving CTA per (sequence,
  * KV head) merges the splits and applies the inverse rotation.
  *   q              device fp16 [batch][num_q_heads][128], 16-byte aligned
  *   seq_lens       device int32 [batch], lengths AFTER any append (tokens to attend)
@@ -256,23 +260,31 @@ KVQ_API int kvq_prefill_attention(kvq_cache* c, int32_t layer, const void* q,
  * geometry and the pool directly and keeps its scratch in one fixed-size device array
  * inside the library (about 8.7 MB, held by every GPU that loads the library until exit).
  *   d              cache geometry (as for kvq_alloc_pages); only read
- *   pool           device pool of kvq_pool_bytes(d) bytes, 16-byte aligned, laid out as
- *                  kvq_rotate_quant_append writes it (caller-owned)
+ *   pool           device pool, 16-byte aligned, laid out as kvq_rotate_quant_append
+ *                  writes it (caller-owned)
+ *   pool_bytes     size of pool; less than kvq_pool_bytes(d) is KVQ_EINVAL
+ *   dev_status     device int32, 4-byte aligned, caller-owned: the kernel ORs KVQ_DEV_*
+ *                  bits into it (the caller reads and clears it); NULL = the bits go to a
+ *                  word inside the library's array that is never read
  *   layer, q, seq_lens, page_table, batch, softmax_scale, out, stream: as for
  *                  kvq_decode_attention
- * Limits of the fixed scratch: batch * num_kv_heads <= 4096 and
- * (batch * num_kv_heads + C) * G <= 4096, C = the kernel's grid (up to 3 CTAs per SM);
- * larger calls return KVQ_EUNSUPPORTED before anything is launched.
- * The first call on a device sets the array up (looks up its device address and zeroes
- * its counters, synchronising the device); make that first call before any stream
- * capture.  Every call shares the array: calls that overlap on the GPU (two streams, or
- * two devices' contexts racing on one device) race on it and must be ordered by the
- * caller.  Device-side range errors are not reported by this call (they still never
- * fault).  Returns KVQ_OK or a negative status. */
-KVQ_API int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, int32_t layer,
-                                         const void* q, const int32_t* seq_lens,
+ * Limits of the fixed scratch: (batch * num_kv_heads + C) * G <= 4096, C = the kernel's
+ * grid (up to 3 CTAs per SM); a larger call returns KVQ_EUNSUPPORTED before anything is
+ * launched.
+ * The first call on a device (and the first after a context reset) sets the array up:
+ * it zeroes the arrival counters, which synchronises the device; make that first call
+ * before any stream capture.  Later calls look up the array's address (a host-side query)
+ * and reuse the launch shape planned for their (G, page size, format, batch) class.
+ * Every call shares the array: calls that overlap on the GPU (two streams, or two
+ * processes' contexts on one device) race on it and must be ordered by the caller.  A
+ * call whose bounded wait gave up (KVQ_DEV_TIMEOUT in dev_status) has undefined outputs,
+ * but every CTA of it still arrives on the counters it uses, so the counters are back at
+ * zero when it ends and later calls are unaffected.  Returns KVQ_OK or a negative status. */
+KVQ_API int kvq_decode_attention_noalloc(const kvq_desc* d, const void* pool, size_t pool_bytes,
+                                         int32_t layer, const void* q, const int32_t* seq_lens,
                                          const int32_t* page_table, int32_t batch,
-                                         float softmax_scale, void* out, void* stream);
+                                         float softmax_scale, void* out, int32_t* dev_status,
+                                         void* stream);
 
 /* Device address of the pool (the caller's buffer, or the library's). NULL for NULL. */
 KVQ_API void* kvq_pool_ptr(const kvq_cache* c);
@@ -282,7 +294,8 @@ KVQ_API void* kvq_pool_ptr(const kvq_cache* c);
 KVQ_API int kvq_get_device_status(kvq_cache* c, int32_t* status, void* stream);
 
 /* Free library-owned memory (the handle, scratch, status word, and the pool if the
- * library allocated it).  Synchronises the device first.  NULL is a no-op.  Returns
+ * library allocated it): the release of the paged cache that kvq_alloc_pages created
+ * ("KVキャッシュを4ビットへ", section "KVキャッシュこそが本当のボトルネックである理由").  Synchronises the device first.  NULL is a no-op.  Returns
  * KVQ_OK, or KVQ_ECUDA if an earlier asynchronous error is found. */
 KVQ_API int kvq_free(kvq_cache* c);
 

@@ -119,22 +119,25 @@ def test_calls_reject_bad_arguments_before_any_cuda_call():
 
 
 def test_noalloc_decode_rejects_bad_arguments_before_any_cuda_call():
-    """The allocation-free decode checks its descriptor, layer, batch, scale, pointers,
-    alignment and the fixed scratch's unit limit before its first CUDA call."""
+    """The allocation-free decode checks its descriptor, pool size, layer, batch, scale,
+    pointers, alignment and the fixed scratch's unit limit before its first CUDA call."""
     L = kvq.lib()
     d = _desc()
     ok = 0x10000  # 16-byte aligned stand-ins; nothing is dereferenced on these paths
-    args = lambda **kw: dict(dict(d=ctypes.byref(d), pool=ok, layer=0, q=ok, lens=ok, pt=ok,  # noqa: E731
-                                  batch=4, scale=0.0, out=ok), **kw)
+    need = kvq.pool_bytes(d)
+    args = lambda **kw: dict(dict(d=ctypes.byref(d), pool=ok, nbytes=need, layer=0, q=ok,  # noqa: E731
+                                  lens=ok, pt=ok, batch=4, scale=0.0, out=ok, st=None), **kw)
 
     def call(a):
-        return L.kvq_decode_attention_noalloc(a["d"], a["pool"], a["layer"], a["q"], a["lens"],
-                                              a["pt"], a["batch"], a["scale"], a["out"], None)
+        return L.kvq_decode_attention_noalloc(a["d"], a["pool"], a["nbytes"], a["layer"], a["q"],
+                                              a["lens"], a["pt"], a["batch"], a["scale"], a["out"],
+                                              a["st"], None)
 
     assert call(args(d=None)) == kvq.KVQ_EINVAL
     for bad in (dict(head_dim=96), dict(num_q_heads=24), dict(hadamard_block=16),
                 dict(page_size=8), dict(kv_format=2), dict(max_batch=5000)):
         assert call(args(d=ctypes.byref(_desc(**bad)))) == kvq.KVQ_EUNSUPPORTED, bad
+    assert call(args(d=ctypes.byref(_desc(num_layers=0)))) == kvq.KVQ_EINVAL
     assert call(args(layer=2)) == kvq.KVQ_EINVAL
     assert call(args(layer=-1)) == kvq.KVQ_EINVAL
     assert call(args(batch=17)) == kvq.KVQ_EINVAL
@@ -147,5 +150,11 @@ def test_noalloc_decode_rejects_bad_arguments_before_any_cuda_call():
         assert call(args(**{name: None})) == kvq.KVQ_EINVAL, name
     for name in ("pool", "q", "out"):
         assert call(args(**{name: ok + 8})) == kvq.KVQ_EINVAL, name
+    assert call(args(st=ok + 2)) == kvq.KVQ_EINVAL          # misaligned status word
+    # a pool smaller than the descriptor's layers: rejected before the kernel could read
+    # past its end
+    assert call(args(nbytes=need - 1)) == kvq.KVQ_EINVAL
+    assert call(args(nbytes=0)) == kvq.KVQ_EINVAL
     big = _desc(num_kv_heads=8, num_q_heads=8, max_batch=4096)
-    assert call(args(d=ctypes.byref(big), batch=513)) == kvq.KVQ_EUNSUPPORTED  # 513 * 8 > 4096
+    assert call(args(d=ctypes.byref(big), nbytes=kvq.pool_bytes(big),
+                     batch=513)) == kvq.KVQ_EUNSUPPORTED  # 513 * 8 units > the counter array

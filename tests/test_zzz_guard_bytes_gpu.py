@@ -84,9 +84,11 @@ def test_calls_write_only_inside_their_buffers(fmt):
         lens = lens + 1
         # the allocation-free decode over the final lengths
         b_na, o_na = _guarded_like(q, dev)
-        kvq.decode_attention_noalloc(d, pool, L, q, t(lens), pt, out=o_na)
+        st_na = torch.zeros(1, dtype=torch.int32, device=dev)
+        kvq.decode_attention_noalloc(d, pool, L, q, t(lens), pt, out=o_na, status=st_na)
         torch.cuda.synchronize()
         assert kvq.get_device_status(cache) == 0
+        assert int(st_na.item()) == 0
         assert _intact(pbuf), "a kernel wrote outside the pool"
         layer_bytes = nbytes // 2
         assert not bool(pool[:layer_bytes].any().item()), "a kernel wrote into the other layer"
