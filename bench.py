@@ -314,32 +314,102 @@ def run_kvq(args, rank, world, local_rank):
     value = whole_job_gbs(world, step_bytes, ms_step)
     peak, peak_kind = _peaks()
 
-    # End to end through the C ABI with host buffers: per step, H2D of q and the step's
-    # K/V rows from pinned memory, the step, D2H of the outputs.
+    # End to end through the C ABI with host buffers.  Every step copies its inputs (q and the
+    # step's K/V rows of all layers) from pinned host memory and its outputs back.  Main leg:
+    # two buffer sets and one captured graph per set; the H2D copies of step s + 1 and the
+    # D2H copies of step s run on their own streams under step s's compute (the copy engines
+    # work beside the SMs).  'serial' = the same with every copy in line on one stream;
+    # 'per_call' = the double-buffered loop issuing the 36 kvq_append_decode_attention calls
+    # per step through the Python binding instead of a graph.
     hq = q.cpu().pin_memory()
     hk, hv = kn.cpu().pin_memory(), vn.cpu().pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     e2e_steps = max(3, min(args.steps, 200))
-
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        kn.copy_(hk, non_blocking=True)
-        vn.copy_(hv, non_blocking=True)
-        graph.replay()
-        hout.copy_(out, non_blocking=True)
-
-    for _ in range(3):
-        e2e_step()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record()
+    s_h2d, s_d2h, s_comp = (torch.cuda.Stream(device=dev) for _ in range(3))
+    bufs = []
+    for b in range(2):
+        qb, knb, vnb, ob = (torch.empty_like(t) for t in (q, kn, vn, out))
+        qb.copy_(q), knb.copy_(kn), vnb.copy_(vn)
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb, stream=side):
+            for l in range(NL):
+                kvq.append_decode_attention(cache, l, knb[l], vnb[l], qb[l], lens_before, ptd, out=ob[l])
+        bufs.append((qb, knb, vnb, ob, gb))
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+
+    def step_calls(b):
+        qb, knb, vnb, ob, _ = bufs[b]
+        for l in range(NL):
+            kvq.append_decode_attention(cache, l, knb[l], vnb[l], qb[l], lens_before, ptd, out=ob[l])
+
+    def e2e_pipelined(K, use_graph=True):
+        ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
+        in_ready, computed, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def h2d(b):
+            qb, knb, vnb, _, _ = bufs[b]
+            qb.copy_(hq, non_blocking=True)
+            knb.copy_(hk, non_blocking=True)
+            vnb.copy_(hv, non_blocking=True)
+            in_ready[b].record(s_h2d)
+
+        with torch.cuda.stream(s_h2d):
+            t0.record(s_h2d)
+            h2d(0)
+        for st in range(K):
+            b = st % 2
+            s_comp.wait_event(in_ready[b])
+            if st >= 2:
+                s_comp.wait_event(out_done[b])     # step st - 2's outputs have left buffer b
+            with torch.cuda.stream(s_comp):
+                if use_graph:
+                    bufs[b][4].replay()
+                else:
+                    step_calls(b)
+                computed[b].record(s_comp)
+            if st + 1 < K:
+                nb = (st + 1) % 2
+                with torch.cuda.stream(s_h2d):
+                    if st >= 1:
+                        s_h2d.wait_event(computed[nb])  # step st - 1 has read buffer nb
+                    h2d(nb)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(computed[b])
+                hout[b].copy_(bufs[b][3], non_blocking=True)
+                out_done[b].record(s_d2h)
+        with torch.cuda.stream(s_d2h):
+            t1.record(s_d2h)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / K
+
+    def e2e_serial(K):
+        qb, knb, vnb, ob, gb = bufs[0]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s_comp):
+            t0.record(s_comp)
+            for _ in range(K):
+                qb.copy_(hq, non_blocking=True)
+                knb.copy_(hk, non_blocking=True)
+                vnb.copy_(hv, non_blocking=True)
+                gb.replay()
+                hout[0].copy_(ob, non_blocking=True)
+            t1.record(s_comp)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / K
+
+    e2e_pipelined(3)
+    barrier()
+    e2e_ms = max_over_ranks(e2e_pipelined(e2e_steps), world, dev)
+    e2e_serial(3)
+    e2e_serial_ms = max_over_ranks(e2e_serial(e2e_steps), world, dev)
+    e2e_pipelined(3, use_graph=False)
+    call_steps = max(3, min(args.steps, 50))
+    e2e_call_ms = max_over_ranks(e2e_pipelined(call_steps, use_graph=False), world, dev)
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
-    d2h = hout.numel() * 2
+    d2h = hout[0].numel() * 2
+    assert kvq.get_device_status(cache) == 0
+    del bufs
 
     del graph
     cache.close()
@@ -365,7 +435,19 @@ def run_kvq(args, rank, world, local_rank):
         "device_status": status,
         "e2e": {"value": round(whole_job_gbs(world, step_bytes, e2e_ms), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "ms_per_step": round(e2e_ms, 5)},
+                "ms_per_step": round(e2e_ms, 5),
+                "how": "per step: H2D of q and the step's K/V rows from pinned host memory, the "
+                       "36-layer step (one captured graph per buffer set), D2H of the outputs; "
+                       "two buffer sets, copies of the neighbouring steps on their own streams "
+                       "under the compute",
+                "serial": {"value": round(whole_job_gbs(world, step_bytes, e2e_serial_ms), 1),
+                           "ms_per_step": round(e2e_serial_ms, 5),
+                           "how": "every copy in line with the step on one stream"},
+                "per_call": {"value": round(whole_job_gbs(world, step_bytes, e2e_call_ms), 1),
+                             "ms_per_step": round(e2e_call_ms, 5), "steps": call_steps,
+                             "how": "as the main leg, the 36 kvq_append_decode_attention calls "
+                                    "per step issued through the Python binding (ctypes), no "
+                                    "graph"}},
     }
     # The timed step is 36 launches of one kernel (the fused append + decode), so that is
     # the roofline kernel: its algorithmic bytes per launch over its mean launch time in

@@ -73,9 +73,12 @@ constexpr int kHalfBytes = kPairs * kD * 2;    // one tensor's rows of a warp st
 constexpr int kSlotBytes = 2 * kHalfBytes;     // K rows, then V rows
 constexpr int kStages = 3;                     // ring slots per warp
 constexpr int kStgStride = 80;                 // staging bytes per row (64 used)
-// A warp's region: ring slots | staging lines | barriers, rounded to 128 bytes so that
-// every region (and so every copy destination) stays 16-byte aligned.
-constexpr int kWarpBytes = (kStages * kSlotBytes + 2 * kPairs * kStgStride + 8 * kStages + 127) / 128 * 128;
+// A warp's region: ring slots | staging lines | sequence cursors (16 B per pair slot) |
+// barriers, rounded to 128 bytes so that every region (and so every copy destination)
+// stays 16-byte aligned.
+constexpr int kCursorBytes = 16 * kPairs;
+constexpr int kWarpBytes =
+    (kStages * kSlotBytes + 2 * kPairs * kStgStride + kCursorBytes + 8 * kStages + 127) / 128 * 128;
 constexpr int kSmemBytes = kWarps * kWarpBytes;
 constexpr int kCtasPerSm = 2;
 static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM must fit");
@@ -149,24 +152,40 @@ struct Dest {
   int h;
 };
 
-__device__ __forceinline__ Dest pair_dest(const AppendParams& p, int gp) {
+// The sequence of a pair slot's current token, kept in shared memory across the warp's
+// stages (whose tokens only increase) as {b, cu_lo, cu_hi, sl}: [cu_lo, cu_hi) = the
+// sequence's tokens in the call, sl = its length before the call.  A token outside the
+// range moves the cursor by a binary search over cu_new_tokens; a token inside it needs no
+// global load.  The four lanes of a pair read and write the same entry with the same
+// values; the warp syncs between stages.
+__device__ __forceinline__ Dest pair_dest(const AppendParams& p, int gp, uint32_t cursor) {
   Dest d;
   // t = gp / num_kv_heads by the host's multiplier (gp < 2^31); pos / S and pos % S by
   // the power-of-two page size.
   const int t = static_cast<int>(__umulhi(static_cast<uint32_t>(gp) << 1, p.heads_magic) >> p.heads_shift);
   d.h = gp - t * p.num_kv_heads;
-  int lo = 0, hi = p.batch;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(p.cu_new_tokens + mid) <= t) lo = mid; else hi = mid;
+  uint4 sc = lds_128(cursor);  // x = b, y = cu_lo, z = cu_hi, w = sl
+  if (t < static_cast<int>(sc.y) || t >= static_cast<int>(sc.z)) {
+    int lo = 0, hi = p.batch;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(p.cu_new_tokens + mid) <= t) lo = mid; else hi = mid;
+    }
+    sc = make_uint4(static_cast<uint32_t>(lo), static_cast<uint32_t>(__ldg(p.cu_new_tokens + lo)),
+                    static_cast<uint32_t>(__ldg(p.cu_new_tokens + lo + 1)),
+                    static_cast<uint32_t>(__ldg(p.seq_lens + lo)));
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(cursor), "r"(sc.x), "r"(sc.y), "r"(sc.z),
+                 "r"(sc.w)
+                 : "memory");
   }
-  const int pos = __ldg(p.seq_lens + lo) + (t - __ldg(p.cu_new_tokens + lo));
+  const int b = static_cast<int>(sc.x);
+  const int pos = static_cast<int>(sc.w) + (t - static_cast<int>(sc.y));
   const int lp = pos >= 0 ? pos >> p.page_shift : 0;
   if (pos < 0 || lp >= p.max_pages_per_seq) {
     d.page = -1;
     d.slot = -1;
   } else {
-    d.page = __ldg(p.page_table + static_cast<size_t>(lo) * p.max_pages_per_seq + lp);
+    d.page = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + lp);
     d.slot = pos & (p.page_size - 1);
   }
   return d;
@@ -451,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) append_kernel(AppendPara
   // This warp's ring, staging lines and barriers.
   const uint32_t ring = smem_addr(smem) + w * kWarpBytes;
   const uint32_t stg = ring + kStages * kSlotBytes;
-  const uint32_t bar0 = stg + 2 * kPairs * kStgStride;
+  const uint32_t cursors = stg + 2 * kPairs * kStgStride;
+  const uint32_t bar0 = cursors + kCursorBytes;
   const int l = lane & 1, rho = lane & 7;
   const int pr = lane >> 2;         // pair within the warp stage
   const int kv = (lane >> 1) & 1;   // 0 = K row, 1 = V row
@@ -477,8 +497,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) append_kernel(AppendPara
   }
   __syncwarp();
 
+  const uint32_t cursor = cursors + 16 * pr;  // this lane's pair slot
+  if ((lane & 3) == 0)  // an empty range: the first lookup searches
+    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(cursor), "r"(0u) : "memory");
+  __syncwarp();
   Dest dcur = {-1, -1, 0};
-  if (gw * kPairs + pr < npairs) dcur = pair_dest(p, gw * kPairs + pr);
+  if (gw * kPairs + pr < npairs) dcur = pair_dest(p, gw * kPairs + pr, cursor);
   bool waited = false;
   int s = 0;
   uint32_t phase = 0;
@@ -488,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) append_kernel(AppendPara
     const bool active = gp < npairs;
     // The next warp stage's destination: its page-table load is in flight meanwhile.
     Dest dnext = {-1, -1, 0};
-    if (j + W < nws && gp + W * kPairs < npairs) dnext = pair_dest(p, gp + W * kPairs);
+    if (j + W < nws && gp + W * kPairs < npairs) dnext = pair_dest(p, gp + W * kPairs, cursor);
 
     if (!mbar_wait_bounded(bar0 + 8 * s, phase, kWaitLimitNs)) {
       // A copy did not land in time: flag it, let this warp's other copies finish

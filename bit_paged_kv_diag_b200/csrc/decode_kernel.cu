@@ -1006,45 +1006,56 @@ __device__ __forceinline__ float4 ld_rec4(const float* a) {
 }
 
 // Merge of at most RMAX records (the common case: a unit's CTAs or a CTA's warps): every
-// lane loads the (m, l) pairs and its o' slice of all records at once (the (m, l) loads
-// are broadcasts), so a query costs one round trip and no cross-lane reduction.  Same
-// contract as merge_records below.
+// lane loads the (m, l) pairs and its o' slice of all records for two of the warp's queries
+// at once (the (m, l) loads are broadcasts), so two queries cost one round trip and no
+// cross-lane reduction.  Same contract as merge_records below.
 template <int G, int QSTEP, bool GLOBAL, int RMAX, typename F>
 __device__ __forceinline__ void merge_few(int nrec, F&& rec, int q0, __half* orow, float* crec,
                                           int lane, const DecodeParams& p) {
+  constexpr int NQW = (G + QSTEP - 1) / QSTEP;  // queries this warp handles (at most)
+  constexpr int QB = NQW < 2 ? NQW : 2;          // queries per round trip
 #pragma unroll 1
-  for (int qi = q0; qi < G; qi += QSTEP) {
-    float2 ml[RMAX];
-    float4 v[RMAX];
+  for (int qb = q0; qb < G; qb += QB * QSTEP) {
+    float2 ml[QB][RMAX];
+    float4 v[QB][RMAX];
 #pragma unroll
-    for (int r = 0; r < RMAX; r++) {
-      ml[r] = make_float2(-CUDART_INF_F, 0.0f);
-      v[r] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      if (r < nrec) {
-        const float* rr = rec(r) + qi * kPartStride;
-        ml[r] = ld_rec2<GLOBAL>(rr + kD);
-        v[r] = ld_rec4<GLOBAL>(rr + 4 * lane);
+    for (int i = 0; i < QB; i++) {
+      const int qi = qb + i * QSTEP;
+#pragma unroll
+      for (int r = 0; r < RMAX; r++) {
+        ml[i][r] = make_float2(-CUDART_INF_F, 0.0f);
+        v[i][r] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (r < nrec && qi < G) {
+          const float* rr = rec(r) + qi * kPartStride;
+          ml[i][r] = ld_rec2<GLOBAL>(rr + kD);
+          v[i][r] = ld_rec4<GLOBAL>(rr + 4 * lane);
+        }
       }
     }
-    float M = ml[0].x;
 #pragma unroll
-    for (int r = 1; r < RMAX; r++) M = fmaxf(M, ml[r].x);
-    float o[4] = {0.0f, 0.0f, 0.0f, 0.0f}, l = 0.0f;
+    for (int i = 0; i < QB; i++) {
+      const int qi = qb + i * QSTEP;
+      if (qi >= G) continue;
+      float M = ml[i][0].x;
 #pragma unroll
-    for (int r = 0; r < RMAX; r++) {
-      const float e = (ml[r].x == -CUDART_INF_F) ? 0.0f : ex2_approx(ml[r].x - M);
-      l += e * ml[r].y;
-      o[0] += e * v[r].x;
-      o[1] += e * v[r].y;
-      o[2] += e * v[r].z;
-      o[3] += e * v[r].w;
-    }
-    if (crec) {
-      float* r = crec + qi * kPartStride;
-      *reinterpret_cast<float4*>(r + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-      if (lane == 0) *reinterpret_cast<float2*>(r + kD) = make_float2(M, l);
-    } else {
-      finish_query(o, l, orow + qi * kD, lane, p);
+      for (int r = 1; r < RMAX; r++) M = fmaxf(M, ml[i][r].x);
+      float o[4] = {0.0f, 0.0f, 0.0f, 0.0f}, l = 0.0f;
+#pragma unroll
+      for (int r = 0; r < RMAX; r++) {
+        const float e = (ml[i][r].x == -CUDART_INF_F) ? 0.0f : ex2_approx(ml[i][r].x - M);
+        l += e * ml[i][r].y;
+        o[0] += e * v[i][r].x;
+        o[1] += e * v[i][r].y;
+        o[2] += e * v[i][r].z;
+        o[3] += e * v[i][r].w;
+      }
+      if (crec) {
+        float* r = crec + qi * kPartStride;
+        *reinterpret_cast<float4*>(r + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+        if (lane == 0) *reinterpret_cast<float2*>(r + kD) = make_float2(M, l);
+      } else {
+        finish_query(o, l, orow + qi * kD, lane, p);
+      }
     }
   }
 }
