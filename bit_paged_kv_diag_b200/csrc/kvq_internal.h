@@ -106,6 +106,8 @@ struct PrefillParams {
 // error).
 int launch_append(const AppendParams& p, int block, int num_sms, cudaStream_t stream);
 int launch_prefill(const PrefillParams& p, int total_q, cudaStream_t stream);
+// Chunked prefill on the 5th-generation tensor cores (INT4 cache).
+int launch_prefill_tc(const PrefillParams& p, int total_q, cudaStream_t stream);
 
 struct DecodeLaunch {
   int grid;          // CTAs (a multiple of the SM count)
