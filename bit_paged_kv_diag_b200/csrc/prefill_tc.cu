@@ -8,16 +8,18 @@
 // is rotated back).  A chunk of C prompt tokens of a sequence, already appended, attends the
 // cache causally: query i of the chunk (position L - C + i) sees positions 0..L - C + i.
 //
-// Work decomposition.  A CTA (8 warps, two threads per query row) takes 128 query rows of one
-// (sequence, KV head): 128 / G consecutive chunk tokens times the G query heads of the KV
-// head.  Row r is lane r of tensor memory; warps w and w + 4 both read the lanes of rows
-// 32(w % 4).., warp w the first half of each tile's columns and of O, warp w + 4 the second.
-// The tile loop is software-pipelined with one CTA barrier per tile: step t runs the softmax of
-// tile t (its QK^T was issued two steps before), then in one phase writes P' of t, expands V of
-// t and the K codes of t + 2, and issues PV of t and QK^T of t + 2 (S is double-buffered in
-// tensor memory, K in shared memory); the tensor cores work on them during step t + 1.  The causal KV range streams in tiles of 64
-// tokens: the tile's pages are bulk-copied (cp.async.bulk, 1-D, no multicast) into one of three
-// raw slots, then the threads expand the token rows into the MMA operand tiles.
+// Work decomposition.  A CTA takes 128 query rows of one (sequence, KV head): 128 / G
+// consecutive chunk tokens times the G query heads of the KV head.  Row r is lane r of tensor
+// memory.  The CTA's 16 warps specialise and hand work to one another through mbarriers, so
+// the softmax, the code expansion and the tensor cores overlap instead of taking turns:
+//   warps 0-7    softmax: warps w and w + 4 both read the lanes of rows 32(w % 4).., warp w
+//                the first half of each tile's columns and of O, warp w + 4 the second;
+//   warps 8-11   expansion: the K and V codes of a tile into the MMA operand tiles, plus
+//                their scales; warp 8 also issues the bulk copies of the raw page data;
+//   warp 12      one lane issues the MMAs: QK^T of tile t, then PV of tile t - 1.
+// S (tensor memory), the K and V operand tiles and the scales are double-buffered by tile
+// parity; the raw page data streams through four slots.  The causal KV range is cut into
+// tiles of 64 tokens, whose pages are bulk-copied (cp.async.bulk, 1-D, no multicast).
 //   QK^T  tcgen05.mma kind::f16, M = 128 rows, N = 64 tokens, K = 128 channels: A = q' cut
 //         into fp16 hi + lo parts (q' * 2^14 / M_r, M_r the power of two >= max |q'_r|), B =
 //         the K codes as exact fp16 integers; both parts accumulate into one fp32 tile S in
@@ -55,7 +57,14 @@ namespace {
 constexpr int kD = 128;
 constexpr int kRowsT = 128;     // query rows per CTA (tensor-memory lanes)
 constexpr int kTokT = 64;       // KV tokens per tile
-constexpr int kThreadsT = 256;  // 8 warps: warps w and w + 4 share the rows of TMEM lanes 32(w % 4)..
+constexpr int kSoftWarps = 8;   // warps w and w + 4 share the rows of TMEM lanes 32(w % 4)..
+constexpr int kSoftThreads = 32 * kSoftWarps;
+constexpr int kExpWarp0 = 8;    // warps 8-11 expand K and V codes; warp 8 also issues copies
+constexpr int kExpWarps = 4;
+constexpr int kExpThreads = 32 * kExpWarps;
+constexpr int kMmaWarp = 12;    // issues the tcgen05 MMAs; warps 13-15 only pad the warpgroup
+constexpr int kThreadsT = 512;
+constexpr int kBarIdExp = 5;    // named barrier of the expansion warps (1-4: softmax row pairs)
 constexpr int kStagesT = 4;     // raw page-data slots
 constexpr uint64_t kWaitT = 2000000000ull;
 constexpr float kLazyT = 8.0f;  // frame slack in log2 units: p <= 2^8 between rescales
@@ -68,15 +77,19 @@ constexpr int kQh = 0;                          // [2 kb][128 rows][128 B] fp16 
 constexpr int kQl = kQh + 2 * kRowsT * 128;     // same, lo
 constexpr int kKs = kQl + 2 * kRowsT * 128;     // [2 buffers][2 kb][64 tokens][128 B] fp16 K codes
 constexpr int kKsBuf = 2 * kTokT * 128;
-constexpr int kVs = kKs + 2 * kKsBuf;           // [2 nb][64 tokens][128 B] bf16 V codes
-constexpr int kPh = kVs + 2 * kTokT * 128;      // [128 rows][128 B] bf16 P' hi
+constexpr int kVs = kKs + 2 * kKsBuf;           // [2 buffers][2 nb][64 tokens][128 B] bf16 V codes
+constexpr int kVsBuf = 2 * kTokT * 128;
+constexpr int kPh = kVs + 2 * kVsBuf;           // [128 rows][128 B] bf16 P' hi
 constexpr int kPl = kPh + kRowsT * 128;         // same, lo
 constexpr int kRing = kPl + kRowsT * 128;       // [4][64 token rows of 132 B]
 constexpr int kSlotT = kTokT * 132;
-constexpr int kSfr = kRing + kStagesT * kSlotT; // row scales [128] fp32
-constexpr int kRed = kSfr + kRowsT * 4;         // row maxima / sums of the two halves [2][128]
-constexpr int kBar = kRed + 2 * kRowsT * 4;     // full[4], qk done[2], pv done
-constexpr int kTmemSlot = kBar + 7 * 8;         // tensor-memory base address
+constexpr int kScl = kRing + kStagesT * kSlotT; // K scales [2][64], V scales [2][64] fp32
+constexpr int kSfr = kScl + 4 * kTokT * 4;      // row scales [128] fp32
+constexpr int kRed = kSfr + kRowsT * 4;         // maxima [2][2][128], sums [2][128] fp32
+constexpr int kBar = kRed + 6 * kRowsT * 4;     // mbarriers, see kBar* below
+constexpr int kBarFull = 0, kBarKReady = 4, kBarVReady = 6, kBarSFull = 8, kBarSFree = 10,
+              kBarPReady = 12, kBarPVDone = 13, kNumBars = 15;
+constexpr int kTmemSlot = kBar + kNumBars * 8;  // tensor-memory base address
 constexpr int kPreq = kTmemSlot + 16;           // query-block prefix [batch + 1]
 
 // Instruction descriptors (kind::f16): fp32 accumulator, M = 128.
@@ -170,11 +183,18 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
+  float* s_kb = reinterpret_cast<float*>(smem + kScl);  // [2][64] K scales of tiles t even / odd
+  float* s_vb = s_kb + 2 * kTokT;                       // [2][64] V scales
   float* sfr = reinterpret_cast<float*>(smem + kSfr);
-  float* red = reinterpret_cast<float*>(smem + kRed);  // [half][row]
+  float* red = reinterpret_cast<float*>(smem + kRed);  // [tile parity][half][row] maxima
+  float* lsum = red + 4 * kRowsT;                      // [half][row] final sums
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlot);
   int32_t* preq = reinterpret_cast<int32_t*>(smem + kPreq);
-  const uint32_t full_s = sbase + kBar, bar_qk = full_s + 8 * kStagesT, bar_pv = bar_qk + 16;
+  const uint32_t bar0 = sbase + kBar;
+  const uint32_t full_s = bar0 + 8 * kBarFull, kready = bar0 + 8 * kBarKReady,
+                 vready = bar0 + 8 * kBarVReady, sfull = bar0 + 8 * kBarSFull,
+                 sfree = bar0 + 8 * kBarSFree, pready = bar0 + 8 * kBarPReady,
+                 pvdone = bar0 + 8 * kBarPVDone;
   __shared__ int warp_sum[kThreadsT / 32];
   __shared__ int running;
 
@@ -183,7 +203,15 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   // call); q, the pool and out are touched after it.
   griddep_launch_dependents();
   if (tid == 0) {
-    for (int k = 0; k < kStagesT + 3; k++) mbar_init(full_s + 8 * k, 1);  // full[4], qk[2], pv
+    for (int k = 0; k < kStagesT; k++) mbar_init(full_s + 8 * k, 1);
+    for (int k = 0; k < 2; k++) {
+      mbar_init(kready + 8 * k, kExpThreads);
+      mbar_init(vready + 8 * k, kExpThreads);
+      mbar_init(sfull + 8 * k, 1);
+      mbar_init(sfree + 8 * k, kSoftThreads);
+      mbar_init(pvdone + 8 * k, 1);
+    }
+    mbar_init(pready, kSoftThreads);
     fence_mbar_init();
     running = 0;
   }
@@ -234,7 +262,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   }
   const int tok_first = qb * QB;                      // first chunk token of the CTA
   const int tok_last = min(C, tok_first + QB) - 1;    // last valid one
-  const int ntile = (L - C + tok_last) / kTokT + 1;
+  const int ntile = (L - C + tok_last) / kTokT + 1;   // >= 1
   const uint64_t pol = l2_policy_evict_first();
 
   // Tensor memory for S and O (one warp allocates; the address goes through shared memory).
@@ -243,360 +271,380 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
     tmem_relinquish();
   }
   griddep_wait();
-  if (w == 0) {
+  if (w == kExpWarp0) {
     for (int t = 0; t < kStagesT && t < ntile; t++)
-      issue_tile_tc<SEFF>(t, b, h, L, sbase + kRing + t * kSlotT, full_s + 8 * t, lane, pol, p);  // slot t
+      issue_tile_tc<SEFF>(t, b, h, L, sbase + kRing + t * kSlotT, full_s + 8 * t, lane, pol, p);
   }
 
-  // q rows: warp w rotates and scales rows 16w..16w+15 (lane: channels 4 lane..4 lane + 3)
-  // and stores q~ = q' * 2^14 / M as fp16 hi + lo parts into the K-major operands.
-  for (int rr = 0; rr < 16; rr++) {
-    const int row = 16 * w + rr;
-    const int ti = tok_first + row / G, gq = row % G;
-    float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (ti < C) {
-      const __half* qrow = p.q + ((static_cast<size_t>(cq0) + ti) * p.num_kv_heads * G + h * G + gq) * kD;
-      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qrow) + lane);
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-      const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      x[0] = a.x; x[1] = a.y; x[2] = c.x; x[3] = c.y;
-    }
-    if (p.hadamard_block > 1) {
-      const float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
-      x[0] = a0 + a2; x[2] = a0 - a2; x[1] = a1 + a3; x[3] = a1 - a3;
+  // q rows: softmax warp w rotates and scales rows 16w..16w+15 (lane: channels 4 lane..
+  // 4 lane + 3) and stores q~ = q' * 2^14 / M as fp16 hi + lo parts into the K-major operands.
+  if (w < kSoftWarps) {
+    for (int rr = 0; rr < 16; rr++) {
+      const int row = 16 * w + rr;
+      const int ti = tok_first + row / G, gq = row % G;
+      float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (ti < C) {
+        const __half* qrow = p.q + ((static_cast<size_t>(cq0) + ti) * p.num_kv_heads * G + h * G + gq) * kD;
+        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qrow) + lane);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+        const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+        x[0] = a.x; x[1] = a.y; x[2] = c.x; x[3] = c.y;
+      }
+      if (p.hadamard_block > 1) {
+        const float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
+        x[0] = a0 + a2; x[2] = a0 - a2; x[1] = a1 + a3; x[3] = a1 - a3;
 #pragma unroll
-      for (int st = 0; st < 5; st++) {
-        if ((4 << st) < p.hadamard_block) {
-          const float sgn = ((lane >> st) & 1) ? -1.0f : 1.0f;
+        for (int st = 0; st < 5; st++) {
+          if ((4 << st) < p.hadamard_block) {
+            const float sgn = ((lane >> st) & 1) ? -1.0f : 1.0f;
 #pragma unroll
-          for (int e = 0; e < 4; e++) x[e] = __fmaf_rn(x[e], sgn, __shfl_xor_sync(kFullT, x[e], 1 << st));
+            for (int e = 0; e < 4; e++) x[e] = __fmaf_rn(x[e], sgn, __shfl_xor_sync(kFullT, x[e], 1 << st));
+          }
         }
       }
-    }
-    float amax = 0.0f;
+      float amax = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 4; e++) {
-      x[e] = x[e] * p.cb * p.q_scale;
-      amax = fmaxf(amax, fabsf(x[e]));
-    }
+      for (int e = 0; e < 4; e++) {
+        x[e] = x[e] * p.cb * p.q_scale;
+        amax = fmaxf(amax, fabsf(x[e]));
+      }
 #pragma unroll
-    for (int d = 1; d < 32; d *= 2) amax = fmaxf(amax, __shfl_xor_sync(kFullT, amax, d));
-    float M = 1.0f;
-    if (amax > 1e-30f) {
-      const uint32_t bits = __float_as_uint(amax);
-      M = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax;
-    }
-    const float inv = __fdiv_rn(16384.0f, M);  // exact: powers of two
-    __half hv[4], lv[4];
+      for (int d = 1; d < 32; d *= 2) amax = fmaxf(amax, __shfl_xor_sync(kFullT, amax, d));
+      float M = 1.0f;
+      if (amax > 1e-30f) {
+        const uint32_t bits = __float_as_uint(amax);
+        M = (bits & 0x7FFFFFu) ? __uint_as_float((bits & 0x7F800000u) + 0x00800000u) : amax;
+      }
+      const float inv = __fdiv_rn(16384.0f, M);  // exact: powers of two
+      __half hv[4], lv[4];
 #pragma unroll
-    for (int e = 0; e < 4; e++) {
-      const float t = x[e] * inv;
-      hv[e] = __float2half_rn(t);
-      lv[e] = __float2half_rn(t - __half2float(hv[e]));
+      for (int e = 0; e < 4; e++) {
+        const float t = x[e] * inv;
+        hv[e] = __float2half_rn(t);
+        lv[e] = __float2half_rn(t - __half2float(hv[e]));
+      }
+      // Channels 4 lane..: K-block lane / 16, chunk (lane % 16) / 2, bytes 8 (lane % 2).
+      const uint32_t off = (lane >> 4) * (kRowsT * 128) + sw_off(row, (lane & 15) >> 1) + 8 * (lane & 1);
+      *reinterpret_cast<uint2*>(smem + kQh + off) = make_uint2(pack_half2(hv[0], hv[1]), pack_half2(hv[2], hv[3]));
+      *reinterpret_cast<uint2*>(smem + kQl + off) = make_uint2(pack_half2(lv[0], lv[1]), pack_half2(lv[2], lv[3]));
+      if (lane == 0) sfr[row] = M * (1.0f / 16384.0f);
     }
-    // Channels 4 lane..: K-block lane / 16, chunk (lane % 16) / 2, bytes 8 (lane % 2).
-    const uint32_t off = (lane >> 4) * (kRowsT * 128) + sw_off(row, (lane & 15) >> 1) + 8 * (lane & 1);
-    *reinterpret_cast<uint2*>(smem + kQh + off) = make_uint2(pack_half2(hv[0], hv[1]), pack_half2(hv[2], hv[3]));
-    *reinterpret_cast<uint2*>(smem + kQl + off) = make_uint2(pack_half2(lv[0], lv[1]), pack_half2(lv[2], lv[3]));
-    if (lane == 0) sfr[row] = M * (1.0f / 16384.0f);
+    fence_proxy_async_smem();  // q~ is read by the tensor cores
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int quarter = w & 3, half = w >> 2;
-  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * quarter) << 16);  // this warp's lanes
-
-  // This thread's row and half: tokens 32 half..32 half + 31 of every tile, channels
-  // 64 half..64 half + 63 of O.
-  const int row = 32 * quarter + lane;
-  const int ti_row = tok_first + row / G;
-  const bool row_valid = ti_row < C;
-  // The row's position: it sees tokens 0..rpos.  Padding rows past the chunk take the last
-  // token's, so that every tile token at or beyond L is masked for them too.
-  const int rpos = min(L - C + ti_row, L - 1);
-  const float sf = sfr[row];
-  float m = -CUDART_INF_F, l = 0.0f;
   bool dead = false;
-  int issued = min(kStagesT, ntile), landed = 0, commits = 0;
-  // Expansion items: warps 0-3 take K (token ej, half ehf), warps 4-7 V, so no warp diverges.
-  const int eid = tid & 127, ej = eid >> 1, ehf = eid & 1;
-  const bool k_role = tid < 128;
 
-  // Expand the K codes (fp16) of tile tt into K buffer tt & 1 (every thread waits for the
-  // tile's raw slot; warps 0-3 expand).
-  auto expand_k = [&](int tt) {
-    const int slot = tt % kStagesT;
-    if (!mbar_wait_bounded(full_s + 8 * slot, static_cast<uint32_t>((tt / kStagesT) & 1), kWaitT)) {
-      dead = true;
-      return;
-    }
-    landed++;
-    if (!k_role) return;
-    const int hf = ehf;
-    const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
-    const int jr = ej % SEFF;
-    const uint4* src = reinterpret_cast<const uint4*>(pg + jr * 64 + 32 * hf);
-    const uint4 c0 = src[0], c1 = src[1];
-    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    uint8_t* kb = smem + kKs + (tt & 1) * kKsBuf + hf * (kTokT * 128);
+  if (w < kSoftWarps) {
+    // ---------------------------------------------------------------- softmax warps --
+    // This thread's row and half: tokens 32 half..32 half + 31 of every tile, channels
+    // 64 half..64 half + 63 of O.
+    const int quarter = w & 3, half = w >> 2;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
+    const int row = 32 * quarter + lane;
+    const int ti_row = tok_first + row / G;
+    const bool row_valid = ti_row < C;
+    // The row's position: it sees tokens 0..rpos.  Padding rows past the chunk take the last
+    // token's, so that every tile token at or beyond L is masked for them too.
+    const int rpos = min(L - C + ti_row, L - 1);
+    const float sf = sfr[row];
+    float m = -CUDART_INF_F, l = 0.0f;
+    for (int t = 0; t < ntile; t++) {
+      const uint32_t par = static_cast<uint32_t>((t >> 1) & 1);
+      if (!dead && !mbar_wait_bounded(sfull + 8 * (t & 1), par, kWaitT)) dead = true;
+      if (!dead && !mbar_wait_bounded(kready + 8 * (t & 1), par, kWaitT)) dead = true;
+      tc_fence_after();
+      uint32_t sraw[32];
+      tmem_ld32(lane_addr + 64 * (t & 1) + 32 * half, sraw);
+      tmem_wait_ld();
+      float kk[32];
+      const float4* s_k4 = reinterpret_cast<const float4*>(s_kb + (t & 1) * kTokT + 32 * half);
 #pragma unroll
-    for (int ch = 0; ch < 8; ch++)  // 16-byte chunk ch = channels 64hf + 8ch .. + 7
-      *reinterpret_cast<uint4*>(kb + sw_off(ej, ch)) =
-          make_uint4(codes_f16x2(cw[ch], 0), codes_f16x2(cw[ch], 1), codes_f16x2(cw[ch], 2),
-                     codes_f16x2(cw[ch], 3));
-  };
-  // Expand tile tt's V codes (bf16) into the V buffer (warps 4-7; the raw slot has landed:
-  // expand_k waited for it).
-  auto expand_v = [&](int tt) {
-    if (k_role) return;
-    const int hf = ehf;
-    const uint8_t* pg = smem + kRing + (tt % kStagesT) * kSlotT + (ej / SEFF) * (SEFF * 132);
-    const int jr = ej % SEFF;
-    const uint4* src = reinterpret_cast<const uint4*>(pg + SEFF * 64 + jr * 64 + 32 * hf);
-    const uint4 c0 = src[0], c1 = src[1];
-    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      for (int e4 = 0; e4 < 8; e4++) {
+        const float4 k4 = s_k4[e4];
+        kk[4 * e4] = k4.x; kk[4 * e4 + 1] = k4.y; kk[4 * e4 + 2] = k4.z; kk[4 * e4 + 3] = k4.w;
+      }
+      // S buffer t & 1 and the K scales of tile t are free for tile t + 2.
+      tc_fence_before();
+      if (!dead) mbar_arrive(sfree + 8 * (t & 1));
+      // Tiles wholly before the CTA's first row need no causal mask (they hold no token at or
+      // beyond L either).
+      const bool masked = t * kTokT + kTokT - 1 > L - C + tok_first;
+      float mx = -CUDART_INF_F;
 #pragma unroll
-    for (int ch = 0; ch < 8; ch++) {
-      const uint32_t wv = cw[ch], wvh = wv >> 4;
-      *reinterpret_cast<uint4*>(smem + kVs + hf * (kTokT * 128) + sw_off(ej, ch)) =
-          make_uint4(codes_bf16x2(wv, wvh, 0), codes_bf16x2(wv, wvh, 1), codes_bf16x2(wv, wvh, 2),
-                     codes_bf16x2(wv, wvh, 3));
-    }
-  };
-  // Eight consecutive K (kind 0) or V (kind 1) scales of tile tt from its raw slot, tokens
-  // j0..j0 + 7 of the tile (j0 a multiple of 8: a group never straddles a page).
-  auto raw_scales8 = [&](int tt, int j0, int kind, float* out8) {
-    const uint8_t* pg = smem + kRing + (tt % kStagesT) * kSlotT + (j0 / SEFF) * (SEFF * 132);
-    const uint4 r = *reinterpret_cast<const uint4*>(pg + SEFF * (128 + 2 * kind) + 2 * (j0 % SEFF));
-    const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&rw[i]));
-      out8[2 * i] = f.x;
-      out8[2 * i + 1] = f.y;
-    }
-  };
-  // Operand descriptors: one base per operand; a k-step adds its byte offset / 16 to the
-  // start-address field (every operand lies in the first 256 KB, so the field never carries).
-  const uint64_t dq_h = smem_desc_sw128(sbase + kQh, 16, 1024), dq_l = smem_desc_sw128(sbase + kQl, 16, 1024);
-  const uint64_t dk0 = smem_desc_sw128(sbase + kKs, 16, 1024);
-  const uint64_t dp_h = smem_desc_sw128(sbase + kPh, 16, 1024), dp_l = smem_desc_sw128(sbase + kPl, 16, 1024);
-  const uint64_t dv0 = smem_desc_sw128(sbase + kVs, kTokT * 128, 1024);
-  // S[tt & 1] = q~hi . K + q~lo . K over 8 k-steps of 16 channels (one thread issues).
-  auto issue_qk = [&](int tt) {
-    const uint64_t dk = dk0 + static_cast<uint64_t>(((tt & 1) * kKsBuf) >> 4);
-#pragma unroll
-    for (int s = 0; s < 8; s++) {
-      const uint64_t qo = static_cast<uint64_t>(((s >> 2) * 16384u + (s & 3) * 32u) >> 4);
-      const uint64_t ko = static_cast<uint64_t>(((s >> 2) * (kTokT * 128u) + (s & 3) * 32u) >> 4);
-      tc_mma_f16_ss(tmem + 64 * (tt & 1), dq_h + qo, dk + ko, kIdescQK, s > 0);
-      tc_mma_f16_ss(tmem + 64 * (tt & 1), dq_l + qo, dk + ko, kIdescQK, 1u);
-    }
-    tc_commit(bar_qk + 8 * (tt & 1));
-  };
-
-  // Prologue: K of tiles 0 and 1 and their QK^T.
-  for (int tt = 0; tt < 2 && tt < ntile; tt++)
-    if (!dead) expand_k(tt);
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const int qk_pro = dead ? 0 : min(2, ntile);  // QK^T launches of the prologue (thread 0)
-  if (tid == 0)
-    for (int tt = 0; tt < qk_pro; tt++) issue_qk(tt);
-
-  for (int t = 0; t < ntile; t++) {
-    // Softmax of tile t.
-    if (!dead && !mbar_wait_bounded(bar_qk + 8 * (t & 1), static_cast<uint32_t>((t >> 1) & 1), kWaitT))
-      dead = true;
-    tc_fence_after();
-    uint32_t sraw[32];
-    tmem_ld32(lane_addr + 64 * (t & 1) + 32 * half, sraw);
-    tmem_wait_ld();
-    // Tiles wholly before the CTA's first row need no causal mask (they hold no token at or
-    // beyond L either; in a masked tile the mask also covers those, whatever their scales).
-    const bool masked = t * kTokT + kTokT - 1 > L - C + tok_first;
-    float mx = -CUDART_INF_F;
-#pragma unroll
-    for (int e8 = 0; e8 < 4; e8++) {
-      float kk[8];
-      raw_scales8(t, 32 * half + 8 * e8, 0, kk);
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const int e = 8 * e8 + i;
-        float v = __uint_as_float(sraw[e]) * (sf * kk[i]);
+      for (int e = 0; e < 32; e++) {
+        float v = __uint_as_float(sraw[e]) * (sf * kk[e]);
         if (masked && t * kTokT + 32 * half + e > rpos) v = -CUDART_INF_F;
         sraw[e] = __float_as_uint(v);
         mx = fmaxf(mx, v);
       }
-    }
-    // The row's maximum over both halves (warps w and w + 4 meet at a 64-thread barrier).
-    red[half * kRowsT + row] = mx;
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
-    mx = fmaxf(mx, red[(half ^ 1) * kRowsT + row]);
-    // Lazy frame: move m only when a score exceeds it by more than kLazyT.
-    float alpha = 1.0f;
-    const bool move = mx > m + kLazyT;
-    if (move) {
-      alpha = m == -CUDART_INF_F ? 0.0f : ex2_approx(m - mx);
-      l *= alpha;
-      m = mx;
-    }
-    float pr[32];
-    float ps = 0.0f;
+      // The row's maximum over both halves (warps w and w + 4 meet at a 64-thread barrier;
+      // the exchange slots alternate with the tile's parity).
+      red[((t & 1) * 2 + half) * kRowsT + row] = mx;
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+      mx = fmaxf(mx, red[((t & 1) * 2 + (half ^ 1)) * kRowsT + row]);
+      // Lazy frame: move m only when a score exceeds it by more than kLazyT.
+      float alpha = 1.0f;
+      const bool move = mx > m + kLazyT;
+      if (move) {
+        alpha = m == -CUDART_INF_F ? 0.0f : ex2_approx(m - mx);
+        l *= alpha;
+        m = mx;
+      }
+      float ps = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 32; e++) {  // ex2(-inf) = +0: masked scores need no test
-      pr[e] = ex2_approx(__uint_as_float(sraw[e]) - m);
-      ps += pr[e];
+      for (int e = 0; e < 32; e++) {  // ex2(-inf) = +0: masked scores need no test
+        const float pe = ex2_approx(__uint_as_float(sraw[e]) - m);
+        sraw[e] = __float_as_uint(pe);
+        ps += pe;
+      }
+      l += ps;
+      // PV of tile t - 1 reads P' and accumulates O: wait for it before touching either.
+      if (t > 0 && !dead &&
+          !mbar_wait_bounded(pvdone + 8 * ((t - 1) & 1), static_cast<uint32_t>(((t - 1) >> 1) & 1), kWaitT))
+        dead = true;
+      tc_fence_after();
+      // Rescale this thread's half of O when a row of the warp moved after its first tile.
+      if (__any_sync(kFullT, move && alpha != 0.0f) && t > 0) {
+#pragma unroll 1
+        for (int q2 = 0; q2 < 2; q2++) {
+          uint32_t o[32];
+          const uint32_t col = kColO + 64 * half + 32 * q2;
+          tmem_ld32(lane_addr + col, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e++) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(lane_addr + col, o);
+        }
+        tmem_wait_st();
+      }
+      // P' = p * s_v as bf16 hi + lo into the K-major A operand (V scales of tile t: vready).
+      if (!dead && !mbar_wait_bounded(vready + 8 * (t & 1), par, kWaitT)) dead = true;
+      const float4* s_v4 = reinterpret_cast<const float4*>(s_vb + (t & 1) * kTokT + 32 * half);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; c4++) {
+        uint32_t ph[4], pl[4];
+        const float4 va = s_v4[2 * c4], vb = s_v4[2 * c4 + 1];
+        const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+        for (int e2 = 0; e2 < 4; e2++) {
+          const int e = 8 * c4 + 2 * e2;
+          const float x0 = __uint_as_float(sraw[e]) * vv[2 * e2];
+          const float x1 = __uint_as_float(sraw[e + 1]) * vv[2 * e2 + 1];
+          ph[e2] = pack_bf16x2(x0, x1);
+          pl[e2] = pack_bf16x2(x0 - bf16_lo(ph[e2]), x1 - bf16_hi(ph[e2]));
+        }
+        const int c8 = 4 * half + c4;
+        *reinterpret_cast<uint4*>(smem + kPh + sw_off(row, c8)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(smem + kPl + sw_off(row, c8)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      if (!dead) mbar_arrive(pready);
     }
-    l += ps;
-    // PV of tile t - 1 reads P' and V and accumulates O: wait for it before touching them.
-    if (!dead && t > 0 && !mbar_wait_bounded(bar_pv, static_cast<uint32_t>((t - 1) & 1), kWaitT))
+    if (!dead && !mbar_wait_bounded(pvdone + 8 * ((ntile - 1) & 1), static_cast<uint32_t>(((ntile - 1) >> 1) & 1),
+                                    kWaitT))
       dead = true;
     tc_fence_after();
-    // Rescale this thread's half of O when a row of the warp moved after its first tile.
-    if (__any_sync(kFullT, move && alpha != 0.0f) && t > 0) {
-#pragma unroll 1
-      for (int q2 = 0; q2 < 2; q2++) {
-        uint32_t o[32];
-        const uint32_t col = kColO + 64 * half + 32 * q2;
-        tmem_ld32(lane_addr + col, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e++) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-        tmem_st32(lane_addr + col, o);
-      }
-      tmem_wait_st();
-    }
-    // V of tile t (the V buffer's last reader, PV of t - 1, has finished) and K of tile
-    // t + 2 (K buffer t & 1 was last read by QK^T of t, which has finished).
-    if (!dead) expand_v(t);
-    if (!dead && t + 2 < ntile) expand_k(t + 2);
-    // P' = p * s_v as bf16 hi + lo into the K-major A operand (P' and PV of t - 1 are done).
-    // The V scales come from the raw slot; in the last tile those at or beyond L are not
-    // data and count as zero (their p is zero as well).
-    const bool tail = (t + 1) * kTokT > L;
-#pragma unroll
-    for (int c4 = 0; c4 < 4; c4++) {
-      uint32_t ph[4], pl[4];
-      float vv[8];
-      raw_scales8(t, 32 * half + 8 * c4, 1, vv);
-      if (tail) {
-#pragma unroll
-        for (int i = 0; i < 8; i++)
-          if (t * kTokT + 32 * half + 8 * c4 + i >= L) vv[i] = 0.0f;
-      }
-#pragma unroll
-      for (int e2 = 0; e2 < 4; e2++) {
-        const int e = 8 * c4 + 2 * e2;
-        const float x0 = pr[e] * vv[2 * e2], x1 = pr[e + 1] * vv[2 * e2 + 1];
-        ph[e2] = pack_bf16x2(x0, x1);
-        pl[e2] = pack_bf16x2(x0 - bf16_lo(ph[e2]), x1 - bf16_hi(ph[e2]));
-      }
-      const int c8 = 4 * half + c4;
-      *reinterpret_cast<uint4*>(smem + kPh + sw_off(row, c8)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-      *reinterpret_cast<uint4*>(smem + kPl + sw_off(row, c8)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (w == 0 && !dead) {
-      // Tile t's raw slot is fully read: refill it with tile t + kStagesT.
-      if (t + kStagesT < ntile) {
-        issue_tile_tc<SEFF>(t + kStagesT, b, h, L, sbase + kRing + (t % kStagesT) * kSlotT,
-                            full_s + 8 * (t % kStagesT), lane, pol, p);
-        issued++;
-      }
-      if (lane == 0) {
-        // QK^T of tile t + 2 goes first, so the commit of PV also covers it.
-        if (t + 2 < ntile) issue_qk(t + 2);
-        // O (+)= P'hi . V + P'lo . V over 4 k-steps of 16 tokens.
-#pragma unroll
-        for (int s = 0; s < 4; s++) {
-          const uint64_t vd = dv0 + static_cast<uint64_t>((2048u * s) >> 4);
-          const uint64_t po = static_cast<uint64_t>((32u * s) >> 4);
-          tc_mma_f16_ss(tmem + kColO, dp_h + po, vd, kIdescPV, (t > 0 || s > 0) ? 1u : 0u);
-          tc_mma_f16_ss(tmem + kColO, dp_l + po, vd, kIdescPV, 1u);
-        }
-        tc_commit(bar_pv);
-      }
-      __syncwarp();
-      commits++;
-    }
-  }
-  if (!dead && ntile > 0 && !mbar_wait_bounded(bar_pv, static_cast<uint32_t>((ntile - 1) & 1), kWaitT))
-    dead = true;
-  tc_fence_after();
-  if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
+    if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
 
-  // o'/l of this half row (the row sum meets the other half's in shared memory).
-  red[half * kRowsT + row] = l;
-  float o[64];
+    // o'/l of this half row (the row sum meets the other half's in shared memory).
+    lsum[half * kRowsT + row] = l;
+    float o[64];
 #pragma unroll
-  for (int q2 = 0; q2 < 2; q2++) {
-    uint32_t r[32];
-    tmem_ld32(lane_addr + kColO + 64 * half + 32 * q2, r);
-    tmem_wait_ld();
+    for (int q2 = 0; q2 < 2; q2++) {
+      uint32_t r[32];
+      tmem_ld32(lane_addr + kColO + 64 * half + 32 * q2, r);
+      tmem_wait_ld();
 #pragma unroll
-    for (int e = 0; e < 32; e++) o[32 * q2 + e] = __uint_as_float(r[e]);
-  }
-  __syncthreads();
-  const float lt = l + red[(half ^ 1) * kRowsT + row];
-  const float il = lt > 0.0f ? __frcp_rn(lt) : 0.0f;
+      for (int e = 0; e < 32; e++) o[32 * q2 + e] = __uint_as_float(r[e]);
+    }
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+    const float lt = l + lsum[(half ^ 1) * kRowsT + row];
+    const float il = lt > 0.0f ? __frcp_rn(lt) : 0.0f;
 #pragma unroll
-  for (int e = 0; e < 64; e++) o[e] *= il;
-  // Inverse block Hadamard: stages h = 1..32 inside the half, h = 64 across the halves
-  // (through the free q operand area, channel-major so a warp's accesses are contiguous).
-  const int block = p.hadamard_block;
+    for (int e = 0; e < 64; e++) o[e] *= il;
+    // Inverse block Hadamard: stages h = 1..32 inside the half, h = 64 across the halves
+    // (through the q operand area, free once the last QK^T has completed; channel-major so a
+    // warp's accesses are contiguous).
+    const int block = p.hadamard_block;
 #pragma unroll
-  for (int hh = 1; hh < 64; hh *= 2) {
-    if (hh < block) {
+    for (int hh = 1; hh < 64; hh *= 2) {
+      if (hh < block) {
 #pragma unroll
-      for (int i = 0; i < 64; i++)
-        if (!(i & hh)) {
-          const float a = o[i], d = o[i + hh];
-          o[i] = a + d;
-          o[i + hh] = a - d;
+        for (int i = 0; i < 64; i++)
+          if (!(i & hh)) {
+            const float a = o[i], d = o[i + hh];
+            o[i] = a + d;
+            o[i + hh] = a - d;
+          }
+      }
+    }
+    if (block == 128) {
+      float* xch = reinterpret_cast<float*>(smem + kQh);  // [half][64 channels][128 rows]
+#pragma unroll
+      for (int e = 0; e < 64; e++) xch[(half * 64 + e) * kRowsT + row] = o[e];
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+#pragma unroll
+      for (int e = 0; e < 64; e++) {
+        const float other = xch[((half ^ 1) * 64 + e) * kRowsT + row];
+        o[e] = half ? other - o[e] : o[e] + other;
+      }
+    }
+    if (row_valid && !dead) {
+      __half* orow = p.out + ((static_cast<size_t>(cq0) + ti_row) * p.num_kv_heads * G + h * G + row % G) * kD +
+                     64 * half;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; c8++) {
+        const float* v = o + 8 * c8;
+        *reinterpret_cast<uint4*>(orow + 8 * c8) = make_uint4(
+            pack_half2(__float2half_rn(v[0] * p.cb), __float2half_rn(v[1] * p.cb)),
+            pack_half2(__float2half_rn(v[2] * p.cb), __float2half_rn(v[3] * p.cb)),
+            pack_half2(__float2half_rn(v[4] * p.cb), __float2half_rn(v[5] * p.cb)),
+            pack_half2(__float2half_rn(v[6] * p.cb), __float2half_rn(v[7] * p.cb)));
+      }
+    }
+  } else if (w < kExpWarp0 + kExpWarps) {
+    // -------------------------------------------------------------- expansion warps --
+    // Item: token ej of the tile, channels 64 ehf..64 ehf + 63, for K and for V.  Warp
+    // kExpWarp0 also issues the bulk copies that refill the raw slots.
+    const int eid = tid - kExpWarp0 * 32, ej = eid >> 1, ehf = eid & 1;
+    int issued = min(kStagesT, ntile), landed = 0;
+    for (int t = 0; t <= ntile; t++) {
+      if (t < ntile) {
+        // K of tile t into K buffer t & 1 (free once the softmax of tile t - 2 has read S and
+        // the K scales, which also means QK^T of t - 2 has completed).
+        const int slot = t % kStagesT;
+        if (!dead && !mbar_wait_bounded(full_s + 8 * slot, static_cast<uint32_t>((t / kStagesT) & 1), kWaitT))
+          dead = true;
+        if (!dead) landed++;
+        if (t >= 2 && !dead &&
+            !mbar_wait_bounded(sfree + 8 * (t & 1), static_cast<uint32_t>(((t - 2) >> 1) & 1), kWaitT))
+          dead = true;
+        if (!dead) {
+          const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
+          const int jr = ej % SEFF;
+          const uint4* src = reinterpret_cast<const uint4*>(pg + jr * 64 + 32 * ehf);
+          const uint4 c0 = src[0], c1 = src[1];
+          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          uint8_t* kb = smem + kKs + (t & 1) * kKsBuf + ehf * (kTokT * 128);
+#pragma unroll
+          for (int ch = 0; ch < 8; ch++)  // 16-byte chunk ch = channels 64 ehf + 8 ch .. + 7
+            *reinterpret_cast<uint4*>(kb + sw_off(ej, ch)) =
+                make_uint4(codes_f16x2(cw[ch], 0), codes_f16x2(cw[ch], 1), codes_f16x2(cw[ch], 2),
+                           codes_f16x2(cw[ch], 3));
+          if (ehf == 0) {
+            const bool live = t * kTokT + ej < L;
+            const __half sc = reinterpret_cast<const __half*>(pg + SEFF * 128)[jr];
+            s_kb[(t & 1) * kTokT + ej] = live ? __half2float(sc) : 0.0f;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(kready + 8 * (t & 1));
         }
-    }
-  }
-  if (block == 128) {
-    float* xch = reinterpret_cast<float*>(smem + kQh);  // [half][64 channels][128 rows]
+      }
+      if (t >= 1) {
+        // V of tile u = t - 1 into V buffer u & 1 (free once PV of u - 2 has completed,
+        // which also means the softmax of u - 2 has read its V scales).
+        const int u = t - 1, slot = u % kStagesT;
+        if (u >= 2 && !dead &&
+            !mbar_wait_bounded(pvdone + 8 * (u & 1), static_cast<uint32_t>(((u - 2) >> 1) & 1), kWaitT))
+          dead = true;
+        if (!dead) {
+          const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
+          const int jr = ej % SEFF;
+          const uint4* src = reinterpret_cast<const uint4*>(pg + SEFF * 64 + jr * 64 + 32 * ehf);
+          const uint4 c0 = src[0], c1 = src[1];
+          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          uint8_t* vb = smem + kVs + (u & 1) * kVsBuf + ehf * (kTokT * 128);
 #pragma unroll
-    for (int e = 0; e < 64; e++) xch[(half * 64 + e) * kRowsT + row] = o[e];
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < 64; e++) {
-      const float other = xch[((half ^ 1) * 64 + e) * kRowsT + row];
-      o[e] = half ? other - o[e] : o[e] + other;
+          for (int ch = 0; ch < 8; ch++) {
+            const uint32_t wv = cw[ch], wvh = wv >> 4;
+            *reinterpret_cast<uint4*>(vb + sw_off(ej, ch)) =
+                make_uint4(codes_bf16x2(wv, wvh, 0), codes_bf16x2(wv, wvh, 1), codes_bf16x2(wv, wvh, 2),
+                           codes_bf16x2(wv, wvh, 3));
+          }
+          if (ehf == 0) {
+            const bool live = u * kTokT + ej < L;
+            const __half sc = reinterpret_cast<const __half*>(pg + SEFF * 130)[jr];
+            s_vb[(u & 1) * kTokT + ej] = live ? __half2float(sc) : 0.0f;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(vready + 8 * (u & 1));
+        }
+        // Raw slot u % kStagesT is fully read: refill it with tile u + kStagesT.
+        asm volatile("bar.sync %0, %1;" ::"r"(kBarIdExp), "r"(kExpThreads) : "memory");
+        if (w == kExpWarp0 && !dead && u + kStagesT < ntile) {
+          issue_tile_tc<SEFF>(u + kStagesT, b, h, L, sbase + kRing + slot * kSlotT, full_s + 8 * slot, lane, pol, p);
+          issued++;
+        }
+      }
     }
-  }
-  if (row_valid && !dead) {
-    __half* orow = p.out + ((static_cast<size_t>(cq0) + ti_row) * p.num_kv_heads * G + h * G + row % G) * kD +
-                   64 * half;
-#pragma unroll
-    for (int c8 = 0; c8 < 8; c8++) {
-      const float* v = o + 8 * c8;
-      *reinterpret_cast<uint4*>(orow + 8 * c8) = make_uint4(
-          pack_half2(__float2half_rn(v[0] * p.cb), __float2half_rn(v[1] * p.cb)),
-          pack_half2(__float2half_rn(v[2] * p.cb), __float2half_rn(v[3] * p.cb)),
-          pack_half2(__float2half_rn(v[4] * p.cb), __float2half_rn(v[5] * p.cb)),
-          pack_half2(__float2half_rn(v[6] * p.cb), __float2half_rn(v[7] * p.cb)));
+    if (dead) {
+      if (lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
+      // Let copies still in flight land (bounded) before shared memory is released.
+      if (w == kExpWarp0 && lane == 0)
+        for (int j = landed; j < issued; j++)
+          mbar_wait_bounded(full_s + 8 * (j % kStagesT), static_cast<uint32_t>((j / kStagesT) & 1), kWaitT);
     }
-  }
-  if (dead) {
-    // Let copies and MMAs still in flight finish (bounded) before shared and tensor memory
-    // are released.
-    if (w == 0 && lane == 0) {
-      for (int j = landed; j < issued; j++)
-        mbar_wait_bounded(full_s + 8 * (j % kStagesT), static_cast<uint32_t>((j / kStagesT) & 1), kWaitT);
-      if (commits > 0)
-        mbar_wait_bounded(bar_pv, static_cast<uint32_t>((commits - 1) & 1), kWaitT);
-      else  // only the prologue's QK^T may be in flight
-        for (int tt = 0; tt < qk_pro; tt++) mbar_wait_bounded(bar_qk + 8 * tt, 0u, kWaitT);
+  } else if (w == kMmaWarp) {
+    // ------------------------------------------------------------------- MMA warp --
+    // One elected lane issues; the whole warp walks the waits so it stays converged.
+    const uint64_t dq_h = smem_desc_sw128(sbase + kQh, 16, 1024), dq_l = smem_desc_sw128(sbase + kQl, 16, 1024);
+    const uint64_t dk0 = smem_desc_sw128(sbase + kKs, 16, 1024);
+    const uint64_t dp_h = smem_desc_sw128(sbase + kPh, 16, 1024), dp_l = smem_desc_sw128(sbase + kPl, 16, 1024);
+    const uint64_t dv0 = smem_desc_sw128(sbase + kVs, kTokT * 128, 1024);
+    uint32_t last_bar = 0, last_par = 0;  // the latest commit (it covers every earlier MMA)
+    for (int t = 0; t <= ntile; t++) {
+      if (t < ntile) {
+        // S[t & 1] = q~hi . K + q~lo . K over 8 k-steps of 16 channels.
+        const uint32_t par = static_cast<uint32_t>((t >> 1) & 1);
+        if (!dead && !mbar_wait_bounded(kready + 8 * (t & 1), par, kWaitT)) dead = true;
+        if (t >= 2 && !dead &&
+            !mbar_wait_bounded(sfree + 8 * (t & 1), static_cast<uint32_t>(((t - 2) >> 1) & 1), kWaitT))
+          dead = true;
+        tc_fence_after();
+        if (!dead && lane == 0) {
+          const uint64_t dk = dk0 + static_cast<uint64_t>(((t & 1) * kKsBuf) >> 4);
+#pragma unroll
+          for (int s = 0; s < 8; s++) {
+            const uint64_t qo = static_cast<uint64_t>(((s >> 2) * (kRowsT * 128u) + (s & 3) * 32u) >> 4);
+            const uint64_t ko = static_cast<uint64_t>(((s >> 2) * (kTokT * 128u) + (s & 3) * 32u) >> 4);
+            tc_mma_f16_ss(tmem + 64 * (t & 1), dq_h + qo, dk + ko, kIdescQK, s > 0);
+            tc_mma_f16_ss(tmem + 64 * (t & 1), dq_l + qo, dk + ko, kIdescQK, 1u);
+          }
+          tc_commit(sfull + 8 * (t & 1));
+        }
+        if (!dead) { last_bar = sfull + 8 * (t & 1); last_par = par; }
+        __syncwarp();
+      }
+      if (t >= 1) {
+        // O (+)= P'hi . V + P'lo . V over 4 k-steps of 16 tokens, tile u = t - 1.
+        const int u = t - 1;
+        const uint32_t par = static_cast<uint32_t>((u >> 1) & 1);
+        if (!dead && !mbar_wait_bounded(pready, static_cast<uint32_t>(u & 1), kWaitT)) dead = true;
+        if (!dead && !mbar_wait_bounded(vready + 8 * (u & 1), par, kWaitT)) dead = true;
+        tc_fence_after();
+        if (!dead && lane == 0) {
+          const uint64_t dv = dv0 + static_cast<uint64_t>(((u & 1) * kVsBuf) >> 4);
+#pragma unroll
+          for (int s = 0; s < 4; s++) {
+            const uint64_t vd = dv + static_cast<uint64_t>((2048u * s) >> 4);
+            const uint64_t po = static_cast<uint64_t>((32u * s) >> 4);
+            tc_mma_f16_ss(tmem + kColO, dp_h + po, vd, kIdescPV, (u > 0 || s > 0) ? 1u : 0u);
+            tc_mma_f16_ss(tmem + kColO, dp_l + po, vd, kIdescPV, 1u);
+          }
+          tc_commit(pvdone + 8 * (u & 1));
+        }
+        if (!dead) { last_bar = pvdone + 8 * (u & 1); last_par = par; }
+        __syncwarp();
+      }
+    }
+    if (dead) {
+      if (lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
+      // Let the MMAs issued so far finish (bounded) before tensor memory is released.
+      if (lane == 0 && last_bar) mbar_wait_bounded(last_bar, last_par, kWaitT);
     }
   }
   tc_fence_before();
