@@ -15,24 +15,31 @@
 //   warps 0-7    softmax: warps w and w + 4 both read the lanes of rows 32(w % 4).., warp w
 //                the first half of each tile's columns and of O, warp w + 4 the second;
 //   warps 8-11   expansion: the K and V codes of a tile into the MMA operand tiles, plus
-//                their scales; warp 8 also issues the bulk copies of the raw page data;
-//   warp 12      one lane issues the MMAs: QK^T of tile t, then PV of tile t - 1.
+//                their scales;
+//   warp 12      one lane issues the MMAs: QK^T of tile t, then PV of tile t - 1;
+//   warp 13      reads the page table and issues the bulk copies of the raw page data.
+// Tensor-core time per instruction hardly depends on N up to 128 here, so the tiles are as
+// wide as the accumulators allow (S of two tiles, O and q~ fill the 512 TMEM columns).
 // S (tensor memory), the K and V operand tiles and the scales are double-buffered by tile
 // parity; the raw page data streams through four slots.  The causal KV range is cut into
-// tiles of 64 tokens, whose pages are bulk-copied (cp.async.bulk, 1-D, no multicast).
-//   QK^T  tcgen05.mma kind::f16, M = 128 rows, N = 64 tokens, K = 128 channels: A = q' cut
-//         into fp16 hi + lo parts (q' * 2^14 / M_r, M_r the power of two >= max |q'_r|), B =
-//         the K codes as exact fp16 integers; both parts accumulate into one fp32 tile S in
-//         tensor memory.  The K scale and the row's M_r / 2^14 multiply the scores.
+// tiles of 128 tokens, whose pages are bulk-copied (cp.async.bulk, 1-D, no multicast).
+//   QK^T  tcgen05.mma kind::f16, M = 128 rows, N = 128 tokens, K = 128 channels: A = q' cut
+//         into fp16 hi + lo parts (q' * 2^14 / M_r, M_r the power of two >= max |q'_r|), held
+//         in tensor memory for the whole CTA; B = the K codes as exact fp16 integers in shared
+//         memory; both parts accumulate into one fp32 tile S in tensor memory.  The K scale
+//         and the row's M_r / 2^14 multiply the scores.
 //   softmax  each thread loads its half row of S (tcgen05.ld), applies the causal mask; the two
 //         halves' maxima meet in shared memory; the row keeps an online maximum m and sum l in
 //         the log2 domain.  The frame m moves only when a
 //         score exceeds it by more than 8 (then the row of O is rescaled in tensor memory),
 //         so p = 2^(score - m) <= 256 and the rescale is rare.
-//   PV    tcgen05.mma kind::f16 in bf16, M = 128 rows, N = 128 channels, K = 64 tokens: A =
+//   PV    tcgen05.mma kind::f16 in bf16, M = 128 rows, N = 128 channels, K = 128 tokens: A =
 //         P' = p * s_v (the V scale folded into the probabilities) as bf16 hi + lo parts (bf16
-//         keeps fp32's range, so P' <= 256 * s_v cannot overflow), B = the V codes as exact
-//         bf16 integers, read channel-major; the accumulator O stays in tensor memory.
+//         keeps fp32's range, so P' <= 256 * s_v cannot overflow), written by each softmax
+//         thread over the S columns it has just read; B = the V codes as exact bf16 integers,
+//         read channel-major from shared memory; the accumulator O stays in tensor memory.
+// With both A operands in tensor memory the tensor cores read only K and V from shared
+// memory, whose bandwidth the MMAs would otherwise share with the expansion.
 // The end: each thread loads its half row of O, divides by l, applies the inverse block
 // Hadamard (stages inside a half in registers, the stage across the halves through shared
 // memory), times c_b, stores fp16.
@@ -56,45 +63,51 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kRowsT = 128;     // query rows per CTA (tensor-memory lanes)
-constexpr int kTokT = 64;       // KV tokens per tile
+constexpr int kTokT = 128;      // KV tokens per tile
 constexpr int kSoftWarps = 8;   // warps w and w + 4 share the rows of TMEM lanes 32(w % 4)..
 constexpr int kSoftThreads = 32 * kSoftWarps;
-constexpr int kExpWarp0 = 8;    // warps 8-11 expand K and V codes; warp 8 also issues copies
+constexpr int kExpWarp0 = 8;    // warps 8-11 expand K and V codes
 constexpr int kExpWarps = 4;
 constexpr int kExpThreads = 32 * kExpWarps;
-constexpr int kMmaWarp = 12;    // issues the tcgen05 MMAs; warps 13-15 only pad the warpgroup
-constexpr int kThreadsT = 512;
-constexpr int kBarIdExp = 5;    // named barrier of the expansion warps (1-4: softmax row pairs)
+constexpr int kMmaWarp = 12;    // issues the tcgen05 MMAs
+constexpr int kProdWarp = 13;   // reads the page table and issues the bulk copies
+constexpr int kThreadsT = 512;  // warps 14-15 only pad the last warpgroup
 constexpr int kStagesT = 4;     // raw page-data slots
 constexpr uint64_t kWaitT = 2000000000ull;
 constexpr float kLazyT = 8.0f;  // frame slack in log2 units: p <= 2^8 between rescales
 constexpr unsigned kFullT = 0xffffffffu;
-constexpr int kTmemCols = 256;  // S of tiles t even / odd: columns [0, 64) / [64, 128); O: [128, 256)
-constexpr int kColO = 128;
+// Tensor-memory columns: S of tiles t even / odd [0, 128) / [128, 256), where P' of the tile
+// replaces S once read; O [256, 384); q~ hi [384, 448) and lo [448, 512) (fp16 pairs).
+constexpr int kTmemCols = 512;
+constexpr int kColO = 256;
+constexpr int kColQh = 384;
+constexpr int kColQl = 448;
 
 // Shared-memory map (bytes from a 1024-byte aligned base).
-constexpr int kQh = 0;                          // [2 kb][128 rows][128 B] fp16 q~ hi
-constexpr int kQl = kQh + 2 * kRowsT * 128;     // same, lo
-constexpr int kKs = kQl + 2 * kRowsT * 128;     // [2 buffers][2 kb][64 tokens][128 B] fp16 K codes
+constexpr int kKs = 0;                          // [2 buffers][2 kb][128 tokens][128 B] fp16 K codes
 constexpr int kKsBuf = 2 * kTokT * 128;
-constexpr int kVs = kKs + 2 * kKsBuf;           // [2 buffers][2 nb][64 tokens][128 B] bf16 V codes
+// q~ passes through the K buffers on its way to tensor memory (before any K is expanded),
+// and the end exchanges O halves there (after the last QK^T).
+constexpr int kQh = kKs;                        // [2 kb][128 rows][128 B] fp16 q~ hi
+constexpr int kQl = kQh + 2 * kRowsT * 128;     // same, lo
+constexpr int kVs = kKs + 2 * kKsBuf;           // [2 buffers][2 nb][128 tokens][128 B] bf16 V codes
 constexpr int kVsBuf = 2 * kTokT * 128;
-constexpr int kPh = kVs + 2 * kVsBuf;           // [128 rows][128 B] bf16 P' hi
-constexpr int kPl = kPh + kRowsT * 128;         // same, lo
-constexpr int kRing = kPl + kRowsT * 128;       // [4][64 token rows of 132 B]
+constexpr int kRing = kVs + 2 * kVsBuf;         // [4][128 token rows of 132 B]
 constexpr int kSlotT = kTokT * 132;
-constexpr int kScl = kRing + kStagesT * kSlotT; // K scales [2][64], V scales [2][64] fp32
+constexpr int kScl = kRing + kStagesT * kSlotT; // K scales [2][128], V scales [2][128] fp32
 constexpr int kSfr = kScl + 4 * kTokT * 4;      // row scales [128] fp32
 constexpr int kRed = kSfr + kRowsT * 4;         // maxima [2][2][128], sums [2][128] fp32
 constexpr int kBar = kRed + 6 * kRowsT * 4;     // mbarriers, see kBar* below
-constexpr int kBarFull = 0, kBarKReady = 4, kBarVReady = 6, kBarSFull = 8, kBarSFree = 10,
-              kBarPReady = 12, kBarPVDone = 13, kNumBars = 15;
+constexpr int kBarFull = 0, kBarEmpty = 4, kBarKReady = 8, kBarVReady = 10, kBarSFull = 12,
+              kBarSFree = 14, kBarPReady = 16, kBarPVDone = 17, kNumBars = 19;
 constexpr int kTmemSlot = kBar + kNumBars * 8;  // tensor-memory base address
 constexpr int kPreq = kTmemSlot + 16;           // query-block prefix [batch + 1]
+static_assert(kQl + 2 * kRowsT * 128 <= kVs, "q~ staging fits the K buffers");
+static_assert(kPreq + 4097 * 4 + 1024 + 1024 <= 232448, "shared memory of the largest batch");
 
 // Instruction descriptors (kind::f16): fp32 accumulator, M = 128.
-//   QK^T: A, B fp16, both K-major, N = 64.   PV: A, B bf16, A K-major, B MN-major, N = 128.
-constexpr uint32_t kIdescQK = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+//   QK^T: A, B fp16, both K-major, N = 128.  PV: A, B bf16, A K-major, B MN-major, N = 128.
+constexpr uint32_t kIdescQK = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) |
                               ((128u >> 4) << 24);
 
@@ -103,26 +116,36 @@ __device__ __forceinline__ uint32_t sw_off(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// Issue the bulk copies of tile t (tokens 64t..) of sequence b, KV head h into a raw slot
-// (warp 0 calls): the slot holds virtual pages of SEFF = min(S, 64) token rows in the pool's
-// block layout [K codes][V codes][K scales][V scales].
+// The raw slot holds virtual pages of SEFF = min(S, 128) token rows in the pool's block layout
+// [K codes][V codes][K scales][V scales].  Copying a tile takes two steps so that the page-
+// table read can be issued well before the copies: tile_page reads this lane's page id of
+// tile t of sequence b (lane i the tile's i-th page when pages are shorter than a tile, else
+// every lane the one page); issue_tile_pages checks it (an id out of range flags
+// KVQ_DEV_BAD_PAGE and reads page 0) and starts the copies into a slot with completion on its
+// barrier.
 template <int SEFF>
-__device__ __forceinline__ void issue_tile_tc(int t, int b, int h, int L, uint32_t slot, uint32_t bar,
-                                              int lane, uint64_t pol, const PrefillParams& p) {
+__device__ __forceinline__ int tile_page(int t, int b, int L, int lane, const PrefillParams& p) {
+  const int sh = p.page_shift;
+  const int t0 = t * kTokT;
+  const int t1 = min(t0 + kTokT, L);  // > t0
+  const int npg = (SEFF < kTokT || p.page_size == kTokT) ? ((t1 - 1) >> sh) - (t0 >> sh) + 1 : 1;
+  if (npg > 1 && lane >= npg) return 0;
+  return __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + (t0 >> sh) + (npg > 1 ? lane : 0));
+}
+
+template <int SEFF>
+__device__ __forceinline__ void issue_tile_pages(int t, int h, int L, int pid, uint32_t slot, uint32_t bar,
+                                                 int lane, uint64_t pol, const PrefillParams& p) {
   const int S = p.page_size, sh = p.page_shift;
   const int t0 = t * kTokT;
   const int t1 = min(t0 + kTokT, L);  // > t0
+  if (pid < 0 || pid >= p.num_pages) {
+    if (lane == 0 || SEFF < kTokT || S == kTokT) atomicOr(p.status, KVQ_DEV_BAD_PAGE_BIT);
+    pid = 0;
+  }
   if (SEFF < kTokT || S == kTokT) {
     const uint32_t blk_bytes = static_cast<uint32_t>(S) * 132u;
     const int npg = ((t1 - 1) >> sh) - (t0 >> sh) + 1;
-    int pid = 0;
-    bool bad = false;
-    if (lane < npg) {
-      pid = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + (t0 >> sh) + lane);
-      bad = pid < 0 || pid >= p.num_pages;
-      if (bad) pid = 0;
-    }
-    if (__any_sync(kFullT, bad) && lane == 0) atomicOr(p.status, KVQ_DEV_BAD_PAGE_BIT);
     if (lane == 0) mbar_arrive_expect_tx(bar, npg * blk_bytes);
     __syncwarp();
     if (lane < npg)
@@ -133,10 +156,6 @@ __device__ __forceinline__ void issue_tile_tc(int t, int b, int h, int L, uint32
     // Pages of 128+ tokens: the tile is part of one page; lanes 0-3 copy its K codes, V
     // codes, K scales and V scales.
     const size_t blk_bytes = static_cast<size_t>(S) * 132u;
-    int pid = __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + (t0 >> sh));
-    const bool bad = pid < 0 || pid >= p.num_pages;
-    if (bad) pid = 0;
-    if (bad && lane == 0) atomicOr(p.status, KVQ_DEV_BAD_PAGE_BIT);
     const size_t o = static_cast<size_t>(t0 & (S - 1));
     const uint8_t* blk = p.pool_layer + (static_cast<size_t>(pid) * p.num_kv_heads + h) * blk_bytes;
     const uint8_t* src = blk + o * 64;
@@ -191,7 +210,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlot);
   int32_t* preq = reinterpret_cast<int32_t*>(smem + kPreq);
   const uint32_t bar0 = sbase + kBar;
-  const uint32_t full_s = bar0 + 8 * kBarFull, kready = bar0 + 8 * kBarKReady,
+  const uint32_t full_s = bar0 + 8 * kBarFull, empty_s = bar0 + 8 * kBarEmpty, kready = bar0 + 8 * kBarKReady,
                  vready = bar0 + 8 * kBarVReady, sfull = bar0 + 8 * kBarSFull,
                  sfree = bar0 + 8 * kBarSFree, pready = bar0 + 8 * kBarPReady,
                  pvdone = bar0 + 8 * kBarPVDone;
@@ -203,7 +222,10 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   // call); q, the pool and out are touched after it.
   griddep_launch_dependents();
   if (tid == 0) {
-    for (int k = 0; k < kStagesT; k++) mbar_init(full_s + 8 * k, 1);
+    for (int k = 0; k < kStagesT; k++) {
+      mbar_init(full_s + 8 * k, 1);
+      mbar_init(empty_s + 8 * k, kExpThreads);
+    }
     for (int k = 0; k < 2; k++) {
       mbar_init(kready + 8 * k, kExpThreads);
       mbar_init(vready + 8 * k, kExpThreads);
@@ -271,9 +293,11 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
     tmem_relinquish();
   }
   griddep_wait();
-  if (w == kExpWarp0) {
+  // The producer warp starts the first kStagesT tiles' copies.
+  if (w == kProdWarp) {
     for (int t = 0; t < kStagesT && t < ntile; t++)
-      issue_tile_tc<SEFF>(t, b, h, L, sbase + kRing + t * kSlotT, full_s + 8 * t, lane, pol, p);
+      issue_tile_pages<SEFF>(t, h, L, tile_page<SEFF>(t, b, L, lane, p), sbase + kRing + t * kSlotT,
+                             full_s + 8 * t, lane, pol, p);
   }
 
   // q rows: softmax warp w rotates and scales rows 16w..16w+15 (lane: channels 4 lane..
@@ -329,13 +353,33 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       *reinterpret_cast<uint2*>(smem + kQl + off) = make_uint2(pack_half2(lv[0], lv[1]), pack_half2(lv[2], lv[3]));
       if (lane == 0) sfr[row] = M * (1.0f / 16384.0f);
     }
-    fence_proxy_async_smem();  // q~ is read by the tensor cores
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool dead = false;
+  // q~ into tensor memory, the A operand of QK^T: softmax thread (row, half) moves channels
+  // 64 half..64 half + 63 of its row, hi and lo parts, as fp16 pairs.
+  if (w < kSoftWarps) {
+    const int row = 32 * (w & 3) + lane, half = w >> 2;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * (w & 3)) << 16);
+#pragma unroll
+    for (int part = 0; part < 2; part++) {
+      uint32_t r[32];
+      const uint8_t* src = smem + (part ? kQl : kQh) + half * (kRowsT * 128);
+#pragma unroll
+      for (int ch = 0; ch < 8; ch++) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + sw_off(row, ch));
+        r[4 * ch] = v.x; r[4 * ch + 1] = v.y; r[4 * ch + 2] = v.z; r[4 * ch + 3] = v.w;
+      }
+      tmem_st32(lane_addr + (part ? kColQl : kColQh) + 32 * half, r);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (w < kSoftWarps) {
     // ---------------------------------------------------------------- softmax warps --
@@ -356,30 +400,37 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       if (!dead && !mbar_wait_bounded(sfull + 8 * (t & 1), par, kWaitT)) dead = true;
       if (!dead && !mbar_wait_bounded(kready + 8 * (t & 1), par, kWaitT)) dead = true;
       tc_fence_after();
-      uint32_t sraw[32];
-      tmem_ld32(lane_addr + 64 * (t & 1) + 32 * half, sraw);
-      tmem_wait_ld();
-      float kk[32];
-      const float4* s_k4 = reinterpret_cast<const float4*>(s_kb + (t & 1) * kTokT + 32 * half);
+      // Scores of this thread's 64 tokens (64 half..): two 32-column loads, scaled by the
+      // row's and the tokens' scales.
+      float sc[64];
 #pragma unroll
-      for (int e4 = 0; e4 < 8; e4++) {
-        const float4 k4 = s_k4[e4];
-        kk[4 * e4] = k4.x; kk[4 * e4 + 1] = k4.y; kk[4 * e4 + 2] = k4.z; kk[4 * e4 + 3] = k4.w;
+      for (int c = 0; c < 2; c++) {
+        uint32_t raw[32];
+        tmem_ld32(lane_addr + kTokT * (t & 1) + 64 * half + 32 * c, raw);
+        tmem_wait_ld();
+        const float4* s_k4 = reinterpret_cast<const float4*>(s_kb + (t & 1) * kTokT + 64 * half + 32 * c);
+#pragma unroll
+        for (int e4 = 0; e4 < 8; e4++) {
+          const float4 k4 = s_k4[e4];
+          sc[32 * c + 4 * e4] = __uint_as_float(raw[4 * e4]) * (sf * k4.x);
+          sc[32 * c + 4 * e4 + 1] = __uint_as_float(raw[4 * e4 + 1]) * (sf * k4.y);
+          sc[32 * c + 4 * e4 + 2] = __uint_as_float(raw[4 * e4 + 2]) * (sf * k4.z);
+          sc[32 * c + 4 * e4 + 3] = __uint_as_float(raw[4 * e4 + 3]) * (sf * k4.w);
+        }
       }
       // S buffer t & 1 and the K scales of tile t are free for tile t + 2.
       tc_fence_before();
       if (!dead) mbar_arrive(sfree + 8 * (t & 1));
       // Tiles wholly before the CTA's first row need no causal mask (they hold no token at or
       // beyond L either).
-      const bool masked = t * kTokT + kTokT - 1 > L - C + tok_first;
-      float mx = -CUDART_INF_F;
+      if (t * kTokT + kTokT - 1 > L - C + tok_first) {
 #pragma unroll
-      for (int e = 0; e < 32; e++) {
-        float v = __uint_as_float(sraw[e]) * (sf * kk[e]);
-        if (masked && t * kTokT + 32 * half + e > rpos) v = -CUDART_INF_F;
-        sraw[e] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
+        for (int e = 0; e < 64; e++)
+          if (t * kTokT + 64 * half + e > rpos) sc[e] = -CUDART_INF_F;
       }
+      float mx = sc[0];
+#pragma unroll
+      for (int e = 1; e < 64; e++) mx = fmaxf(mx, sc[e]);
       // The row's maximum over both halves (warps w and w + 4 meet at a 64-thread barrier;
       // the exchange slots alternate with the tile's parity).
       red[((t & 1) * 2 + half) * kRowsT + row] = mx;
@@ -395,10 +446,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       }
       float ps = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 32; e++) {  // ex2(-inf) = +0: masked scores need no test
-        const float pe = ex2_approx(__uint_as_float(sraw[e]) - m);
-        sraw[e] = __float_as_uint(pe);
-        ps += pe;
+      for (int e = 0; e < 64; e++) {  // ex2(-inf) = +0: masked scores need no test
+        sc[e] = ex2_approx(sc[e] - m);
+        ps += sc[e];
       }
       l += ps;
       // PV of tile t - 1 reads P' and accumulates O: wait for it before touching either.
@@ -420,27 +470,31 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
         }
         tmem_wait_st();
       }
-      // P' = p * s_v as bf16 hi + lo into the K-major A operand (V scales of tile t: vready).
+      // P' = p * s_v as bf16 hi + lo pairs over this thread's own S columns (the A operand
+      // of PV): 32-token chunk c at columns 64 half + 32 c, hi in [0, 16), lo in [16, 32)
+      // (V scales of tile t: vready).
       if (!dead && !mbar_wait_bounded(vready + 8 * (t & 1), par, kWaitT)) dead = true;
-      const float4* s_v4 = reinterpret_cast<const float4*>(s_vb + (t & 1) * kTokT + 32 * half);
 #pragma unroll
-      for (int c4 = 0; c4 < 4; c4++) {
-        uint32_t ph[4], pl[4];
-        const float4 va = s_v4[2 * c4], vb = s_v4[2 * c4 + 1];
-        const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+      for (int c = 0; c < 2; c++) {
+        const float4* s_v4 = reinterpret_cast<const float4*>(s_vb + (t & 1) * kTokT + 64 * half + 32 * c);
+        uint32_t pp[32];
 #pragma unroll
-        for (int e2 = 0; e2 < 4; e2++) {
-          const int e = 8 * c4 + 2 * e2;
-          const float x0 = __uint_as_float(sraw[e]) * vv[2 * e2];
-          const float x1 = __uint_as_float(sraw[e + 1]) * vv[2 * e2 + 1];
-          ph[e2] = pack_bf16x2(x0, x1);
-          pl[e2] = pack_bf16x2(x0 - bf16_lo(ph[e2]), x1 - bf16_hi(ph[e2]));
+        for (int c4 = 0; c4 < 4; c4++) {
+          const float4 va = s_v4[2 * c4], vb = s_v4[2 * c4 + 1];
+          const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 4; e2++) {
+            const int e = 8 * c4 + 2 * e2;
+            const float x0 = sc[32 * c + e] * vv[2 * e2];
+            const float x1 = sc[32 * c + e + 1] * vv[2 * e2 + 1];
+            const uint32_t hi2 = pack_bf16x2(x0, x1);
+            pp[e >> 1] = hi2;
+            pp[16 + (e >> 1)] = pack_bf16x2(x0 - bf16_lo(hi2), x1 - bf16_hi(hi2));
+          }
         }
-        const int c8 = 4 * half + c4;
-        *reinterpret_cast<uint4*>(smem + kPh + sw_off(row, c8)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-        *reinterpret_cast<uint4*>(smem + kPl + sw_off(row, c8)) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        tmem_st32(lane_addr + kTokT * (t & 1) + 64 * half + 32 * c, pp);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       if (!dead) mbar_arrive(pready);
     }
@@ -508,10 +562,8 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
     }
   } else if (w < kExpWarp0 + kExpWarps) {
     // -------------------------------------------------------------- expansion warps --
-    // Item: token ej of the tile, channels 64 ehf..64 ehf + 63, for K and for V.  Warp
-    // kExpWarp0 also issues the bulk copies that refill the raw slots.
-    const int eid = tid - kExpWarp0 * 32, ej = eid >> 1, ehf = eid & 1;
-    int issued = min(kStagesT, ntile), landed = 0;
+    // Items: tokens ej and ej + 64 of the tile, channels 64 ehf..64 ehf + 63, for K and V.
+    const int eid = tid - kExpWarp0 * 32, ej0 = eid >> 1, ehf = eid & 1;
     for (int t = 0; t <= ntile; t++) {
       if (t < ntile) {
         // K of tile t into K buffer t & 1 (free once the softmax of tile t - 2 has read S and
@@ -519,26 +571,29 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
         const int slot = t % kStagesT;
         if (!dead && !mbar_wait_bounded(full_s + 8 * slot, static_cast<uint32_t>((t / kStagesT) & 1), kWaitT))
           dead = true;
-        if (!dead) landed++;
         if (t >= 2 && !dead &&
             !mbar_wait_bounded(sfree + 8 * (t & 1), static_cast<uint32_t>(((t - 2) >> 1) & 1), kWaitT))
           dead = true;
         if (!dead) {
-          const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
-          const int jr = ej % SEFF;
-          const uint4* src = reinterpret_cast<const uint4*>(pg + jr * 64 + 32 * ehf);
-          const uint4 c0 = src[0], c1 = src[1];
-          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          uint8_t* kb = smem + kKs + (t & 1) * kKsBuf + ehf * (kTokT * 128);
 #pragma unroll
-          for (int ch = 0; ch < 8; ch++)  // 16-byte chunk ch = channels 64 ehf + 8 ch .. + 7
-            *reinterpret_cast<uint4*>(kb + sw_off(ej, ch)) =
-                make_uint4(codes_f16x2(cw[ch], 0), codes_f16x2(cw[ch], 1), codes_f16x2(cw[ch], 2),
-                           codes_f16x2(cw[ch], 3));
-          if (ehf == 0) {
-            const bool live = t * kTokT + ej < L;
-            const __half sc = reinterpret_cast<const __half*>(pg + SEFF * 128)[jr];
-            s_kb[(t & 1) * kTokT + ej] = live ? __half2float(sc) : 0.0f;
+          for (int it = 0; it < 2; it++) {
+            const int ej = ej0 + 64 * it;
+            const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
+            const int jr = ej % SEFF;
+            const uint4* src = reinterpret_cast<const uint4*>(pg + jr * 64 + 32 * ehf);
+            const uint4 c0 = src[0], c1 = src[1];
+            const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            uint8_t* kb = smem + kKs + (t & 1) * kKsBuf + ehf * (kTokT * 128);
+#pragma unroll
+            for (int ch = 0; ch < 8; ch++)  // 16-byte chunk ch = channels 64 ehf + 8 ch .. + 7
+              *reinterpret_cast<uint4*>(kb + sw_off(ej, ch)) =
+                  make_uint4(codes_f16x2(cw[ch], 0), codes_f16x2(cw[ch], 1), codes_f16x2(cw[ch], 2),
+                             codes_f16x2(cw[ch], 3));
+            if (ehf == 0) {
+              const bool live = t * kTokT + ej < L;
+              const __half sk = reinterpret_cast<const __half*>(pg + SEFF * 128)[jr];
+              s_kb[(t & 1) * kTokT + ej] = live ? __half2float(sk) : 0.0f;
+            }
           }
           fence_proxy_async_smem();
           mbar_arrive(kready + 8 * (t & 1));
@@ -552,48 +607,45 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
             !mbar_wait_bounded(pvdone + 8 * (u & 1), static_cast<uint32_t>(((u - 2) >> 1) & 1), kWaitT))
           dead = true;
         if (!dead) {
-          const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
-          const int jr = ej % SEFF;
-          const uint4* src = reinterpret_cast<const uint4*>(pg + SEFF * 64 + jr * 64 + 32 * ehf);
-          const uint4 c0 = src[0], c1 = src[1];
-          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          uint8_t* vb = smem + kVs + (u & 1) * kVsBuf + ehf * (kTokT * 128);
+          uint32_t cw[2][8];
+          float vs[2] = {0.0f, 0.0f};
 #pragma unroll
-          for (int ch = 0; ch < 8; ch++) {
-            const uint32_t wv = cw[ch], wvh = wv >> 4;
-            *reinterpret_cast<uint4*>(vb + sw_off(ej, ch)) =
-                make_uint4(codes_bf16x2(wv, wvh, 0), codes_bf16x2(wv, wvh, 1), codes_bf16x2(wv, wvh, 2),
-                           codes_bf16x2(wv, wvh, 3));
+          for (int it = 0; it < 2; it++) {
+            const int ej = ej0 + 64 * it;
+            const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
+            const int jr = ej % SEFF;
+            const uint4* src = reinterpret_cast<const uint4*>(pg + SEFF * 64 + jr * 64 + 32 * ehf);
+            const uint4 c0 = src[0], c1 = src[1];
+            cw[it][0] = c0.x; cw[it][1] = c0.y; cw[it][2] = c0.z; cw[it][3] = c0.w;
+            cw[it][4] = c1.x; cw[it][5] = c1.y; cw[it][6] = c1.z; cw[it][7] = c1.w;
+            if (ehf == 0 && u * kTokT + ej < L)
+              vs[it] = __half2float(reinterpret_cast<const __half*>(pg + SEFF * 130)[jr]);
           }
-          if (ehf == 0) {
-            const bool live = u * kTokT + ej < L;
-            const __half sc = reinterpret_cast<const __half*>(pg + SEFF * 130)[jr];
-            s_vb[(u & 1) * kTokT + ej] = live ? __half2float(sc) : 0.0f;
+          // The raw slot of tile u is fully read: the producer may refill it.
+          mbar_arrive(empty_s + 8 * slot);
+#pragma unroll
+          for (int it = 0; it < 2; it++) {
+            const int ej = ej0 + 64 * it;
+            uint8_t* vb = smem + kVs + (u & 1) * kVsBuf + ehf * (kTokT * 128);
+#pragma unroll
+            for (int ch = 0; ch < 8; ch++) {
+              const uint32_t wv = cw[it][ch], wvh = wv >> 4;
+              *reinterpret_cast<uint4*>(vb + sw_off(ej, ch)) =
+                  make_uint4(codes_bf16x2(wv, wvh, 0), codes_bf16x2(wv, wvh, 1), codes_bf16x2(wv, wvh, 2),
+                             codes_bf16x2(wv, wvh, 3));
+            }
+            if (ehf == 0) s_vb[(u & 1) * kTokT + ej] = vs[it];
           }
           fence_proxy_async_smem();
           mbar_arrive(vready + 8 * (u & 1));
         }
-        // Raw slot u % kStagesT is fully read: refill it with tile u + kStagesT.
-        asm volatile("bar.sync %0, %1;" ::"r"(kBarIdExp), "r"(kExpThreads) : "memory");
-        if (w == kExpWarp0 && !dead && u + kStagesT < ntile) {
-          issue_tile_tc<SEFF>(u + kStagesT, b, h, L, sbase + kRing + slot * kSlotT, full_s + 8 * slot, lane, pol, p);
-          issued++;
-        }
       }
     }
-    if (dead) {
-      if (lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
-      // Let copies still in flight land (bounded) before shared memory is released.
-      if (w == kExpWarp0 && lane == 0)
-        for (int j = landed; j < issued; j++)
-          mbar_wait_bounded(full_s + 8 * (j % kStagesT), static_cast<uint32_t>((j / kStagesT) & 1), kWaitT);
-    }
+    if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
   } else if (w == kMmaWarp) {
     // ------------------------------------------------------------------- MMA warp --
     // One elected lane issues; the whole warp walks the waits so it stays converged.
-    const uint64_t dq_h = smem_desc_sw128(sbase + kQh, 16, 1024), dq_l = smem_desc_sw128(sbase + kQl, 16, 1024);
     const uint64_t dk0 = smem_desc_sw128(sbase + kKs, 16, 1024);
-    const uint64_t dp_h = smem_desc_sw128(sbase + kPh, 16, 1024), dp_l = smem_desc_sw128(sbase + kPl, 16, 1024);
     const uint64_t dv0 = smem_desc_sw128(sbase + kVs, kTokT * 128, 1024);
     uint32_t last_bar = 0, last_par = 0;  // the latest commit (it covers every earlier MMA)
     for (int t = 0; t <= ntile; t++) {
@@ -608,11 +660,10 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
         if (!dead && lane == 0) {
           const uint64_t dk = dk0 + static_cast<uint64_t>(((t & 1) * kKsBuf) >> 4);
 #pragma unroll
-          for (int s = 0; s < 8; s++) {
-            const uint64_t qo = static_cast<uint64_t>(((s >> 2) * (kRowsT * 128u) + (s & 3) * 32u) >> 4);
+          for (int s = 0; s < 8; s++) {  // k-step s: channels 16 s.., q~ columns 8 s..
             const uint64_t ko = static_cast<uint64_t>(((s >> 2) * (kTokT * 128u) + (s & 3) * 32u) >> 4);
-            tc_mma_f16_ss(tmem + 64 * (t & 1), dq_h + qo, dk + ko, kIdescQK, s > 0);
-            tc_mma_f16_ss(tmem + 64 * (t & 1), dq_l + qo, dk + ko, kIdescQK, 1u);
+            tc_mma_f16_ts(tmem + kTokT * (t & 1), tmem + kColQh + 8 * s, dk + ko, kIdescQK, s > 0);
+            tc_mma_f16_ts(tmem + kTokT * (t & 1), tmem + kColQl + 8 * s, dk + ko, kIdescQK, 1u);
           }
           tc_commit(sfull + 8 * (t & 1));
         }
@@ -629,11 +680,11 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
         if (!dead && lane == 0) {
           const uint64_t dv = dv0 + static_cast<uint64_t>(((u & 1) * kVsBuf) >> 4);
 #pragma unroll
-          for (int s = 0; s < 4; s++) {
+          for (int s = 0; s < 8; s++) {  // k-step s: tokens 16 s.., P' of half s / 4, chunk (s / 2) % 2
             const uint64_t vd = dv + static_cast<uint64_t>((2048u * s) >> 4);
-            const uint64_t po = static_cast<uint64_t>((32u * s) >> 4);
-            tc_mma_f16_ss(tmem + kColO, dp_h + po, vd, kIdescPV, (u > 0 || s > 0) ? 1u : 0u);
-            tc_mma_f16_ss(tmem + kColO, dp_l + po, vd, kIdescPV, 1u);
+            const uint32_t pa = tmem + kTokT * (u & 1) + 32 * (s >> 1) + 8 * (s & 1);
+            tc_mma_f16_ts(tmem + kColO, pa, vd, kIdescPV, (u > 0 || s > 0) ? 1u : 0u);
+            tc_mma_f16_ts(tmem + kColO, pa + 16, vd, kIdescPV, 1u);
           }
           tc_commit(pvdone + 8 * (u & 1));
         }
@@ -646,6 +697,32 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       // Let the MMAs issued so far finish (bounded) before tensor memory is released.
       if (lane == 0 && last_bar) mbar_wait_bounded(last_bar, last_par, kWaitT);
     }
+  } else if (w == kProdWarp) {
+    // ----------------------------------------------------------------- producer warp --
+    // Tile t (t >= kStagesT) refills slot t % kStagesT once the expansion has released tile
+    // t - kStagesT; its page ids are read one tile ahead, so the read overlaps that wait.
+    int issued = min(kStagesT, ntile);
+    int pid_next = kStagesT < ntile ? tile_page<SEFF>(kStagesT, b, L, lane, p) : 0;
+    for (int t = kStagesT; t < ntile && !dead; t++) {
+      const int pid_after = t + 1 < ntile ? tile_page<SEFF>(t + 1, b, L, lane, p) : 0;
+      const int slot = t % kStagesT;
+      // Lane 0 waits and tells the others, so the warp stays converged for the copies.
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_bounded(empty_s + 8 * slot, static_cast<uint32_t>((t / kStagesT - 1) & 1), kWaitT);
+      if (!__shfl_sync(kFullT, ok, 0)) {
+        dead = true;
+        break;
+      }
+      issue_tile_pages<SEFF>(t, h, L, pid_next, sbase + kRing + slot * kSlotT, full_s + 8 * slot, lane, pol, p);
+      issued++;
+      pid_next = pid_after;
+    }
+    if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
+    // Before shared memory is released, the last copies into each slot must have landed
+    // (bounded; earlier ones were consumed by the expansion before their slot was reused).
+    if (lane == 0)
+      for (int j = max(0, issued - kStagesT); j < issued; j++)
+        mbar_wait_bounded(full_s + 8 * (j % kStagesT), static_cast<uint32_t>((j / kStagesT) & 1), kWaitT);
   }
   tc_fence_before();
   __syncthreads();
@@ -658,6 +735,7 @@ void* prefill_tc_ptr(int seff) {
   if (seff == 16) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 16>);
   if (seff == 32) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 32>);
   if (seff == 64) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 64>);
+  if (seff == 128) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 128>);
   return nullptr;
 }
 
