@@ -400,23 +400,21 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       if (!dead && !mbar_wait_bounded(sfull + 8 * (t & 1), par, kWaitT)) dead = true;
       if (!dead && !mbar_wait_bounded(kready + 8 * (t & 1), par, kWaitT)) dead = true;
       tc_fence_after();
-      // Scores of this thread's 64 tokens (64 half..): two 32-column loads, scaled by the
-      // row's and the tokens' scales.
-      float sc[64];
+      // This thread's 64 tokens (64 half..): u = S * s_k, in pairs.  The row scale sf > 0
+      // commutes with the maximum, so the score sf * u is formed only inside the exponent.
+      uint32_t raw[64];
+      tmem_ld32(lane_addr + kTokT * (t & 1) + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(raw));
+      tmem_ld32(lane_addr + kTokT * (t & 1) + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
+      tmem_wait_ld();
+      uint64_t u2[32];
+      const float4* s_k4 = reinterpret_cast<const float4*>(s_kb + (t & 1) * kTokT + 64 * half);
 #pragma unroll
-      for (int c = 0; c < 2; c++) {
-        uint32_t raw[32];
-        tmem_ld32(lane_addr + kTokT * (t & 1) + 64 * half + 32 * c, raw);
-        tmem_wait_ld();
-        const float4* s_k4 = reinterpret_cast<const float4*>(s_kb + (t & 1) * kTokT + 64 * half + 32 * c);
-#pragma unroll
-        for (int e4 = 0; e4 < 8; e4++) {
-          const float4 k4 = s_k4[e4];
-          sc[32 * c + 4 * e4] = __uint_as_float(raw[4 * e4]) * (sf * k4.x);
-          sc[32 * c + 4 * e4 + 1] = __uint_as_float(raw[4 * e4 + 1]) * (sf * k4.y);
-          sc[32 * c + 4 * e4 + 2] = __uint_as_float(raw[4 * e4 + 2]) * (sf * k4.z);
-          sc[32 * c + 4 * e4 + 3] = __uint_as_float(raw[4 * e4 + 3]) * (sf * k4.w);
-        }
+      for (int e4 = 0; e4 < 16; e4++) {
+        const float4 k4 = s_k4[e4];
+        u2[2 * e4] = f2_mul(f2_pack(__uint_as_float(raw[4 * e4]), __uint_as_float(raw[4 * e4 + 1])),
+                            f2_pack(k4.x, k4.y));
+        u2[2 * e4 + 1] = f2_mul(f2_pack(__uint_as_float(raw[4 * e4 + 2]), __uint_as_float(raw[4 * e4 + 3])),
+                                f2_pack(k4.z, k4.w));
       }
       // S buffer t & 1 and the K scales of tile t are free for tile t + 2.
       tc_fence_before();
@@ -425,12 +423,22 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       // beyond L either).
       if (t * kTokT + kTokT - 1 > L - C + tok_first) {
 #pragma unroll
-        for (int e = 0; e < 64; e++)
-          if (t * kTokT + 64 * half + e > rpos) sc[e] = -CUDART_INF_F;
+        for (int e2 = 0; e2 < 32; e2++) {
+          float2 v = f2_unpack(u2[e2]);
+          const int pos = t * kTokT + 64 * half + 2 * e2;
+          if (pos > rpos) v.x = -CUDART_INF_F;
+          if (pos + 1 > rpos) v.y = -CUDART_INF_F;
+          u2[e2] = f2_pack(v.x, v.y);
+        }
       }
-      float mx = sc[0];
+      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
 #pragma unroll
-      for (int e = 1; e < 64; e++) mx = fmaxf(mx, sc[e]);
+      for (int e2 = 0; e2 < 32; e2++) {
+        const float2 v = f2_unpack(u2[e2]);
+        mx0 = fmaxf(mx0, v.x);
+        mx1 = fmaxf(mx1, v.y);
+      }
+      float mx = fmaxf(mx0, mx1) * sf;
       // The row's maximum over both halves (warps w and w + 4 meet at a 64-thread barrier;
       // the exchange slots alternate with the tile's parity).
       red[((t & 1) * 2 + half) * kRowsT + row] = mx;
@@ -444,13 +452,17 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
         l *= alpha;
         m = mx;
       }
-      float ps = 0.0f;
+      // p = 2^(sf * u - m); ex2(-inf) = +0, so masked scores need no test.
+      const uint64_t sf2 = f2_pack(sf, sf), nm2 = f2_pack(-m, -m);
+      uint64_t ps2 = f2_pack(0.0f, 0.0f);
 #pragma unroll
-      for (int e = 0; e < 64; e++) {  // ex2(-inf) = +0: masked scores need no test
-        sc[e] = ex2_approx(sc[e] - m);
-        ps += sc[e];
+      for (int e2 = 0; e2 < 32; e2++) {
+        const float2 a = f2_unpack(f2_fma(u2[e2], sf2, nm2));
+        u2[e2] = f2_pack(ex2_approx(a.x), ex2_approx(a.y));
+        ps2 = f2_add(ps2, u2[e2]);
       }
-      l += ps;
+      const float2 psum = f2_unpack(ps2);
+      l += psum.x + psum.y;
       // PV of tile t - 1 reads P' and accumulates O: wait for it before touching either.
       if (t > 0 && !dead &&
           !mbar_wait_bounded(pvdone + 8 * ((t - 1) & 1), static_cast<uint32_t>(((t - 1) >> 1) & 1), kWaitT))
@@ -479,17 +491,17 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
         const float4* s_v4 = reinterpret_cast<const float4*>(s_vb + (t & 1) * kTokT + 64 * half + 32 * c);
         uint32_t pp[32];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; c4++) {
-          const float4 va = s_v4[2 * c4], vb = s_v4[2 * c4 + 1];
-          const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+        for (int c4 = 0; c4 < 8; c4++) {
+          const float4 va = s_v4[c4];
+          const uint64_t x2[2] = {f2_mul(u2[16 * c + 2 * c4], f2_pack(va.x, va.y)),
+                                  f2_mul(u2[16 * c + 2 * c4 + 1], f2_pack(va.z, va.w))};
 #pragma unroll
-          for (int e2 = 0; e2 < 4; e2++) {
-            const int e = 8 * c4 + 2 * e2;
-            const float x0 = sc[32 * c + e] * vv[2 * e2];
-            const float x1 = sc[32 * c + e + 1] * vv[2 * e2 + 1];
-            const uint32_t hi2 = pack_bf16x2(x0, x1);
-            pp[e >> 1] = hi2;
-            pp[16 + (e >> 1)] = pack_bf16x2(x0 - bf16_lo(hi2), x1 - bf16_hi(hi2));
+          for (int j = 0; j < 2; j++) {
+            const float2 x = f2_unpack(x2[j]);
+            const uint32_t hi2 = pack_bf16x2(x.x, x.y);
+            const float2 lo = f2_unpack(f2_sub(x2[j], f2_pack(bf16_lo(hi2), bf16_hi(hi2))));
+            pp[2 * c4 + j] = hi2;
+            pp[16 + 2 * c4 + j] = pack_bf16x2(lo.x, lo.y);
           }
         }
         tmem_st32(lane_addr + kTokT * (t & 1) + 64 * half + 32 * c, pp);
