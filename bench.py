@@ -927,7 +927,9 @@ def run_prefill_bench(dev, reps=5, fmt=0):
             "note": "algorithmic FLOPs 4*128 per (query row, visible token); the kernel runs "
                     + ("QK^T as fp16 q hi+lo against the dequantised fp16 K stage and PV as "
                        "fp16 on mma.sync (NVFP4 cache)" if fmt else
-                       "QK^T as three int8 slices and PV as fp16 hi+lo on mma.sync")}
+                       "QK^T (q~ fp16 hi + lo against exact fp16 K codes) and PV (P' bf16 hi + lo "
+                       "against exact bf16 V codes) as tcgen05 MMAs, so the tensor cores execute twice "
+                       "the algorithmic FLOPs")}
 
 
 # ------------------------------------------------------------- CPU oracle arm --
