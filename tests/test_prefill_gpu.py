@@ -28,7 +28,7 @@ def test_prefill_workloads(name, lengths, chunks):
 
 
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
-@pytest.mark.parametrize("page_size", [16, 32, 64, 256])
+@pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])
 def test_prefill_group_and_page_size_grid(group, page_size):
     w = dataclasses.replace(W["qwen3_4b_decode"], num_kv_heads=2, num_q_heads=2 * group,
                             page_size=page_size, block=64)
