@@ -925,8 +925,9 @@ def run_prefill_bench(dev, reps=5, fmt=0):
             "workload": "chunked_prefill: 16 sequences x 512-token chunk after 3584 cached "
                         "tokens, Qwen3-4B heads (8 KV / 32 q), b = 128, page 16",
             "note": "algorithmic FLOPs 4*128 per (query row, visible token); the kernel runs "
-                    + ("QK^T as fp16 q hi+lo against the dequantised fp16 K stage and PV as "
-                       "fp16 on mma.sync (NVFP4 cache)" if fmt else
+                    + ("QK^T (q~ fp16 hi + lo against K dequantised exactly to fp16) and PV (p as "
+                       "fp16 hi + lo against V dequantised exactly to fp16) as tcgen05 MMAs (NVFP4 "
+                       "cache), twice the algorithmic FLOPs on the tensor cores" if fmt else
                        "QK^T (q~ fp16 hi + lo against exact fp16 K codes) and PV (P' bf16 hi + lo "
                        "against exact bf16 V codes) as tcgen05 MMAs, so the tensor cores execute twice "
                        "the algorithmic FLOPs")}

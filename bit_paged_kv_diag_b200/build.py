@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkvq.so")
 SOURCES = ["kvq_api.cu", "append_kernel.cu", "decode_kernel.cu", "kvq_noalloc.cu",
-           "prefill_kernel.cu", "prefill_tc.cu"]
+           "prefill_tc.cu"]
 HEADERS = ["kvq_internal.h", "kvq_ptx.cuh"]
 
 NVCC_FLAGS = [

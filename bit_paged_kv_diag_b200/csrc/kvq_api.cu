@@ -348,8 +348,7 @@ int kvq_prefill_attention(kvq_cache* c, int32_t layer, const void* q, const int3
   p.q_scale = static_cast<float>(sm * 1.4426950408889634);  // log2(e)
   p.cb = c->cb;
   p.fp4 = c->d.kv_format == KVQ_FORMAT_NVFP4;
-  const int rc = p.fp4 ? kvq::launch_prefill(p, total_q, static_cast<cudaStream_t>(stream))
-                       : kvq::launch_prefill_tc(p, total_q, static_cast<cudaStream_t>(stream));
+  const int rc = kvq::launch_prefill_tc(p, total_q, static_cast<cudaStream_t>(stream));
   if (rc == -1) return KVQ_EUNSUPPORTED;
   return rc == 0 ? KVQ_OK : KVQ_ECUDA;
 }

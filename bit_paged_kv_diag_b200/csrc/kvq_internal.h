@@ -105,8 +105,7 @@ struct PrefillParams {
 // Host-side launchers (return 0 on success, <0 on an unsupported shape or a launch
 // error).
 int launch_append(const AppendParams& p, int block, int num_sms, cudaStream_t stream);
-int launch_prefill(const PrefillParams& p, int total_q, cudaStream_t stream);
-// Chunked prefill on the 5th-generation tensor cores (INT4 cache).
+// Chunked prefill on the 5th-generation tensor cores (INT4 and NVFP4 caches).
 int launch_prefill_tc(const PrefillParams& p, int total_q, cudaStream_t stream);
 
 struct DecodeLaunch {

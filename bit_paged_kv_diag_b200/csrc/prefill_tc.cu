@@ -72,7 +72,6 @@ constexpr int kExpThreads = 32 * kExpWarps;
 constexpr int kMmaWarp = 12;    // issues the tcgen05 MMAs
 constexpr int kProdWarp = 13;   // reads the page table and issues the bulk copies
 constexpr int kThreadsT = 512;  // warps 14-15 only pad the last warpgroup
-constexpr int kStagesT = 4;     // raw page-data slots
 constexpr uint64_t kWaitT = 2000000000ull;
 constexpr float kLazyT = 8.0f;  // frame slack in log2 units: p <= 2^8 between rescales
 constexpr unsigned kFullT = 0xffffffffu;
@@ -92,24 +91,37 @@ constexpr int kQh = kKs;                        // [2 kb][128 rows][128 B] fp16 
 constexpr int kQl = kQh + 2 * kRowsT * 128;     // same, lo
 constexpr int kVs = kKs + 2 * kKsBuf;           // [2 buffers][2 nb][128 tokens][128 B] bf16 V codes
 constexpr int kVsBuf = 2 * kTokT * 128;
-constexpr int kRing = kVs + 2 * kVsBuf;         // [4][128 token rows of 132 B]
-constexpr int kSlotT = kTokT * 132;
-constexpr int kScl = kRing + kStagesT * kSlotT; // K scales [2][128], V scales [2][128] fp32
-constexpr int kSfr = kScl + 4 * kTokT * 4;      // row scales [128] fp32
-constexpr int kRed = kSfr + kRowsT * 4;         // maxima [2][2][128], sums [2][128] fp32
-constexpr int kBar = kRed + 6 * kRowsT * 4;     // mbarriers, see kBar* below
+constexpr int kRing = kVs + 2 * kVsBuf;         // raw page-data slots, see TcFmt
 constexpr int kBarFull = 0, kBarEmpty = 4, kBarKReady = 8, kBarVReady = 10, kBarSFull = 12,
               kBarSFree = 14, kBarPReady = 16, kBarPVDone = 17, kNumBars = 19;
-constexpr int kTmemSlot = kBar + kNumBars * 8;  // tensor-memory base address
-constexpr int kPreq = kTmemSlot + 16;           // query-block prefix [batch + 1]
 static_assert(kQl + 2 * kRowsT * 128 <= kVs, "q~ staging fits the K buffers");
-static_assert(kPreq + 4097 * 4 + 1024 + 1024 <= 232448, "shared memory of the largest batch");
+
+// What depends on the cache format: a (token, KV head) row is 132 B in INT4 ([64 B K codes]
+// [64 B V codes] and one fp16 scale each) and 144 B in NVFP4 (the same codes, then 8 E4M3
+// block scales each); the raw slots (4 INT4, 3 NVFP4) and the rest of the map follow.
+template <bool FP4>
+struct TcFmt {
+  static constexpr int kRowB = FP4 ? 144 : 132;
+  static constexpr int kScB = FP4 ? 8 : 2;        // scale bytes per token, K or V
+  static constexpr int kStages = FP4 ? 3 : 4;
+  static constexpr int kSlot = kTokT * kRowB;     // [128 token rows] in page-block layout
+  static constexpr int kScl = kRing + kStages * kSlot;  // K [2][128], V [2][128] fp32 multipliers
+  static constexpr int kSfr = kScl + 4 * kTokT * 4;     // row scales [128] fp32
+  static constexpr int kRed = kSfr + kRowsT * 4;        // maxima [2][2][128], sums [2][128]
+  static constexpr int kBar = kRed + 6 * kRowsT * 4;    // mbarriers, see kBar* above
+  static constexpr int kTmemSlot = kBar + kNumBars * 8; // tensor-memory base address
+  static constexpr int kPreq = kTmemSlot + 16;          // query-block prefix [batch + 1]
+  static_assert(kStages <= 4, "four full / empty barriers");
+  static_assert(kPreq + 4097 * 4 + 1024 + 1024 <= 232448, "shared memory of the largest batch");
+};
 
 // Instruction descriptors (kind::f16): fp32 accumulator, M = 128.
-//   QK^T: A, B fp16, both K-major, N = 128.  PV: A, B bf16, A K-major, B MN-major, N = 128.
+//   QK^T: A, B fp16, both K-major, N = 128.  PV: A, B bf16 (INT4) or fp16 (NVFP4), A K-major,
+//   B MN-major, N = 128.
 constexpr uint32_t kIdescQK = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) |
                               ((128u >> 4) << 24);
+constexpr uint32_t kIdescPVh = (1u << 4) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
 // Byte offset of the 16-byte chunk `chunk` of row `row` in a 128-byte swizzled operand.
 __device__ __forceinline__ uint32_t sw_off(int row, int chunk) {
@@ -123,7 +135,7 @@ __device__ __forceinline__ uint32_t sw_off(int row, int chunk) {
 // every lane the one page); issue_tile_pages checks it (an id out of range flags
 // KVQ_DEV_BAD_PAGE and reads page 0) and starts the copies into a slot with completion on its
 // barrier.
-template <int SEFF>
+template <int SEFF, bool FP4>
 __device__ __forceinline__ int tile_page(int t, int b, int L, int lane, const PrefillParams& p) {
   const int sh = p.page_shift;
   const int t0 = t * kTokT;
@@ -133,7 +145,7 @@ __device__ __forceinline__ int tile_page(int t, int b, int L, int lane, const Pr
   return __ldg(p.page_table + static_cast<size_t>(b) * p.max_pages_per_seq + (t0 >> sh) + (npg > 1 ? lane : 0));
 }
 
-template <int SEFF>
+template <int SEFF, bool FP4>
 __device__ __forceinline__ void issue_tile_pages(int t, int h, int L, int pid, uint32_t slot, uint32_t bar,
                                                  int lane, uint64_t pol, const PrefillParams& p) {
   const int S = p.page_size, sh = p.page_shift;
@@ -144,7 +156,7 @@ __device__ __forceinline__ void issue_tile_pages(int t, int h, int L, int pid, u
     pid = 0;
   }
   if (SEFF < kTokT || S == kTokT) {
-    const uint32_t blk_bytes = static_cast<uint32_t>(S) * 132u;
+    const uint32_t blk_bytes = static_cast<uint32_t>(S) * TcFmt<FP4>::kRowB;
     const int npg = ((t1 - 1) >> sh) - (t0 >> sh) + 1;
     if (lane == 0) mbar_arrive_expect_tx(bar, npg * blk_bytes);
     __syncwarp();
@@ -155,15 +167,20 @@ __device__ __forceinline__ void issue_tile_pages(int t, int h, int L, int pid, u
   } else {
     // Pages of 128+ tokens: the tile is part of one page; lanes 0-3 copy its K codes, V
     // codes, K scales and V scales.
-    const size_t blk_bytes = static_cast<size_t>(S) * 132u;
+    constexpr int sb = TcFmt<FP4>::kScB;
+    const size_t blk_bytes = static_cast<size_t>(S) * TcFmt<FP4>::kRowB;
     const size_t o = static_cast<size_t>(t0 & (S - 1));
     const uint8_t* blk = p.pool_layer + (static_cast<size_t>(pid) * p.num_kv_heads + h) * blk_bytes;
     const uint8_t* src = blk + o * 64;
     uint32_t dst = slot, bytes = kTokT * 64;
     if (lane == 1) { src = blk + static_cast<size_t>(S) * 64 + o * 64; dst = slot + kTokT * 64; }
-    if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * 2; dst = slot + kTokT * 128; bytes = kTokT * 2; }
-    if (lane == 3) { src = blk + static_cast<size_t>(S) * 130 + o * 2; dst = slot + kTokT * 130; bytes = kTokT * 2; }
-    if (lane == 0) mbar_arrive_expect_tx(bar, kSlotT);
+    if (lane == 2) { src = blk + static_cast<size_t>(S) * 128 + o * sb; dst = slot + kTokT * 128; bytes = kTokT * sb; }
+    if (lane == 3) {
+      src = blk + static_cast<size_t>(S) * (128 + sb) + o * sb;
+      dst = slot + kTokT * (128 + sb);
+      bytes = kTokT * sb;
+    }
+    if (lane == 0) mbar_arrive_expect_tx(bar, TcFmt<FP4>::kSlot);
     __syncwarp();
     if (lane < 4) bulk_copy_g2s(dst, src, bytes, bar, pol);
   }
@@ -188,6 +205,57 @@ __device__ __forceinline__ uint32_t codes_bf16x2(uint32_t lo, uint32_t hi, int k
   return x;
 }
 
+// NVFP4: one byte of two E2M1 codes (low nibble first) -> fp16x2; two E4M3 bytes -> fp16x2.
+// Both exact (the formats' values are fp16 values).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2_t(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+      : "=r"(r)
+      : "r"(byte));
+  return r;
+}
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_t(uint32_t b) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(b)));
+  return h;
+}
+__device__ __forceinline__ uint32_t hmul2_t(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// NVFP4 row half: channels 64 hf..64 hf + 63 of K (kv 0) or V (kv 1) of token row jr of a
+// virtual page, dequantised to fp16 (E2M1 value x E4M3 block scale has at most 6 significant
+// bits and lies in [2^-10, 2688]: exact) into row ej of a 128-byte swizzled operand tile.
+// A token past the sequence's end takes scale 0, so its (arbitrary) bytes become zeros.
+template <int SEFF>
+__device__ __forceinline__ void expand_fp4_half(const uint8_t* pg, int jr, int kv, int hf, bool live,
+                                                uint8_t* dst, int ej) {
+  const uint4* src = reinterpret_cast<const uint4*>(pg + kv * SEFF * 64 + jr * 64 + 32 * hf);
+  const uint4 c0 = src[0], c1 = src[1];
+  const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const uint32_t sc = live ? *reinterpret_cast<const uint32_t*>(pg + SEFF * 128 + kv * SEFF * 8 + jr * 8 + 4 * hf)
+                           : 0u;
+  const uint32_t s01 = e4m3x2_to_f16x2_t(sc & 0xFFFFu), s23 = e4m3x2_to_f16x2_t(sc >> 16);
+  const uint32_t sdup[4] = {prmt(s01, s01, 0x1010u), prmt(s01, s01, 0x3232u), prmt(s23, s23, 0x1010u),
+                            prmt(s23, s23, 0x3232u)};  // blocks 4 hf .. 4 hf + 3, both halves
+#pragma unroll
+  for (int ch = 0; ch < 8; ch++) {  // 16-byte chunk ch = channels 64 hf + 8 ch .. + 7, block ch / 2
+    uint32_t hv[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) hv[k] = hmul2_t(e2m1x2_to_f16x2_t(cw[ch] >> (8 * k)), sdup[ch >> 1]);
+    *reinterpret_cast<uint4*>(dst + sw_off(ej, ch)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(a), "f"(b));
@@ -196,20 +264,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-template <int G, int SEFF>
+template <int G, int SEFF, bool FP4>
 __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams p) {
+  using F = TcFmt<FP4>;
   constexpr int QB = kRowsT / G;  // chunk tokens per CTA
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
-  float* s_kb = reinterpret_cast<float*>(smem + kScl);  // [2][64] K scales of tiles t even / odd
+  float* s_kb = reinterpret_cast<float*>(smem + F::kScl);  // [2][64] K scales of tiles t even / odd
   float* s_vb = s_kb + 2 * kTokT;                       // [2][64] V scales
-  float* sfr = reinterpret_cast<float*>(smem + kSfr);
-  float* red = reinterpret_cast<float*>(smem + kRed);  // [tile parity][half][row] maxima
+  float* sfr = reinterpret_cast<float*>(smem + F::kSfr);
+  float* red = reinterpret_cast<float*>(smem + F::kRed);  // [tile parity][half][row] maxima
   float* lsum = red + 4 * kRowsT;                      // [half][row] final sums
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTmemSlot);
-  int32_t* preq = reinterpret_cast<int32_t*>(smem + kPreq);
-  const uint32_t bar0 = sbase + kBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F::kTmemSlot);
+  int32_t* preq = reinterpret_cast<int32_t*>(smem + F::kPreq);
+  const uint32_t bar0 = sbase + F::kBar;
   const uint32_t full_s = bar0 + 8 * kBarFull, empty_s = bar0 + 8 * kBarEmpty, kready = bar0 + 8 * kBarKReady,
                  vready = bar0 + 8 * kBarVReady, sfull = bar0 + 8 * kBarSFull,
                  sfree = bar0 + 8 * kBarSFree, pready = bar0 + 8 * kBarPReady,
@@ -222,7 +291,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   // call); q, the pool and out are touched after it.
   griddep_launch_dependents();
   if (tid == 0) {
-    for (int k = 0; k < kStagesT; k++) {
+    for (int k = 0; k < F::kStages; k++) {
       mbar_init(full_s + 8 * k, 1);
       mbar_init(empty_s + 8 * k, kExpThreads);
     }
@@ -293,10 +362,10 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
     tmem_relinquish();
   }
   griddep_wait();
-  // The producer warp starts the first kStagesT tiles' copies.
+  // The producer warp starts the copies of the first tiles, one per raw slot.
   if (w == kProdWarp) {
-    for (int t = 0; t < kStagesT && t < ntile; t++)
-      issue_tile_pages<SEFF>(t, h, L, tile_page<SEFF>(t, b, L, lane, p), sbase + kRing + t * kSlotT,
+    for (int t = 0; t < F::kStages && t < ntile; t++)
+      issue_tile_pages<SEFF, FP4>(t, h, L, tile_page<SEFF, FP4>(t, b, L, lane, p), sbase + kRing + t * F::kSlot,
                              full_s + 8 * t, lane, pol, p);
   }
 
@@ -498,10 +567,18 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
 #pragma unroll
           for (int j = 0; j < 2; j++) {
             const float2 x = f2_unpack(x2[j]);
-            const uint32_t hi2 = pack_bf16x2(x.x, x.y);
-            const float2 lo = f2_unpack(f2_sub(x2[j], f2_pack(bf16_lo(hi2), bf16_hi(hi2))));
-            pp[2 * c4 + j] = hi2;
-            pp[16 + 2 * c4 + j] = pack_bf16x2(lo.x, lo.y);
+            if constexpr (FP4) {  // P' = p <= 256 as fp16 hi + lo (V carries its scales)
+              const uint32_t hi2 = pack_f16x2(x.x, x.y);
+              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hi2));
+              const float2 lo = f2_unpack(f2_sub(x2[j], f2_pack(hf.x, hf.y)));
+              pp[2 * c4 + j] = hi2;
+              pp[16 + 2 * c4 + j] = pack_f16x2(lo.x, lo.y);
+            } else {
+              const uint32_t hi2 = pack_bf16x2(x.x, x.y);
+              const float2 lo = f2_unpack(f2_sub(x2[j], f2_pack(bf16_lo(hi2), bf16_hi(hi2))));
+              pp[2 * c4 + j] = hi2;
+              pp[16 + 2 * c4 + j] = pack_bf16x2(lo.x, lo.y);
+            }
           }
         }
         tmem_st32(lane_addr + kTokT * (t & 1) + 64 * half + 32 * c, pp);
@@ -580,8 +657,8 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       if (t < ntile) {
         // K of tile t into K buffer t & 1 (free once the softmax of tile t - 2 has read S and
         // the K scales, which also means QK^T of t - 2 has completed).
-        const int slot = t % kStagesT;
-        if (!dead && !mbar_wait_bounded(full_s + 8 * slot, static_cast<uint32_t>((t / kStagesT) & 1), kWaitT))
+        const int slot = t % F::kStages;
+        if (!dead && !mbar_wait_bounded(full_s + 8 * slot, static_cast<uint32_t>((t / F::kStages) & 1), kWaitT))
           dead = true;
         if (t >= 2 && !dead &&
             !mbar_wait_bounded(sfree + 8 * (t & 1), static_cast<uint32_t>(((t - 2) >> 1) & 1), kWaitT))
@@ -590,8 +667,14 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
 #pragma unroll
           for (int it = 0; it < 2; it++) {
             const int ej = ej0 + 64 * it;
-            const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
+            const uint8_t* pg = smem + kRing + slot * F::kSlot + (ej / SEFF) * (SEFF * F::kRowB);
             const int jr = ej % SEFF;
+            if constexpr (FP4) {
+              const bool live = t * kTokT + ej < L;
+              expand_fp4_half<SEFF>(pg, jr, 0, ehf, live, smem + kKs + (t & 1) * kKsBuf + ehf * (kTokT * 128), ej);
+              if (ehf == 0) s_kb[(t & 1) * kTokT + ej] = live ? 1.0f : 0.0f;
+              continue;
+            }
             const uint4* src = reinterpret_cast<const uint4*>(pg + jr * 64 + 32 * ehf);
             const uint4 c0 = src[0], c1 = src[1];
             const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -614,17 +697,32 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       if (t >= 1) {
         // V of tile u = t - 1 into V buffer u & 1 (free once PV of u - 2 has completed,
         // which also means the softmax of u - 2 has read its V scales).
-        const int u = t - 1, slot = u % kStagesT;
+        const int u = t - 1, slot = u % F::kStages;
         if (u >= 2 && !dead &&
             !mbar_wait_bounded(pvdone + 8 * (u & 1), static_cast<uint32_t>(((u - 2) >> 1) & 1), kWaitT))
           dead = true;
-        if (!dead) {
+        if (FP4 && !dead) {
+#pragma unroll
+          for (int it = 0; it < 2; it++) {
+            const int ej = ej0 + 64 * it;
+            const uint8_t* pg = smem + kRing + slot * F::kSlot + (ej / SEFF) * (SEFF * F::kRowB);
+            const bool live = u * kTokT + ej < L;
+            expand_fp4_half<SEFF>(pg, ej % SEFF, 1, ehf, live, smem + kVs + (u & 1) * kVsBuf + ehf * (kTokT * 128),
+                                  ej);
+            if (ehf == 0) s_vb[(u & 1) * kTokT + ej] = live ? 1.0f : 0.0f;
+          }
+          // The raw slot of tile u is fully read: the producer may refill it.
+          mbar_arrive(empty_s + 8 * slot);
+          fence_proxy_async_smem();
+          mbar_arrive(vready + 8 * (u & 1));
+        }
+        if (!FP4 && !dead) {
           uint32_t cw[2][8];
           float vs[2] = {0.0f, 0.0f};
 #pragma unroll
           for (int it = 0; it < 2; it++) {
             const int ej = ej0 + 64 * it;
-            const uint8_t* pg = smem + kRing + slot * kSlotT + (ej / SEFF) * (SEFF * 132);
+            const uint8_t* pg = smem + kRing + slot * F::kSlot + (ej / SEFF) * (SEFF * F::kRowB);
             const int jr = ej % SEFF;
             const uint4* src = reinterpret_cast<const uint4*>(pg + SEFF * 64 + jr * 64 + 32 * ehf);
             const uint4 c0 = src[0], c1 = src[1];
@@ -695,8 +793,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
           for (int s = 0; s < 8; s++) {  // k-step s: tokens 16 s.., P' of half s / 4, chunk (s / 2) % 2
             const uint64_t vd = dv + static_cast<uint64_t>((2048u * s) >> 4);
             const uint32_t pa = tmem + kTokT * (u & 1) + 32 * (s >> 1) + 8 * (s & 1);
-            tc_mma_f16_ts(tmem + kColO, pa, vd, kIdescPV, (u > 0 || s > 0) ? 1u : 0u);
-            tc_mma_f16_ts(tmem + kColO, pa + 16, vd, kIdescPV, 1u);
+            constexpr uint32_t idesc = FP4 ? kIdescPVh : kIdescPV;
+            tc_mma_f16_ts(tmem + kColO, pa, vd, idesc, (u > 0 || s > 0) ? 1u : 0u);
+            tc_mma_f16_ts(tmem + kColO, pa + 16, vd, idesc, 1u);
           }
           tc_commit(pvdone + 8 * (u & 1));
         }
@@ -711,21 +810,21 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
     }
   } else if (w == kProdWarp) {
     // ----------------------------------------------------------------- producer warp --
-    // Tile t (t >= kStagesT) refills slot t % kStagesT once the expansion has released tile
-    // t - kStagesT; its page ids are read one tile ahead, so the read overlaps that wait.
-    int issued = min(kStagesT, ntile);
-    int pid_next = kStagesT < ntile ? tile_page<SEFF>(kStagesT, b, L, lane, p) : 0;
-    for (int t = kStagesT; t < ntile && !dead; t++) {
-      const int pid_after = t + 1 < ntile ? tile_page<SEFF>(t + 1, b, L, lane, p) : 0;
-      const int slot = t % kStagesT;
+    // Tile t refills slot t % kStages once the expansion has released tile t - kStages; its
+    // page ids are read one tile ahead, so the read overlaps that wait.
+    int issued = min(F::kStages, ntile);
+    int pid_next = F::kStages < ntile ? tile_page<SEFF, FP4>(F::kStages, b, L, lane, p) : 0;
+    for (int t = F::kStages; t < ntile && !dead; t++) {
+      const int pid_after = t + 1 < ntile ? tile_page<SEFF, FP4>(t + 1, b, L, lane, p) : 0;
+      const int slot = t % F::kStages;
       // Lane 0 waits and tells the others, so the warp stays converged for the copies.
       bool ok = true;
-      if (lane == 0) ok = mbar_wait_bounded(empty_s + 8 * slot, static_cast<uint32_t>((t / kStagesT - 1) & 1), kWaitT);
+      if (lane == 0) ok = mbar_wait_bounded(empty_s + 8 * slot, static_cast<uint32_t>((t / F::kStages - 1) & 1), kWaitT);
       if (!__shfl_sync(kFullT, ok, 0)) {
         dead = true;
         break;
       }
-      issue_tile_pages<SEFF>(t, h, L, pid_next, sbase + kRing + slot * kSlotT, full_s + 8 * slot, lane, pol, p);
+      issue_tile_pages<SEFF, FP4>(t, h, L, pid_next, sbase + kRing + slot * F::kSlot, full_s + 8 * slot, lane, pol, p);
       issued++;
       pid_next = pid_after;
     }
@@ -733,8 +832,8 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
     // Before shared memory is released, the last copies into each slot must have landed
     // (bounded; earlier ones were consumed by the expansion before their slot was reused).
     if (lane == 0)
-      for (int j = max(0, issued - kStagesT); j < issued; j++)
-        mbar_wait_bounded(full_s + 8 * (j % kStagesT), static_cast<uint32_t>((j / kStagesT) & 1), kWaitT);
+      for (int j = max(0, issued - F::kStages); j < issued; j++)
+        mbar_wait_bounded(full_s + 8 * (j % F::kStages), static_cast<uint32_t>((j / F::kStages) & 1), kWaitT);
   }
   tc_fence_before();
   __syncthreads();
@@ -742,43 +841,45 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   if (w == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int G>
+template <int G, bool FP4>
 void* prefill_tc_ptr(int seff) {
-  if (seff == 16) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 16>);
-  if (seff == 32) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 32>);
-  if (seff == 64) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 64>);
-  if (seff == 128) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 128>);
+  if (seff == 16) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 16, FP4>);
+  if (seff == 32) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 32, FP4>);
+  if (seff == 64) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 64, FP4>);
+  if (seff == 128) return reinterpret_cast<void*>(&prefill_tc_kernel<G, 128, FP4>);
   return nullptr;
 }
 
+template <bool FP4>
 void* pick_prefill_tc(int group, int seff) {
   switch (group) {
-    case 1: return prefill_tc_ptr<1>(seff);
-    case 2: return prefill_tc_ptr<2>(seff);
-    case 4: return prefill_tc_ptr<4>(seff);
-    case 8: return prefill_tc_ptr<8>(seff);
+    case 1: return prefill_tc_ptr<1, FP4>(seff);
+    case 2: return prefill_tc_ptr<2, FP4>(seff);
+    case 4: return prefill_tc_ptr<4, FP4>(seff);
+    case 8: return prefill_tc_ptr<8, FP4>(seff);
     default: return nullptr;
   }
 }
 
-size_t prefill_tc_smem(int max_batch) {
-  return static_cast<size_t>(kPreq) + static_cast<size_t>(max_batch + 1) * sizeof(int32_t) + 1024;
+size_t prefill_tc_smem(int max_batch, bool fp4) {
+  const int preq = fp4 ? TcFmt<true>::kPreq : TcFmt<false>::kPreq;
+  return static_cast<size_t>(preq) + static_cast<size_t>(max_batch + 1) * sizeof(int32_t) + 1024;
 }
 
 }  // namespace
 
 int launch_prefill_tc(const PrefillParams& p, int total_q, cudaStream_t stream) {
   const int seff = p.page_size < kTokT ? p.page_size : kTokT;
-  void* fn = pick_prefill_tc(p.group, seff);
+  void* fn = p.fp4 ? pick_prefill_tc<true>(p.group, seff) : pick_prefill_tc<false>(p.group, seff);
   if (!fn) return -1;
   if (p.batch == 0 || total_q == 0) return 0;
   const int QB = kRowsT / p.group;
   const long long blocks = (static_cast<long long>(total_q) + QB - 1) / QB + p.batch;
   const long long grid = blocks * p.num_kv_heads;
   if (grid > 0x7fffffffLL) return -1;
-  const size_t smem = prefill_tc_smem(p.batch);
+  const size_t smem = prefill_tc_smem(p.batch, p.fp4 != 0);
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(prefill_tc_smem(4096))) != cudaSuccess)
+                           static_cast<int>(prefill_tc_smem(4096, p.fp4 != 0))) != cudaSuccess)
     return -2;
   PrefillParams q = p;
   q.total_q = total_q;

@@ -232,10 +232,9 @@ KVQ_API int kvq_append_decode_attention(kvq_cache* c, int32_t layer, const void*
  * at position seq_lens[b] - C_b + i, attends positions 0 .. seq_lens[b] - C_b + i.  The
  * pages' attention over the paged cache ("KVキャッシュを4ビットへ", section
  * "KVキャッシュこそが本当のボトルネックである理由") for the many-query case a serving
- * engine runs on the same cache; decode is the case C_b = 1.  On an INT4 cache the call
- * runs on the 5th-generation tensor cores (tcgen05 MMAs, S and O in tensor memory, one
- * CTA of 128 query rows per SM, 512 tensor-memory columns); on an NVFP4 cache on the
- * warp-level mma.sync path.
+ * engine runs on the same cache; decode is the case C_b = 1.  Runs on the 5th-generation
+ * tensor cores (tcgen05 MMAs, S and O in tensor memory, one CTA of 128 query rows per SM,
+ * 512 tensor-memory columns) for both cache formats.
  *   q              device fp16 [total_q][num_q_heads][128], the chunks concatenated in
  *                  order of b, 16-byte aligned
  *   cu_q           device int32 [batch+1], chunk offsets into q (cu_q[0] = 0)
