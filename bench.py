@@ -80,12 +80,13 @@ def append_bytes(tokens, num_kv_heads, row_bytes=132):
 BYTES_PER_TOKEN_HEAD_NVFP4 = 2 * 64 + 2 * 8
 
 # A write larger than the 126 MB L2 between timed calls whose inputs and outputs would fit.
-FLUSH_BYTES = 256 << 20
+FLUSH_BYTES = 512 << 20
 
 
 def _timed_calls(fn, reps, flush=None):
-    """Mean device time (ms) of fn() over reps calls, events around each call on the
-    current stream; with flush, a write of that buffer before every call (not timed)."""
+    """Median device time (ms) of fn() over reps calls, events around each call on the
+    current stream; with flush, a write of that buffer (512 MB, four times L2) before every
+    call, not timed."""
     import torch
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(reps)]
@@ -96,7 +97,7 @@ def _timed_calls(fn, reps, flush=None):
         fn()
         b.record()
     torch.cuda.synchronize()
-    return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    return float(np.median([a.elapsed_time(b) for a, b in ev]))
 
 
 # --------------------------------------------------------------------- clocks --
@@ -534,8 +535,9 @@ def run_append_bench(dev, reps=20):
         cache.close()
     res["workload"] = ("prefill_append: 8 x 8192 tokens, 8 KV heads, page 16, Student-t(3); "
                        "b1 = plain INT4 (no rotation)")
-    res["timing"] = ("events around each call, a 256 MB write between calls (flushes the "
-                     "126 MB L2)")
+    res["timing"] = ("median of 20 calls, events around each, a 512 MB write between calls "
+                     "(flushes the 126 MB L2; its dirty lines are written back during the next "
+                     "call)")
     res["traffic"] = _traffic("append", append_bytes(T, H))
     return res
 

@@ -12,12 +12,14 @@
 // consecutive chunk tokens times the G query heads of the KV head.  Row r is lane r of tensor
 // memory.  The CTA's 16 warps specialise and hand work to one another through mbarriers, so
 // the softmax, the code expansion and the tensor cores overlap instead of taking turns:
-//   warps 0-7    softmax: warps w and w + 4 both read the lanes of rows 32(w % 4).., warp w
-//                the first half of each tile's columns and of O, warp w + 4 the second;
-//   warps 8-11   expansion: the K and V codes of a tile into the MMA operand tiles, plus
+//   warps 0-15   softmax: warps q, q + 4, q + 8, q + 12 all read the lanes of rows 32q..,
+//                warp q + 4j the j-th 32 columns of each tile and of O (four threads per
+//                row: the special-function unit's exponentials and the other phases of
+//                the warps sharing an SMSP overlap better than with two);
+//   warps 16-19  expansion: the K and V codes of a tile into the MMA operand tiles, plus
 //                their scales;
-//   warp 12      one lane issues the MMAs: QK^T of tile t, then PV of tile t - 1;
-//   warp 13      reads the page table and issues the bulk copies of the raw page data.
+//   warp 20      one lane issues the MMAs: QK^T of tile t, then PV of tile t - 1;
+//   warp 21      reads the page table and issues the bulk copies of the raw page data.
 // Tensor-core time per instruction hardly depends on N up to 128 here, so the tiles are as
 // wide as the accumulators allow (S of two tiles, O and q~ fill the 512 TMEM columns).
 // S (tensor memory), the K and V operand tiles and the scales are double-buffered by tile
@@ -28,11 +30,11 @@
 //         in tensor memory for the whole CTA; B = the K codes as exact fp16 integers in shared
 //         memory; both parts accumulate into one fp32 tile S in tensor memory.  The K scale
 //         and the row's M_r / 2^14 multiply the scores.
-//   softmax  each thread loads its half row of S (tcgen05.ld), applies the causal mask; the two
-//         halves' maxima meet in shared memory; the row keeps an online maximum m and sum l in
-//         the log2 domain.  The frame m moves only when a
-//         score exceeds it by more than 8 (then the row of O is rescaled in tensor memory),
-//         so p = 2^(score - m) <= 256 and the rescale is rare.
+//   softmax  each thread loads its quarter row of S (tcgen05.ld), applies the causal mask;
+//         the four quarters' maxima meet in shared memory; the row keeps an online maximum m
+//         and sum l in the log2 domain.  The frame m moves only when a score exceeds it by
+//         more than 8 (then the row of O is rescaled in tensor memory), so
+//         p = 2^(score - m) <= 256 and the rescale is rare.
 //   PV    tcgen05.mma kind::f16 in bf16, M = 128 rows, N = 128 channels, K = 128 tokens: A =
 //         P' = p * s_v (the V scale folded into the probabilities) as bf16 hi + lo parts (bf16
 //         keeps fp32's range, so P' <= 256 * s_v cannot overflow), written by each softmax
@@ -40,9 +42,10 @@
 //         read channel-major from shared memory; the accumulator O stays in tensor memory.
 // With both A operands in tensor memory the tensor cores read only K and V from shared
 // memory, whose bandwidth the MMAs would otherwise share with the expansion.
-// The end: each thread loads its half row of O, divides by l, applies the inverse block
-// Hadamard (stages inside a half in registers, the stage across the halves through shared
-// memory), times c_b, stores fp16.
+// The end: each thread loads its quarter row of O, divides by l, applies the inverse block
+// Hadamard (stages inside a quarter in registers, the two stages across quarters through
+// shared memory), times c_b, stores fp16.  On the NVFP4 cache the expansion dequantises K
+// and V exactly to fp16 (block scales folded in), and PV runs in fp16 with P' = p.
 //
 // Shared-memory operands use the 128-byte swizzle of the tensor core's canonical layouts: 8
 // rows of 128 bytes per 1024-byte atom, the 16-byte chunk index XOR the row within the atom.
@@ -64,14 +67,14 @@ namespace {
 constexpr int kD = 128;
 constexpr int kRowsT = 128;     // query rows per CTA (tensor-memory lanes)
 constexpr int kTokT = 128;      // KV tokens per tile
-constexpr int kSoftWarps = 8;   // warps w and w + 4 share the rows of TMEM lanes 32(w % 4)..
+constexpr int kSoftWarps = 16;  // warps q, q + 4, q + 8, q + 12 share the rows of TMEM lanes 32q..
 constexpr int kSoftThreads = 32 * kSoftWarps;
-constexpr int kExpWarp0 = 8;    // warps 8-11 expand K and V codes
+constexpr int kExpWarp0 = 16;   // warps 16-19 expand K and V codes
 constexpr int kExpWarps = 4;
 constexpr int kExpThreads = 32 * kExpWarps;
-constexpr int kMmaWarp = 12;    // issues the tcgen05 MMAs
-constexpr int kProdWarp = 13;   // reads the page table and issues the bulk copies
-constexpr int kThreadsT = 512;  // warps 14-15 only pad the last warpgroup
+constexpr int kMmaWarp = 20;    // issues the tcgen05 MMAs
+constexpr int kProdWarp = 21;   // reads the page table and issues the bulk copies
+constexpr int kThreadsT = 704;
 constexpr uint64_t kWaitT = 2000000000ull;
 constexpr float kLazyT = 8.0f;  // frame slack in log2 units: p <= 2^8 between rescales
 constexpr unsigned kFullT = 0xffffffffu;
@@ -107,8 +110,8 @@ struct TcFmt {
   static constexpr int kSlot = kTokT * kRowB;     // [128 token rows] in page-block layout
   static constexpr int kScl = kRing + kStages * kSlot;  // K [2][128], V [2][128] fp32 multipliers
   static constexpr int kSfr = kScl + 4 * kTokT * 4;     // row scales [128] fp32
-  static constexpr int kRed = kSfr + kRowsT * 4;        // maxima [2][2][128], sums [2][128]
-  static constexpr int kBar = kRed + 6 * kRowsT * 4;    // mbarriers, see kBar* above
+  static constexpr int kRed = kSfr + kRowsT * 4;        // maxima [2][4][128], sums [4][128]
+  static constexpr int kBar = kRed + 12 * kRowsT * 4;   // mbarriers, see kBar* above
   static constexpr int kTmemSlot = kBar + kNumBars * 8; // tensor-memory base address
   static constexpr int kPreq = kTmemSlot + 16;          // query-block prefix [batch + 1]
   static_assert(kStages <= 4, "four full / empty barriers");
@@ -274,8 +277,8 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   float* s_kb = reinterpret_cast<float*>(smem + F::kScl);  // [2][64] K scales of tiles t even / odd
   float* s_vb = s_kb + 2 * kTokT;                       // [2][64] V scales
   float* sfr = reinterpret_cast<float*>(smem + F::kSfr);
-  float* red = reinterpret_cast<float*>(smem + F::kRed);  // [tile parity][half][row] maxima
-  float* lsum = red + 4 * kRowsT;                      // [half][row] final sums
+  float* red = reinterpret_cast<float*>(smem + F::kRed);  // [tile parity][part][row] maxima
+  float* lsum = red + 8 * kRowsT;                         // [part][row] final sums
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + F::kTmemSlot);
   int32_t* preq = reinterpret_cast<int32_t*>(smem + F::kPreq);
   const uint32_t bar0 = sbase + F::kBar;
@@ -372,8 +375,8 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   // q rows: softmax warp w rotates and scales rows 16w..16w+15 (lane: channels 4 lane..
   // 4 lane + 3) and stores q~ = q' * 2^14 / M as fp16 hi + lo parts into the K-major operands.
   if (w < kSoftWarps) {
-    for (int rr = 0; rr < 16; rr++) {
-      const int row = 16 * w + rr;
+    for (int rr = 0; rr < kRowsT / kSoftWarps; rr++) {
+      const int row = (kRowsT / kSoftWarps) * w + rr;
       const int ti = tok_first + row / G, gq = row % G;
       float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       if (ti < C) {
@@ -428,21 +431,21 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool dead = false;
-  // q~ into tensor memory, the A operand of QK^T: softmax thread (row, half) moves channels
-  // 64 half..64 half + 63 of its row, hi and lo parts, as fp16 pairs.
+  // q~ into tensor memory, the A operand of QK^T: softmax thread (row, part) moves channels
+  // 32 part..32 part + 31 of its row, hi and lo parts, as fp16 pairs (16 columns each).
   if (w < kSoftWarps) {
-    const int row = 32 * (w & 3) + lane, half = w >> 2;
+    const int row = 32 * (w & 3) + lane, part = w >> 2;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * (w & 3)) << 16);
 #pragma unroll
-    for (int part = 0; part < 2; part++) {
-      uint32_t r[32];
-      const uint8_t* src = smem + (part ? kQl : kQh) + half * (kRowsT * 128);
+    for (int hl = 0; hl < 2; hl++) {
+      uint32_t r[16];
+      const uint8_t* src = smem + (hl ? kQl : kQh) + (part >> 1) * (kRowsT * 128);
 #pragma unroll
-      for (int ch = 0; ch < 8; ch++) {
-        const uint4 v = *reinterpret_cast<const uint4*>(src + sw_off(row, ch));
-        r[4 * ch] = v.x; r[4 * ch + 1] = v.y; r[4 * ch + 2] = v.z; r[4 * ch + 3] = v.w;
+      for (int c = 0; c < 4; c++) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + sw_off(row, 4 * (part & 1) + c));
+        r[4 * c] = v.x; r[4 * c + 1] = v.y; r[4 * c + 2] = v.z; r[4 * c + 3] = v.w;
       }
-      tmem_st32(lane_addr + (part ? kColQl : kColQh) + 32 * half, r);
+      tmem_st16(lane_addr + (hl ? kColQl : kColQh) + 16 * part, r);
     }
     tmem_wait_st();
   }
@@ -452,9 +455,10 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
 
   if (w < kSoftWarps) {
     // ---------------------------------------------------------------- softmax warps --
-    // This thread's row and half: tokens 32 half..32 half + 31 of every tile, channels
-    // 64 half..64 half + 63 of O.
-    const int quarter = w & 3, half = w >> 2;
+    // This thread's row and part: tokens 32 part..32 part + 31 of every tile, channels
+    // 32 part..32 part + 31 of O.  The four parts of a row are warps q, q + 4, q + 8, q + 12
+    // (q = the row's TMEM lane quarter); they meet at a 128-thread named barrier.
+    const int quarter = w & 3, part = w >> 2;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
     const int row = 32 * quarter + lane;
     const int ti_row = tok_first + row / G;
@@ -469,16 +473,15 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       if (!dead && !mbar_wait_bounded(sfull + 8 * (t & 1), par, kWaitT)) dead = true;
       if (!dead && !mbar_wait_bounded(kready + 8 * (t & 1), par, kWaitT)) dead = true;
       tc_fence_after();
-      // This thread's 64 tokens (64 half..): u = S * s_k, in pairs.  The row scale sf > 0
-      // commutes with the maximum, so the score sf * u is formed only inside the exponent.
-      uint32_t raw[64];
-      tmem_ld32(lane_addr + kTokT * (t & 1) + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(raw));
-      tmem_ld32(lane_addr + kTokT * (t & 1) + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
+      // u = S * s_k for this thread's 32 tokens, in pairs.  The row scale sf > 0 commutes
+      // with the maximum, so the score sf * u is formed only inside the exponent.
+      uint32_t raw[32];
+      tmem_ld32(lane_addr + kTokT * (t & 1) + 32 * part, raw);
       tmem_wait_ld();
-      uint64_t u2[32];
-      const float4* s_k4 = reinterpret_cast<const float4*>(s_kb + (t & 1) * kTokT + 64 * half);
+      uint64_t u2[16];
+      const float4* s_k4 = reinterpret_cast<const float4*>(s_kb + (t & 1) * kTokT + 32 * part);
 #pragma unroll
-      for (int e4 = 0; e4 < 16; e4++) {
+      for (int e4 = 0; e4 < 8; e4++) {
         const float4 k4 = s_k4[e4];
         u2[2 * e4] = f2_mul(f2_pack(__uint_as_float(raw[4 * e4]), __uint_as_float(raw[4 * e4 + 1])),
                             f2_pack(k4.x, k4.y));
@@ -492,9 +495,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       // beyond L either).
       if (t * kTokT + kTokT - 1 > L - C + tok_first) {
 #pragma unroll
-        for (int e2 = 0; e2 < 32; e2++) {
+        for (int e2 = 0; e2 < 16; e2++) {
           float2 v = f2_unpack(u2[e2]);
-          const int pos = t * kTokT + 64 * half + 2 * e2;
+          const int pos = t * kTokT + 32 * part + 2 * e2;
           if (pos > rpos) v.x = -CUDART_INF_F;
           if (pos + 1 > rpos) v.y = -CUDART_INF_F;
           u2[e2] = f2_pack(v.x, v.y);
@@ -502,17 +505,18 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       }
       float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
 #pragma unroll
-      for (int e2 = 0; e2 < 32; e2++) {
+      for (int e2 = 0; e2 < 16; e2++) {
         const float2 v = f2_unpack(u2[e2]);
         mx0 = fmaxf(mx0, v.x);
         mx1 = fmaxf(mx1, v.y);
       }
       float mx = fmaxf(mx0, mx1) * sf;
-      // The row's maximum over both halves (warps w and w + 4 meet at a 64-thread barrier;
-      // the exchange slots alternate with the tile's parity).
-      red[((t & 1) * 2 + half) * kRowsT + row] = mx;
-      asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
-      mx = fmaxf(mx, red[((t & 1) * 2 + (half ^ 1)) * kRowsT + row]);
+      // The row's maximum over its four parts (the exchange slots alternate with the tile's
+      // parity, so a slot is rewritten only after every part has passed the next barrier).
+      red[((t & 1) * 4 + part) * kRowsT + row] = mx;
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + quarter) : "memory");
+#pragma unroll
+      for (int q2 = 1; q2 < 4; q2++) mx = fmaxf(mx, red[((t & 1) * 4 + (part ^ q2)) * kRowsT + row]);
       // Lazy frame: move m only when a score exceeds it by more than kLazyT.
       float alpha = 1.0f;
       const bool move = mx > m + kLazyT;
@@ -525,7 +529,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
       const uint64_t sf2 = f2_pack(sf, sf), nm2 = f2_pack(-m, -m);
       uint64_t ps2 = f2_pack(0.0f, 0.0f);
 #pragma unroll
-      for (int e2 = 0; e2 < 32; e2++) {
+      for (int e2 = 0; e2 < 16; e2++) {
         const float2 a = f2_unpack(f2_fma(u2[e2], sf2, nm2));
         u2[e2] = f2_pack(ex2_approx(a.x), ex2_approx(a.y));
         ps2 = f2_add(ps2, u2[e2]);
@@ -537,37 +541,31 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
           !mbar_wait_bounded(pvdone + 8 * ((t - 1) & 1), static_cast<uint32_t>(((t - 1) >> 1) & 1), kWaitT))
         dead = true;
       tc_fence_after();
-      // Rescale this thread's half of O when a row of the warp moved after its first tile.
+      // Rescale this thread's part of O when a row of the warp moved after its first tile.
       if (__any_sync(kFullT, move && alpha != 0.0f) && t > 0) {
-#pragma unroll 1
-        for (int q2 = 0; q2 < 2; q2++) {
-          uint32_t o[32];
-          const uint32_t col = kColO + 64 * half + 32 * q2;
-          tmem_ld32(lane_addr + col, o);
-          tmem_wait_ld();
+        uint32_t o[32];
+        tmem_ld32(lane_addr + kColO + 32 * part, o);
+        tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; e++) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(lane_addr + col, o);
-        }
-        tmem_wait_st();
+        for (int e = 0; e < 32; e++) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        tmem_st32(lane_addr + kColO + 32 * part, o);
       }
-      // P' = p * s_v as bf16 hi + lo pairs over this thread's own S columns (the A operand
-      // of PV): 32-token chunk c at columns 64 half + 32 c, hi in [0, 16), lo in [16, 32)
-      // (V scales of tile t: vready).
+      // P' = p * s_v as hi + lo pairs over this thread's own S columns (the A operand of PV):
+      // columns 32 part + [0, 16) hi, + [16, 32) lo; bf16 on INT4, fp16 on NVFP4 (where V
+      // carries its scales and s_v = 1).  The V scales of tile t come with vready.
       if (!dead && !mbar_wait_bounded(vready + 8 * (t & 1), par, kWaitT)) dead = true;
-#pragma unroll
-      for (int c = 0; c < 2; c++) {
-        const float4* s_v4 = reinterpret_cast<const float4*>(s_vb + (t & 1) * kTokT + 64 * half + 32 * c);
+      {
+        const float4* s_v4 = reinterpret_cast<const float4*>(s_vb + (t & 1) * kTokT + 32 * part);
         uint32_t pp[32];
 #pragma unroll
         for (int c4 = 0; c4 < 8; c4++) {
           const float4 va = s_v4[c4];
-          const uint64_t x2[2] = {f2_mul(u2[16 * c + 2 * c4], f2_pack(va.x, va.y)),
-                                  f2_mul(u2[16 * c + 2 * c4 + 1], f2_pack(va.z, va.w))};
+          const uint64_t x2[2] = {f2_mul(u2[2 * c4], f2_pack(va.x, va.y)),
+                                  f2_mul(u2[2 * c4 + 1], f2_pack(va.z, va.w))};
 #pragma unroll
           for (int j = 0; j < 2; j++) {
             const float2 x = f2_unpack(x2[j]);
-            if constexpr (FP4) {  // P' = p <= 256 as fp16 hi + lo (V carries its scales)
+            if constexpr (FP4) {  // P' = p <= 256 as fp16 hi + lo
               const uint32_t hi2 = pack_f16x2(x.x, x.y);
               const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hi2));
               const float2 lo = f2_unpack(f2_sub(x2[j], f2_pack(hf.x, hf.y)));
@@ -581,7 +579,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
             }
           }
         }
-        tmem_st32(lane_addr + kTokT * (t & 1) + 64 * half + 32 * c, pp);
+        tmem_st32(lane_addr + kTokT * (t & 1) + 32 * part, pp);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -593,31 +591,32 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
     tc_fence_after();
     if (dead && lane == 0) atomicOr(p.status, KVQ_DEV_TIMEOUT_BIT);
 
-    // o'/l of this half row (the row sum meets the other half's in shared memory).
-    lsum[half * kRowsT + row] = l;
-    float o[64];
-#pragma unroll
-    for (int q2 = 0; q2 < 2; q2++) {
+    // o'/l of this part of the row (the row sum gathers the four parts' in shared memory).
+    lsum[part * kRowsT + row] = l;
+    float o[32];
+    {
       uint32_t r[32];
-      tmem_ld32(lane_addr + kColO + 64 * half + 32 * q2, r);
+      tmem_ld32(lane_addr + kColO + 32 * part, r);
       tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; e++) o[32 * q2 + e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 32; e++) o[e] = __uint_as_float(r[e]);
     }
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
-    const float lt = l + lsum[(half ^ 1) * kRowsT + row];
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + quarter) : "memory");
+    float lt = 0.0f;
+#pragma unroll
+    for (int q2 = 0; q2 < 4; q2++) lt += lsum[q2 * kRowsT + row];
     const float il = lt > 0.0f ? __frcp_rn(lt) : 0.0f;
 #pragma unroll
-    for (int e = 0; e < 64; e++) o[e] *= il;
-    // Inverse block Hadamard: stages h = 1..32 inside the half, h = 64 across the halves
-    // (through the q operand area, free once the last QK^T has completed; channel-major so a
+    for (int e = 0; e < 32; e++) o[e] *= il;
+    // Inverse block Hadamard: stages h = 1..16 inside the part, h = 32 and 64 across parts
+    // (through the K buffers, free once the last QK^T has completed; channel-major so a
     // warp's accesses are contiguous).
     const int block = p.hadamard_block;
 #pragma unroll
-    for (int hh = 1; hh < 64; hh *= 2) {
+    for (int hh = 1; hh < 32; hh *= 2) {
       if (hh < block) {
 #pragma unroll
-        for (int i = 0; i < 64; i++)
+        for (int i = 0; i < 32; i++)
           if (!(i & hh)) {
             const float a = o[i], d = o[i + hh];
             o[i] = a + d;
@@ -625,22 +624,27 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
           }
       }
     }
-    if (block == 128) {
-      float* xch = reinterpret_cast<float*>(smem + kQh);  // [half][64 channels][128 rows]
+    float* xch = reinterpret_cast<float*>(smem + kQh);  // [part][32 channels][128 rows]
 #pragma unroll
-      for (int e = 0; e < 64; e++) xch[(half * 64 + e) * kRowsT + row] = o[e];
-      asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+    for (int st = 0; st < 2; st++) {
+      const int hp = 1 << st;  // partner part: channels differ by 32 hp
+      if ((32 << st) < block) {
 #pragma unroll
-      for (int e = 0; e < 64; e++) {
-        const float other = xch[((half ^ 1) * 64 + e) * kRowsT + row];
-        o[e] = half ? other - o[e] : o[e] + other;
+        for (int e = 0; e < 32; e++) xch[(part * 32 + e) * kRowsT + row] = o[e];
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + quarter) : "memory");
+#pragma unroll
+        for (int e = 0; e < 32; e++) {
+          const float other = xch[((part ^ hp) * 32 + e) * kRowsT + row];
+          o[e] = (part & hp) ? other - o[e] : o[e] + other;
+        }
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + quarter) : "memory");
       }
     }
     if (row_valid && !dead) {
       __half* orow = p.out + ((static_cast<size_t>(cq0) + ti_row) * p.num_kv_heads * G + h * G + row % G) * kD +
-                     64 * half;
+                     32 * part;
 #pragma unroll
-      for (int c8 = 0; c8 < 8; c8++) {
+      for (int c8 = 0; c8 < 4; c8++) {
         const float* v = o + 8 * c8;
         *reinterpret_cast<uint4*>(orow + 8 * c8) = make_uint4(
             pack_half2(__float2half_rn(v[0] * p.cb), __float2half_rn(v[1] * p.cb)),
