@@ -165,10 +165,11 @@ def test_nvfp4_prefill_append_full_size():
     _full_size_parity(W["prefill_append"], 128, 203, fmt=1)
 
 
-def test_chunked_prefill_full_size():
-    """16 sequences x a 512-token chunk after 3584 cached tokens (one layer): sampled query
-    rows of the chunk against the oracle (query i of a chunk is the one query of a chunk of
-    length 1 over the first L - C + i + 1 tokens)."""
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_chunked_prefill_full_size(fmt):
+    """16 sequences x a 512-token chunk after 3584 cached tokens (one layer), on the INT4
+    and the NVFP4 cache: sampled query rows of the chunk against the oracle (query i of a
+    chunk is the one query of a chunk of length 1 over the first L - C + i + 1 tokens)."""
     import torch
 
     import bit_paged_kv_diag_b200 as kvq
@@ -180,7 +181,7 @@ def test_chunked_prefill_full_size():
     S, H = w.page_size, w.num_kv_heads
     P = workloads.pool_pages(w, cap)
     mp = int((cap.max() + S - 1) // S)
-    desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, w.batch, mp)
+    desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, w.batch, mp, fmt)
     pool = torch.zeros(kvq.pool_bytes(desc), dtype=torch.uint8, device=dev)
     cache, pt = kvq.alloc_pages(desc, cap, None, pool=pool)
     ptd = torch.from_numpy(pt).to(dev)
@@ -197,12 +198,12 @@ def test_chunked_prefill_full_size():
     host_pool = pool.cpu().numpy()
     host_out = out.float().cpu().numpy()
     cache.close()
-    g = oracle.Geometry(1, H, w.num_q_heads, 128, w.block, S, P, mp)
-    rng = np.random.default_rng(104)
+    g = oracle.Geometry(1, H, w.num_q_heads, 128, w.block, S, P, mp, fmt)
+    rng = np.random.default_rng(104 + fmt)
     for b in rng.choice(w.batch, 3, replace=False):
         for i in sorted({0, int(chunk[b]) - 1, *rng.integers(0, int(chunk[b]), 4).tolist()}):
             row = int(cu_q[b]) + i
             pos = int(cap[b] - chunk[b]) + i
             ref = oracle.prefill_attention(g, host_pool, 0, q[row:row + 1], np.array([0, 1], np.int32),
                                            np.array([pos + 1], np.int32), pt[b:b + 1])
-            check_outputs(host_out[row:row + 1], ref, f"chunked prefill b={b} i={i}")
+            check_outputs(host_out[row:row + 1], ref, f"chunked prefill fmt={fmt} b={b} i={i}")

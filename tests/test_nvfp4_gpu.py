@@ -93,7 +93,7 @@ def test_nvfp4_prefill_workloads(name, lengths, chunks):
 
 
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
-@pytest.mark.parametrize("page_size", [16, 32, 64, 256])
+@pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])
 def test_nvfp4_prefill_group_and_page_size_grid(group, page_size):
     import dataclasses
     from harness import prefill_parity
