@@ -93,3 +93,15 @@ def test_prefill_and_fused_bad_inputs_set_status_without_fault():
     assert st & kvq.KVQ_DEV_BAD_POS and st & kvq.KVQ_DEV_BAD_PAGE
     assert kvq.get_device_status(cache) == 0
     cache.close()
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_prefill_at_the_batch_limit(fmt):
+    """4096 sequences (the descriptor's maximum, where the kernel's per-sequence prefix takes
+    the most shared memory) of 0..6 cached tokens with chunks of 0..2 tokens."""
+    import numpy as np
+    rng = np.random.default_rng(4096 + fmt)
+    lengths = rng.integers(0, 7, 4096)
+    chunks = rng.integers(0, 3, 4096)
+    w = dataclasses.replace(W["tiny"], batch=4096)
+    prefill_parity(make_case(w, lengths, chunks, max_batch=4096, fmt=fmt))
