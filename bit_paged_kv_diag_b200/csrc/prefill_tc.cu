@@ -1,5 +1,6 @@
-// prefill_tc.cu -- causal chunked-prefill attention over the rotated-INT4 paged KV cache on
-// the 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory), sm_100a.
+// prefill_tc.cu -- causal chunked-prefill attention over the paged KV cache (rotated INT4 or
+// NVFP4) on the 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory),
+// sm_100a.
 //
 // Method: "KVキャッシュを4ビットへ — SAW-INT4とシステムを踏まえたINT4量子化"
 // (youngju.dev): section "KVキャッシュこそが本当のボトルネックである理由" (attention runs
@@ -10,7 +11,7 @@
 //
 // Work decomposition.  A CTA takes 128 query rows of one (sequence, KV head): 128 / G
 // consecutive chunk tokens times the G query heads of the KV head.  Row r is lane r of tensor
-// memory.  The CTA's 16 warps specialise and hand work to one another through mbarriers, so
+// memory.  The CTA's 22 warps specialise and hand work to one another through mbarriers, so
 // the softmax, the code expansion and the tensor cores overlap instead of taking turns:
 //   warps 0-15   softmax: warps q, q + 4, q + 8, q + 12 all read the lanes of rows 32q..,
 //                warp q + 4j the j-th 32 columns of each tile and of O (four threads per
@@ -23,8 +24,9 @@
 // Tensor-core time per instruction hardly depends on N up to 128 here, so the tiles are as
 // wide as the accumulators allow (S of two tiles, O and q~ fill the 512 TMEM columns).
 // S (tensor memory), the K and V operand tiles and the scales are double-buffered by tile
-// parity; the raw page data streams through four slots.  The causal KV range is cut into
-// tiles of 128 tokens, whose pages are bulk-copied (cp.async.bulk, 1-D, no multicast).
+// parity; the raw page data streams through four slots (three on NVFP4).  The causal KV
+// range is cut into tiles of 128 tokens, whose pages are bulk-copied (cp.async.bulk, 1-D,
+// no multicast).
 //   QK^T  tcgen05.mma kind::f16, M = 128 rows, N = 128 tokens, K = 128 channels: A = q' cut
 //         into fp16 hi + lo parts (q' * 2^14 / M_r, M_r the power of two >= max |q'_r|), held
 //         in tensor memory for the whole CTA; B = the K codes as exact fp16 integers in shared
@@ -89,7 +91,7 @@ constexpr int kColQl = 448;
 constexpr int kKs = 0;                          // [2 buffers][2 kb][128 tokens][128 B] fp16 K codes
 constexpr int kKsBuf = 2 * kTokT * 128;
 // q~ passes through the K buffers on its way to tensor memory (before any K is expanded),
-// and the end exchanges O halves there (after the last QK^T).
+// and the end exchanges the four parts of O there (after the last QK^T).
 constexpr int kQh = kKs;                        // [2 kb][128 rows][128 B] fp16 q~ hi
 constexpr int kQl = kQh + 2 * kRowsT * 128;     // same, lo
 constexpr int kVs = kKs + 2 * kKsBuf;           // [2 buffers][2 nb][128 tokens][128 B] bf16 V codes
@@ -274,8 +276,8 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
-  float* s_kb = reinterpret_cast<float*>(smem + F::kScl);  // [2][64] K scales of tiles t even / odd
-  float* s_vb = s_kb + 2 * kTokT;                       // [2][64] V scales
+  float* s_kb = reinterpret_cast<float*>(smem + F::kScl);  // [2][128] K multipliers, tiles t even / odd
+  float* s_vb = s_kb + 2 * kTokT;                          // [2][128] V multipliers
   float* sfr = reinterpret_cast<float*>(smem + F::kSfr);
   float* red = reinterpret_cast<float*>(smem + F::kRed);  // [tile parity][part][row] maxima
   float* lsum = red + 8 * kRowsT;                         // [part][row] final sums
@@ -372,8 +374,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) prefill_tc_kernel(PrefillParams 
                              full_s + 8 * t, lane, pol, p);
   }
 
-  // q rows: softmax warp w rotates and scales rows 16w..16w+15 (lane: channels 4 lane..
-  // 4 lane + 3) and stores q~ = q' * 2^14 / M as fp16 hi + lo parts into the K-major operands.
+  // q rows: softmax warp w rotates and scales rows 8w..8w+7 (lane: channels 4 lane..
+  // 4 lane + 3) and stores q~ = q' * 2^14 / M as fp16 hi + lo parts into swizzled staging
+  // tiles, from which each softmax thread moves its part of its row into tensor memory.
   if (w < kSoftWarps) {
     for (int rr = 0; rr < kRowsT / kSoftWarps; rr++) {
       const int row = (kRowsT / kSoftWarps) * w + rr;
