@@ -207,3 +207,48 @@ def test_chunked_prefill_full_size(fmt):
             ref = oracle.prefill_attention(g, host_pool, 0, q[row:row + 1], np.array([0, 1], np.int32),
                                            np.array([pos + 1], np.int32), pt[b:b + 1])
             check_outputs(host_out[row:row + 1], ref, f"chunked prefill fmt={fmt} b={b} i={i}")
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_chunked_prefill_long_context(fmt):
+    """The long-context shape (4 KV / 32 query heads, G = 8, page 64, b = 64): a 256-token
+    chunk after 32 512 and after 65 280 cached tokens, so a CTA walks up to 512 KV tiles
+    and its softmax frame moves across hundreds of them; sampled query rows against the
+    oracle."""
+    import torch
+
+    import bit_paged_kv_diag_b200 as kvq
+    w = W["long_context"]
+    dev = torch.device("cuda")
+    chunk = np.array([256, 256], np.int32)
+    cap = np.array([32768, 65536], np.int32)
+    S, H, B = w.page_size, w.num_kv_heads, len(cap)
+    P = int(((cap + S - 1) // S).sum())
+    mp = int((cap.max() + S - 1) // S)
+    desc = kvq.Desc(1, H, w.num_q_heads, 128, w.block, S, P, B, mp, fmt)
+    pool = torch.zeros(kvq.pool_bytes(desc), dtype=torch.uint8, device=dev)
+    cache, pt = kvq.alloc_pages(desc, cap, None, pool=pool)
+    ptd = torch.from_numpy(pt).to(dev)
+    k = workloads.kv_rows_torch(w, 0, 0, int(cap.sum()), stream=1, device=dev)
+    v = workloads.kv_rows_torch(w, 0, 1, int(cap.sum()), stream=1, device=dev)
+    kvq.rotate_quant_append(cache, 0, k, v, torch.from_numpy(workloads.cu_seqlens(cap)).to(dev),
+                            torch.zeros(B, dtype=torch.int32, device=dev), ptd)
+    del k, v
+    cu_q = workloads.cu_seqlens(chunk)
+    q = workloads.q_rows_chunk(w, 0, int(cu_q[-1]))
+    out = kvq.prefill_attention(cache, 0, torch.from_numpy(q).to(dev),
+                                torch.from_numpy(cu_q).to(dev), torch.from_numpy(cap).to(dev), ptd)
+    torch.cuda.synchronize()
+    assert kvq.get_device_status(cache) == 0
+    host_pool = pool.cpu().numpy()
+    host_out = out.float().cpu().numpy()
+    cache.close()
+    g = oracle.Geometry(1, H, w.num_q_heads, 128, w.block, S, P, mp, fmt)
+    rng = np.random.default_rng(204 + fmt)
+    for b in range(B):
+        for i in sorted({0, int(chunk[b]) - 1, *rng.integers(0, int(chunk[b]), 3).tolist()}):
+            row = int(cu_q[b]) + i
+            pos = int(cap[b] - chunk[b]) + i
+            ref = oracle.prefill_attention(g, host_pool, 0, q[row:row + 1], np.array([0, 1], np.int32),
+                                           np.array([pos + 1], np.int32), pt[b:b + 1])
+            check_outputs(host_out[row:row + 1], ref, f"long-context prefill fmt={fmt} b={b} i={i}")
